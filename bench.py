@@ -1,0 +1,468 @@
+#!/usr/bin/env python3
+"""Decode-step benchmark for the FSQ decode-attention library on B200.
+
+One step = the hot path over one batch: append this step's token of every
+batch row to the packed code cache (encoder GEMM -> FSQ -> pack, written at
+row T-1) and run single-token GQA decode attention over the T cached tokens.
+Metric: context tokens/s (B*T per step) and code GB/s (B*T*G/2 per step).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl fsq|reference]
+                    [--workload qwen3_8b_32x] [--B 16] [--T 131072] [--variant absorbed]
+
+With N > 1 it runs under torch.distributed.run, one rank per GPU; batch rows
+are sharded across ranks (each rank owns B rows of its own; weak scaling) and
+no collective touches the data path.  `--impl reference` times the fp64 CPU
+oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = ("qwen3_8b_32x", 16, 131072)
+SECOND_WORKLOAD = ("qwen3_8b_97x", 16, 131072)
+L2_BYTES = 126 * 1024 * 1024
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def src_digest():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "fsq_latent_decode_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def traffic_record(kernel, workload_key):
+    """Per-launch DRAM traffic from the committed ncu summary, or None when the
+    kernel sources changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    rec = d.get(kernel, {}).get(workload_key)
+    if not rec or rec.get("src_digest") != src_digest():
+        return None
+    return rec.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle reasons sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.f = None
+
+    def start(self):
+        try:
+            self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.flush()
+        rows = [r.split(",") for r in open(self.f.name).read().strip().splitlines() if r.count(",") >= 8]
+        os.unlink(self.f.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i] and "Not" not in r[5 + i]})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+class RawEvents:
+    """cudaEvent_t pairs created through the CUDA runtime directly, so that the
+    library can record them inside its C-ABI call; timed with
+    cudaEventElapsedTime."""
+
+    def __init__(self, n):
+        import ctypes
+        self.rt = None
+        for name in ("libcudart.so.12", "libcudart.so"):
+            try:
+                self.rt = ctypes.CDLL(name)
+                break
+            except OSError:
+                continue
+        if self.rt is None:
+            raise RuntimeError("libcudart not found")
+        self.ct = ctypes
+        self.ev = []
+        for _ in range(n):
+            a, b = ctypes.c_void_p(), ctypes.c_void_p()
+            assert self.rt.cudaEventCreate(ctypes.byref(a)) == 0 and self.rt.cudaEventCreate(ctypes.byref(b)) == 0
+            self.ev.append((a.value, b.value))
+
+    def pair(self, i):
+        class _E:  # the binding reads .cuda_event
+            def __init__(self, h):
+                self.cuda_event = h
+        a, b = self.ev[i]
+        return (_E(a), _E(b))
+
+    def elapsed_ms(self, i):
+        ms = self.ct.c_float()
+        a, b = self.ev[i]
+        rc = self.rt.cudaEventElapsedTime(self.ct.byref(ms), self.ct.c_void_p(a), self.ct.c_void_p(b))
+        if rc != 0:
+            raise RuntimeError(f"cudaEventElapsedTime failed ({rc})")
+        return ms.value
+
+    def close(self):
+        for a, b in self.ev:
+            self.rt.cudaEventDestroy(self.ct.c_void_p(a))
+            self.rt.cudaEventDestroy(self.ct.c_void_p(b))
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+# --------------------------------------------------------------------------- GPU arm
+def build_state(torch, F, synth, wl, B, T, rank, device, n_copies):
+    """Device-resident cache(s) plus the step's new-token rows, weights and
+    queries.  Cached rows are the library's FSQ codes of seeded pre-activations
+    u ~ N(0, 4), the law of E x for the seeded E and x (so the full cache does
+    not need x materialised); each step's new token goes through the whole
+    append path (encoder GEMM, FSQ, pack)."""
+    G, C = wl.G, wl.C
+    half = G // 2
+    T_max = T
+    while (T_max * half) % 16:
+        T_max += 1
+    seed = synth.workload_seed(0, rank, B, T, G)
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    E = synth.normal((G, C), (4.0 / C) ** 0.5, gen, device=device)
+    W_kv, q = synth.decoder_inputs(B, wl.n_q, wl.n_kv, wl.d_h, G, gen, device=device)
+    caches = []
+    chunk = 1 << 16
+    for c in range(n_copies):
+        cache = torch.empty((B, T_max, half), dtype=torch.uint8, device=device)
+        flat = cache.view(B * T_max, half)
+        for b in range(B):
+            for t0 in range(0, T, chunk):
+                n = min(chunk, T - t0)
+                u = synth.preactivations(n, G, gen, device=device)
+                F.quantize_pack_f32(u, out=flat[b * T_max + t0: b * T_max + t0 + n])
+        caches.append(cache)
+    x_new = synth.normal((B, C), 1.0, gen, device=device)
+    torch.cuda.synchronize()
+    return dict(E=E, W_kv=W_kv, q=q, caches=caches, x_new=x_new, T_max=T_max)
+
+
+def run_gpu(args, wl_name, B, T, torch, F, synth, dist, rank, world, device, timed=True):
+    wl = synth.WORKLOADS[wl_name]
+    G = wl.G
+    half = G // 2
+    code_bytes = B * T * half
+    n_copies = max(1, math.ceil(2 * L2_BYTES / code_bytes)) if code_bytes < 2 * L2_BYTES else 1
+    n_copies = min(n_copies, 8)
+    st = build_state(torch, F, synth, wl, B, T, rank, device, n_copies)
+    q, W_kv, E, x_new = st["q"], st["W_kv"], st["E"], st["x_new"]
+    T_max = st["T_max"]
+    bstride = T_max * half
+    ws = F.Workspace(device)
+    out = torch.empty((B, wl.n_q, wl.d_h), dtype=torch.bfloat16, device=device)
+    stream = torch.cuda.current_stream()
+    qp = F.quant_params()
+    nbytes_ws = F.workspace_size(B, T, wl.n_q, wl.n_kv, wl.d_h, G, F.attn_opts(variant=args.variant))
+    wbuf = ws.get(nbytes_ws)
+    sptr = stream.cuda_stream
+
+    def step(i, prof=None):
+        cache = st["caches"][i % n_copies]
+        # append this step's token of every batch row at position T-1 (rows strided by the batch stride)
+        rc = F.encode_pack_raw(x_new.data_ptr(), B, wl.C, wl.C, E.data_ptr(), G, qp,
+                               cache.data_ptr() + (T - 1) * half, bstride, sptr)
+        if rc:
+            raise F.FsqError(rc, "fsq_encode_pack")
+        opts = F.attn_opts(variant=args.variant, prof_events=prof)
+        rc = F.decode_attn_raw(q.data_ptr(), B, wl.n_q, wl.d_h, cache.data_ptr(), bstride, T, G,
+                               W_kv.data_ptr(), wl.n_kv, opts, wbuf.data_ptr(), wbuf.numel(), out.data_ptr(), sptr)
+        if rc:
+            raise F.FsqError(rc, "fsq_decode_attn")
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    K = args.steps
+    evs = RawEvents(K)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(torch.cuda.current_device()) if (timed and rank == 0) else None
+    if clocks:
+        clocks.start()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(K):
+        step(i, evs.pair(i))
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop() if clocks else None
+    ms = t0.elapsed_time(t1) / K
+    kern_ms = sum(evs.elapsed_ms(i) for i in range(K)) / K
+    evs.close()
+    if dist is not None:
+        t = torch.tensor([ms, kern_ms], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, kern_ms = float(t[0]), float(t[1])
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if timed:
+        q_h = q.cpu().pin_memory()
+        x_h = x_new.cpu().pin_memory()
+        o_h = torch.empty((B, wl.n_q, wl.d_h), dtype=torch.bfloat16).pin_memory()
+        q_d = torch.empty_like(q)
+        x_d = torch.empty_like(x_new)
+
+        def e2e_step(i):
+            q_d.copy_(q_h, non_blocking=True)
+            x_d.copy_(x_h, non_blocking=True)
+            cache = st["caches"][i % n_copies]
+            rc = F.encode_pack_raw(x_d.data_ptr(), B, wl.C, wl.C, E.data_ptr(), G, qp,
+                                   cache.data_ptr() + (T - 1) * half, bstride, sptr)
+            if rc:
+                raise F.FsqError(rc, "fsq_encode_pack")
+            rc = F.decode_attn_raw(q_d.data_ptr(), B, wl.n_q, wl.d_h, cache.data_ptr(), bstride, T, G,
+                                   W_kv.data_ptr(), wl.n_kv, F.attn_opts(variant=args.variant), wbuf.data_ptr(),
+                                   wbuf.numel(), out.data_ptr(), sptr)
+            if rc:
+                raise F.FsqError(rc, "fsq_decode_attn")
+            o_h.copy_(out, non_blocking=True)
+
+        for i in range(args.warmup):
+            e2e_step(i)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(K):
+            e2e_step(i)
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = a.elapsed_time(b) / K
+        if dist is not None:
+            t = torch.tensor([e_ms], device=device, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t[0])
+        e2e = {"value": world * B * T / (e_ms * 1e-3), "unit": "context tokens/s",
+               "h2d_bytes_per_step": q_h.numel() * 2 + x_h.numel() * 2, "d2h_bytes_per_step": o_h.numel() * 2,
+               "ms_per_step": e_ms}
+    return dict(ms=ms, kern_ms=kern_ms, clocks=clk, e2e=e2e, n_copies=n_copies, wl=wl, B=B, T=T,
+                code_bytes=code_bytes)
+
+
+def roofline(res, peaks, kernel_name):
+    wl, B, T = res["wl"], res["B"], res["T"]
+    G, n_q, d_h = wl.G, wl.n_q, wl.d_h
+    bytes_alg = B * T * (G // 2)
+    flops_alg = B * T * 4 * n_q * G  # scores + latent pooling; per-query W_k^T q and W_v run outside this kernel
+    t = res["kern_ms"] * 1e-3
+    t_b = bytes_alg / (peaks["hbm_gbs"] * 1e9)
+    t_f = flops_alg / (peaks["bf16_tflops"] * 1e12)
+    key = f"{wl.name}_B{B}_T{T}"
+    traffic = traffic_record(kernel_name, key)
+    if t_f >= t_b:
+        ach = flops_alg / t / 1e12
+        r = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+             "frac": ach / peaks["bf16_tflops"]}
+    else:
+        ach = bytes_alg / t / 1e9
+        r = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"]}
+    r.update({"traffic": traffic, "kernel": kernel_name, "kernel_ms": res["kern_ms"],
+              "code_gbs": bytes_alg / t / 1e9, "frac_of_roofline": max(t_b, t_f) / t,
+              "algorithmic_bytes": bytes_alg, "algorithmic_flops": flops_alg,
+              "peak_source": peaks["source"] + " (burst)"})
+    return r
+
+
+def _oracle_setup(wl_name, Ts):
+    from fsq_latent_decode_b200 import synth
+    from oracle import fsq_oracle as O
+    wl = synth.WORKLOADS[wl_name]
+    gen = synth._gen(123)
+    W, q = synth.decoder_inputs(1, wl.n_q, wl.n_kv, wl.d_h, wl.G, gen)
+    u = synth.preactivations(Ts, wl.G, gen).numpy()
+    codes = O.quantize_pack(u)[None]
+    qn, Wn = q.float().numpy(), W.float().numpy()
+    return lambda: O.decode_attn(qn, codes, Wn, wl.n_kv, wl.G), wl
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return int(max([i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"] or [1]))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline_oracle(wl_name, T, budget_s=20.0):
+    """The fp64 oracle as it stands, timed on one batch row of the workload."""
+    Ts = min(T, 8192)
+    fn, wl = _oracle_setup(wl_name, Ts)
+    reps, el = 0, 0.0
+    while True:
+        t0 = time.perf_counter()
+        fn()
+        el += time.perf_counter() - t0
+        reps += 1
+        if reps >= 50 or el * (reps + 1) / reps > budget_s:
+            break
+    return {"value": reps * Ts / el, "unit": "context tokens/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"fp64 oracle decode of 1 batch row x {Ts} cached tokens (all {wl.n_q} heads, K and V expanded "
+                      f"through W_kv), {reps} repetitions in {el:.1f} s"}
+
+
+def reference_arm(wl_name, T, K, W, total_budget_s=150.0):
+    """--impl reference: the oracle as the reference arm, K timed steps of a
+    bounded sample (one batch row, Ts cached tokens) sized to end in minutes."""
+    cal_fn, _ = _oracle_setup(wl_name, 1024)
+    t0 = time.perf_counter()
+    cal_fn()
+    per_tok = (time.perf_counter() - t0) / 1024
+    Ts = int(total_budget_s / max(1, K + W) / max(per_tok, 1e-9))
+    Ts = max(256, min(T, 8192, Ts))
+    fn, wl = _oracle_setup(wl_name, Ts)
+    for _ in range(W):
+        fn()
+    t0 = time.perf_counter()
+    for _ in range(K):
+        fn()
+    el = time.perf_counter() - t0
+    val = K * Ts / el
+    cb = {"value": val, "unit": "context tokens/s", "cores": _blas_threads(), "kind": "oracle",
+          "sample": f"per step: fp64 oracle decode of 1 batch row x {Ts} cached tokens (all {wl.n_q} heads)"}
+    return val, el / K * 1e3, cb
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="fsq", choices=["fsq", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD[0])
+    ap.add_argument("--B", type=int, default=None)
+    ap.add_argument("--T", type=int, default=None)
+    ap.add_argument("--variant", default="absorbed", choices=["absorbed", "expand"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-second", action="store_true", help="skip the G=84 companion measurement")
+    args = ap.parse_args()
+    rank, world, local = dist_env()
+    wl_name = args.workload
+    from fsq_latent_decode_b200 import synth
+    wl = synth.WORKLOADS[wl_name]
+    B = args.B if args.B is not None else (DEFAULT_WORKLOAD[1] if wl_name == DEFAULT_WORKLOAD[0] else wl.batches[-1])
+    T = args.T if args.T is not None else (DEFAULT_WORKLOAD[2] if wl_name == DEFAULT_WORKLOAD[0] else wl.lengths[-1])
+    config = {"workload": f"{wl_name}: Qwen3-8B-shaped layer, n_q={wl.n_q} n_kv={wl.n_kv} d_h={wl.d_h} G={wl.G} "
+                          f"({wl.G // 2} B/token), C={wl.C}, batch {B} per GPU, T={T}",
+              "B_per_gpu": B, "T": T, "G": wl.G, "n_q": wl.n_q, "n_kv": wl.n_kv, "d_h": wl.d_h, "C": wl.C,
+              "variant": args.variant, "parallelism": f"replicas x{world} (batch rows sharded, no collective)"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        val, ms, cb = reference_arm(wl_name, T, max(1, args.steps), max(0, args.warmup))
+        line = {"impl": "reference", "metric": "FSQ decode-attn context tok/s & code GB/s, Qwen3-8B G=256/84; % roofline",
+                "value": val, "unit": "context tokens/s", "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f64", "data": "synthetic (seeded; codes = oracle FSQ of u ~ N(0,4))", "config": config,
+                "cpu_baseline": cb,
+                "e2e": {"value": val, "unit": "context tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return 0
+
+    import torch
+    import fsq_latent_decode_b200 as F
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist_mod
+        torch.cuda.set_device(local)
+        dist_mod.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        dist = dist_mod
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    peaks = load_peaks()
+    kernel_name = "absorbed_split" if args.variant == "absorbed" else "expand_split"
+    res = run_gpu(args, wl_name, B, T, torch, F, synth, dist, rank, world, device)
+    also = None
+    if not args.no_second and wl_name == DEFAULT_WORKLOAD[0] and args.B is None and args.T is None:
+        r2 = run_gpu(args, SECOND_WORKLOAD[0], SECOND_WORKLOAD[1], SECOND_WORKLOAD[2], torch, F, synth, dist, rank,
+                     world, device, timed=False)
+        rf2 = roofline(r2, peaks, kernel_name)
+        also = {"workload": f"{SECOND_WORKLOAD[0]} B={SECOND_WORKLOAD[1]} T={SECOND_WORKLOAD[2]} G=84",
+                "value": world * r2["B"] * r2["T"] / (r2["ms"] * 1e-3), "unit": "context tokens/s",
+                "ms_per_step": r2["ms"], "code_gbs": rf2["code_gbs"], "roofline": rf2,
+                "l2": f"{r2['n_copies']} rotating caches"}
+    cb = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = cpu_baseline_oracle(wl_name, T)
+    if rank == 0:
+        rf = roofline(res, peaks, kernel_name)
+        value = world * B * T / (res["ms"] * 1e-3)
+        config["l2"] = ("codes larger than L2 (%.0f MB per cache)" % (res["code_bytes"] / 1e6) if res["n_copies"] == 1
+                        else f"{res['n_copies']} rotating caches > 2x L2")
+        line = {"metric": "FSQ decode-attn context tok/s & code GB/s, Qwen3-8B G=256/84; % roofline",
+                "value": value, "unit": "context tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": res["ms"], "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f32",
+                "data": "synthetic (seeded; cache = FSQ codes of u ~ N(0,4), the law of E x; new token x ~ N(0,1) appended each step)",
+                "config": config, "code_gbs": world * res["code_bytes"] / (res["ms"] * 1e-3) / 1e9,
+                "roofline": rf, "cpu_baseline": cb, "e2e": res["e2e"], "clocks": res["clocks"],
+                "gpu_launches": args.steps * 4, "also": also}
+        print(json.dumps(line))
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

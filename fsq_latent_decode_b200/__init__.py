@@ -1,0 +1,17 @@
+"""fsq_latent_decode_b200 — B200 (sm_100a) CUDA library for Transformer-FSQ's
+decode hot path: append tokens to a nibble-packed 4-bit FSQ code cache and
+run single-token GQA attention directly over the codes.
+
+The compute lives in libfsq.so (C ABI, include/fsq.h); this package is its
+ctypes binding plus seeded synthetic inputs.  PyTorch only provides device
+memory and streams.
+"""
+from ._abi import (  # noqa: F401
+    EXPORTED, FSQ_OK, FSQ_ERR_CUDA, FSQ_ERR_INVALID_ARG, FSQ_ERR_MISALIGNED, FSQ_ERR_TIMEOUT,
+    FSQ_ERR_UNSUPPORTED, FSQ_ERR_WORKSPACE, AttnOpts, FsqError, QuantParams, Workspace, attn_opts,
+    decode_attn, decode_attn_raw, encode_pack, encode_pack_raw, lib, quant_params, quantize_pack_f32,
+    quantize_pack_f32_raw, status_string, thresholds, workspace_size, workspace_status,
+)
+
+__all__ = ["encode_pack", "quantize_pack_f32", "decode_attn", "attn_opts", "thresholds", "workspace_size",
+           "Workspace", "FsqError"]

@@ -1,0 +1,219 @@
+"""ctypes binding of libfsq.so (declared in include/fsq.h).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  If the shared library is missing the import fails loudly; there is
+no fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import math
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libfsq.so")
+
+FSQ_OK = 0
+FSQ_ERR_INVALID_ARG = -1
+FSQ_ERR_UNSUPPORTED = -2
+FSQ_ERR_MISALIGNED = -3
+FSQ_ERR_WORKSPACE = -4
+FSQ_ERR_CUDA = -5
+FSQ_ERR_TIMEOUT = -6
+
+VARIANT_AUTO, VARIANT_ABSORBED, VARIANT_EXPAND = 0, 1, 2
+VARIANTS = {"auto": VARIANT_AUTO, "absorbed": VARIANT_ABSORBED, "expand": VARIANT_EXPAND}
+
+# Every symbol include/fsq.h declares.
+EXPORTED = ("fsq_attn_opts_default", "fsq_thresholds", "fsq_encode_pack", "fsq_quantize_pack_f32",
+            "fsq_decode_attn_workspace_size", "fsq_decode_attn", "fsq_workspace_status",
+            "fsq_status_string", "fsq_format_version")
+
+
+class QuantParams(C.Structure):
+    _fields_ = [("h", C.c_float), ("delta", C.c_float)]
+
+
+class AttnOpts(C.Structure):
+    _fields_ = [("variant", C.c_int), ("scale", C.c_float), ("num_splits", C.c_int),
+                ("rope_knorm", C.c_int), ("rope_base", C.c_float), ("knorm_gain", C.c_void_p),
+                ("knorm_eps", C.c_float), ("out_fp32", C.c_int), ("prof_events", C.c_void_p * 2)]
+
+
+class FsqError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} ({status})")
+
+
+def _load() -> C.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run `python -m fsq_latent_decode_b200.build` "
+                          "(the CUDA library is required; there is no CPU fallback)")
+    lib = C.CDLL(LIB_PATH)
+    i64, i32, vp, f32 = C.c_int64, C.c_int, C.c_void_p, C.c_float
+    lib.fsq_attn_opts_default.argtypes = [C.POINTER(AttnOpts)]
+    lib.fsq_attn_opts_default.restype = None
+    lib.fsq_thresholds.argtypes = [QuantParams, C.POINTER(C.c_float)]
+    lib.fsq_thresholds.restype = i32
+    lib.fsq_encode_pack.argtypes = [vp, i64, i64, i64, vp, i32, QuantParams, vp, i64, vp]
+    lib.fsq_encode_pack.restype = i32
+    lib.fsq_quantize_pack_f32.argtypes = [vp, i64, i32, QuantParams, vp, i64, vp]
+    lib.fsq_quantize_pack_f32.restype = i32
+    lib.fsq_decode_attn_workspace_size.argtypes = [i64, i64, i32, i32, i32, i32, C.POINTER(AttnOpts)]
+    lib.fsq_decode_attn_workspace_size.restype = C.c_size_t
+    lib.fsq_decode_attn.argtypes = [vp, i64, i32, i32, vp, i64, i64, i32, vp, i32, C.POINTER(AttnOpts),
+                                    vp, C.c_size_t, vp, vp]
+    lib.fsq_decode_attn.restype = i32
+    lib.fsq_workspace_status.argtypes = [vp, C.c_size_t, vp]
+    lib.fsq_workspace_status.restype = i32
+    lib.fsq_status_string.argtypes = [i32]
+    lib.fsq_status_string.restype = C.c_char_p
+    lib.fsq_format_version.argtypes = []
+    lib.fsq_format_version.restype = i32
+    return lib
+
+
+lib = _load()
+
+
+def status_string(s: int) -> str:
+    return lib.fsq_status_string(int(s)).decode()
+
+
+def _check(st: int, what: str):
+    if st != FSQ_OK:
+        raise FsqError(st, what)
+
+
+def quant_params(h: float = 7.5, delta: float = 0.5) -> QuantParams:
+    return QuantParams(float(h), float(delta))
+
+
+def thresholds(h: float = 7.5, delta: float = 0.5):
+    buf = (C.c_float * 15)()
+    _check(lib.fsq_thresholds(quant_params(h, delta), buf), "fsq_thresholds")
+    return [buf[i] for i in range(15)]
+
+
+def attn_opts(variant="auto", scale=0.0, num_splits=0, rope_knorm=False, rope_base=1.0e6,
+              knorm_gain=None, knorm_eps=1e-6, out_fp32=False, prof_events=None) -> AttnOpts:
+    o = AttnOpts()
+    lib.fsq_attn_opts_default(C.byref(o))
+    o.variant = VARIANTS[variant] if isinstance(variant, str) else int(variant)
+    o.scale = float(scale)
+    o.num_splits = int(num_splits)
+    o.rope_knorm = int(bool(rope_knorm))
+    o.rope_base = float(rope_base)
+    o.knorm_gain = None if knorm_gain is None else int(knorm_gain.data_ptr())
+    o.knorm_eps = float(knorm_eps)
+    o.out_fp32 = int(bool(out_fp32))
+    if prof_events is not None:  # a pair of objects exposing a raw cudaEvent_t as .cuda_event
+        o.prof_events[0] = int(prof_events[0].cuda_event)
+        o.prof_events[1] = int(prof_events[1].cuda_event)
+    return o
+
+
+def _stream_ptr(stream) -> int:
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(s.cuda_stream)
+
+
+def _ptr(t) -> int:
+    return int(t.data_ptr())
+
+
+# ---------------------------------------------------------------- raw C-ABI calls (pointers in, status out)
+def encode_pack_raw(x_ptr, n_tok, ldx, C_, E_ptr, G, qp, codes_ptr, ldc, stream_ptr) -> int:
+    return lib.fsq_encode_pack(x_ptr, n_tok, ldx, C_, E_ptr, G, qp, codes_ptr, ldc, stream_ptr)
+
+
+def quantize_pack_f32_raw(u_ptr, n_tok, G, qp, codes_ptr, ldc, stream_ptr) -> int:
+    return lib.fsq_quantize_pack_f32(u_ptr, n_tok, G, qp, codes_ptr, ldc, stream_ptr)
+
+
+def workspace_size(B, T, n_q, n_kv, d_h, G, opts: AttnOpts | None = None) -> int:
+    return int(lib.fsq_decode_attn_workspace_size(B, T, n_q, n_kv, d_h, G,
+                                                  None if opts is None else C.byref(opts)))
+
+
+def decode_attn_raw(q_ptr, B, n_q, d_h, codes_ptr, bstride, T, G, wkv_ptr, n_kv, opts, ws_ptr, ws_bytes,
+                    o_ptr, stream_ptr) -> int:
+    return lib.fsq_decode_attn(q_ptr, B, n_q, d_h, codes_ptr, bstride, T, G, wkv_ptr, n_kv,
+                               None if opts is None else C.byref(opts), ws_ptr, ws_bytes, o_ptr, stream_ptr)
+
+
+def workspace_status(ws, stream=None) -> int:
+    return lib.fsq_workspace_status(_ptr(ws), ws.numel() * ws.element_size(), _stream_ptr(stream))
+
+
+# ---------------------------------------------------------------- tensor-level wrappers (torch for memory only)
+def encode_pack(x, E, h=7.5, delta=0.5, out=None, stream=None):
+    """codes[n_tok, G/2] (uint8) for bf16 rows x[n_tok, C] through E[G, C]."""
+    import torch
+    n_tok, C_ = x.shape
+    G = E.shape[0]
+    if out is None:
+        out = torch.empty((n_tok, G // 2), dtype=torch.uint8, device=x.device)
+    ldc = out.stride(0) if out.dim() == 2 else G // 2
+    st = encode_pack_raw(_ptr(x), n_tok, x.stride(0), C_, _ptr(E), G, quant_params(h, delta), _ptr(out), ldc,
+                         _stream_ptr(stream))
+    _check(st, "fsq_encode_pack")
+    return out
+
+
+def quantize_pack_f32(u, h=7.5, delta=0.5, out=None, stream=None):
+    import torch
+    n_tok, G = u.shape
+    if out is None:
+        out = torch.empty((n_tok, G // 2), dtype=torch.uint8, device=u.device)
+    st = quantize_pack_f32_raw(_ptr(u), n_tok, G, quant_params(h, delta), _ptr(out), out.stride(0),
+                               _stream_ptr(stream))
+    _check(st, "fsq_quantize_pack_f32")
+    return out
+
+
+class Workspace:
+    """Caller-owned device workspace, grown on demand (torch allocates it)."""
+
+    def __init__(self, device="cuda"):
+        self.device = device
+        self.buf = None
+
+    def get(self, nbytes: int):
+        import torch
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=self.device)
+        return self.buf
+
+
+def decode_attn(q, codes, W_kv, T, n_kv, G, code_batch_stride=None, opts=None, workspace=None, out=None,
+                stream=None):
+    """o[B, n_q, d_h] = GQA decode attention over codes[B, T_max, G/2] (first T rows)."""
+    import torch
+    B, n_q, d_h = q.shape
+    if opts is None:
+        opts = attn_opts()
+    if code_batch_stride is None:
+        # a size-1 leading dim may carry any stride (numpy gives 0); use the row extent then
+        if codes.dim() == 3 and codes.shape[0] > 1:
+            code_batch_stride = codes.stride(0)
+        elif codes.dim() == 3:
+            code_batch_stride = codes.shape[1] * codes.shape[2]
+        else:
+            code_batch_stride = T * (G // 2)
+    nbytes = workspace_size(B, T, n_q, n_kv, d_h, G, opts)
+    if nbytes == 0:
+        raise FsqError(FSQ_ERR_INVALID_ARG, "fsq_decode_attn_workspace_size")
+    ws = (workspace or Workspace(q.device)).get(nbytes)
+    if out is None:
+        out = torch.empty((B, n_q, d_h), dtype=torch.float32 if opts.out_fp32 else torch.bfloat16, device=q.device)
+    st = decode_attn_raw(_ptr(q), B, n_q, d_h, _ptr(codes), code_batch_stride, T, G, _ptr(W_kv), n_kv, opts,
+                         _ptr(ws), ws.numel(), _ptr(out), _stream_ptr(stream))
+    _check(st, "fsq_decode_attn")
+    return out
+
+
+def default_scale(d_h: int) -> float:
+    return 1.0 / math.sqrt(d_h)

@@ -1,0 +1,260 @@
+// C ABI of the library: argument validation, launch planning, dispatch.
+// Every check that can fail runs before any CUDA call, so invalid requests
+// return synchronously without touching the device.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "common.cuh"
+
+namespace fsq {
+cudaError_t launch_encode_pack_simt(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C, const uint16_t *E,
+                                    int G, const Thresholds &th, uint8_t *codes, int64_t ldc, cudaStream_t s);
+cudaError_t launch_quantize_pack_f32(const float *u, int64_t n_tok, int G, const Thresholds &th, uint8_t *codes,
+                                     int64_t ldc, cudaStream_t s);
+cudaError_t launch_absorbed_simt(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
+                                 int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv, float scale, int S,
+                                 int64_t tps, float *qa, float *part, uint32_t *err, void *o, int out_fp32,
+                                 void *const *prof, cudaStream_t st);
+cudaError_t launch_expand_simt(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
+                               int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv, float scale, int S,
+                               int64_t tps, int rope_knorm, float rope_base, const uint16_t *gain, float eps,
+                               float *part, uint32_t *err, void *o, int out_fp32, void *const *prof,
+                               cudaStream_t st);
+int simt_max_nq();
+int simt_max_grp();
+bool absorbed_tc_supported(int n_q, int G);
+size_t absorbed_tc_qphys_bytes(int n_q, int G);
+cudaError_t launch_absorbed_tc(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
+                               int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv, float scale, int S,
+                               int64_t tps, uint8_t *qphys, float *corr, float *part, uint32_t *err, void *o,
+                               int out_fp32, void *const *prof, cudaStream_t st);
+
+namespace {
+
+constexpr int kMaxSplits = 1024;
+constexpr bool kEnableTc = false;  // tensor-core absorbed kernel (being validated)
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+fsq_status check_quant(fsq_quant_params qp) {
+  if (!(qp.delta > 0.f) || !(qp.h > qp.delta)) return FSQ_ERR_INVALID_ARG;
+  if (!(qp.h - qp.delta <= 7.5f) || !(qp.h + qp.delta <= 8.5f)) return FSQ_ERR_INVALID_ARG;
+  return FSQ_OK;
+}
+
+// Smallest float not below x (x finite).
+float ceil_to_float(double x) {
+  float f = (float)x;
+  if ((double)f < x) f = nextafterf(f, INFINITY);
+  return f;
+}
+
+void make_thresholds(fsq_quant_params qp, float out[15]) {
+  const double h = qp.h, dl = qp.delta;
+  const double a = atanh(dl / h);
+  for (int k = 0; k < 15; ++k) {
+    const double m = (double)(k - 8);         // boundary between levels m and m+1
+    const double arg = (m + 0.5 + dl) / h;    // tanh(u + a) at u~ = m + 1/2
+    if (arg >= 1.0) out[k] = INFINITY;
+    else if (arg <= -1.0) out[k] = -INFINITY;
+    else out[k] = ceil_to_float(atanh(arg) - a);
+  }
+}
+
+struct Plan {
+  int variant;
+  bool tc;        // tensor-core kernel (absorbed form)
+  int S;          // splits per batch row
+  int64_t tps;    // tokens per split
+  size_t off_qa, off_corr, off_part, total;
+};
+
+fsq_status plan_decode(int64_t B, int64_t T, int n_q, int n_kv, int d_h, int G, const fsq_attn_opts &op, Plan *p) {
+  if (B < 0 || T < 1 || n_q < 1 || n_kv < 1 || d_h < 1 || G < 2) return FSQ_ERR_INVALID_ARG;
+  if (n_q % n_kv) return FSQ_ERR_INVALID_ARG;
+  if (G % 2) return FSQ_ERR_UNSUPPORTED;
+  if (G > FSQ_MAX_G || d_h != FSQ_HEAD_DIM) return FSQ_ERR_UNSUPPORTED;
+  if (op.variant < FSQ_VARIANT_AUTO || op.variant > FSQ_VARIANT_EXPAND) return FSQ_ERR_INVALID_ARG;
+  if (op.num_splits < 0) return FSQ_ERR_INVALID_ARG;
+  if (op.rope_knorm != 0 && op.rope_knorm != 1) return FSQ_ERR_INVALID_ARG;
+  int variant = op.variant;
+  if (variant == FSQ_VARIANT_AUTO) variant = op.rope_knorm ? FSQ_VARIANT_EXPAND : FSQ_VARIANT_ABSORBED;
+  if (variant == FSQ_VARIANT_ABSORBED && op.rope_knorm) return FSQ_ERR_UNSUPPORTED;
+  if (variant == FSQ_VARIANT_ABSORBED && n_q > simt_max_nq()) return FSQ_ERR_UNSUPPORTED;
+  if (variant == FSQ_VARIANT_EXPAND && n_q / n_kv > simt_max_grp()) return FSQ_ERR_UNSUPPORTED;
+  if (op.rope_knorm && !(op.rope_base > 1.f && op.knorm_eps >= 0.f)) return FSQ_ERR_INVALID_ARG;
+
+  const int64_t Bc = B > 0 ? B : 1;
+  const bool tc = kEnableTc && variant == FSQ_VARIANT_ABSORBED && absorbed_tc_supported(n_q, G);
+  const int64_t ctas_per_row = variant == FSQ_VARIANT_EXPAND ? n_kv : 1;
+  int64_t S = op.num_splits;
+  if (S == 0) {
+    if (tc) {
+      // one CTA per SM (each holds all of TMEM): fill the 148 SMs in a single wave
+      S = kNumSMs / Bc;
+      if (S < 1) S = 1;
+    } else {
+      const int64_t target = 2 * kNumSMs;
+      S = (target + Bc * ctas_per_row - 1) / (Bc * ctas_per_row);
+      const int64_t max_by_len = (T + 255) / 256;
+      if (S > max_by_len) S = max_by_len;
+    }
+  }
+  if (S < 1) S = 1;
+  if (S > kMaxSplits) S = kMaxSplits;
+  if (S > T) S = T;
+  int64_t tps = (T + S - 1) / S;
+  if (tc) tps = (tps + 127) / 128 * 128;  // whole 128-token tiles, 16-byte aligned split starts
+  S = (T + tps - 1) / tps;  // no empty splits
+  p->variant = variant;
+  p->tc = tc;
+  p->S = (int)S;
+  p->tps = tps;
+  const int acc_len = variant == FSQ_VARIANT_EXPAND ? d_h : G;
+  size_t off = kWsHeader;
+  p->off_qa = off;
+  if (tc) off = align_up(off + absorbed_tc_qphys_bytes(n_q, G) * (size_t)Bc, 256);
+  else if (variant == FSQ_VARIANT_ABSORBED) off = align_up(off + sizeof(float) * (size_t)Bc * n_q * G, 256);
+  p->off_corr = off;
+  if (tc) off = align_up(off + sizeof(float) * (size_t)Bc * n_q, 256);
+  p->off_part = off;
+  off = align_up(off + sizeof(float) * (size_t)Bc * S * n_q * (2 + acc_len), 256);
+  p->total = off;
+  return FSQ_OK;
+}
+
+fsq_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FSQ_OK : FSQ_ERR_CUDA; }
+
+}  // namespace
+}  // namespace fsq
+
+using namespace fsq;
+
+extern "C" {
+
+void fsq_attn_opts_default(fsq_attn_opts *opts) {
+  if (!opts) return;
+  memset(opts, 0, sizeof(*opts));
+  opts->variant = FSQ_VARIANT_AUTO;
+  opts->scale = 0.f;
+  opts->num_splits = 0;
+  opts->rope_knorm = 0;
+  opts->rope_base = 1.0e6f;
+  opts->knorm_gain = nullptr;
+  opts->knorm_eps = 1.0e-6f;
+  opts->out_fp32 = 0;
+  opts->prof_events[0] = opts->prof_events[1] = nullptr;
+}
+
+fsq_status fsq_thresholds(fsq_quant_params qp, float theta_out[15]) {
+  if (!theta_out) return FSQ_ERR_INVALID_ARG;
+  fsq_status st = check_quant(qp);
+  if (st != FSQ_OK) return st;
+  make_thresholds(qp, theta_out);
+  return FSQ_OK;
+}
+
+fsq_status fsq_encode_pack(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C, const uint16_t *E, int G,
+                           fsq_quant_params qp, uint8_t *codes, int64_t ldc_bytes, fsq_stream_t stream) {
+  if (n_tok < 0 || C < 1 || G < 2) return FSQ_ERR_INVALID_ARG;
+  if (G % 2 || G > FSQ_MAX_G || C % 64) return FSQ_ERR_UNSUPPORTED;
+  if (ldx < C || ldc_bytes < G / 2) return FSQ_ERR_INVALID_ARG;
+  fsq_status st = check_quant(qp);
+  if (st != FSQ_OK) return st;
+  if (n_tok == 0) return FSQ_OK;
+  if (!x || !E || !codes) return FSQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(E) || ldx % 8) return FSQ_ERR_MISALIGNED;
+  Thresholds th;
+  make_thresholds(qp, th.th);
+  return from_cuda(launch_encode_pack_simt(x, n_tok, ldx, C, E, G, th, codes, ldc_bytes, (cudaStream_t)stream));
+}
+
+fsq_status fsq_quantize_pack_f32(const float *u, int64_t n_tok, int G, fsq_quant_params qp, uint8_t *codes,
+                                 int64_t ldc_bytes, fsq_stream_t stream) {
+  if (n_tok < 0 || G < 2) return FSQ_ERR_INVALID_ARG;
+  if (G % 2 || G > FSQ_MAX_G) return FSQ_ERR_UNSUPPORTED;
+  if (ldc_bytes < G / 2) return FSQ_ERR_INVALID_ARG;
+  fsq_status st = check_quant(qp);
+  if (st != FSQ_OK) return st;
+  if (n_tok == 0) return FSQ_OK;
+  if (!u || !codes) return FSQ_ERR_INVALID_ARG;
+  if (!aligned16(u)) return FSQ_ERR_MISALIGNED;
+  Thresholds th;
+  make_thresholds(qp, th.th);
+  return from_cuda(launch_quantize_pack_f32(u, n_tok, G, th, codes, ldc_bytes, (cudaStream_t)stream));
+}
+
+size_t fsq_decode_attn_workspace_size(int64_t B, int64_t T, int n_q, int n_kv, int d_h, int G,
+                                      const fsq_attn_opts *opts) {
+  fsq_attn_opts op;
+  if (opts) op = *opts;
+  else fsq_attn_opts_default(&op);
+  Plan p;
+  if (plan_decode(B, T, n_q, n_kv, d_h, G, op, &p) != FSQ_OK) return 0;
+  return p.total;
+}
+
+fsq_status fsq_decode_attn(const uint16_t *q, int64_t B, int n_q, int d_h, const uint8_t *codes,
+                           int64_t code_batch_stride_bytes, int64_t T, int G, const uint16_t *W_kv, int n_kv,
+                           const fsq_attn_opts *opts, void *workspace, size_t workspace_bytes, void *o,
+                           fsq_stream_t stream) {
+  fsq_attn_opts op;
+  if (opts) op = *opts;
+  else fsq_attn_opts_default(&op);
+  Plan p;
+  fsq_status st = plan_decode(B, T, n_q, n_kv, d_h, G, op, &p);
+  if (st != FSQ_OK) return st;
+  if (B == 0) return FSQ_OK;
+  if (!q || !codes || !W_kv || !o) return FSQ_ERR_INVALID_ARG;
+  if (code_batch_stride_bytes < T * (G / 2)) return FSQ_ERR_INVALID_ARG;
+  if (!aligned16(codes) || code_batch_stride_bytes % 16) return FSQ_ERR_MISALIGNED;
+  if (!aligned16(q) || !aligned16(W_kv) || !aligned16(o)) return FSQ_ERR_MISALIGNED;
+  if (!workspace || workspace_bytes < p.total) return FSQ_ERR_WORKSPACE;
+  if ((uintptr_t)workspace & 255u) return FSQ_ERR_MISALIGNED;
+  const float scale = op.scale > 0.f ? op.scale : 1.f / sqrtf((float)d_h);
+  char *ws = (char *)workspace;
+  uint32_t *err = (uint32_t *)ws;
+  float *part = (float *)(ws + p.off_part);
+  cudaStream_t s = (cudaStream_t)stream;
+  cudaError_t e;
+  if (p.tc) {
+    e = launch_absorbed_tc(q, codes, code_batch_stride_bytes, B, T, n_q, n_kv, d_h, G, W_kv, scale, p.S, p.tps,
+                           (uint8_t *)(ws + p.off_qa), (float *)(ws + p.off_corr), part, err, o, op.out_fp32,
+                           op.prof_events, s);
+  } else if (p.variant == FSQ_VARIANT_ABSORBED) {
+    e = launch_absorbed_simt(q, codes, code_batch_stride_bytes, B, T, n_q, n_kv, d_h, G, W_kv, scale, p.S, p.tps,
+                             (float *)(ws + p.off_qa), part, err, o, op.out_fp32, op.prof_events, s);
+  } else {
+    e = launch_expand_simt(q, codes, code_batch_stride_bytes, B, T, n_q, n_kv, d_h, G, W_kv, scale, p.S, p.tps,
+                           op.rope_knorm, op.rope_base, op.knorm_gain, op.knorm_eps, part, err, o, op.out_fp32,
+                           op.prof_events, s);
+  }
+  return from_cuda(e);
+}
+
+fsq_status fsq_workspace_status(const void *workspace, size_t workspace_bytes, fsq_stream_t stream) {
+  if (!workspace || workspace_bytes < kWsHeader) return FSQ_ERR_INVALID_ARG;
+  uint32_t v = 0;
+  cudaError_t e = cudaMemcpyAsync(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);
+  if (e != cudaSuccess) return FSQ_ERR_CUDA;
+  return v == 0 ? FSQ_OK : (fsq_status)(-(int)v);
+}
+
+const char *fsq_status_string(fsq_status s) {
+  switch (s) {
+    case FSQ_OK: return "ok";
+    case FSQ_ERR_INVALID_ARG: return "invalid argument";
+    case FSQ_ERR_UNSUPPORTED: return "unsupported shape or option";
+    case FSQ_ERR_MISALIGNED: return "pointer or stride not 16-byte aligned";
+    case FSQ_ERR_WORKSPACE: return "workspace missing or too small";
+    case FSQ_ERR_CUDA: return "CUDA error";
+    case FSQ_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+int fsq_format_version(void) { return FSQ_FORMAT_VERSION; }
+
+}  // extern "C"

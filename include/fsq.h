@@ -1,0 +1,173 @@
+/*
+ * fsq.h — C ABI of the B200 (sm_100a) library for Transformer-FSQ's decode
+ * hot path: appending tokens to a KV cache that holds only nibble-packed
+ * 4-bit FSQ latent codes, and single-token grouped-query attention read
+ * directly from those codes through the shared decoder W_kv.
+ *
+ * Sources (page titles):
+ *  [S] "Transformer-FSQ: Discrete Latents for Extreme KV-Cache Compression",
+ *      picx.dev summary — Theoretical Basis (eq. 2), Methodology/Architecture
+ *      (eqs. 4, 5), Key Design Innovation (eq. 6), Closed-Form Conversion
+ *      (eq. 8, row order of W_kv), Byte Budgeting.
+ *  [D] Transformer-FSQ slide deck — frames "A wide product code uses four
+ *      bits per coordinate" (L=16, b=4, h=7.5075, delta=0.5, ceil(G*b/8)
+ *      bytes per token), "Attention pools codes before decoding values"
+ *      (eqs. 5-6), "The kernel reads codes and never writes reconstructed
+ *      K/V" (read codes, unpack in registers, tensor cores, online softmax,
+ *      merge partials, apply W_v once).
+ *
+ * Conventions shared by every call
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *    never allocates device memory, never synchronises the host (except
+ *    fsq_workspace_status, which says so) and keeps no global state.
+ *  - bf16 means IEEE bfloat16 stored as uint16; row-major throughout.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default).
+ *  - Argument errors are returned synchronously, before anything is
+ *    launched.  A failed launch returns FSQ_ERR_CUDA.  A bounded device-side
+ *    wait that gives up records FSQ_ERR_TIMEOUT in the workspace's error word
+ *    (see fsq_workspace_status) instead of hanging or trapping.
+ *
+ * Cache format (FSQ_FORMAT_VERSION 1)
+ *  - A token's G levels z_i in {-8..7} are stored as nibbles n_i = z_i + 8.
+ *    Byte i of the token's row holds coordinate 2i in its low nibble and
+ *    coordinate 2i+1 in its high nibble.  A row is exactly G/2 bytes; no
+ *    scale, zero point or norm is stored ([S] Summary; [D] product-code frame).
+ *  - A layer's cache is [B, T_max, G/2] bytes; row t of batch b starts at
+ *    codes + b*code_batch_stride_bytes + t*G/2.
+ */
+#ifndef FSQ_H_
+#define FSQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FSQ_FORMAT_VERSION 1
+#define FSQ_LEVELS 16
+#define FSQ_MAX_G 256
+#define FSQ_HEAD_DIM 128
+
+#if defined(__GNUC__)
+#define FSQ_API __attribute__((visibility("default")))
+#else
+#define FSQ_API
+#endif
+
+typedef struct CUstream_st *fsq_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  FSQ_OK = 0,
+  FSQ_ERR_INVALID_ARG = -1, /* null pointer, bad size, bad parameter */
+  FSQ_ERR_UNSUPPORTED = -2, /* valid request outside the supported shapes */
+  FSQ_ERR_MISALIGNED = -3,  /* pointer or stride not 16-byte aligned */
+  FSQ_ERR_WORKSPACE = -4,   /* workspace missing or too small */
+  FSQ_ERR_CUDA = -5,        /* a CUDA launch or runtime call failed */
+  FSQ_ERR_TIMEOUT = -6      /* a bounded device wait gave up (device-recorded) */
+} fsq_status;
+
+/* eq. (2) of [S]: u~ = h*tanh(u + atanh(delta/h)) - delta, level = round(u~).
+ * Requires 0 < delta < h, h - delta <= 7.5 and h + delta <= 8.5 so that every
+ * level lies in {-8..7}.  The acceptance default is {7.5, 0.5}; the deck
+ * prints h=7.5075 for L=16 ([D] product-code frame). */
+typedef struct {
+  float h;
+  float delta;
+} fsq_quant_params;
+
+enum {
+  FSQ_VARIANT_AUTO = 0,     /* library picks (ABSORBED when rope_knorm == 0) */
+  FSQ_VARIANT_ABSORBED = 1, /* score with W_k^T q, pool codes, apply W_v once */
+  FSQ_VARIANT_EXPAND = 2    /* rebuild K and V per tile through W_kv, then GQA */
+};
+
+typedef struct {
+  int variant;            /* FSQ_VARIANT_* */
+  float scale;            /* softmax scale; <= 0 selects 1/sqrt(d_h) */
+  int num_splits;         /* token-range splits per batch row; 0 = automatic */
+  int rope_knorm;         /* 1: k_t = RoPE_t(N_k(W_k z_t)) ([S] eq. 5); EXPAND only */
+  float rope_base;        /* RoPE base (rope_knorm == 1) */
+  const uint16_t *knorm_gain; /* device bf16 [d_h] RMS-norm gain, NULL = ones */
+  float knorm_eps;        /* RMS-norm epsilon */
+  int out_fp32;           /* 0: o is bf16; 1: o is fp32 */
+  void *prof_events[2];   /* optional cudaEvent_t pair: recorded on `stream`
+                             right before and right after the main attention
+                             kernel (for timing it alone); NULL = none */
+} fsq_attn_opts;
+
+/* Fills *opts with {AUTO, 1/sqrt(d_h), auto splits, rope off, 1e6, NULL,
+ * 1e-6, bf16 output, no profiling events}. */
+FSQ_API void fsq_attn_opts_default(fsq_attn_opts *opts);
+
+/* Host-side: the 15 ascending u-space decision thresholds the kernels
+ * compare against.  A level is -8 + #{k : u >= theta_k}.  theta_k is the
+ * smallest fp32 value not below the exact preimage of the half-integer
+ * boundary m + 1/2 (m = -8..6) under eq. (2), so for any fp32 u the count
+ * equals the exact rounding of eq. (2) except at an exact tie.  Unreachable
+ * boundaries are +/-infinity.  Returns FSQ_ERR_INVALID_ARG for bad params. */
+FSQ_API fsq_status fsq_thresholds(fsq_quant_params qp, float theta_out[15]);
+
+/* Append path ([S] eq. 4 then packing; [D] product-code frame):
+ *   u = E x_t (bf16 operands, fp32 accumulation), level = eq. (2), packed.
+ *  x      bf16 [n_tok, ldx], row t = x_t (C used entries)      — read
+ *  E      bf16 [G, C] encoder                                    — read
+ *  codes  uint8 [n_tok, ldc_bytes]; row t gets G/2 bytes          — written
+ * To append at position T of a [T_max, G/2] cache pass codes + T*G/2 and
+ * ldc_bytes = G/2.  Needs: G even, 2 <= G <= 256; C a positive multiple of
+ * 64; ldx >= C and ldx % 8 == 0; x and E 16-byte aligned.  n_tok == 0 is a
+ * no-op.  Codes are bit-exact with eq. (2) applied to the fp32 u; the fp32 u
+ * itself differs from exact arithmetic by the GEMM's rounding. */
+FSQ_API fsq_status fsq_encode_pack(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C,
+                           const uint16_t *E, int G, fsq_quant_params qp,
+                           uint8_t *codes, int64_t ldc_bytes, fsq_stream_t stream);
+
+/* Quantiser + packing alone on given fp32 pre-activations u [n_tok, G]
+ * (row-major, contiguous).  Same codes as fsq_encode_pack would write for
+ * that u.  Used to test eq. (2) in isolation. */
+FSQ_API fsq_status fsq_quantize_pack_f32(const float *u, int64_t n_tok, int G, fsq_quant_params qp,
+                                 uint8_t *codes, int64_t ldc_bytes, fsq_stream_t stream);
+
+/* Bytes of device workspace fsq_decode_attn needs for this shape and
+ * options (0 if the arguments are invalid).  Depends only on its
+ * arguments. */
+FSQ_API size_t fsq_decode_attn_workspace_size(int64_t B, int64_t T, int n_q, int n_kv, int d_h, int G,
+                                      const fsq_attn_opts *opts);
+
+/* Single-token GQA decode attention over the packed code cache.
+ * For batch row b and query head h, with kv head j = h / (n_q / n_kv):
+ *   k_t = W_k^(j) z_t (RoPE_t(N_k(.)) when opts->rope_knorm), v_t = W_v^(j) z_t
+ *   o_h = sum_t softmax_t(scale * q_h . k_t) v_t                 ([S] eq. 5)
+ * over cached tokens t = 0..T-1 (the caller appends the current token first;
+ * cached token t sits at position t).  ABSORBED evaluates the same sum as
+ * (W_k^T q_h) . z_t and W_v (sum_t a_t z_t) ([S] eq. 6).
+ *  q        bf16 [B, n_q, d_h], already projected/normed/rotated by the caller
+ *  codes    uint8 cache, rows as in the format above
+ *  W_kv     bf16 [2*n_kv*d_h, G]; rows [W_k; W_v] ([S] eq. 8), head j of W_k
+ *           is rows j*d_h..j*d_h+d_h-1, head j of W_v rows (n_kv+j)*d_h..
+ *  o        [B, n_q, d_h], bf16 or fp32 (opts->out_fp32)          — written
+ *  workspace  >= fsq_decode_attn_workspace_size(...) bytes, 256-byte aligned,
+ *             owned by the caller; contents need no initialisation
+ * Needs: d_h == 128, n_q % n_kv == 0, G even, 2 <= G <= 256, T >= 1; codes
+ * and code_batch_stride_bytes 16-byte aligned, code_batch_stride_bytes >=
+ * T*G/2; q, W_kv, o 16-byte aligned.  B == 0 is a no-op.  opts may be NULL
+ * (defaults). */
+FSQ_API fsq_status fsq_decode_attn(const uint16_t *q, int64_t B, int n_q, int d_h,
+                           const uint8_t *codes, int64_t code_batch_stride_bytes, int64_t T, int G,
+                           const uint16_t *W_kv, int n_kv, const fsq_attn_opts *opts,
+                           void *workspace, size_t workspace_bytes, void *o, fsq_stream_t stream);
+
+/* Reads the device error word of a workspace last used by fsq_decode_attn
+ * (blocking copy: synchronises with `stream`).  Returns FSQ_OK or the
+ * recorded device status (e.g. FSQ_ERR_TIMEOUT); clears nothing. */
+FSQ_API fsq_status fsq_workspace_status(const void *workspace, size_t workspace_bytes, fsq_stream_t stream);
+
+FSQ_API const char *fsq_status_string(fsq_status s);
+FSQ_API int fsq_format_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FSQ_H_ */

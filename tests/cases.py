@@ -1,0 +1,65 @@
+"""Seeded test inputs shared by the parity tests (no method arithmetic here
+except through the oracle, which makes every stored code)."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+from fsq_latent_decode_b200 import synth
+from oracle import fsq_oracle as O
+
+TOL = 5e-3  # max|delta| / max|ref| for attention outputs (bf16 operands, fp32 accumulation)
+
+
+def padded_len(T: int, G: int) -> int:
+    """Smallest T_max >= T whose batch stride T_max*G/2 is a multiple of 16 bytes."""
+    half = G // 2
+    t = T
+    while (t * half) % 16:
+        t += 1
+    return max(t, 1)
+
+
+def oracle_cache(B, T, G, seed, h=7.5, rows=None, T_max=None):
+    """Packed cache [B, T_max, G/2] (numpy uint8).
+
+    Rows in `rows` (default: all) hold the oracle's eq.-(2) codes of seeded
+    pre-activations u ~ N(0, 4) (the law of E x for the seeded E and x);
+    other rows hold uniform random bytes (every byte is a valid code pair)."""
+    T_max = padded_len(T, G) if T_max is None else T_max
+    rows = range(B) if rows is None else rows
+    codes = np.empty((B, T_max, G // 2), dtype=np.uint8)
+    gen = synth._gen(synth.workload_seed(seed, 99))
+    codes[:] = synth.random_bytes((B, T_max, G // 2), gen).numpy()
+    hq = float(np.float32(h))
+    for b in rows:
+        g = synth._gen(synth.workload_seed(seed, b))
+        chunk = 1 << 18
+        for t0 in range(0, T, chunk):
+            n = min(chunk, T - t0)
+            u = synth.preactivations(n, G, g).numpy()
+            codes[b, t0:t0 + n] = O.quantize_pack(u, hq)
+    return codes
+
+
+def rel_err(got, ref) -> float:
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    m = np.isfinite(ref)
+    return float(np.abs(got[m] - ref[m]).max() / np.abs(ref[m]).max())
+
+
+def decoder_weights(n_q, n_kv, G, B, seed, d_h=128):
+    gen = synth._gen(synth.workload_seed(seed, 7))
+    W_kv, q = synth.decoder_inputs(B, n_q, n_kv, d_h, G, gen)
+    return W_kv, q
+
+
+def gemm_error_bound(x, E):
+    """fp32 forward-error bound gamma_C * sum_c |E_ic x_tc| of the encoder GEMM."""
+    Cdim = x.shape[1]
+    u = 2.0 ** -24
+    gam = Cdim * u / (1 - Cdim * u)
+    return gam * (np.abs(np.asarray(x, np.float64)) @ np.abs(np.asarray(E, np.float64)).T)

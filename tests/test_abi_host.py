@@ -1,0 +1,113 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every symbol include/fsq.h declares, computes its threshold table and
+workspace plans, and rejects bad arguments before touching the device."""
+import ctypes as C
+import math
+import os
+import re
+
+import numpy as np
+import pytest
+
+import fsq_latent_decode_b200 as F
+from fsq_latent_decode_b200 import _abi
+from oracle import fsq_oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "fsq.h")).read()
+    return sorted(set(re.findall(r"FSQ_API\s+[^;(]*?\b(fsq_\w+)\s*\(", src)))
+
+
+def test_header_symbols_are_exported():
+    names = declared_symbols()
+    assert len(names) >= 9
+    assert sorted(_abi.EXPORTED) == names
+    for n in names:
+        assert hasattr(F.lib, n), n
+
+
+def test_format_version_and_status_strings():
+    assert F.lib.fsq_format_version() == 1
+    for s in range(0, -7, -1):
+        assert F.status_string(s) and F.status_string(s) != "unknown status"
+
+
+@pytest.mark.parametrize("h", [7.5, 7.5075])
+def test_threshold_table_agrees_with_oracle(h):
+    th = np.array(F.thresholds(h, 0.5), dtype=np.float32)
+    assert np.all(np.diff(th) > 0)
+    h = float(np.float32(h))  # the library's h is an fp32 parameter; evaluate the oracle there
+    for k, t in enumerate(th):
+        below = np.nextafter(t, np.float32(-np.inf), dtype=np.float32)
+        # the oracle (literal tanh) puts theta_k in level k-7 and the fp32 value
+        # just below it in level k-8: theta_k is the first fp32 of the new level
+        lv = O.fsq_quantize(np.array([float(t), float(below)], dtype=np.float64), h, 0.5)
+        assert lv[0] == k - 7 and lv[1] == k - 8, (k, t)
+
+
+def test_threshold_param_checks():
+    for h, d in [(7.5, 0.0), (0.4, 0.5), (9.0, 0.5), (7.9, 0.7)]:
+        with pytest.raises(F.FsqError):
+            F.thresholds(h, d)
+
+
+def _opts(**kw):
+    return F.attn_opts(**kw)
+
+
+def test_workspace_plan_is_deterministic_and_validates():
+    ws = F.workspace_size(16, 131072, 32, 8, 128, 256, _opts())
+    assert ws > 0 and ws % 256 == 0
+    assert ws == F.workspace_size(16, 131072, 32, 8, 128, 256, _opts())
+    assert F.workspace_size(1, 1, 16, 8, 128, 84, _opts()) > 0
+    assert F.workspace_size(1, 0, 16, 8, 128, 84, _opts()) == 0          # T = 0
+    assert F.workspace_size(1, 10, 16, 8, 64, 84, _opts()) == 0          # d_h != 128
+    assert F.workspace_size(1, 10, 12, 8, 128, 84, _opts()) == 0         # n_q % n_kv
+    assert F.workspace_size(1, 10, 16, 8, 128, 85, _opts()) == 0         # odd G
+    assert F.workspace_size(1, 10, 16, 8, 128, 258, _opts()) == 0        # G > 256
+    assert F.workspace_size(1, 10, 16, 8, 128, 84, _opts(variant="absorbed", rope_knorm=True)) == 0
+    assert F.workspace_size(1, 10, 16, 8, 128, 84, _opts(rope_knorm=True)) > 0  # auto -> expand
+
+
+def test_invalid_arguments_return_before_launch():
+    qp = F.quant_params()
+    null = None
+    # encode: bad shapes / params / nulls
+    assert F.encode_pack_raw(null, 4, 64, 64, null, 256, qp, null, 128, null) == F.FSQ_ERR_INVALID_ARG
+    assert F.encode_pack_raw(8, 4, 64, 63, 8, 256, qp, 8, 128, null) == F.FSQ_ERR_UNSUPPORTED
+    assert F.encode_pack_raw(16, 4, 64, 64, 16, 255, qp, 16, 128, null) == F.FSQ_ERR_UNSUPPORTED
+    assert F.encode_pack_raw(16, 4, 32, 64, 16, 256, qp, 16, 128, null) == F.FSQ_ERR_INVALID_ARG
+    assert F.encode_pack_raw(16, 4, 64, 64, 16, 256, qp, 16, 64, null) == F.FSQ_ERR_INVALID_ARG
+    assert F.encode_pack_raw(17, 4, 64, 64, 16, 256, qp, 16, 128, null) == F.FSQ_ERR_MISALIGNED
+    assert F.encode_pack_raw(16, 4, 68, 64, 16, 256, qp, 16, 128, null) == F.FSQ_ERR_MISALIGNED
+    assert F.encode_pack_raw(16, 4, 64, 64, 16, 256, F.quant_params(9.0, 0.5), 16, 128, null) == F.FSQ_ERR_INVALID_ARG
+    assert F.encode_pack_raw(null, 0, 64, 64, null, 256, qp, null, 128, null) == F.FSQ_OK  # empty: no-op
+    assert F.quantize_pack_f32_raw(null, 3, 256, qp, null, 128, null) == F.FSQ_ERR_INVALID_ARG
+    assert F.quantize_pack_f32_raw(8, 3, 256, qp, 16, 128, null) == F.FSQ_ERR_MISALIGNED
+    # decode
+    o = _opts()
+    args = dict(q=16, B=1, n_q=16, d_h=128, codes=16, bs=4096, T=32, G=256, w=16, n_kv=8)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        ws = kw.get("ws", 256)
+        wsb = kw.get("wsb", 1 << 30)
+        return F.decode_attn_raw(a["q"], a["B"], a["n_q"], a["d_h"], a["codes"], a["bs"], a["T"], a["G"], a["w"],
+                                 a["n_kv"], o, ws, wsb, 16, None)
+
+    assert call(T=0) == F.FSQ_ERR_INVALID_ARG
+    assert call(d_h=64) == F.FSQ_ERR_UNSUPPORTED
+    assert call(n_q=12) == F.FSQ_ERR_INVALID_ARG
+    assert call(G=85) == F.FSQ_ERR_UNSUPPORTED
+    assert call(codes=None) == F.FSQ_ERR_INVALID_ARG
+    assert call(bs=100) == F.FSQ_ERR_INVALID_ARG          # stride < T*G/2
+    assert call(bs=4104) == F.FSQ_ERR_MISALIGNED          # stride % 16
+    assert call(codes=24) == F.FSQ_ERR_MISALIGNED
+    assert call(q=18) == F.FSQ_ERR_MISALIGNED
+    assert call(wsb=16) == F.FSQ_ERR_WORKSPACE
+    assert call(ws=None) == F.FSQ_ERR_WORKSPACE
+    assert call(ws=272) == F.FSQ_ERR_MISALIGNED
+    assert call(B=0, q=None, codes=None, w=None) == F.FSQ_OK  # empty batch: no-op

@@ -1,0 +1,210 @@
+"""GPU parity: the CUDA library (through its C ABI) against the fp64 oracle.
+
+Codes: bit-exact, except inputs whose exact u lies within a stated band of a
+rounding boundary (counted and reported).  Attention: max|delta|/max|ref| <=
+5e-3 with bf16 operands and fp32 accumulation."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import fsq_latent_decode_b200 as F
+from fsq_latent_decode_b200 import synth
+from oracle import fsq_oracle as O
+
+from cases import TOL, decoder_weights, gemm_error_bound, oracle_cache, padded_len, rel_err
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _dev(t):
+    return t.to(DEV) if isinstance(t, torch.Tensor) else torch.from_numpy(np.ascontiguousarray(t)).to(DEV)
+
+
+# ---------------------------------------------------------------- quantiser alone
+@pytest.mark.parametrize("G", [84, 256])
+@pytest.mark.parametrize("h", [7.5, 7.5075])
+@pytest.mark.parametrize("n_tok", [1, 7, 129, 4099])
+def test_quantize_pack_bit_exact(G, h, n_tok):
+    gen = synth._gen(synth.workload_seed(11, G, n_tok))
+    u = synth.preactivations(n_tok, G, gen)
+    # plant exact thresholds and their fp32 neighbours
+    th = np.array(F.thresholds(h, 0.5), dtype=np.float32)
+    flat = u.view(-1)
+    k = min(flat.numel(), 45)
+    planted = np.concatenate([th, np.nextafter(th, np.float32(np.inf)), np.nextafter(th, np.float32(-np.inf))])
+    flat[:k] = torch.from_numpy(planted[:k])
+    got = F.quantize_pack_f32(_dev(u), h, 0.5).cpu().numpy()
+    hq = float(np.float32(h))
+    ref = O.quantize_pack(u.numpy().astype(np.float64), hq)
+    mism = got != ref
+    if mism.any():
+        lv_g = O.unpack(got, G)
+        lv_r = O.unpack(ref, G)
+        bad = lv_g != lv_r
+        d = O.fsq_boundary_distance(u.numpy()[bad].astype(np.float64), hq)
+        assert (d < 1e-6).all(), f"{bad.sum()} mismatches outside the 1e-6 band"
+        print(f"quantize G={G} h={h}: {int(bad.sum())} codes within 1e-6 of a boundary differ")
+
+
+# ---------------------------------------------------------------- encoder + FSQ + pack
+@pytest.mark.parametrize("n_tok,C,G", [(1024, 1024, 256), (4096, 2048, 256), (4096, 4096, 256), (4096, 4096, 84),
+                                       (1, 1024, 84), (37, 2048, 256), (129, 4096, 84)])
+def test_encode_pack_parity(n_tok, C, G):
+    gen = synth._gen(synth.workload_seed(21, n_tok, C, G))
+    x, E = synth.encoder_inputs(n_tok, C, G, gen)
+    got = F.encode_pack(_dev(x), _dev(E)).cpu().numpy()
+    lv_r, u = O.encode(x.float().numpy(), E.float().numpy())
+    ref = O.pack(lv_r)
+    lv_g = O.unpack(got, G)
+    bad = lv_g != lv_r
+    n_bad = int(bad.sum())
+    if n_bad:
+        d = O.fsq_boundary_distance(u[bad])
+        bound = gemm_error_bound(x.float().numpy(), E.float().numpy())[bad]
+        assert (np.abs(lv_g[bad] - lv_r[bad]) == 1).all()
+        assert (d <= bound * 2.0 + 1e-7).all(), "code mismatch farther from a boundary than the fp32 GEMM bound"
+        print(f"encode n={n_tok} C={C} G={G}: {n_bad} of {lv_r.size} codes differ; "
+              f"{int((d < 1e-6).sum())} within 1e-6 of a boundary, all within the fp32 GEMM bound")
+    assert n_bad <= max(2, lv_r.size // 2000)
+
+
+# ---------------------------------------------------------------- decode attention
+def _decode(q, codes, W, T, n_kv, G, **kw):
+    opts = F.attn_opts(**kw)
+    return F.decode_attn(_dev(q), _dev(codes), _dev(W), T, n_kv, G, opts=opts)
+
+
+SMALL = [
+    # B, n_q, n_kv, G, T
+    (1, 16, 8, 256, 1), (1, 16, 8, 256, 2), (2, 16, 8, 256, 7), (1, 16, 8, 84, 8), (3, 32, 8, 84, 9),
+    (1, 32, 8, 256, 127), (2, 32, 8, 256, 128), (1, 32, 8, 84, 129), (2, 16, 8, 84, 1000), (1, 32, 8, 256, 4099),
+    (3, 8, 2, 12, 300), (1, 4, 4, 2, 65),
+]
+
+
+@pytest.mark.parametrize("variant", ["absorbed", "expand"])
+@pytest.mark.parametrize("B,n_q,n_kv,G,T", SMALL)
+def test_decode_parity_small(variant, B, n_q, n_kv, G, T):
+    codes = oracle_cache(B, T, G, seed=31 + T)
+    W, q = decoder_weights(n_q, n_kv, G, B, seed=32 + T)
+    got = _decode(q, codes, W, T, n_kv, G, variant=variant, out_fp32=True).cpu().numpy()
+    ref = O.decode_attn(q.float().numpy(), codes[:, :T], W.float().numpy(), n_kv, G)
+    assert rel_err(got, ref) <= TOL
+
+
+@pytest.mark.parametrize("splits", [1, 3, 64, 1024])
+def test_decode_split_counts_agree(splits):
+    B, n_q, n_kv, G, T = 2, 32, 8, 84, 3001
+    codes = oracle_cache(B, T, G, seed=41)
+    W, q = decoder_weights(n_q, n_kv, G, B, seed=42)
+    ref = O.decode_attn(q.float().numpy(), codes[:, :T], W.float().numpy(), n_kv, G)
+    for variant in ("absorbed", "expand"):
+        got = _decode(q, codes, W, T, n_kv, G, variant=variant, num_splits=splits, out_fp32=True).cpu().numpy()
+        assert rel_err(got, ref) <= TOL
+
+
+def test_decode_bf16_output_and_scale():
+    B, n_q, n_kv, G, T = 2, 32, 8, 256, 513
+    codes = oracle_cache(B, T, G, seed=51)
+    W, q = decoder_weights(n_q, n_kv, G, B, seed=52)
+    ref = O.decode_attn(q.float().numpy(), codes[:, :T], W.float().numpy(), n_kv, G, scale=0.05)
+    got = _decode(q, codes, W, T, n_kv, G, scale=0.05)
+    assert got.dtype == torch.bfloat16
+    assert rel_err(got.float().cpu().numpy(), ref) <= TOL
+
+
+@pytest.mark.parametrize("G,T", [(84, 1), (256, 300), (84, 4099)])
+def test_decode_rope_knorm_expand(G, T):
+    B, n_q, n_kv = 2, 32, 8
+    codes = oracle_cache(B, T, G, seed=61)
+    W, q = decoder_weights(n_q, n_kv, G, B, seed=62)
+    gen = synth._gen(63)
+    gain = (1.0 + 0.1 * torch.randn(128, generator=gen)).to(torch.bfloat16)
+    rk = dict(gain=gain.float().numpy(), eps=1e-6, base=1.0e6)
+    ref = O.decode_attn(q.float().numpy(), codes[:, :T], W.float().numpy(), n_kv, G, rope_knorm=rk)
+    got = _decode(q, codes, W, T, n_kv, G, rope_knorm=True, rope_base=1.0e6, knorm_gain=_dev(gain),
+                  knorm_eps=1e-6, out_fp32=True).cpu().numpy()
+    assert rel_err(got, ref) <= TOL
+
+
+def test_decode_leaves_neighbouring_memory_alone():
+    B, n_q, n_kv, G, T = 2, 16, 8, 84, 257
+    codes = oracle_cache(B, T, G, seed=71)
+    W, q = decoder_weights(n_q, n_kv, G, B, seed=72)
+    buf = torch.full((B * n_q * 128 + 2 * 4096,), 12345.0, device=DEV)
+    out = buf[4096:4096 + B * n_q * 128].view(B, n_q, 128)
+    F.decode_attn(_dev(q), _dev(codes), _dev(W), T, n_kv, G, opts=F.attn_opts(out_fp32=True), out=out)
+    torch.cuda.synchronize()
+    assert (buf[:4096] == 12345.0).all() and (buf[-4096:] == 12345.0).all()
+    ref = O.decode_attn(q.float().numpy(), codes[:, :T], W.float().numpy(), n_kv, G)
+    assert rel_err(out.cpu().numpy(), ref) <= TOL
+
+
+# ---------------------------------------------------------------- the seeded workloads
+def test_tiny_workload_end_to_end():
+    wl = synth.WORKLOADS["tiny_0p6b"]
+    gen = synth._gen(0)
+    T = wl.lengths[0]
+    x, E = synth.encoder_inputs(T, wl.C, wl.G, gen)
+    W, q = synth.decoder_inputs(1, wl.n_q, wl.n_kv, wl.d_h, wl.G, gen)
+    # append path on the GPU vs the oracle
+    got_codes = F.encode_pack(_dev(x), _dev(E)).cpu().numpy()
+    lv_r, u = O.encode(x.float().numpy(), E.float().numpy())
+    ref_codes = O.pack(lv_r)
+    bad = O.unpack(got_codes, wl.G) != lv_r
+    if bad.any():
+        d = O.fsq_boundary_distance(u[bad])
+        assert (d <= 2 * gemm_error_bound(x.float().numpy(), E.float().numpy())[bad] + 1e-7).all()
+    # decode over the oracle's codes, both variants
+    codes = ref_codes[None]
+    ref = O.decode_attn(q.float().numpy(), codes, W.float().numpy(), wl.n_kv, wl.G)
+    for variant in ("absorbed", "expand"):
+        got = _decode(q, codes, W, T, wl.n_kv, wl.G, variant=variant, out_fp32=True).cpu().numpy()
+        assert rel_err(got, ref) <= TOL
+
+
+FULL = [
+    ("qwen3_1p7b_32x", 1, 32768), ("qwen3_1p7b_32x", 4, 32768), ("qwen3_1p7b_32x", 8, 32768),
+    ("qwen3_8b_32x", 1, 8192), ("qwen3_8b_32x", 4, 32768), ("qwen3_8b_32x", 16, 131072),
+    ("qwen3_8b_97x", 1, 8192), ("qwen3_8b_97x", 4, 32768), ("qwen3_8b_97x", 16, 131072),
+    ("long_8b_97x", 1, 1 << 20),
+]
+
+
+@pytest.mark.parametrize("name,B,T", FULL)
+def test_full_size_workloads_sampled(name, B, T):
+    """Full-size caches at the benchmark's launch configuration; the oracle
+    checks sampled batch rows (first and last), every head of those rows."""
+    wl = synth.WORKLOADS[name]
+    rows = sorted({0, B - 1})
+    codes = oracle_cache(B, T, wl.G, seed=1000 + B, rows=rows)
+    W, q = decoder_weights(wl.n_q, wl.n_kv, wl.G, B, seed=2000 + B)
+    heads = None if T <= 131072 else [0, 7, 8, 31]
+    ref = O.decode_attn(q.float().numpy(), codes[:, :T], W.float().numpy(), wl.n_kv, wl.G, rows=rows, heads=heads)
+    got = _decode(q, codes, W, T, wl.n_kv, wl.G).float().cpu().numpy()
+    assert rel_err(got, ref) <= TOL
+    assert np.isfinite(got).all()
+
+
+@pytest.mark.parametrize("name", ["qwen3_1p7b_32x", "long_8b_97x"])
+def test_workload_append_leg(name):
+    """The workload's append leg: encode n_new tokens straight into the cache rows
+    after T (codes written in place), checked against the oracle."""
+    wl = synth.WORKLOADS[name]
+    gen = synth._gen(synth.workload_seed(5, wl.C))
+    x, E = synth.encoder_inputs(wl.n_new, wl.C, wl.G, gen)
+    T0 = 4096
+    cache = torch.zeros((T0 + wl.n_new + 16, wl.G // 2), dtype=torch.uint8, device=DEV)
+    F.encode_pack(_dev(x), _dev(E), out=cache[T0:T0 + wl.n_new])
+    got = cache.cpu().numpy()
+    assert (got[:T0] == 0).all() and (got[T0 + wl.n_new:] == 0).all()
+    lv_r, u = O.encode(x.float().numpy(), E.float().numpy())
+    bad = O.unpack(got[T0:T0 + wl.n_new], wl.G) != lv_r
+    assert bad.sum() <= max(2, lv_r.size // 2000)
+    if bad.any():
+        d = O.fsq_boundary_distance(u[bad])
+        assert (d <= 2 * gemm_error_bound(x.float().numpy(), E.float().numpy())[bad] + 1e-7).all()
