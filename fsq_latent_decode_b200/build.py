@@ -1,6 +1,6 @@
 """Builds libfsq.so in-tree from csrc/*.cu for sm_100a (B200) with nvcc.
 
-    python -m fsq_latent_decode_b200.build [--force] [--verbose]
+    python fsq_latent_decode_b200/build.py [--force] [--verbose]
 
 Objects go to fsq_latent_decode_b200/_build/; the shared library is written
 next to this file.  Rebuilds only when a source or header is newer than the

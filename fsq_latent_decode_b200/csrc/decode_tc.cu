@@ -96,6 +96,7 @@ struct Misc {
   uint32_t abort;
   uint32_t vote[4];
   float red[4][64];
+  float fac[4][64];
   float corr[64];
 };
 
@@ -351,12 +352,11 @@ __global__ void __launch_bounds__(384, 1) absorbed_split_tc(Params p) {
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     for (int n = stid; n < NQ; n += 128) ms.corr[n] = p.corr[(size_t)b * NQ + n];
     named_bar(1, 128);
-    float m[NQ], lsum[NQ], cr[NQ];
+    float m[NQ], lsum[NQ];
 #pragma unroll
     for (int n = 0; n < NQ; ++n) {
       m[n] = -INFINITY;
       lsum[n] = 0.f;
-      cr[n] = ms.corr[n];
     }
     const int r = 32 * q + lane;                  // token row within the tile
     const int kap = kappa_of_token(r);            // its K position in the pooling operand
@@ -374,11 +374,11 @@ __global__ void __launch_bounds__(384, 1) absorbed_split_tc(Params p) {
       __syncwarp();
       if (lane == 0) mbar_arrive(&ms.s_free[sb]);
       const bool valid = (t0 + (int64_t)i * kTile + r) < t1;
-      float s[NQ];
+      float *s = reinterpret_cast<float *>(raw);  // scores in place of the raw MMA values
       bool need = false;
 #pragma unroll
       for (int n = 0; n < NQ; ++n) {
-        s[n] = valid ? (__uint_as_float(raw[n]) - cr[n]) : -INFINITY;
+        s[n] = valid ? (__uint_as_float(raw[n]) - ms.corr[n]) : -INFINITY;
         need |= s[n] > m[n] + kTau;
       }
       const bool wneed = __any_sync(0xffffffffu, need);
@@ -395,14 +395,15 @@ __global__ void __launch_bounds__(384, 1) absorbed_split_tc(Params p) {
           if (lane == 0) ms.red[q][n] = v;
         }
         named_bar(1, 128);
-        float f[NQ];
+        float *f = ms.fac[q];  // this warp's copy of the rescale factors
 #pragma unroll
         for (int n = 0; n < NQ; ++n) {
           const float mt = fmaxf(fmaxf(ms.red[0][n], ms.red[1][n]), fmaxf(ms.red[2][n], ms.red[3][n]));
           const float mn = fmaxf(m[n], mt);
-          f[n] = exp2f(m[n] - mn);  // 0 on the first tile
+          const float fn = exp2f(m[n] - mn);  // 0 on the first tile
           m[n] = mn;
-          lsum[n] *= f[n];
+          lsum[n] *= fn;
+          if (lane == 0) f[n] = fn;
         }
         named_bar(1, 128);
         if (i > 0) {
@@ -464,14 +465,14 @@ __global__ void __launch_bounds__(384, 1) absorbed_split_tc(Params p) {
         if (lane == 0) ms.red[q][n] = v;
       }
       named_bar(1, 128);
-      float Lt[NQ];
-#pragma unroll
-      for (int n = 0; n < NQ; ++n) Lt[n] = (ms.red[0][n] + ms.red[1][n]) + (ms.red[2][n] + ms.red[3][n]);
+      if (stid < NQ) ms.fac[0][stid] = (ms.red[0][stid] + ms.red[1][stid]) + (ms.red[2][stid] + ms.red[3][stid]);
+      named_bar(1, 128);
+      const float *Lt = ms.fac[0];
       float *out = p.part + (((size_t)b * p.S + split) * NQ) * (2 + G);
-      if (stid < NQ) {
-        out[(size_t)stid * (2 + G)] = m[stid];
-        out[(size_t)stid * (2 + G) + 1] = Lt[stid];
-      }
+#pragma unroll
+      for (int n = 0; n < NQ; ++n)
+        if (stid == n) out[(size_t)n * (2 + G)] = m[n];
+      if (stid < NQ) out[(size_t)stid * (2 + G) + 1] = Lt[stid];
       // TMEM lane L of sub-partition q in half h holds coordinate
       // 128h + 32q + 8((L%8)/2) + L/8 + 4(L%2), scaled by 16 when (L/8) is odd.
       const int cb = lane >> 3, sl = lane & 7;

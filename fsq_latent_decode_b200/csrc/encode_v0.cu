@@ -59,6 +59,44 @@ __global__ void __launch_bounds__(256) encode_pack_simt(const uint16_t *__restri
   }
 }
 
+// Few-token append (a decode step appends one token per batch row): one warp
+// per (token, byte), i.e. per pair of coordinates (2i, 2i+1); 16-byte loads of
+// the token's row and the two encoder rows, fp32 accumulation, warp reduction.
+__global__ void __launch_bounds__(256) encode_pack_rows(const uint16_t *__restrict__ x, int64_t n_tok, int64_t ldx,
+                                                        int64_t C, const uint16_t *__restrict__ E, int G,
+                                                        Thresholds th, uint8_t *__restrict__ codes, int64_t ldc) {
+  const int half = G / 2;
+  const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid >= n_tok * half) return;
+  const int64_t t = wid / half;
+  const int by = (int)(wid % half);
+  const uint4 *xr = reinterpret_cast<const uint4 *>(x + t * ldx);
+  const uint4 *e0 = reinterpret_cast<const uint4 *>(E + (int64_t)(2 * by) * C);
+  const uint4 *e1 = reinterpret_cast<const uint4 *>(E + (int64_t)(2 * by + 1) * C);
+  float a0 = 0.f, a1 = 0.f;
+  for (int64_t k = lane; k < C / 8; k += 32) {
+    const uint4 xv = xr[k], v0 = e0[k], v1 = e1[k];
+    const uint32_t xs[4] = {xv.x, xv.y, xv.z, xv.w};
+    const uint32_t s0[4] = {v0.x, v0.y, v0.z, v0.w};
+    const uint32_t s1[4] = {v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float xl = __uint_as_float(xs[j] << 16), xh = __uint_as_float(xs[j] & 0xFFFF0000u);
+      a0 = fmaf(xl, __uint_as_float(s0[j] << 16), a0);
+      a0 = fmaf(xh, __uint_as_float(s0[j] & 0xFFFF0000u), a0);
+      a1 = fmaf(xl, __uint_as_float(s1[j] << 16), a1);
+      a1 = fmaf(xh, __uint_as_float(s1[j] & 0xFFFF0000u), a1);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    a0 += __shfl_xor_sync(0xffffffffu, a0, o);
+    a1 += __shfl_xor_sync(0xffffffffu, a1, o);
+  }
+  if (lane == 0) codes[t * ldc + by] = (uint8_t)(fsq_nibble(a0, th) | (fsq_nibble(a1, th) << 4));
+}
+
 __global__ void quantize_pack_f32_kernel(const float *__restrict__ u, int64_t n_tok, int G, Thresholds th,
                                          uint8_t *__restrict__ codes, int64_t ldc) {
   const int half = G / 2;
@@ -75,6 +113,11 @@ __global__ void quantize_pack_f32_kernel(const float *__restrict__ u, int64_t n_
 cudaError_t launch_encode_pack_simt(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C,
                                     const uint16_t *E, int G, const Thresholds &th, uint8_t *codes,
                                     int64_t ldc, cudaStream_t s) {
+  if (n_tok <= 64) {
+    const int64_t warps = n_tok * (G / 2);
+    encode_pack_rows<<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(x, n_tok, ldx, C, E, G, th, codes, ldc);
+    return cudaGetLastError();
+  }
   dim3 grid((unsigned)((n_tok + kEncTok - 1) / kEncTok));
   encode_pack_simt<<<grid, 256, 0, s>>>(x, n_tok, ldx, C, E, G, th, codes, ldc);
   return cudaGetLastError();
