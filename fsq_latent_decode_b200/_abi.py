@@ -27,7 +27,8 @@ VARIANTS = {"auto": VARIANT_AUTO, "absorbed": VARIANT_ABSORBED, "expand": VARIAN
 # Every symbol include/fsq.h declares.
 EXPORTED = ("fsq_attn_opts_default", "fsq_thresholds", "fsq_encode_pack", "fsq_quantize_pack_f32",
             "fsq_decode_attn_workspace_size", "fsq_decode_attn", "fsq_workspace_status",
-            "fsq_status_string", "fsq_format_version")
+            "fsq_status_string", "fsq_format_version", "fsq_decode_attn_noalloc")
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class QuantParams(C.Structure):
@@ -48,7 +49,7 @@ class FsqError(RuntimeError):
 
 def _load() -> C.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is not built; run `python -m fsq_latent_decode_b200.build` "
+        raise ImportError(f"{LIB_PATH} is not built; run `python fsq_latent_decode_b200/build.py` "
                           "(the CUDA library is required; there is no CPU fallback)")
     lib = C.CDLL(LIB_PATH)
     i64, i32, vp, f32 = C.c_int64, C.c_int, C.c_void_p, C.c_float
@@ -65,6 +66,9 @@ def _load() -> C.CDLL:
     lib.fsq_decode_attn.argtypes = [vp, i64, i32, i32, vp, i64, i64, i32, vp, i32, C.POINTER(AttnOpts),
                                     vp, C.c_size_t, vp, vp]
     lib.fsq_decode_attn.restype = i32
+    lib.fsq_decode_attn_noalloc.argtypes = [vp, i64, i32, i32, vp, i64, i64, i32, vp, i32, C.POINTER(AttnOpts),
+                                            vp, vp]
+    lib.fsq_decode_attn_noalloc.restype = i32
     lib.fsq_workspace_status.argtypes = [vp, C.c_size_t, vp]
     lib.fsq_workspace_status.restype = i32
     lib.fsq_status_string.argtypes = [i32]
@@ -142,6 +146,12 @@ def decode_attn_raw(q_ptr, B, n_q, d_h, codes_ptr, bstride, T, G, wkv_ptr, n_kv,
                     o_ptr, stream_ptr) -> int:
     return lib.fsq_decode_attn(q_ptr, B, n_q, d_h, codes_ptr, bstride, T, G, wkv_ptr, n_kv,
                                None if opts is None else C.byref(opts), ws_ptr, ws_bytes, o_ptr, stream_ptr)
+
+
+def decode_attn_noalloc_raw(q_ptr, B, n_q, d_h, codes_ptr, bstride, T, G, wkv_ptr, n_kv, opts, o_ptr,
+                            stream_ptr) -> int:
+    return lib.fsq_decode_attn_noalloc(q_ptr, B, n_q, d_h, codes_ptr, bstride, T, G, wkv_ptr, n_kv,
+                                       None if opts is None else C.byref(opts), o_ptr, stream_ptr)
 
 
 def workspace_status(ws, stream=None) -> int:

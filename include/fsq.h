@@ -158,6 +158,32 @@ FSQ_API fsq_status fsq_decode_attn(const uint16_t *q, int64_t B, int n_q, int d_
                            const uint16_t *W_kv, int n_kv, const fsq_attn_opts *opts,
                            void *workspace, size_t workspace_bytes, void *o, fsq_stream_t stream);
 
+/* Allocation-free decode attention.  There is no counterpart in the paper:
+ * this entry point exists for callers that cannot allocate device memory at
+ * the point where they decode — for example a plugin whose host framework
+ * owns every device allocation, or a latency-bound decode loop in which a
+ * cudaMalloc (which may synchronise the device) is not acceptable.
+ * Same arguments, semantics and result as fsq_decode_attn, minus the
+ * workspace: the scratch comes from a file-scope device array of
+ * FSQ_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads
+ * the library holds until the process exits.  Nothing is allocated: no
+ * cudaMalloc, cudaFree or allocating library routine is called.
+ *  - The first call on a device looks up that array's device address
+ *    (cudaGetSymbolAddress, with the device current); make that first call
+ *    before any stream capture.
+ *  - Requests whose fsq_decode_attn_workspace_size exceeds
+ *    FSQ_NOALLOC_SCRATCH_BYTES return FSQ_ERR_WORKSPACE before any launch
+ *    (use fsq_decode_attn with a workspace of your own for those).
+ *  - All calls on a device share the one array and it keeps the last call's
+ *    contents (every value a call relies on is rewritten by that call).
+ *    Calls that can overlap on the GPU (different streams without ordering)
+ *    race on it and must be serialised by the caller. */
+#define FSQ_NOALLOC_SCRATCH_BYTES (16u << 20)
+FSQ_API fsq_status fsq_decode_attn_noalloc(const uint16_t *q, int64_t B, int n_q, int d_h,
+                                           const uint8_t *codes, int64_t code_batch_stride_bytes, int64_t T,
+                                           int G, const uint16_t *W_kv, int n_kv, const fsq_attn_opts *opts,
+                                           void *o, fsq_stream_t stream);
+
 /* Reads the device error word of a workspace last used by fsq_decode_attn
  * (blocking copy: synchronises with `stream`).  Returns FSQ_OK or the
  * recorded device status (e.g. FSQ_ERR_TIMEOUT); clears nothing. */
