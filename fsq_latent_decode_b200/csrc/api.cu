@@ -33,7 +33,7 @@ cudaError_t launch_absorbed_tc(const uint16_t *q, const uint8_t *codes, int64_t 
 namespace {
 
 constexpr int kMaxSplits = 1024;
-constexpr bool kEnableTc = false;  // tensor-core absorbed kernel (being validated)
+constexpr bool kEnableTc = true;  // tensor-core absorbed kernel (being validated)
 
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 

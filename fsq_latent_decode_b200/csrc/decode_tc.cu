@@ -19,11 +19,13 @@
 //   -> softmax warps read S from TMEM, keep the running max, write P (fp16)
 //      to shared memory, rescale ACC in TMEM when the max grows.
 //
-// Nibbles are turned into fp16 with one LOP3 per pair: OR-ing the nibble into
-// the bit pattern of 1024.0 gives 1024 + n exactly (ulp 1), or 1024 + 16 n for
-// the high nibble of a byte.  The constant 1024 and the per-position factor
-// 1 or 16 are folded into Q' (score side) and into a per-row correction of
-// ACC (pooling side), so no per-value subtract is needed.
+// Nibbles are turned into fp16 without a per-value subtract.  Score operand:
+// one LOP3 per pair ORs the nibble into the bit pattern of 1024.0, giving
+// 1024 + n exactly (ulp 1), or 1024 + 16 n for the high nibble of a byte; the
+// constant and the factor 1 or 16 are folded into Q' and a per-head score
+// offset.  Pooling operand: a shift and a LOP3 per pair give 16 + n; ACC is
+// corrected by 24 l per head at the end (16 for the bias, 8 for the level
+// offset), keeping the long fp32 accumulation well conditioned.
 //
 // Warp roles (12 warps): 0 loads code tiles and owns TMEM, 1 issues MMAs,
 // 2-3 stage Q' once, 4-7 dequantise (TMEM sub-partitions 0-3), 8-11 softmax.
@@ -102,6 +104,15 @@ struct Misc {
 
 __device__ __forceinline__ uint32_t lop_lo(uint32_t w) { return (w & 0x000F000Fu) | 0x64006400u; }
 __device__ __forceinline__ uint32_t lop_hi(uint32_t w) { return (w & 0x00F000F0u) | 0x64006400u; }
+// Nibble j (bits 4j..4j+3) of both half-words moved to mantissa bits 6..9 of
+// the pattern of 16.0: the fp16 pair (16 + n_lo, 16 + n_hi), exact.  Used for
+// the pooling operand, whose fp32 accumulator runs over a whole split: a bias
+// of 16 keeps its cancellation (acc = D - 24 l) small.
+template <int J>
+__device__ __forceinline__ uint32_t nib16(uint32_t w) {
+  const uint32_t x = (J == 0) ? (w << 6) : (J == 1) ? (w << 2) : (J == 2) ? (w >> 2) : (w >> 6);
+  return (x & 0x03C003C0u) | 0x4C004C00u;
+}
 
 // Physical K position of token r in the pooling operand (see the 16x256b store below).
 __device__ __forceinline__ int kappa_of_token(int r) {
@@ -325,11 +336,10 @@ __global__ void __launch_bounds__(384, 1) absorbed_split_tc(Params p) {
               uint32_t x;
               if constexpr (G == 256) x = *reinterpret_cast<const uint32_t *>(src);
               else x = lds_u32_a2(src);
-              const uint32_t x8 = x >> 8;
-              t[e][0] = movmatrix_trans(lop_lo(x));
-              t[e][1] = movmatrix_trans(lop_hi(x));
-              t[e][2] = movmatrix_trans(lop_lo(x8));
-              t[e][3] = movmatrix_trans(lop_hi(x8));
+              t[e][0] = movmatrix_trans(nib16<0>(x));
+              t[e][1] = movmatrix_trans(nib16<1>(x));
+              t[e][2] = movmatrix_trans(nib16<2>(x));
+              t[e][3] = movmatrix_trans(nib16<3>(x));
             }
             tmem_st_16x256b(cbase + 8 * j, t[0][0], t[1][0], t[0][1], t[1][1]);
             tmem_st_16x256b(cbase + (16u << 16) + 8 * j, t[0][2], t[1][2], t[0][3], t[1][3]);
@@ -474,9 +484,8 @@ __global__ void __launch_bounds__(384, 1) absorbed_split_tc(Params p) {
         if (stid == n) out[(size_t)n * (2 + G)] = m[n];
       if (stid < NQ) out[(size_t)stid * (2 + G) + 1] = Lt[stid];
       // TMEM lane L of sub-partition q in half h holds coordinate
-      // 128h + 32q + 8((L%8)/2) + L/8 + 4(L%2), scaled by 16 when (L/8) is odd.
+      // 128h + 32q + 8((L%8)/2) + L/8 + 4(L%2); its values were 16 + nibble.
       const int cb = lane >> 3, sl = lane & 7;
-      const float scl = (cb & 1) ? (1.f / 16.f) : 1.f;
 #pragma unroll
       for (int h = 0; h < C::NH; ++h) {
         const int g = 128 * h + 32 * q + 8 * (sl >> 1) + cb + 4 * (sl & 1);
@@ -489,7 +498,7 @@ __global__ void __launch_bounds__(384, 1) absorbed_split_tc(Params p) {
 #pragma unroll
           for (int n = 0; n < NQ; ++n) {
             const float d = __uint_as_float(a[n]);
-            out[(size_t)n * (2 + G) + 2 + g] = (d - 1024.f * Lt[n]) * scl - 8.f * Lt[n];
+            out[(size_t)n * (2 + G) + 2 + g] = d - 24.f * Lt[n];
           }
         }
       }
