@@ -12,25 +12,36 @@
 // never writes reconstructed K/V": read packed codes, unpack in registers,
 // tensor cores, online softmax, merge partials):
 //   bulk copy (1-D, 16-B aligned) of the packed rows into a shared-memory ring
-//   -> dequant warps unpack nibbles in registers straight into two TMEM
-//      operand layouts: token-major Z (A of the score MMA) and, through 8x8
-//      register transposes, coordinate-major Z^T (A of the pooling MMA)
-//   -> one thread issues both MMAs (A from TMEM, B from shared memory)
+//   -> score-dequant warps unpack each token's nibbles in registers into
+//      token-major Z in TMEM (A of the score MMA, double-buffered)
+//   -> pool-dequant warps build coordinate-major Z^T in TMEM (A of the pooling
+//      MMA, in two 64-token chunks): an 8x8 register transpose (movmatrix) of
+//      the still-packed 16-bit groups of four nibbles, then the nibbles are
+//      unpacked, so one transpose serves four coordinates
+//   -> four issuer threads (two for the score MMAs of even / odd tiles, two for
+//      the pooling MMAs) keep the tensor core fed: a single issuing thread
+//      cannot issue small-N MMAs as fast as the tensor core retires them
 //   -> softmax warps read S from TMEM, keep the running max, write P (fp16)
 //      to shared memory, rescale ACC in TMEM when the max grows.
 //
-// Nibbles are turned into fp16 without a per-value subtract.  Score operand:
-// one LOP3 per pair ORs the nibble into the bit pattern of 1024.0, giving
-// 1024 + n exactly (ulp 1), or 1024 + 16 n for the high nibble of a byte; the
-// constant and the factor 1 or 16 are folded into Q' and a per-head score
-// offset.  Pooling operand: a shift and a LOP3 per pair give 16 + n; ACC is
-// corrected by 24 l per head at the end (16 for the bias, 8 for the level
-// offset), keeping the long fp32 accumulation well conditioned.
+// Nibbles become fp16 without a per-value subtract.  Score operand: one LOP3
+// per pair ORs the nibble into the bit pattern of 1024.0, giving 1024 + n
+// exactly (ulp 1), or 1024 + 16 n for the high nibble of a byte; the constant
+// and the factor 1 or 16 are folded into Q' and a per-head score offset.
+// Pooling operand: a shift and a LOP3 per pair give 16 + n; ACC is corrected
+// by 24 l per head at the end (16 for the bias, 8 for the level offset),
+// keeping the split-long fp32 accumulation well conditioned.
 //
-// Warp roles (12 warps): 0 loads code tiles and owns TMEM, 1 issues MMAs,
-// 2-3 stage Q' once, 4-7 dequantise (TMEM sub-partitions 0-3), 8-11 softmax.
-// Every wait is bounded; on a timeout the CTA records FSQ_ERR_TIMEOUT in the
-// workspace error word and all roles drain and exit.
+// Warps (17): 0 loads code tiles and owns TMEM; 1-2 issue score MMAs; 3 and 16
+// issue pooling MMAs; 4-7 score dequant, 8-11 softmax, 12-15 pooling dequant
+// (each group of four covers TMEM sub-partitions 0-3).  Every wait is
+// bounded; on a timeout the CTA records FSQ_ERR_TIMEOUT in the workspace error
+// word and all roles drain and exit.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
 #include "common.cuh"
 #include "tc_ptx.cuh"
 
@@ -41,8 +52,9 @@ using namespace ptx;
 
 constexpr int kTile = 128;
 constexpr int kStages = 4;
-constexpr float kTau = 8.f;                  // rescale when a score exceeds the running max by 2^8
-constexpr uint64_t kWaitLimitNs = 1000000000ull;  // 1 s per wait
+constexpr int kThreads = 17 * 32;
+constexpr float kTau = 8.f;                        // rescale when a score exceeds the running max by 2^8
+constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s per wait
 
 template <int G, int NQ>
 struct Cfg {
@@ -52,24 +64,30 @@ struct Cfg {
   static constexpr int SCOLS = KPAD / 2;             // TMEM columns of token-major Z
   static constexpr int NH = (G + 127) / 128;         // 128-row halves of the pooling MMA
   static constexpr int TILE_BYTES = kTile * HALF;
-  static constexpr int STAGE_BYTES = (TILE_BYTES + 16 + 127) / 128 * 128;  // + over-read pad
+  // G=256: 128-byte rows arrive by a 2-D TMA copy in 128-byte-swizzle mode, so
+  // that both dequant access patterns are free of shared-memory bank conflicts.
+  // Other G: 1-D bulk copy of the contiguous rows (+16 bytes for over-reads).
+  static constexpr bool TMA = (HALF == 128);
+  static constexpr int STAGE_BYTES = TMA ? TILE_BYTES : (TILE_BYTES + 16 + 127) / 128 * 128;
   static constexpr int Q_BYTES = NQ * KPAD * 2;      // Q' in the K-major no-swizzle layout
   static constexpr int P_BYTES = kTile * NQ * 2;     // P in the MN-major no-swizzle layout
-  // TMEM columns
+  // TMEM columns: Z (score A) x2 | Z^T chunks (pool A) x2 | S x2 | ACC
+  static constexpr int CS_COLS = (SCOLS + 15) / 16 * 16;
+  static constexpr int CP_CHUNK = NH * 32;           // one 64-token chunk of Z^T
   static constexpr int OFF_CS = 0;
-  static constexpr int OFF_CP = (SCOLS + 15) / 16 * 16;
-  static constexpr int CP_BUF = NH * 64;
-  static constexpr int OFF_S = OFF_CP + 2 * CP_BUF;
+  static constexpr int OFF_CP = 2 * CS_COLS;
+  static constexpr int OFF_S = OFF_CP + 2 * CP_CHUNK;
   static constexpr int OFF_ACC = OFF_S + 2 * NQ;
-  static constexpr int TMEM_USED = OFF_ACC + NH * NQ;
-  static constexpr int TMEM_COLS = 512;
+  static constexpr int ACC_COLS = 2 * NQ;            // NH=2: one per half; NH=1: one per chunk
+  static constexpr int TMEM_USED = OFF_ACC + ACC_COLS;
+  static constexpr int TMEM_COLS = TMEM_USED <= 256 ? 256 : 512;
   static_assert(TMEM_USED <= 512, "TMEM plan exceeds 512 columns");
   // shared memory
   static constexpr int SM_CODES = 0;
   static constexpr int SM_Q = SM_CODES + kStages * STAGE_BYTES;
   static constexpr int SM_P = SM_Q + Q_BYTES;
   static constexpr int SM_MISC = SM_P + 2 * P_BYTES;
-  static constexpr int SM_TOTAL = SM_MISC + 2048;
+  static constexpr int SM_TOTAL = SM_MISC + 4096;
   static constexpr int LBO_Q = (NQ / 8) * 128;       // K-chunk stride of Q'
   static constexpr int SBO_P = (kTile / 8) * 128;    // N-group stride of P
 };
@@ -89,25 +107,26 @@ struct Params {
 
 struct Misc {
   uint64_t full[kStages], empty[kStages];
-  uint64_t cs_ready, cs_free;
+  uint64_t cs_ready[2], cs_free[2];
   uint64_t cp_ready[2], cp_free[2];
   uint64_t s_full[2], s_free[2];
   uint64_t p_full[2], p_free[2];
-  uint64_t acc_full, q_full, mma_done;
+  uint64_t acc_full, q_full, done[5];
   uint32_t tmem_base;
   uint32_t abort;
-  uint32_t vote[4];
+  uint32_t vote[2][4];
   float red[4][64];
   float fac[4][64];
+  float m[64];
+  float cm[4][64];   // per softmax warp: score offset + running max, per head
   float corr[64];
 };
 
+// Score operand pairs from one packed word (bias 1024, factor 1 / 16 / 1 / 16).
 __device__ __forceinline__ uint32_t lop_lo(uint32_t w) { return (w & 0x000F000Fu) | 0x64006400u; }
 __device__ __forceinline__ uint32_t lop_hi(uint32_t w) { return (w & 0x00F000F0u) | 0x64006400u; }
-// Nibble j (bits 4j..4j+3) of both half-words moved to mantissa bits 6..9 of
-// the pattern of 16.0: the fp16 pair (16 + n_lo, 16 + n_hi), exact.  Used for
-// the pooling operand, whose fp32 accumulator runs over a whole split: a bias
-// of 16 keeps its cancellation (acc = D - 24 l) small.
+// Nibble J (bits 4J..4J+3) of both half-words moved to mantissa bits 6..9 of
+// the pattern of 16.0: the fp16 pair (16 + n_lo, 16 + n_hi), exact.
 template <int J>
 __device__ __forceinline__ uint32_t nib16(uint32_t w) {
   const uint32_t x = (J == 0) ? (w << 6) : (J == 1) ? (w << 2) : (J == 2) ? (w >> 2) : (w >> 6);
@@ -119,14 +138,73 @@ __device__ __forceinline__ int kappa_of_token(int r) {
   return (r & ~15) | (((r >> 1) & 3) << 2) | (((r >> 3) & 1) << 1) | (r & 1);
 }
 
+// 128-byte-swizzle layout of a TMA tile: 16-byte chunk c of row r sits at chunk c ^ (r % 8).
+__device__ __forceinline__ int swz(int r, int chunk) { return r * 128 + ((chunk ^ (r & 7)) << 4); }
+
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int c0, int c1, int c2, uint64_t *bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // 32-bit little-endian load from a 2-byte aligned shared address
 __device__ __forceinline__ uint32_t lds_u32_a2(const uint8_t *p) {
   const uint16_t *h = reinterpret_cast<const uint16_t *>(p);
   return (uint32_t)h[0] | ((uint32_t)h[1] << 16);
 }
 
+// Blocking wait with a suspend hint: the thread sleeps in the barrier instead
+// of spinning.  Gives up after `limit_ns` or once *abort is set.
+__device__ __forceinline__ bool wait_bar(uint64_t *b, uint32_t parity, volatile uint32_t *abort, uint64_t limit_ns) {
+  const uint32_t a = smem_u32(b);
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(a), "r"(parity), "r"(20000u)
+      : "memory");
+  if (ok) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(a), "r"(parity), "r"(200000u)
+        : "memory");
+    if (ok) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
+__device__ __forceinline__ void tmem_st_16x256b_x4(uint32_t taddr, const uint32_t *r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x256b.x4.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+template <int NQ>
+__device__ __forceinline__ void tmem_ld_nq(uint32_t ta, uint32_t *r) {
+  if constexpr (NQ == 32) tmem_ld32(ta, r);
+  else tmem_ld16(ta, r);
+}
+template <int NQ>
+__device__ __forceinline__ void tmem_st_nq(uint32_t ta, const uint32_t *r) {
+  if constexpr (NQ == 32) tmem_st32(ta, r);
+  else tmem_st16(ta, r);
+}
+
 template <int G, int NQ>
-__global__ void __launch_bounds__(384, 1) absorbed_split_tc(Params p) {
+__global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_constant__ CUtensorMap tmap, Params p) {
   using C = Cfg<G, NQ>;
   extern __shared__ __align__(1024) uint8_t smem[];
   Misc &ms = *reinterpret_cast<Misc *>(smem + C::SM_MISC);
@@ -137,25 +215,26 @@ __global__ void __launch_bounds__(384, 1) absorbed_split_tc(Params p) {
   const int n_tiles = (int)((t1 - t0 + kTile - 1) / kTile);
   const uint8_t *gcodes = p.codes + (int64_t)b * p.bstride + t0 * C::HALF;
   volatile uint32_t *abort = &ms.abort;
+  constexpr uint32_t kPoolIssuers = 2;
 
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&ms.full[s], 1);
-      mbar_init(&ms.empty[s], 4);
+      mbar_init(&ms.empty[s], 8);
     }
-    mbar_init(&ms.cs_ready, 4);
-    mbar_init(&ms.cs_free, 1);
     for (int i = 0; i < 2; ++i) {
+      mbar_init(&ms.cs_ready[i], 4);
+      mbar_init(&ms.cs_free[i], 1);
       mbar_init(&ms.cp_ready[i], 4);
-      mbar_init(&ms.cp_free[i], 1);
+      mbar_init(&ms.cp_free[i], C::NH == 2 ? 2 : 1);
       mbar_init(&ms.s_full[i], 1);
       mbar_init(&ms.s_free[i], 4);
       mbar_init(&ms.p_full[i], 4);
-      mbar_init(&ms.p_free[i], 1);
+      mbar_init(&ms.p_free[i], kPoolIssuers);
     }
-    mbar_init(&ms.acc_full, 1);
+    mbar_init(&ms.acc_full, kPoolIssuers);
     mbar_init(&ms.q_full, 1);
-    mbar_init(&ms.mma_done, 1);
+    for (int i = 0; i < 5; ++i) mbar_init(&ms.done[i], 1);
     ms.abort = 0;
     fence_mbar_init();
   }
@@ -180,22 +259,25 @@ __global__ void __launch_bounds__(384, 1) absorbed_split_tc(Params p) {
       mbar_arrive_expect_tx(&ms.q_full, C::Q_BYTES);
       bulk_g2s(smem + C::SM_Q, p.qphys + (size_t)b * C::Q_BYTES, C::Q_BYTES, &ms.q_full);
     }
-    int issued_phase[kStages];
-#pragma unroll
-    for (int s = 0; s < kStages; ++s) issued_phase[s] = -1;
+    int issued = 0;
     bool ok = true;
-    for (int i = 0; i < n_tiles && ok; ++i) {
+    for (int i = 0; i < n_tiles; ++i) {
       const int st = i % kStages;
       const uint32_t ph = (uint32_t)(i / kStages) & 1u;
-      if (!mbar_wait(&ms.empty[st], ph ^ 1u, abort, p.wait_ns)) {
-        if (lane == 0) fail();
+      if (!wait_bar(&ms.empty[st], ph ^ 1u, abort, p.wait_ns)) {
         ok = false;
         break;
       }
       const int64_t rows = min((int64_t)kTile, t1 - (t0 + (int64_t)i * kTile));
       uint8_t *dst = ring + st * C::STAGE_BYTES;
       const uint8_t *src = gcodes + (int64_t)i * kTile * C::HALF;
-      if (rows == kTile) {
+      if constexpr (C::TMA) {
+        // rows past T arrive as zeros; rows past this split's end are masked by the softmax
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&ms.full[st], C::TILE_BYTES);
+          tma_load_3d(dst, &tmap, 0, (int)(t0 + (int64_t)i * kTile), b, &ms.full[st]);
+        }
+      } else if (rows == kTile) {
         if (lane == 0) {
           mbar_arrive_expect_tx(&ms.full[st], C::TILE_BYTES);
           bulk_g2s(dst, src, C::TILE_BYTES, &ms.full[st]);
@@ -207,247 +289,274 @@ __global__ void __launch_bounds__(384, 1) absorbed_split_tc(Params p) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&ms.full[st]);
       }
-      issued_phase[st] = (int)ph;
+      issued = i + 1;
     }
     if (!ok) {
-      // let copies already in flight land before the CTA exits
-      for (int s = 0; s < kStages; ++s)
-        if (issued_phase[s] >= 0) mbar_wait(&ms.full[s], (uint32_t)issued_phase[s], abort, p.wait_ns / 4 + 1);
+      if (lane == 0) fail();
+      // let the copies still in flight land before the CTA exits
+      for (int i = max(0, issued - kStages); i < issued; ++i)
+        wait_bar(&ms.full[i % kStages], (uint32_t)(i / kStages) & 1u, abort, p.wait_ns / 4 + 1);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------------ score-MMA issuers (even / odd tiles)
     if (lane == 0) {
-      const uint32_t id_s = idesc_f16(128, NQ, 0, 0);
-      const uint32_t id_p = idesc_f16(128, NQ, 0, 1);
-      const uint32_t qs = smem_u32(smem + C::SM_Q);
-      const uint32_t pbase = smem_u32(smem + C::SM_P);
-      bool ok = mbar_wait(&ms.q_full, 0, abort, p.wait_ns);
-      auto pool = [&](int j) -> bool {
-        const int pb = j & 1;
-        const uint32_t par = (uint32_t)(j >> 1) & 1u;
-        if (!mbar_wait(&ms.p_full[pb], par, abort, p.wait_ns)) return false;
-        if (!mbar_wait(&ms.cp_ready[pb], par, abort, p.wait_ns)) return false;
-        tc_fence_after();
-#pragma unroll
-        for (int h = 0; h < C::NH; ++h) {
-#pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk) {
-            const uint64_t bd = smem_desc(pbase + pb * C::P_BYTES + kk * 256, 128, C::SBO_P);
-            mma_ts(tm + C::OFF_ACC + h * NQ, tm + C::OFF_CP + pb * C::CP_BUF + h * 64 + kk * 8, bd, id_p,
-                   (j > 0 || kk > 0) ? 1u : 0u);
-          }
-        }
-        tc_commit(&ms.p_free[pb]);
-        tc_commit(&ms.cp_free[pb]);
-        return true;
-      };
-      for (int i = 0; i < n_tiles && ok; ++i) {
-        const int sb = i & 1;
-        ok = mbar_wait(&ms.cs_ready, (uint32_t)i & 1u, abort, p.wait_ns) &&
-             mbar_wait(&ms.s_free[sb], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort, p.wait_ns);
+      const int sb = warp - 1;
+      constexpr uint32_t id_s = idesc_f16(128, NQ, 0, 0);
+      const uint64_t qd0 = smem_desc(smem_u32(smem + C::SM_Q), C::LBO_Q, 128);
+      bool ok = wait_bar(&ms.q_full, 0, abort, p.wait_ns);
+      for (int i = sb; i < n_tiles && ok; i += 2) {
+        const uint32_t par = (uint32_t)(i >> 1) & 1u;
+        ok = wait_bar(&ms.cs_ready[sb], par, abort, p.wait_ns) &&
+             wait_bar(&ms.s_free[sb], par ^ 1u, abort, p.wait_ns);
         if (!ok) break;
         tc_fence_after();
+        const uint32_t a0 = tm + C::OFF_CS + sb * C::CS_COLS;
+        const uint32_t d = tm + C::OFF_S + sb * NQ;
 #pragma unroll
-        for (int k = 0; k < C::KPAD / 16; ++k) {
-          const uint64_t bd = smem_desc(qs + k * 2 * C::LBO_Q, C::LBO_Q, 128);
-          mma_ts(tm + C::OFF_S + sb * NQ, tm + C::OFF_CS + k * 8, bd, id_s, k > 0 ? 1u : 0u);
-        }
+        for (int k = 0; k < C::KPAD / 16; ++k)
+          mma_ts(d, a0 + k * 8, qd0 + (uint64_t)((k * 2 * C::LBO_Q) >> 4), id_s, k > 0 ? 1u : 0u);
         tc_commit(&ms.s_full[sb]);
-        tc_commit(&ms.cs_free);
-        if (i > 0) ok = pool(i - 1);
+        tc_commit(&ms.cs_free[sb]);
       }
-      if (ok && n_tiles > 0) ok = pool(n_tiles - 1);
+      if (!ok) fail();
+      tc_commit(&ms.done[sb]);
+      wait_bar(&ms.done[sb], 0, abort, p.wait_ns);
+    }
+  } else if (warp == 3 || warp == 16) {
+    // ------------------------------------------------------------ pooling-MMA issuers
+    if (lane == 0) {
+      const int k_iss = warp == 3 ? 0 : 1;  // NH=2: half k_iss, both chunks; NH=1: chunk k_iss
+      constexpr uint32_t id_p = idesc_f16(128, NQ, 0, 1);
+      const uint64_t pd0 = smem_desc(smem_u32(smem + C::SM_P), 128, C::SBO_P);
+      bool ok = true;
+      for (int i = 0; i < n_tiles && ok; ++i) {
+        const int pb = i & 1;
+        ok = wait_bar(&ms.p_full[pb], (uint32_t)(i >> 1) & 1u, abort, p.wait_ns);
+        if (!ok) break;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          if (C::NH == 1 && c != k_iss) continue;
+          if (!wait_bar(&ms.cp_ready[c], (uint32_t)i & 1u, abort, p.wait_ns)) { ok = false; break; }
+          tc_fence_after();
+          const int h = C::NH == 2 ? k_iss : 0;
+          const uint32_t d = tm + C::OFF_ACC + k_iss * NQ;
+          const uint32_t a0 = tm + C::OFF_CP + c * C::CP_CHUNK + h * 32;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t bd = pd0 + (uint64_t)((pb * C::P_BYTES + (4 * c + kk) * 256) >> 4);
+            const bool first = (i == 0) && (C::NH == 1 ? kk == 0 : (c == 0 && kk == 0));
+            mma_ts(d, a0 + kk * 8, bd, id_p, first ? 0u : 1u);
+          }
+          tc_commit(&ms.cp_free[c]);
+        }
+        if (!ok) break;
+        tc_commit(&ms.p_free[pb]);
+      }
       if (ok) tc_commit(&ms.acc_full);
       else fail();
-      // every MMA issued by this thread has completed once mma_done flips
-      tc_commit(&ms.mma_done);
-      mbar_wait(&ms.mma_done, 0, abort, p.wait_ns);
+      tc_commit(&ms.done[2 + k_iss]);
+      wait_bar(&ms.done[2 + k_iss], 0, abort, p.wait_ns);
     }
   } else if (warp >= 4 && warp < 8) {
-    // ------------------------------------------------------------ dequant
+    // ------------------------------------------------------------ score dequant: token row -> TMEM lane
     const int q = warp - 4;
+    const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+    bool ok = true;
+    for (int i = 0; i < n_tiles; ++i) {
+      const int st = i % kStages, sb = i & 1;
+      const uint8_t *tile = smem + C::SM_CODES + st * C::STAGE_BYTES;
+      if (!wait_bar(&ms.full[st], (uint32_t)(i / kStages) & 1u, abort, p.wait_ns) ||
+          !wait_bar(&ms.cs_free[sb], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort, p.wait_ns)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint8_t *row = tile + (32 * q + lane) * C::HALF;
+      const uint32_t cbase = tm + lane_base + C::OFF_CS + sb * C::CS_COLS;
+#pragma unroll
+      for (int c0 = 0; c0 < C::KW; c0 += 8) {
+        const int nw = (C::KW - c0) < 8 ? (C::KW - c0) : 8;
+        uint32_t w[8];
+        if constexpr (C::TMA) {
+          const int rr = 32 * q + lane;
+          const uint4 v0 = *reinterpret_cast<const uint4 *>(tile + swz(rr, c0 / 4));
+          const uint4 v1 = *reinterpret_cast<const uint4 *>(tile + swz(rr, c0 / 4 + 1));
+          w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
+          w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+        } else {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int kw = c0 + k;
+            if (4 * kw + 4 <= C::HALF) w[k] = lds_u32_a2(row + 4 * kw);
+            else if (4 * kw + 2 <= C::HALF) w[k] = *reinterpret_cast<const uint16_t *>(row + 4 * kw);
+            else w[k] = 0u;
+          }
+        }
+        uint32_t r[32];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          if (k < nw) {
+            const uint32_t x = w[k], x8 = x >> 8;
+            r[4 * k + 0] = lop_lo(x);
+            r[4 * k + 1] = lop_hi(x);
+            r[4 * k + 2] = lop_lo(x8);
+            r[4 * k + 3] = lop_hi(x8);
+          }
+        }
+        if (nw == 8) tmem_st32(cbase + 4 * c0, r);
+        else if (nw == 4) tmem_st16(cbase + 4 * c0, r);
+        else if (nw == 2) tmem_st8(cbase + 4 * c0, r);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ms.empty[st]);  // this warp is done with the stage
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ms.cs_ready[sb]);
+    }
+    if (!ok && lane == 0) fail();
+  } else if (warp >= 12 && warp < 16) {
+    // ------------------------------------------------------------ pooling dequant: coordinates -> TMEM lanes
+    const int q = warp - 12;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     bool ok = true;
     for (int i = 0; i < n_tiles && ok; ++i) {
       const int st = i % kStages;
       const uint8_t *tile = smem + C::SM_CODES + st * C::STAGE_BYTES;
-      if (!mbar_wait(&ms.full[st], (uint32_t)(i / kStages) & 1u, abort, p.wait_ns)) { ok = false; break; }
-      // token-major Z: this thread's token row -> TMEM lane (32q + lane)
-      if (!mbar_wait(&ms.cs_free, ((uint32_t)i & 1u) ^ 1u, abort, p.wait_ns)) { ok = false; break; }
-      tc_fence_after();
-      {
-        const uint8_t *row = tile + (32 * q + lane) * C::HALF;
-        uint32_t w[C::KW];
-        if constexpr (G == 256) {
+      if (!wait_bar(&ms.full[st], (uint32_t)(i / kStages) & 1u, abort, p.wait_ns)) { ok = false; break; }
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
-            uint4 v = *reinterpret_cast<const uint4 *>(row + 16 * k);
-            w[4 * k] = v.x; w[4 * k + 1] = v.y; w[4 * k + 2] = v.z; w[4 * k + 3] = v.w;
-          }
-        } else {
+      for (int c = 0; c < 2; ++c) {
+        if (!wait_bar(&ms.cp_free[c], ((uint32_t)i & 1u) ^ 1u, abort, p.wait_ns)) { ok = false; break; }
+        tc_fence_after();
 #pragma unroll
-          for (int k = 0; k < C::KW; ++k) {
-            if (4 * k + 4 <= C::HALF) w[k] = lds_u32_a2(row + 4 * k);
-            else if (4 * k + 2 <= C::HALF) w[k] = *reinterpret_cast<const uint16_t *>(row + 4 * k);
-            else w[k] = 0u;
-          }
-        }
-        constexpr int CH = 8;  // words per TMEM store (32 columns)
+        for (int h = 0; h < C::NH; ++h) {
+          const int byte0 = 64 * h + 16 * q;  // first byte of this warp's 32 coordinates
+          if (byte0 >= C::HALF) continue;
+          uint32_t lo[16], hi[16];
 #pragma unroll
-        for (int c0 = 0; c0 < C::KW; c0 += CH) {
-          uint32_t r[32];
-          const int nw = (C::KW - c0) < CH ? (C::KW - c0) : CH;
-#pragma unroll
-          for (int k = 0; k < CH; ++k) {
-            if (k < nw) {
-              const uint32_t x = w[c0 + k], x8 = x >> 8;
-              r[4 * k + 0] = lop_lo(x);
-              r[4 * k + 1] = lop_hi(x);
-              r[4 * k + 2] = lop_lo(x8);
-              r[4 * k + 3] = lop_hi(x8);
-            }
-          }
-          const uint32_t ta = tm + lane_base + C::OFF_CS + 4 * c0;
-          if (nw == 8) tmem_st32(ta, r);
-          else if (nw == 4) tmem_st16(ta, r);
-          else if (nw == 2) tmem_st8(ta, r);
-        }
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ms.cs_ready);
-      // coordinate-major Z^T via 8x8 transposes -> TMEM lanes = coordinates
-      const int pb = i & 1;
-      if (!mbar_wait(&ms.cp_free[pb], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort, p.wait_ns)) { ok = false; break; }
-      tc_fence_after();
-#pragma unroll
-      for (int h = 0; h < C::NH; ++h) {
-        const int byte0 = 64 * h + 16 * q;  // first byte of this warp's 32 coordinates
-        if (byte0 < C::HALF) {
-          const uint32_t cbase = tm + lane_base + C::OFF_CP + pb * C::CP_BUF + h * 64;
-#pragma unroll 2
-          for (int j = 0; j < kTile / 16; ++j) {
-            uint32_t t[2][4];
+          for (int j = 0; j < 4; ++j) {
 #pragma unroll
             for (int e = 0; e < 2; ++e) {
-              const int tb = 2 * j + e;
-              const uint8_t *src = tile + (8 * tb + (lane >> 2)) * C::HALF + byte0 + 4 * (lane & 3);
+              const int tb = 8 * c + 2 * j + e;  // 8-token block within the tile
+              const int rr = 8 * tb + (lane >> 2);
               uint32_t x;
-              if constexpr (G == 256) x = *reinterpret_cast<const uint32_t *>(src);
-              else x = lds_u32_a2(src);
-              t[e][0] = movmatrix_trans(nib16<0>(x));
-              t[e][1] = movmatrix_trans(nib16<1>(x));
-              t[e][2] = movmatrix_trans(nib16<2>(x));
-              t[e][3] = movmatrix_trans(nib16<3>(x));
+              if constexpr (C::TMA) x = *reinterpret_cast<const uint32_t *>(tile + swz(rr, byte0 >> 4) + 4 * (lane & 3));
+              else x = lds_u32_a2(tile + rr * C::HALF + byte0 + 4 * (lane & 3));
+              // transpose 16-bit groups of four nibbles: this thread now holds one
+              // group (four coordinates) of two tokens, then unpack each coordinate
+              const uint32_t y = movmatrix_trans(x);
+              lo[4 * j + e] = nib16<0>(y);
+              lo[4 * j + 2 + e] = nib16<1>(y);
+              hi[4 * j + e] = nib16<2>(y);
+              hi[4 * j + 2 + e] = nib16<3>(y);
             }
-            tmem_st_16x256b(cbase + 8 * j, t[0][0], t[1][0], t[0][1], t[1][1]);
-            tmem_st_16x256b(cbase + (16u << 16) + 8 * j, t[0][2], t[1][2], t[0][3], t[1][3]);
           }
+          const uint32_t cb = tm + lane_base + C::OFF_CP + c * C::CP_CHUNK + h * 32;
+          tmem_st_16x256b_x4(cb, lo);
+          tmem_st_16x256b_x4(cb + (16u << 16), hi);
         }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ms.cp_ready[c]);
       }
-      tmem_st_wait();
-      tc_fence_before();
+      if (!ok) break;
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&ms.cp_ready[pb]);
-        mbar_arrive(&ms.empty[st]);
-      }
+      if (lane == 0) mbar_arrive(&ms.empty[st]);
     }
     if (!ok && lane == 0) fail();
-  } else if (warp >= 8) {
+  } else if (warp >= 8 && warp < 12) {
     // ------------------------------------------------------------ softmax
     const int q = warp - 8;
     const int stid = tid - 256;  // 0..127
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     for (int n = stid; n < NQ; n += 128) ms.corr[n] = p.corr[(size_t)b * NQ + n];
     named_bar(1, 128);
-    float m[NQ], lsum[NQ];
+    float *cm = ms.cm[q];  // score offset + running max m, per head (this warp's copy)
+    float lsum[NQ];
+    if (lane == 0)
+      for (int n = 0; n < NQ; ++n) cm[n] = ms.corr[n];  // provisional m = 0; the first tile always rescales
+    __syncwarp();
 #pragma unroll
-    for (int n = 0; n < NQ; ++n) {
-      m[n] = -INFINITY;
-      lsum[n] = 0.f;
-    }
-    const int r = 32 * q + lane;                  // token row within the tile
-    const int kap = kappa_of_token(r);            // its K position in the pooling operand
+    for (int n = 0; n < NQ; ++n) lsum[n] = 0.f;
+    const int r = 32 * q + lane;        // token row within the tile
+    const int kap = kappa_of_token(r);  // its K position in the pooling operand
     bool ok = true;
     for (int i = 0; i < n_tiles && ok; ++i) {
       const int sb = i & 1;
       const uint32_t par = (uint32_t)(i >> 1) & 1u;
-      if (!mbar_wait(&ms.s_full[sb], par, abort, p.wait_ns)) { ok = false; break; }
+      if (!wait_bar(&ms.s_full[sb], par, abort, p.wait_ns)) { ok = false; break; }
       tc_fence_after();
       uint32_t raw[NQ];
-      if constexpr (NQ == 32) tmem_ld32(tm + lane_base + C::OFF_S + sb * NQ, raw);
-      else tmem_ld16(tm + lane_base + C::OFF_S + sb * NQ, raw);
+      tmem_ld_nq<NQ>(tm + lane_base + C::OFF_S + sb * NQ, raw);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ms.s_free[sb]);
       const bool valid = (t0 + (int64_t)i * kTile + r) < t1;
-      float *s = reinterpret_cast<float *>(raw);  // scores in place of the raw MMA values
-      bool need = false;
+      float *x = reinterpret_cast<float *>(raw);  // x = score - m, in place
+      bool need = (i == 0);
 #pragma unroll
       for (int n = 0; n < NQ; ++n) {
-        s[n] = valid ? (__uint_as_float(raw[n]) - ms.corr[n]) : -INFINITY;
-        need |= s[n] > m[n] + kTau;
+        x[n] = valid ? (__uint_as_float(raw[n]) - cm[n]) : -INFINITY;
+        need |= x[n] > kTau;
       }
-      const bool wneed = __any_sync(0xffffffffu, need);
-      if (lane == 0) ms.vote[q] = wneed ? 1u : 0u;
+      const uint32_t wneed = __any_sync(0xffffffffu, need) ? 1u : 0u;
+      if (lane == 0) ms.vote[i & 1][q] = wneed;
       named_bar(1, 128);
-      const bool any = (ms.vote[0] | ms.vote[1] | ms.vote[2] | ms.vote[3]) != 0u;
-      named_bar(1, 128);
+      const bool any = (ms.vote[i & 1][0] | ms.vote[i & 1][1] | ms.vote[i & 1][2] | ms.vote[i & 1][3]) != 0u;
       if (any) {
+        // raise the running max: m <- m + max(0, tile max of x) (the first tile: m <- its max)
 #pragma unroll
         for (int n = 0; n < NQ; ++n) {
-          float v = s[n];
+          float v = x[n];
 #pragma unroll
           for (int off = 16; off; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
           if (lane == 0) ms.red[q][n] = v;
         }
         named_bar(1, 128);
-        float *f = ms.fac[q];  // this warp's copy of the rescale factors
+        float *f = ms.fac[q];
 #pragma unroll
         for (int n = 0; n < NQ; ++n) {
-          const float mt = fmaxf(fmaxf(ms.red[0][n], ms.red[1][n]), fmaxf(ms.red[2][n], ms.red[3][n]));
-          const float mn = fmaxf(m[n], mt);
-          const float fn = exp2f(m[n] - mn);  // 0 on the first tile
-          m[n] = mn;
+          const float d = fmaxf(fmaxf(ms.red[0][n], ms.red[1][n]), fmaxf(ms.red[2][n], ms.red[3][n]));
+          const float sh = (i == 0) ? d : fmaxf(d, 0.f);
+          const float fn = (i == 0) ? 0.f : exp2f(-sh);
+          x[n] -= sh;
           lsum[n] *= fn;
-          if (lane == 0) f[n] = fn;
+          if (lane == 0) {
+            f[n] = fn;
+            cm[n] += sh;
+          }
         }
-        named_bar(1, 128);
+        __syncwarp();
         if (i > 0) {
           // ACC must hold every earlier tile before it is rescaled
           const int pj = (i - 1) & 1;
-          if (!mbar_wait(&ms.p_free[pj], (uint32_t)((i - 1) >> 1) & 1u, abort, p.wait_ns)) { ok = false; break; }
+          if (!wait_bar(&ms.p_free[pj], (uint32_t)((i - 1) >> 1) & 1u, abort, p.wait_ns)) { ok = false; break; }
           tc_fence_after();
-#pragma unroll
-          for (int h = 0; h < C::NH; ++h) {
-            uint32_t a[NQ];
-            const uint32_t ta = tm + lane_base + C::OFF_ACC + h * NQ;
-            if constexpr (NQ == 32) tmem_ld32(ta, a);
-            else tmem_ld16(ta, a);
+#pragma unroll 1
+          for (int cc = 0; cc < 2 * NQ; cc += 16) {  // both ACC blocks, 16 columns at a time
+            uint32_t a[16];
+            const uint32_t ta = tm + lane_base + C::OFF_ACC + cc;
+            tmem_ld16(ta, a);
             tmem_ld_wait();
 #pragma unroll
-            for (int n = 0; n < NQ; ++n) a[n] = __float_as_uint(__uint_as_float(a[n]) * f[n]);
-            if constexpr (NQ == 32) tmem_st32(ta, a);
-            else tmem_st16(ta, a);
+            for (int n = 0; n < 16; ++n) a[n] = __float_as_uint(__uint_as_float(a[n]) * f[(cc + n) % NQ]);
+            tmem_st16(ta, a);
           }
           tmem_st_wait();
         }
       }
-      // P row of this token (fp16), MN-major: 4 chunks of 8 heads
+      // P row of this token (fp16), MN-major: NQ/8 chunks of 8 heads
       const int pb = i & 1;
-      if (!mbar_wait(&ms.p_free[pb], par ^ 1u, abort, p.wait_ns)) { ok = false; break; }
+      if (!wait_bar(&ms.p_free[pb], par ^ 1u, abort, p.wait_ns)) { ok = false; break; }
       uint8_t *prow = smem + C::SM_P + pb * C::P_BYTES + (kap >> 3) * 128 + (kap & 7) * 16;
 #pragma unroll
       for (int g8 = 0; g8 < NQ / 8; ++g8) {
         uint32_t h2[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const float p0 = exp2f(s[8 * g8 + 2 * k] - m[8 * g8 + 2 * k]);
-          const float p1 = exp2f(s[8 * g8 + 2 * k + 1] - m[8 * g8 + 2 * k + 1]);
-          const __half2 hv = __floats2half2_rn(p0, p1);
+          const __half2 hv = __floats2half2_rn(exp2f(x[8 * g8 + 2 * k]), exp2f(x[8 * g8 + 2 * k + 1]));
           const float2 back = __half22float2(hv);
           lsum[8 * g8 + 2 * k] += back.x;
           lsum[8 * g8 + 2 * k + 1] += back.y;
@@ -461,7 +570,7 @@ __global__ void __launch_bounds__(384, 1) absorbed_split_tc(Params p) {
       if (lane == 0) mbar_arrive(&ms.p_full[pb]);
     }
     // ------------------------------------------------------------ epilogue: ACC -> partials
-    if (ok) ok = mbar_wait(&ms.acc_full, 0, abort, p.wait_ns);
+    if (ok) ok = wait_bar(&ms.acc_full, 0, abort, p.wait_ns);
     if (!ok) {
       if (lane == 0) fail();
     } else {
@@ -474,37 +583,49 @@ __global__ void __launch_bounds__(384, 1) absorbed_split_tc(Params p) {
         for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
         if (lane == 0) ms.red[q][n] = v;
       }
+      if (stid == 0) {
+#pragma unroll
+        for (int n = 0; n < NQ; ++n) ms.m[n] = ms.cm[0][n] - ms.corr[n];
+      }
       named_bar(1, 128);
       if (stid < NQ) ms.fac[0][stid] = (ms.red[0][stid] + ms.red[1][stid]) + (ms.red[2][stid] + ms.red[3][stid]);
       named_bar(1, 128);
       const float *Lt = ms.fac[0];
       float *out = p.part + (((size_t)b * p.S + split) * NQ) * (2 + G);
-#pragma unroll
-      for (int n = 0; n < NQ; ++n)
-        if (stid == n) out[(size_t)n * (2 + G)] = m[n];
-      if (stid < NQ) out[(size_t)stid * (2 + G) + 1] = Lt[stid];
+      if (stid < NQ) {
+        out[(size_t)stid * (2 + G)] = ms.m[stid];
+        out[(size_t)stid * (2 + G) + 1] = Lt[stid];
+      }
       // TMEM lane L of sub-partition q in half h holds coordinate
-      // 128h + 32q + 8((L%8)/2) + L/8 + 4(L%2); its values were 16 + nibble.
-      const int cb = lane >> 3, sl = lane & 7;
+      // 128h + 32q + 8((L%8)/2) + 4(L%2) + L/8 (see the pooling dequant); values
+      // are 16 + nibble.  NH=1 keeps one ACC copy per 64-token chunk: add them.
+      const int jn = lane >> 3, sl = lane & 7;
+      if constexpr (C::NH == 2) {
+#pragma unroll 1
+        for (int h = 0; h < 2; ++h) {
+          uint32_t a[NQ];
+          tmem_ld_nq<NQ>(tm + lane_base + C::OFF_ACC + h * NQ, a);
+          tmem_ld_wait();
+          const int g = 128 * h + 32 * q + 8 * (sl >> 1) + 4 * (sl & 1) + jn;
 #pragma unroll
-      for (int h = 0; h < C::NH; ++h) {
-        const int g = 128 * h + 32 * q + 8 * (sl >> 1) + cb + 4 * (sl & 1);
-        uint32_t a[NQ];
-        const uint32_t ta = tm + lane_base + C::OFF_ACC + h * NQ;
-        if constexpr (NQ == 32) tmem_ld32(ta, a);
-        else tmem_ld16(ta, a);
+          for (int n = 0; n < NQ; ++n) out[(size_t)n * (2 + G) + 2 + g] = __uint_as_float(a[n]) - 24.f * Lt[n];
+        }
+      } else {
+        uint32_t a0[NQ], a1[NQ];
+        tmem_ld_nq<NQ>(tm + lane_base + C::OFF_ACC, a0);
+        tmem_ld_nq<NQ>(tm + lane_base + C::OFF_ACC + NQ, a1);
         tmem_ld_wait();
+        const int g = 32 * q + 8 * (sl >> 1) + 4 * (sl & 1) + jn;
         if (g < G) {
 #pragma unroll
           for (int n = 0; n < NQ; ++n) {
-            const float d = __uint_as_float(a[n]);
+            const float d = __uint_as_float(a0[n]) + __uint_as_float(a1[n]);
             out[(size_t)n * (2 + G) + 2 + g] = d - 24.f * Lt[n];
           }
         }
       }
     }
   }
-  // warps 2-3 have no role after set-up
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -571,6 +692,36 @@ __global__ void absorb_query_tc(const uint16_t *__restrict__ q, const uint16_t *
   }
 }
 
+// Tensor map of the code cache as a 3-D byte tensor [B][T][row bytes]: the
+// box is one 128-row tile of one batch row, swizzled 128 B.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, []() {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+cudaError_t make_code_tensor_map(CUtensorMap *map, const uint8_t *codes, int64_t bstride, int64_t T, int64_t B,
+                                 int row_bytes) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+  if (!enc) return cudaErrorNotSupported;
+  if (T > 0x7fffffffLL || B > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const cuuint64_t dims[3] = {(cuuint64_t)row_bytes, (cuuint64_t)T, (cuuint64_t)B};
+  const cuuint64_t strides[2] = {(cuuint64_t)row_bytes, (cuuint64_t)bstride};
+  const cuuint32_t box[3] = {(cuuint32_t)row_bytes, (cuuint32_t)kTile, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t *>(codes), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 template <int G, int NQ>
 cudaError_t launch(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T, int n_kv,
                    const uint16_t *W_kv, float scale, int S, int64_t tps, uint8_t *qphys, float *corr, float *part,
@@ -584,8 +735,14 @@ cudaError_t launch(const uint16_t *q, const uint8_t *codes, int64_t bstride, int
   e = cudaFuncSetAttribute(absorbed_split_tc<G, NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   Params p{codes, bstride, T, tps, S, qphys, corr, part, err, kWaitLimitNs};
+  CUtensorMap tmap;
+  memset(&tmap, 0, sizeof(tmap));
+  if constexpr (C::TMA) {
+    e = make_code_tensor_map(&tmap, codes, bstride, T, B, C::HALF);
+    if (e != cudaSuccess) return e;
+  }
   if (prof[0]) cudaEventRecord((cudaEvent_t)prof[0], st);
-  absorbed_split_tc<G, NQ><<<dim3(S, (unsigned)B), 384, smem, st>>>(p);
+  absorbed_split_tc<G, NQ><<<dim3(S, (unsigned)B), kThreads, smem, st>>>(tmap, p);
   e = cudaGetLastError();
   if (prof[1]) cudaEventRecord((cudaEvent_t)prof[1], st);
   return e;
