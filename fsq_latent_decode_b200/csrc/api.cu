@@ -117,7 +117,7 @@ fsq_status plan_decode(int64_t B, int64_t T, int n_q, int n_kv, int d_h, int G, 
   if (tc) off = align_up(off + absorbed_tc_qphys_bytes(n_q, G) * (size_t)Bc, 256);
   else if (variant == FSQ_VARIANT_ABSORBED) off = align_up(off + sizeof(float) * (size_t)Bc * n_q * G, 256);
   p->off_corr = off;
-  if (tc) off = align_up(off + sizeof(float) * (size_t)Bc * n_q, 256);
+  if (tc) off = align_up(off + 2 * sizeof(float) * (size_t)Bc * n_q, 256);
   p->off_part = off;
   off = align_up(off + sizeof(float) * (size_t)Bc * S * n_q * (2 + acc_len), 256);
   p->total = off;

@@ -24,13 +24,14 @@
 //   -> softmax warps read S from TMEM, keep the running max, write P (fp16)
 //      to shared memory, rescale ACC in TMEM when the max grows.
 //
-// Nibbles become fp16 without a per-value subtract.  Score operand: one LOP3
-// per pair ORs the nibble into the bit pattern of 1024.0, giving 1024 + n
-// exactly (ulp 1), or 1024 + 16 n for the high nibble of a byte; the constant
-// and the factor 1 or 16 are folded into Q' and a per-head score offset.
-// Pooling operand: a shift and a LOP3 per pair give 16 + n; ACC is corrected
-// by 24 l per head at the end (16 for the bias, 8 for the level offset),
-// keeping the split-long fp32 accumulation well conditioned.
+// Score MMA (kind::i8): the codes enter as unsigned bytes n = level + 8 (one
+// LOP3 or SHF+LOP3 per four nibbles), and Q' is split per head into two int8
+// terms, Q' ~ sigma (128 a + b), stacked along N (2 n_q columns), so the score
+// is exact integer arithmetic on a 15-bit Q': s = sigma (128 S_a + S_b) minus a
+// per-head offset for the -8 level shift.  Pooling MMA (kind::f16): a shift
+// and a LOP3 per pair give the fp16 values 16 + n; ACC is corrected by 24 l
+// per head at the end (16 for the bias, 8 for the level offset), keeping the
+// split-long fp32 accumulation well conditioned.
 //
 // Warps (17): 0 loads code tiles and owns TMEM; 1-2 issue score MMAs; 3 and 16
 // issue pooling MMAs; 4-7 score dequant, 8-11 softmax, 12-15 pooling dequant
@@ -59,9 +60,10 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s per wait
 template <int G, int NQ>
 struct Cfg {
   static constexpr int HALF = G / 2;                 // bytes per token row
-  static constexpr int KPAD = (G + 15) / 16 * 16;    // K of the score MMA
+  static constexpr int KPAD = (G + 31) / 32 * 32;    // K of the score MMA (32 per kind::i8 step)
   static constexpr int KW = KPAD / 8;                // 32-bit code words (8 coordinates) per padded row
-  static constexpr int SCOLS = KPAD / 2;             // TMEM columns of token-major Z
+  static constexpr int SCOLS = KPAD / 4;             // TMEM columns of token-major Z (4 bytes per column)
+  static constexpr int NS = 2 * NQ;                  // score-MMA N: the a and b terms of every head
   static constexpr int NH = (G + 127) / 128;         // 128-row halves of the pooling MMA
   static constexpr int TILE_BYTES = kTile * HALF;
   // G=256: 128-byte rows arrive by a 2-D TMA copy in 128-byte-swizzle mode, so
@@ -69,7 +71,7 @@ struct Cfg {
   // Other G: 1-D bulk copy of the contiguous rows (+16 bytes for over-reads).
   static constexpr bool TMA = (HALF == 128);
   static constexpr int STAGE_BYTES = TMA ? TILE_BYTES : (TILE_BYTES + 16 + 127) / 128 * 128;
-  static constexpr int Q_BYTES = NQ * KPAD * 2;      // Q' in the K-major no-swizzle layout
+  static constexpr int Q_BYTES = NS * KPAD;          // int8 Q' terms in the K-major no-swizzle layout
   static constexpr int P_BYTES = kTile * NQ * 2;     // P in the MN-major no-swizzle layout
   // TMEM columns: Z (score A) x2 | Z^T chunks (pool A) x2 | S x2 | ACC
   static constexpr int CS_COLS = (SCOLS + 15) / 16 * 16;
@@ -77,7 +79,7 @@ struct Cfg {
   static constexpr int OFF_CS = 0;
   static constexpr int OFF_CP = 2 * CS_COLS;
   static constexpr int OFF_S = OFF_CP + 2 * CP_CHUNK;
-  static constexpr int OFF_ACC = OFF_S + 2 * NQ;
+  static constexpr int OFF_ACC = OFF_S + 2 * NS;
   static constexpr int ACC_COLS = 2 * NQ;            // NH=2: one per half; NH=1: one per chunk
   static constexpr int TMEM_USED = OFF_ACC + ACC_COLS;
   static constexpr int TMEM_COLS = TMEM_USED <= 256 ? 256 : 512;
@@ -88,7 +90,7 @@ struct Cfg {
   static constexpr int SM_P = SM_Q + Q_BYTES;
   static constexpr int SM_MISC = SM_P + 2 * P_BYTES;
   static constexpr int SM_TOTAL = SM_MISC + 4096;
-  static constexpr int LBO_Q = (NQ / 8) * 128;       // K-chunk stride of Q'
+  static constexpr int LBO_Q = (NS / 8) * 128;       // 16-byte K-chunk stride of Q'
   static constexpr int SBO_P = (kTile / 8) * 128;    // N-group stride of P
 };
 
@@ -99,7 +101,7 @@ struct Params {
   int64_t tps;
   int S;
   const uint8_t *qphys;  // per batch row: Q' bytes in the shared-memory layout
-  const float *corr;     // per batch row: [NQ] score offsets
+  const float *corr;     // per batch row: [NQ] sigma, then [NQ] score offsets
   float *part;           // [B][S][NQ][2 + G]
   uint32_t *err;
   uint64_t wait_ns;
@@ -120,11 +122,26 @@ struct Misc {
   float m[64];
   float cm[4][64];   // per softmax warp: score offset + running max, per head
   float corr[64];
+  float sig[64];
 };
 
-// Score operand pairs from one packed word (bias 1024, factor 1 / 16 / 1 / 16).
-__device__ __forceinline__ uint32_t lop_lo(uint32_t w) { return (w & 0x000F000Fu) | 0x64006400u; }
-__device__ __forceinline__ uint32_t lop_hi(uint32_t w) { return (w & 0x00F000F0u) | 0x64006400u; }
+// Score operand bytes from one packed word: even coordinates, then odd ones.
+__device__ __forceinline__ uint32_t nib_even(uint32_t w) { return w & 0x0F0F0F0Fu; }
+__device__ __forceinline__ uint32_t nib_odd(uint32_t w) { return (w >> 4) & 0x0F0F0F0Fu; }
+
+// Instruction descriptor for kind::i8: D s32, A unsigned, B signed.
+__host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
+  return (2u << 4) | (0u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+__device__ __forceinline__ void mma_ts_i8(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Nibble J (bits 4J..4J+3) of both half-words moved to mantissa bits 6..9 of
 // the pattern of 16.0: the fp16 pair (16 + n_lo, 16 + n_hi), exact.
 template <int J>
@@ -301,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
     // ------------------------------------------------------------ score-MMA issuers (even / odd tiles)
     if (lane == 0) {
       const int sb = warp - 1;
-      constexpr uint32_t id_s = idesc_f16(128, NQ, 0, 0);
+      constexpr uint32_t id_s = idesc_i8(128, C::NS);
       const uint64_t qd0 = smem_desc(smem_u32(smem + C::SM_Q), C::LBO_Q, 128);
       bool ok = wait_bar(&ms.q_full, 0, abort, p.wait_ns);
       for (int i = sb; i < n_tiles && ok; i += 2) {
@@ -311,10 +328,10 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
         if (!ok) break;
         tc_fence_after();
         const uint32_t a0 = tm + C::OFF_CS + sb * C::CS_COLS;
-        const uint32_t d = tm + C::OFF_S + sb * NQ;
+        const uint32_t d = tm + C::OFF_S + sb * C::NS;
 #pragma unroll
-        for (int k = 0; k < C::KPAD / 16; ++k)
-          mma_ts(d, a0 + k * 8, qd0 + (uint64_t)((k * 2 * C::LBO_Q) >> 4), id_s, k > 0 ? 1u : 0u);
+        for (int k = 0; k < C::KPAD / 32; ++k)
+          mma_ts_i8(d, a0 + k * 8, qd0 + (uint64_t)((k * 2 * C::LBO_Q) >> 4), id_s, k > 0 ? 1u : 0u);
         tc_commit(&ms.s_full[sb]);
         tc_commit(&ms.cs_free[sb]);
       }
@@ -373,39 +390,38 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
       tc_fence_after();
       const uint8_t *row = tile + (32 * q + lane) * C::HALF;
       const uint32_t cbase = tm + lane_base + C::OFF_CS + sb * C::CS_COLS;
+      // word k (coordinates 8k..8k+7) -> TMEM columns 2k (even coordinates) and 2k+1 (odd)
 #pragma unroll
-      for (int c0 = 0; c0 < C::KW; c0 += 8) {
-        const int nw = (C::KW - c0) < 8 ? (C::KW - c0) : 8;
-        uint32_t w[8];
+      for (int c0 = 0; c0 < C::KW; c0 += 16) {
+        const int nw = (C::KW - c0) < 16 ? (C::KW - c0) : 16;
+        uint32_t r[32];
         if constexpr (C::TMA) {
           const int rr = 32 * q + lane;
-          const uint4 v0 = *reinterpret_cast<const uint4 *>(tile + swz(rr, c0 / 4));
-          const uint4 v1 = *reinterpret_cast<const uint4 *>(tile + swz(rr, c0 / 4 + 1));
-          w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
-          w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const uint4 u = *reinterpret_cast<const uint4 *>(tile + swz(rr, c0 / 4 + v));
+            r[8 * v + 0] = nib_even(u.x); r[8 * v + 1] = nib_odd(u.x);
+            r[8 * v + 2] = nib_even(u.y); r[8 * v + 3] = nib_odd(u.y);
+            r[8 * v + 4] = nib_even(u.z); r[8 * v + 5] = nib_odd(u.z);
+            r[8 * v + 6] = nib_even(u.w); r[8 * v + 7] = nib_odd(u.w);
+          }
         } else {
 #pragma unroll
-          for (int k = 0; k < 8; ++k) {
+          for (int k = 0; k < 16; ++k) {
             const int kw = c0 + k;
-            if (4 * kw + 4 <= C::HALF) w[k] = lds_u32_a2(row + 4 * kw);
-            else if (4 * kw + 2 <= C::HALF) w[k] = *reinterpret_cast<const uint16_t *>(row + 4 * kw);
-            else w[k] = 0u;
+            uint32_t w = 0u;
+            if (4 * kw + 4 <= C::HALF) w = lds_u32_a2(row + 4 * kw);
+            else if (4 * kw + 2 <= C::HALF) w = *reinterpret_cast<const uint16_t *>(row + 4 * kw);
+            r[2 * k] = nib_even(w);
+            r[2 * k + 1] = nib_odd(w);
           }
         }
-        uint32_t r[32];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-          if (k < nw) {
-            const uint32_t x = w[k], x8 = x >> 8;
-            r[4 * k + 0] = lop_lo(x);
-            r[4 * k + 1] = lop_hi(x);
-            r[4 * k + 2] = lop_lo(x8);
-            r[4 * k + 3] = lop_hi(x8);
-          }
+        if (nw == 16) {
+          tmem_st32(cbase + 2 * c0, r);
+        } else {
+          if (nw >= 8) tmem_st16(cbase + 2 * c0, r);
+          if (nw % 8 == 4) tmem_st8(cbase + 2 * c0 + 2 * (nw - 4), r + 2 * (nw - 4));
         }
-        if (nw == 8) tmem_st32(cbase + 4 * c0, r);
-        else if (nw == 4) tmem_st16(cbase + 4 * c0, r);
-        else if (nw == 2) tmem_st8(cbase + 4 * c0, r);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&ms.empty[st]);  // this warp is done with the stage
@@ -470,7 +486,10 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
     const int q = warp - 8;
     const int stid = tid - 256;  // 0..127
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-    for (int n = stid; n < NQ; n += 128) ms.corr[n] = p.corr[(size_t)b * NQ + n];
+    for (int n = stid; n < NQ; n += 128) {
+      ms.sig[n] = p.corr[(size_t)b * 2 * NQ + n];
+      ms.corr[n] = p.corr[(size_t)b * 2 * NQ + NQ + n];
+    }
     named_bar(1, 128);
     float *cm = ms.cm[q];  // score offset + running max m, per head (this warp's copy)
     float lsum[NQ];
@@ -487,20 +506,25 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
       const uint32_t par = (uint32_t)(i >> 1) & 1u;
       if (!wait_bar(&ms.s_full[sb], par, abort, p.wait_ns)) { ok = false; break; }
       tc_fence_after();
-      uint32_t raw[NQ];
-      tmem_ld_nq<NQ>(tm + lane_base + C::OFF_S + sb * NQ, raw);
-      tmem_ld_wait();
+      const bool valid = (t0 + (int64_t)i * kTile + r) < t1;
+      float x[NQ];  // score - m
+      bool need = (i == 0);
+#pragma unroll
+      for (int n0 = 0; n0 < NQ; n0 += 16) {
+        uint32_t ra[16], rb[16];
+        tmem_ld16(tm + lane_base + C::OFF_S + sb * C::NS + n0, ra);       // a terms
+        tmem_ld16(tm + lane_base + C::OFF_S + sb * C::NS + NQ + n0, rb);  // b terms
+        tmem_ld_wait();
+#pragma unroll
+        for (int n = 0; n < 16; ++n) {
+          const int y = (int)ra[n] * 128 + (int)rb[n];  // exact: |y| < 2^27
+          x[n0 + n] = valid ? fmaf((float)y, ms.sig[n0 + n], -cm[n0 + n]) : -INFINITY;
+          need |= x[n0 + n] > kTau;
+        }
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ms.s_free[sb]);
-      const bool valid = (t0 + (int64_t)i * kTile + r) < t1;
-      float *x = reinterpret_cast<float *>(raw);  // x = score - m, in place
-      bool need = (i == 0);
-#pragma unroll
-      for (int n = 0; n < NQ; ++n) {
-        x[n] = valid ? (__uint_as_float(raw[n]) - cm[n]) : -INFINITY;
-        need |= x[n] > kTau;
-      }
       const uint32_t wneed = __any_sync(0xffffffffu, need) ? 1u : 0u;
       if (lane == 0) ms.vote[i & 1][q] = wneed;
       named_bar(1, 128);
@@ -635,60 +659,68 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
 }
 
 // ---------------------------------------------------------------- prologue
-// Per (b, h): q'_g = c * sum_d W_k[j*d_h + d][g] q[b][h][d] (c = scale*log2 e), rounded
-// to fp16; written at its physical K position kappa, divided by the position's
-// nibble factor (1 or 16), in the K-major no-swizzle layout of the score MMA's B
-// operand.  corr[b][h] = 1024 * sum_kappa Q'[kappa] + 8 * sum_g q'_g, the part of
-// the raw MMA score that the nibble bias and the -8 level offset contribute.
+// Per (b, h): q'_g = c * sum_d W_k[j*d_h + d][g] q[b][h][d] (c = scale*log2 e),
+// split into two int8 terms q'_g ~ sigma (128 a_g + b_g) with sigma =
+// max_g |q'_g| / (127*128).  Written in the K-major no-swizzle layout of the
+// score MMA's B operand: rows h (a terms) and NQ + h (b terms), K position
+// kappa = 8w + 4e + i for coordinate 8w + 2i + e (the dequant's byte order).
+// corr[b] = [sigma_h] then [sigma_h * 8 * sum_g (128 a_g + b_g)]: the score is
+// sigma (128 S_a + S_b) - offset, the offset removing the +8 of the bytes.
 template <int G, int NQ>
 __global__ void absorb_query_tc(const uint16_t *__restrict__ q, const uint16_t *__restrict__ W_kv, int n_kv,
                                 float c, uint8_t *__restrict__ qphys, float *__restrict__ corr, uint32_t *err) {
   using C = Cfg<G, NQ>;
   constexpr int D = FSQ_HEAD_DIM;
   __shared__ float qs[D];
-  __shared__ float red[2][8];
+  __shared__ float qv[C::KPAD];
+  __shared__ float red[8];
+  __shared__ int ired[8];
   const int h = blockIdx.x, b = blockIdx.y;
   const int j = h / (NQ / n_kv);
   if (h == 0 && b == 0 && threadIdx.x == 0) *err = 0u;
   for (int d = threadIdx.x; d < D; d += blockDim.x) qs[d] = bf16_to_f32(q[((int64_t)b * NQ + h) * D + d]);
   __syncthreads();
-  float sum_q = 0.f, sum_phys = 0.f;
-  uint8_t *dst = qphys + (size_t)b * C::Q_BYTES;
-  for (int kap = threadIdx.x; kap < C::KPAD; kap += blockDim.x) {
-    // kappa = 8w + 2cc + e  <->  coordinate 8w + cc + 4e, nibble factor 16 when cc is odd
-    const int w = kap >> 3, cc = (kap >> 1) & 3, e = kap & 1;
-    const int g = 8 * w + cc + 4 * e;
+  float amax = 0.f;
+  for (int g = threadIdx.x; g < C::KPAD; g += blockDim.x) {
     float v = 0.f;
     if (g < G) {
       const uint16_t *wk = W_kv + (int64_t)j * D * G + g;
       for (int d = 0; d < D; ++d) v = fmaf(bf16_to_f32(wk[(int64_t)d * G]), qs[d], v);
       v *= c;
     }
-    const __half hq = __float2half_rn(v);
-    const float vq = __half2float(hq);          // the value the MMA multiplies (times its factor)
-    const float f = (cc & 1) ? 16.f : 1.f;
-    const __half hp = __float2half_rn(vq / f);  // exact: division by a power of two
-    sum_q += vq;
-    sum_phys += __half2float(hp);
-    const int off = (kap >> 3) * C::LBO_Q + (h >> 3) * 128 + (h & 7) * 16 + (kap & 7) * 2;
-    *reinterpret_cast<__half *>(dst + off) = hp;
+    qv[g] = v;
+    amax = fmaxf(amax, fabsf(v));
   }
-  for (int o = 16; o; o >>= 1) {
-    sum_q += __shfl_xor_sync(0xffffffffu, sum_q, o);
-    sum_phys += __shfl_xor_sync(0xffffffffu, sum_phys, o);
+  for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  float am = 0.f;
+  for (int i = 0; i < (int)(blockDim.x >> 5); ++i) am = fmaxf(am, red[i]);
+  const float sigma = am > 0.f ? am / (127.f * 128.f) : 1.f;
+  int isum = 0;
+  uint8_t *dst = qphys + (size_t)b * C::Q_BYTES;
+  for (int kap = threadIdx.x; kap < C::KPAD; kap += blockDim.x) {
+    const int w = kap >> 3, e = (kap >> 2) & 1, i4 = kap & 3;
+    const int g = 8 * w + 2 * i4 + e;
+    const float t = qv[g] / sigma;
+    int a = __float2int_rn(t / 128.f);
+    a = max(-127, min(127, a));
+    int bt = __float2int_rn(t - 128.f * (float)a);
+    bt = max(-127, min(127, bt));
+    isum += 128 * a + bt;
+    // K-major no swizzle, 8-bit: 16-byte K chunk kappa/16, 8-row group n/8, row n%8, byte kappa%16
+    const int base = (kap >> 4) * C::LBO_Q + (kap & 15);
+    dst[base + (h >> 3) * 128 + (h & 7) * 16] = (uint8_t)(int8_t)a;
+    dst[base + ((NQ + h) >> 3) * 128 + ((NQ + h) & 7) * 16] = (uint8_t)(int8_t)bt;
   }
-  if ((threadIdx.x & 31) == 0) {
-    red[0][threadIdx.x >> 5] = sum_q;
-    red[1][threadIdx.x >> 5] = sum_phys;
-  }
+  for (int o = 16; o; o >>= 1) isum += __shfl_xor_sync(0xffffffffu, isum, o);
+  if ((threadIdx.x & 31) == 0) ired[threadIdx.x >> 5] = isum;
   __syncthreads();
   if (threadIdx.x == 0) {
-    float a = 0.f, bsum = 0.f;
-    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) {
-      a += red[0][i];
-      bsum += red[1][i];
-    }
-    corr[(size_t)b * NQ + h] = 1024.f * bsum + 8.f * a;
+    long long tot = 0;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) tot += ired[i];
+    corr[(size_t)b * 2 * NQ + h] = sigma;
+    corr[(size_t)b * 2 * NQ + NQ + h] = (float)((double)sigma * 8.0 * (double)tot);
   }
 }
 
@@ -753,8 +785,8 @@ cudaError_t launch(const uint16_t *q, const uint8_t *codes, int64_t bstride, int
 bool absorbed_tc_supported(int n_q, int G) { return (n_q == 16 || n_q == 32) && (G == 256 || G == 84); }
 
 size_t absorbed_tc_qphys_bytes(int n_q, int G) {
-  const int kpad = (G + 15) / 16 * 16;
-  return (size_t)n_q * kpad * 2;
+  const int kpad = (G + 31) / 32 * 32;
+  return (size_t)2 * n_q * kpad;
 }
 
 cudaError_t merge_absorbed_launch(const float *part, int S, int64_t B, int n_q, int n_kv, int d_h, int G,
