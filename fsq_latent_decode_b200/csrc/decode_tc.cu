@@ -18,9 +18,9 @@
 //      MMA, in two 64-token chunks): an 8x8 register transpose (movmatrix) of
 //      the still-packed 16-bit groups of four nibbles, then the nibbles are
 //      unpacked, so one transpose serves four coordinates
-//   -> four issuer threads (two for the score MMAs of even / odd tiles, two for
-//      the pooling MMAs) keep the tensor core fed: a single issuing thread
-//      cannot issue small-N MMAs as fast as the tensor core retires them
+//   -> three issuer threads (score MMAs; pooling MMAs of each 128-row half or
+//      chunk) keep the tensor core fed: a single issuing thread cannot issue
+//      small-N MMAs as fast as the tensor core retires them
 //   -> softmax warps read S from TMEM, keep the running max, write P (fp16)
 //      to shared memory, rescale ACC in TMEM when the max grows.
 //
@@ -33,9 +33,10 @@
 // per head at the end (16 for the bias, 8 for the level offset), keeping the
 // split-long fp32 accumulation well conditioned.
 //
-// Warps (17): 0 loads code tiles and owns TMEM; 1-2 issue score MMAs; 3 and 16
-// issue pooling MMAs; 4-7 score dequant, 8-11 softmax, 12-15 pooling dequant
-// (each group of four covers TMEM sub-partitions 0-3).  Every wait is
+// Warps (20): 0 loads code tiles and owns TMEM; 1 issues score MMAs; 2-3 issue
+// pooling MMAs; 4-7 score dequant, 8-11 softmax, 12-15 and 16-19 pooling
+// dequant for the first and second 64-token chunk of every tile (each group
+// of four covers TMEM sub-partitions 0-3).  Every wait is
 // bounded; on a timeout the CTA records FSQ_ERR_TIMEOUT in the workspace error
 // word and all roles drain and exit.
 #include <cuda.h>
@@ -53,7 +54,7 @@ using namespace ptx;
 
 constexpr int kTile = 128;
 constexpr int kStages = 4;
-constexpr int kThreads = 17 * 32;
+constexpr int kThreads = 20 * 32;
 constexpr float kTau = 8.f;                        // rescale when a score exceeds the running max by 2^8
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s per wait
 
@@ -73,13 +74,13 @@ struct Cfg {
   static constexpr int STAGE_BYTES = TMA ? TILE_BYTES : (TILE_BYTES + 16 + 127) / 128 * 128;
   static constexpr int Q_BYTES = NS * KPAD;          // int8 Q' terms in the K-major no-swizzle layout
   static constexpr int P_BYTES = kTile * NQ * 2;     // P in the MN-major no-swizzle layout
-  // TMEM columns: Z (score A) x2 | Z^T chunks (pool A) x2 | S x2 | ACC
+  // TMEM columns: Z (score A) x2 | Z^T 64-token chunks (pool A) x4 | S | ACC
   static constexpr int CS_COLS = (SCOLS + 15) / 16 * 16;
   static constexpr int CP_CHUNK = NH * 32;           // one 64-token chunk of Z^T
   static constexpr int OFF_CS = 0;
   static constexpr int OFF_CP = 2 * CS_COLS;
-  static constexpr int OFF_S = OFF_CP + 2 * CP_CHUNK;
-  static constexpr int OFF_ACC = OFF_S + 2 * NS;
+  static constexpr int OFF_S = OFF_CP + 4 * CP_CHUNK;
+  static constexpr int OFF_ACC = OFF_S + NS;
   static constexpr int ACC_COLS = 2 * NQ;            // NH=2: one per half; NH=1: one per chunk
   static constexpr int TMEM_USED = OFF_ACC + ACC_COLS;
   static constexpr int TMEM_COLS = TMEM_USED <= 256 ? 256 : 512;
@@ -89,7 +90,7 @@ struct Cfg {
   static constexpr int SM_Q = SM_CODES + kStages * STAGE_BYTES;
   static constexpr int SM_P = SM_Q + Q_BYTES;
   static constexpr int SM_MISC = SM_P + 2 * P_BYTES;
-  static constexpr int SM_TOTAL = SM_MISC + 4096;
+  static constexpr int SM_TOTAL = SM_MISC + 8192;  // >= sizeof(Misc), checked below
   static constexpr int LBO_Q = (NS / 8) * 128;       // 16-byte K-chunk stride of Q'
   static constexpr int SBO_P = (kTile / 8) * 128;    // N-group stride of P
 };
@@ -110,8 +111,8 @@ struct Params {
 struct Misc {
   uint64_t full[kStages], empty[kStages];
   uint64_t cs_ready[2], cs_free[2];
-  uint64_t cp_ready[2], cp_free[2];
-  uint64_t s_full[2], s_free[2];
+  uint64_t cp_ready[4], cp_free[4];
+  uint64_t s_full, s_free;
   uint64_t p_full[2], p_free[2];
   uint64_t acc_full, q_full, done[5];
   uint32_t tmem_base;
@@ -126,6 +127,8 @@ struct Misc {
 };
 
 // Score operand bytes from one packed word: even coordinates, then odd ones.
+static_assert(sizeof(Misc) <= 8192, "Misc block exceeds its shared-memory reservation");
+
 __device__ __forceinline__ uint32_t nib_even(uint32_t w) { return w & 0x0F0F0F0Fu; }
 __device__ __forceinline__ uint32_t nib_odd(uint32_t w) { return (w >> 4) & 0x0F0F0F0Fu; }
 
@@ -153,6 +156,13 @@ __device__ __forceinline__ uint32_t nib16(uint32_t w) {
 // Physical K position of token r in the pooling operand (see the 16x256b store below).
 __device__ __forceinline__ int kappa_of_token(int r) {
   return (r & ~15) | (((r >> 1) & 3) << 2) | (((r >> 3) & 1) << 1) | (r & 1);
+}
+
+// 2^x on the special-function unit (inputs <= 8 here; -inf gives 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
 }
 
 // 128-byte-swizzle layout of a TMA tile: 16-byte chunk c of row r sits at chunk c ^ (r % 8).
@@ -237,18 +247,20 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&ms.full[s], 1);
-      mbar_init(&ms.empty[s], 8);
+      mbar_init(&ms.empty[s], 12);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ms.cs_ready[i], 4);
       mbar_init(&ms.cs_free[i], 1);
-      mbar_init(&ms.cp_ready[i], 4);
-      mbar_init(&ms.cp_free[i], C::NH == 2 ? 2 : 1);
-      mbar_init(&ms.s_full[i], 1);
-      mbar_init(&ms.s_free[i], 4);
       mbar_init(&ms.p_full[i], 4);
       mbar_init(&ms.p_free[i], kPoolIssuers);
     }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&ms.cp_ready[i], 4);
+      mbar_init(&ms.cp_free[i], C::NH == 2 ? 2 : 1);
+    }
+    mbar_init(&ms.s_full, 1);
+    mbar_init(&ms.s_free, 4);
     mbar_init(&ms.acc_full, kPoolIssuers);
     mbar_init(&ms.q_full, 1);
     for (int i = 0; i < 5; ++i) mbar_init(&ms.done[i], 1);
@@ -314,35 +326,34 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
       for (int i = max(0, issued - kStages); i < issued; ++i)
         wait_bar(&ms.full[i % kStages], (uint32_t)(i / kStages) & 1u, abort, p.wait_ns / 4 + 1);
     }
-  } else if (warp == 1 || warp == 2) {
-    // ------------------------------------------------------------ score-MMA issuers (even / odd tiles)
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ score-MMA issuer
     if (lane == 0) {
-      const int sb = warp - 1;
       constexpr uint32_t id_s = idesc_i8(128, C::NS);
       const uint64_t qd0 = smem_desc(smem_u32(smem + C::SM_Q), C::LBO_Q, 128);
       bool ok = wait_bar(&ms.q_full, 0, abort, p.wait_ns);
-      for (int i = sb; i < n_tiles && ok; i += 2) {
-        const uint32_t par = (uint32_t)(i >> 1) & 1u;
-        ok = wait_bar(&ms.cs_ready[sb], par, abort, p.wait_ns) &&
-             wait_bar(&ms.s_free[sb], par ^ 1u, abort, p.wait_ns);
+      for (int i = 0; i < n_tiles && ok; ++i) {
+        const int sb = i & 1;
+        ok = wait_bar(&ms.cs_ready[sb], (uint32_t)(i >> 1) & 1u, abort, p.wait_ns) &&
+             wait_bar(&ms.s_free, ((uint32_t)i & 1u) ^ 1u, abort, p.wait_ns);
         if (!ok) break;
         tc_fence_after();
         const uint32_t a0 = tm + C::OFF_CS + sb * C::CS_COLS;
-        const uint32_t d = tm + C::OFF_S + sb * C::NS;
+        const uint32_t d = tm + C::OFF_S;
 #pragma unroll
         for (int k = 0; k < C::KPAD / 32; ++k)
           mma_ts_i8(d, a0 + k * 8, qd0 + (uint64_t)((k * 2 * C::LBO_Q) >> 4), id_s, k > 0 ? 1u : 0u);
-        tc_commit(&ms.s_full[sb]);
+        tc_commit(&ms.s_full);
         tc_commit(&ms.cs_free[sb]);
       }
       if (!ok) fail();
-      tc_commit(&ms.done[sb]);
-      wait_bar(&ms.done[sb], 0, abort, p.wait_ns);
+      tc_commit(&ms.done[0]);
+      wait_bar(&ms.done[0], 0, abort, p.wait_ns);
     }
-  } else if (warp == 3 || warp == 16) {
+  } else if (warp == 2 || warp == 3) {
     // ------------------------------------------------------------ pooling-MMA issuers
     if (lane == 0) {
-      const int k_iss = warp == 3 ? 0 : 1;  // NH=2: half k_iss, both chunks; NH=1: chunk k_iss
+      const int k_iss = warp - 2;  // NH=2: half k_iss, both chunks; NH=1: chunk k_iss
       constexpr uint32_t id_p = idesc_f16(128, NQ, 0, 1);
       const uint64_t pd0 = smem_desc(smem_u32(smem + C::SM_P), 128, C::SBO_P);
       bool ok = true;
@@ -353,18 +364,19 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           if (C::NH == 1 && c != k_iss) continue;
-          if (!wait_bar(&ms.cp_ready[c], (uint32_t)i & 1u, abort, p.wait_ns)) { ok = false; break; }
+          const int cb = 2 * pb + c;  // chunk buffer
+          if (!wait_bar(&ms.cp_ready[cb], (uint32_t)(i >> 1) & 1u, abort, p.wait_ns)) { ok = false; break; }
           tc_fence_after();
           const int h = C::NH == 2 ? k_iss : 0;
           const uint32_t d = tm + C::OFF_ACC + k_iss * NQ;
-          const uint32_t a0 = tm + C::OFF_CP + c * C::CP_CHUNK + h * 32;
+          const uint32_t a0 = tm + C::OFF_CP + cb * C::CP_CHUNK + h * 32;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t bd = pd0 + (uint64_t)((pb * C::P_BYTES + (4 * c + kk) * 256) >> 4);
             const bool first = (i == 0) && (C::NH == 1 ? kk == 0 : (c == 0 && kk == 0));
             mma_ts(d, a0 + kk * 8, bd, id_p, first ? 0u : 1u);
           }
-          tc_commit(&ms.cp_free[c]);
+          tc_commit(&ms.cp_free[cb]);
         }
         if (!ok) break;
         tc_commit(&ms.p_free[pb]);
@@ -431,54 +443,56 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
       if (lane == 0) mbar_arrive(&ms.cs_ready[sb]);
     }
     if (!ok && lane == 0) fail();
-  } else if (warp >= 12 && warp < 16) {
+  } else if (warp >= 12 && warp < 20) {
     // ------------------------------------------------------------ pooling dequant: coordinates -> TMEM lanes
-    const int q = warp - 12;
+    // group c = 0 / 1 builds 64-token chunk c of every tile into chunk buffer 2 (i % 2) + c
+    const int q = warp & 3;
+    const int c = (warp - 12) >> 2;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     bool ok = true;
     for (int i = 0; i < n_tiles && ok; ++i) {
       const int st = i % kStages;
+      const int cb = 2 * (i & 1) + c;
       const uint8_t *tile = smem + C::SM_CODES + st * C::STAGE_BYTES;
-      if (!wait_bar(&ms.full[st], (uint32_t)(i / kStages) & 1u, abort, p.wait_ns)) { ok = false; break; }
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        if (!wait_bar(&ms.cp_free[c], ((uint32_t)i & 1u) ^ 1u, abort, p.wait_ns)) { ok = false; break; }
-        tc_fence_after();
-#pragma unroll
-        for (int h = 0; h < C::NH; ++h) {
-          const int byte0 = 64 * h + 16 * q;  // first byte of this warp's 32 coordinates
-          if (byte0 >= C::HALF) continue;
-          uint32_t lo[16], hi[16];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int tb = 8 * c + 2 * j + e;  // 8-token block within the tile
-              const int rr = 8 * tb + (lane >> 2);
-              uint32_t x;
-              if constexpr (C::TMA) x = *reinterpret_cast<const uint32_t *>(tile + swz(rr, byte0 >> 4) + 4 * (lane & 3));
-              else x = lds_u32_a2(tile + rr * C::HALF + byte0 + 4 * (lane & 3));
-              // transpose 16-bit groups of four nibbles: this thread now holds one
-              // group (four coordinates) of two tokens, then unpack each coordinate
-              const uint32_t y = movmatrix_trans(x);
-              lo[4 * j + e] = nib16<0>(y);
-              lo[4 * j + 2 + e] = nib16<1>(y);
-              hi[4 * j + e] = nib16<2>(y);
-              hi[4 * j + 2 + e] = nib16<3>(y);
-            }
-          }
-          const uint32_t cb = tm + lane_base + C::OFF_CP + c * C::CP_CHUNK + h * 32;
-          tmem_st_16x256b_x4(cb, lo);
-          tmem_st_16x256b_x4(cb + (16u << 16), hi);
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ms.cp_ready[c]);
+      if (!wait_bar(&ms.full[st], (uint32_t)(i / kStages) & 1u, abort, p.wait_ns) ||
+          !wait_bar(&ms.cp_free[cb], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort, p.wait_ns)) {
+        ok = false;
+        break;
       }
-      if (!ok) break;
+      tc_fence_after();
+#pragma unroll
+      for (int h = 0; h < C::NH; ++h) {
+        const int byte0 = 64 * h + 16 * q;  // first byte of this warp's 32 coordinates
+        if (byte0 >= C::HALF) continue;
+        uint32_t lo[16], hi[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int tb = 8 * c + 2 * j + e;  // 8-token block within the tile
+            const int rr = 8 * tb + (lane >> 2);
+            uint32_t x;
+            if constexpr (C::TMA) x = *reinterpret_cast<const uint32_t *>(tile + swz(rr, byte0 >> 4) + 4 * (lane & 3));
+            else x = lds_u32_a2(tile + rr * C::HALF + byte0 + 4 * (lane & 3));
+            // transpose 16-bit groups of four nibbles: this thread now holds one
+            // group (four coordinates) of two tokens, then unpack each coordinate
+            const uint32_t y = movmatrix_trans(x);
+            lo[4 * j + e] = nib16<0>(y);
+            lo[4 * j + 2 + e] = nib16<1>(y);
+            hi[4 * j + e] = nib16<2>(y);
+            hi[4 * j + 2 + e] = nib16<3>(y);
+          }
+        }
+        const uint32_t cbase = tm + lane_base + C::OFF_CP + cb * C::CP_CHUNK + h * 32;
+        tmem_st_16x256b_x4(cbase, lo);
+        tmem_st_16x256b_x4(cbase + (16u << 16), hi);
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&ms.empty[st]);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ms.cp_ready[cb]);
     }
     if (!ok && lane == 0) fail();
   } else if (warp >= 8 && warp < 12) {
@@ -502,9 +516,8 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
     const int kap = kappa_of_token(r);  // its K position in the pooling operand
     bool ok = true;
     for (int i = 0; i < n_tiles && ok; ++i) {
-      const int sb = i & 1;
       const uint32_t par = (uint32_t)(i >> 1) & 1u;
-      if (!wait_bar(&ms.s_full[sb], par, abort, p.wait_ns)) { ok = false; break; }
+      if (!wait_bar(&ms.s_full, (uint32_t)i & 1u, abort, p.wait_ns)) { ok = false; break; }
       tc_fence_after();
       const bool valid = (t0 + (int64_t)i * kTile + r) < t1;
       float x[NQ];  // score - m
@@ -512,8 +525,8 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
 #pragma unroll
       for (int n0 = 0; n0 < NQ; n0 += 16) {
         uint32_t ra[16], rb[16];
-        tmem_ld16(tm + lane_base + C::OFF_S + sb * C::NS + n0, ra);       // a terms
-        tmem_ld16(tm + lane_base + C::OFF_S + sb * C::NS + NQ + n0, rb);  // b terms
+        tmem_ld16(tm + lane_base + C::OFF_S + n0, ra);       // a terms
+        tmem_ld16(tm + lane_base + C::OFF_S + NQ + n0, rb);  // b terms
         tmem_ld_wait();
 #pragma unroll
         for (int n = 0; n < 16; ++n) {
@@ -524,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ms.s_free[sb]);
+      if (lane == 0) mbar_arrive(&ms.s_free);
       const uint32_t wneed = __any_sync(0xffffffffu, need) ? 1u : 0u;
       if (lane == 0) ms.vote[i & 1][q] = wneed;
       named_bar(1, 128);
@@ -580,7 +593,7 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
         uint32_t h2[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const __half2 hv = __floats2half2_rn(exp2f(x[8 * g8 + 2 * k]), exp2f(x[8 * g8 + 2 * k + 1]));
+          const __half2 hv = __floats2half2_rn(ex2_approx(x[8 * g8 + 2 * k]), ex2_approx(x[8 * g8 + 2 * k + 1]));
           const float2 back = __half22float2(hv);
           lsum[8 * g8 + 2 * k] += back.x;
           lsum[8 * g8 + 2 * k + 1] += back.y;
