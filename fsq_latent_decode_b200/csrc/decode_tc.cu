@@ -33,10 +33,11 @@
 // per head at the end (16 for the bias, 8 for the level offset), keeping the
 // split-long fp32 accumulation well conditioned.
 //
-// Warps (20): 0 loads code tiles and owns TMEM; 1 issues score MMAs; 2-3 issue
-// pooling MMAs; 4-7 score dequant, 8-11 softmax, 12-15 and 16-19 pooling
-// dequant for the first and second 64-token chunk of every tile (each group
-// of four covers TMEM sub-partitions 0-3).  Every wait is
+// Warps (24): 0 loads code tiles and owns TMEM; 1 issues score MMAs; 2-3 issue
+// pooling MMAs; 4-7 score dequant; 12-15 and 16-19 pooling dequant for the
+// first and second 64-token chunk of every tile; 8-11 and 20-23 softmax for
+// the first and second half of the heads (each group of four covers TMEM
+// sub-partitions 0-3).  Every wait is
 // bounded; on a timeout the CTA records FSQ_ERR_TIMEOUT in the workspace error
 // word and all roles drain and exit.
 #include <cuda.h>
@@ -54,7 +55,7 @@ using namespace ptx;
 
 constexpr int kTile = 128;
 constexpr int kStages = 4;
-constexpr int kThreads = 20 * 32;
+constexpr int kThreads = 24 * 32;
 constexpr float kTau = 8.f;                        // rescale when a score exceeds the running max by 2^8
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s per wait
 
@@ -117,11 +118,12 @@ struct Misc {
   uint64_t acc_full, q_full, done[5];
   uint32_t tmem_base;
   uint32_t abort;
-  uint32_t vote[2][4];
+  uint32_t vote[2][2][4];
   float red[4][64];
-  float fac[4][64];
+  float fac[8][64];
   float m[64];
-  float cm[4][64];   // per softmax warp: score offset + running max, per head
+  float lt[64];
+  float cm[8][64];   // per softmax warp: score offset + running max, per head
   float corr[64];
   float sig[64];
 };
@@ -182,31 +184,32 @@ __device__ __forceinline__ uint32_t lds_u32_a2(const uint8_t *p) {
   return (uint32_t)h[0] | ((uint32_t)h[1] << 16);
 }
 
-// Blocking wait with a suspend hint: the thread sleeps in the barrier instead
-// of spinning.  Gives up after `limit_ns` or once *abort is set.
-__device__ __forceinline__ bool wait_bar(uint64_t *b, uint32_t parity, volatile uint32_t *abort, uint64_t limit_ns) {
-  const uint32_t a = smem_u32(b);
+// Bounded barrier wait: non-blocking probes with a short sleep between them,
+// so that a waiting warp neither spins on the issue port nor oversleeps the
+// phase flip.  Gives up after `limit_ns` or once *abort is set.
+__device__ __forceinline__ bool bar_test(uint32_t a, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(a), "r"(parity), "r"(20000u)
+      : "r"(a), "r"(parity)
       : "memory");
-  if (ok) return true;
+  return ok != 0;
+}
+__device__ __forceinline__ bool wait_bar(uint64_t *b, uint32_t parity, volatile uint32_t *abort, uint64_t limit_ns,
+                                         uint32_t sleep_ns = 20) {
+  const uint32_t a = smem_u32(b);
+  if (bar_test(a, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  while (true) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(a), "r"(parity), "r"(200000u)
-        : "memory");
-    if (ok) return true;
-    if (*abort) return false;
-    if (globaltimer_ns() - t0 > limit_ns) return false;
+  for (uint32_t it = 1;; ++it) {
+    if (sleep_ns) __nanosleep(sleep_ns);
+    if (bar_test(a, parity)) return true;
+    if ((it & 255u) == 0u) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > limit_ns) return false;
+    }
   }
 }
 
@@ -217,6 +220,23 @@ __device__ __forceinline__ void tmem_st_16x256b_x4(uint32_t taddr, const uint32_
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
       "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t *r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr)
+               : "memory");
+}
+template <int HQ>
+__device__ __forceinline__ void tmem_ld_hq(uint32_t ta, uint32_t *r) {
+  if constexpr (HQ == 16) tmem_ld16(ta, r);
+  else tmem_ld8(ta, r);
+}
+template <int HQ>
+__device__ __forceinline__ void tmem_st_hq(uint32_t ta, const uint32_t *r) {
+  if constexpr (HQ == 16) tmem_st16(ta, r);
+  else tmem_st8(ta, r);
 }
 
 template <int NQ>
@@ -252,7 +272,7 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ms.cs_ready[i], 4);
       mbar_init(&ms.cs_free[i], 1);
-      mbar_init(&ms.p_full[i], 4);
+      mbar_init(&ms.p_full[i], 8);
       mbar_init(&ms.p_free[i], kPoolIssuers);
     }
     for (int i = 0; i < 4; ++i) {
@@ -260,7 +280,7 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
       mbar_init(&ms.cp_free[i], C::NH == 2 ? 2 : 1);
     }
     mbar_init(&ms.s_full, 1);
-    mbar_init(&ms.s_free, 4);
+    mbar_init(&ms.s_free, 8);
     mbar_init(&ms.acc_full, kPoolIssuers);
     mbar_init(&ms.q_full, 1);
     for (int i = 0; i < 5; ++i) mbar_init(&ms.done[i], 1);
@@ -495,23 +515,29 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
       if (lane == 0) mbar_arrive(&ms.cp_ready[cb]);
     }
     if (!ok && lane == 0) fail();
-  } else if (warp >= 8 && warp < 12) {
+  } else if ((warp >= 8 && warp < 12) || warp >= 20) {
     // ------------------------------------------------------------ softmax
-    const int q = warp - 8;
-    const int stid = tid - 256;  // 0..127
+    // two groups of four warps (8-11, 20-23); each group owns half the heads
+    constexpr int HQ = NQ / 2;
+    const int q = warp & 3;
+    const int hh = warp >= 20 ? 1 : 0;  // head half
+    const int h0 = hh * HQ;             // first head of this warp
+    const int sw = 4 * hh + q;          // softmax warp index 0..7
+    const int gtid = 32 * q + lane;     // thread index within the group
+    const int barid = 1 + hh;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-    for (int n = stid; n < NQ; n += 128) {
-      ms.sig[n] = p.corr[(size_t)b * 2 * NQ + n];
-      ms.corr[n] = p.corr[(size_t)b * 2 * NQ + NQ + n];
+    if (gtid < HQ) {
+      ms.sig[h0 + gtid] = p.corr[(size_t)b * 2 * NQ + h0 + gtid];
+      ms.corr[h0 + gtid] = p.corr[(size_t)b * 2 * NQ + NQ + h0 + gtid];
     }
-    named_bar(1, 128);
-    float *cm = ms.cm[q];  // score offset + running max m, per head (this warp's copy)
-    float lsum[NQ];
+    named_bar(barid, 128);
+    float *cm = ms.cm[sw];  // score offset + running max m, per head (this warp's copy)
+    float lsum[HQ];
     if (lane == 0)
-      for (int n = 0; n < NQ; ++n) cm[n] = ms.corr[n];  // provisional m = 0; the first tile always rescales
+      for (int n = 0; n < HQ; ++n) cm[n] = ms.corr[h0 + n];  // provisional m = 0; the first tile rescales
     __syncwarp();
 #pragma unroll
-    for (int n = 0; n < NQ; ++n) lsum[n] = 0.f;
+    for (int n = 0; n < HQ; ++n) lsum[n] = 0.f;
     const int r = 32 * q + lane;        // token row within the tile
     const int kap = kappa_of_token(r);  // its K position in the pooling operand
     bool ok = true;
@@ -520,42 +546,43 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
       if (!wait_bar(&ms.s_full, (uint32_t)i & 1u, abort, p.wait_ns)) { ok = false; break; }
       tc_fence_after();
       const bool valid = (t0 + (int64_t)i * kTile + r) < t1;
-      float x[NQ];  // score - m
+      float x[HQ];  // score - m
       bool need = (i == 0);
-#pragma unroll
-      for (int n0 = 0; n0 < NQ; n0 += 16) {
-        uint32_t ra[16], rb[16];
-        tmem_ld16(tm + lane_base + C::OFF_S + n0, ra);       // a terms
-        tmem_ld16(tm + lane_base + C::OFF_S + NQ + n0, rb);  // b terms
+      {
+        uint32_t ra[HQ], rb[HQ];
+        tmem_ld_hq<HQ>(tm + lane_base + C::OFF_S + h0, ra);       // a terms
+        tmem_ld_hq<HQ>(tm + lane_base + C::OFF_S + NQ + h0, rb);  // b terms
         tmem_ld_wait();
 #pragma unroll
-        for (int n = 0; n < 16; ++n) {
+        for (int n = 0; n < HQ; ++n) {
           const int y = (int)ra[n] * 128 + (int)rb[n];  // exact: |y| < 2^27
-          x[n0 + n] = valid ? fmaf((float)y, ms.sig[n0 + n], -cm[n0 + n]) : -INFINITY;
-          need |= x[n0 + n] > kTau;
+          x[n] = valid ? fmaf((float)y, ms.sig[h0 + n], -cm[n]) : -INFINITY;
+          need |= x[n] > kTau;
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ms.s_free);
       const uint32_t wneed = __any_sync(0xffffffffu, need) ? 1u : 0u;
-      if (lane == 0) ms.vote[i & 1][q] = wneed;
-      named_bar(1, 128);
-      const bool any = (ms.vote[i & 1][0] | ms.vote[i & 1][1] | ms.vote[i & 1][2] | ms.vote[i & 1][3]) != 0u;
+      if (lane == 0) ms.vote[hh][i & 1][q] = wneed;
+      named_bar(barid, 128);
+      const uint32_t *vt = ms.vote[hh][i & 1];
+      const bool any = (vt[0] | vt[1] | vt[2] | vt[3]) != 0u;
       if (any) {
         // raise the running max: m <- m + max(0, tile max of x) (the first tile: m <- its max)
 #pragma unroll
-        for (int n = 0; n < NQ; ++n) {
+        for (int n = 0; n < HQ; ++n) {
           float v = x[n];
 #pragma unroll
           for (int off = 16; off; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-          if (lane == 0) ms.red[q][n] = v;
+          if (lane == 0) ms.red[q][h0 + n] = v;
         }
-        named_bar(1, 128);
-        float *f = ms.fac[q];
+        named_bar(barid, 128);
+        float *f = ms.fac[sw];
 #pragma unroll
-        for (int n = 0; n < NQ; ++n) {
-          const float d = fmaxf(fmaxf(ms.red[0][n], ms.red[1][n]), fmaxf(ms.red[2][n], ms.red[3][n]));
+        for (int n = 0; n < HQ; ++n) {
+          const int hn = h0 + n;
+          const float d = fmaxf(fmaxf(ms.red[0][hn], ms.red[1][hn]), fmaxf(ms.red[2][hn], ms.red[3][hn]));
           const float sh = (i == 0) ? d : fmaxf(d, 0.f);
           const float fn = (i == 0) ? 0.f : exp2f(-sh);
           x[n] -= sh;
@@ -572,24 +599,24 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
           if (!wait_bar(&ms.p_free[pj], (uint32_t)((i - 1) >> 1) & 1u, abort, p.wait_ns)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll 1
-          for (int cc = 0; cc < 2 * NQ; cc += 16) {  // both ACC blocks, 16 columns at a time
-            uint32_t a[16];
-            const uint32_t ta = tm + lane_base + C::OFF_ACC + cc;
-            tmem_ld16(ta, a);
+          for (int blk = 0; blk < 2; ++blk) {  // both ACC blocks, this warp's head columns
+            uint32_t a[HQ];
+            const uint32_t ta = tm + lane_base + C::OFF_ACC + blk * NQ + h0;
+            tmem_ld_hq<HQ>(ta, a);
             tmem_ld_wait();
 #pragma unroll
-            for (int n = 0; n < 16; ++n) a[n] = __float_as_uint(__uint_as_float(a[n]) * f[(cc + n) % NQ]);
-            tmem_st16(ta, a);
+            for (int n = 0; n < HQ; ++n) a[n] = __float_as_uint(__uint_as_float(a[n]) * f[n]);
+            tmem_st_hq<HQ>(ta, a);
           }
           tmem_st_wait();
         }
       }
-      // P row of this token (fp16), MN-major: NQ/8 chunks of 8 heads
+      // P row of this token (fp16) for this warp's heads, MN-major: HQ/8 chunks of 8 heads
       const int pb = i & 1;
       if (!wait_bar(&ms.p_free[pb], par ^ 1u, abort, p.wait_ns)) { ok = false; break; }
-      uint8_t *prow = smem + C::SM_P + pb * C::P_BYTES + (kap >> 3) * 128 + (kap & 7) * 16;
+      uint8_t *prow = smem + C::SM_P + pb * C::P_BYTES + (kap >> 3) * 128 + (kap & 7) * 16 + (h0 / 8) * C::SBO_P;
 #pragma unroll
-      for (int g8 = 0; g8 < NQ / 8; ++g8) {
+      for (int g8 = 0; g8 < HQ / 8; ++g8) {
         uint32_t h2[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -614,50 +641,48 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
       tc_fence_after();
       // L~ = sum over the CTA's tokens of the fp16 weights actually pooled
 #pragma unroll
-      for (int n = 0; n < NQ; ++n) {
+      for (int n = 0; n < HQ; ++n) {
         float v = lsum[n];
 #pragma unroll
         for (int off = 16; off; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-        if (lane == 0) ms.red[q][n] = v;
+        if (lane == 0) ms.red[q][h0 + n] = v;
       }
-      if (stid == 0) {
-#pragma unroll
-        for (int n = 0; n < NQ; ++n) ms.m[n] = ms.cm[0][n] - ms.corr[n];
+      named_bar(barid, 128);
+      if (gtid < HQ) {
+        const int hn = h0 + gtid;
+        ms.lt[hn] = (ms.red[0][hn] + ms.red[1][hn]) + (ms.red[2][hn] + ms.red[3][hn]);
+        ms.m[hn] = ms.cm[4 * hh][gtid] - ms.corr[hn];
       }
-      named_bar(1, 128);
-      if (stid < NQ) ms.fac[0][stid] = (ms.red[0][stid] + ms.red[1][stid]) + (ms.red[2][stid] + ms.red[3][stid]);
-      named_bar(1, 128);
-      const float *Lt = ms.fac[0];
+      named_bar(barid, 128);
+      const float *Lt = ms.lt;
       float *out = p.part + (((size_t)b * p.S + split) * NQ) * (2 + G);
-      if (stid < NQ) {
-        out[(size_t)stid * (2 + G)] = ms.m[stid];
-        out[(size_t)stid * (2 + G) + 1] = Lt[stid];
+      if (gtid < HQ) {
+        out[(size_t)(h0 + gtid) * (2 + G)] = ms.m[h0 + gtid];
+        out[(size_t)(h0 + gtid) * (2 + G) + 1] = Lt[h0 + gtid];
       }
       // TMEM lane L of sub-partition q in half h holds coordinate
       // 128h + 32q + 8((L%8)/2) + 4(L%2) + L/8 (see the pooling dequant); values
       // are 16 + nibble.  NH=1 keeps one ACC copy per 64-token chunk: add them.
       const int jn = lane >> 3, sl = lane & 7;
+      uint32_t a0[HQ], a1[HQ];
+      tmem_ld_hq<HQ>(tm + lane_base + C::OFF_ACC + h0, a0);
+      tmem_ld_hq<HQ>(tm + lane_base + C::OFF_ACC + NQ + h0, a1);
+      tmem_ld_wait();
       if constexpr (C::NH == 2) {
-#pragma unroll 1
+#pragma unroll
         for (int h = 0; h < 2; ++h) {
-          uint32_t a[NQ];
-          tmem_ld_nq<NQ>(tm + lane_base + C::OFF_ACC + h * NQ, a);
-          tmem_ld_wait();
           const int g = 128 * h + 32 * q + 8 * (sl >> 1) + 4 * (sl & 1) + jn;
 #pragma unroll
-          for (int n = 0; n < NQ; ++n) out[(size_t)n * (2 + G) + 2 + g] = __uint_as_float(a[n]) - 24.f * Lt[n];
+          for (int n = 0; n < HQ; ++n)
+            out[(size_t)(h0 + n) * (2 + G) + 2 + g] = __uint_as_float(h ? a1[n] : a0[n]) - 24.f * Lt[h0 + n];
         }
       } else {
-        uint32_t a0[NQ], a1[NQ];
-        tmem_ld_nq<NQ>(tm + lane_base + C::OFF_ACC, a0);
-        tmem_ld_nq<NQ>(tm + lane_base + C::OFF_ACC + NQ, a1);
-        tmem_ld_wait();
         const int g = 32 * q + 8 * (sl >> 1) + 4 * (sl & 1) + jn;
         if (g < G) {
 #pragma unroll
-          for (int n = 0; n < NQ; ++n) {
+          for (int n = 0; n < HQ; ++n) {
             const float d = __uint_as_float(a0[n]) + __uint_as_float(a1[n]);
-            out[(size_t)n * (2 + G) + 2 + g] = d - 24.f * Lt[n];
+            out[(size_t)(h0 + n) * (2 + G) + 2 + g] = d - 24.f * Lt[h0 + n];
           }
         }
       }
