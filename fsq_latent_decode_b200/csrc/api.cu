@@ -23,7 +23,7 @@ cudaError_t launch_expand_simt(const uint16_t *q, const uint8_t *codes, int64_t 
                                cudaStream_t st);
 int simt_max_nq();
 int simt_max_grp();
-bool absorbed_tc_supported(int n_q, int G);
+bool absorbed_tc_supported(int n_q, int n_kv, int G);
 size_t absorbed_tc_qphys_bytes(int n_q, int G);
 cudaError_t launch_absorbed_tc(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
                                int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv, float scale, int S,
@@ -86,7 +86,7 @@ fsq_status plan_decode(int64_t B, int64_t T, int n_q, int n_kv, int d_h, int G, 
   if (op.rope_knorm && !(op.rope_base > 1.f && op.knorm_eps >= 0.f)) return FSQ_ERR_INVALID_ARG;
 
   const int64_t Bc = B > 0 ? B : 1;
-  const bool tc = kEnableTc && variant == FSQ_VARIANT_ABSORBED && absorbed_tc_supported(n_q, G);
+  const bool tc = kEnableTc && variant == FSQ_VARIANT_ABSORBED && absorbed_tc_supported(n_q, n_kv, G);
   const int64_t ctas_per_row = variant == FSQ_VARIANT_EXPAND ? n_kv : 1;
   int64_t S = op.num_splits;
   if (S == 0) {

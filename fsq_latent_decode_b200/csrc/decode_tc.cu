@@ -704,62 +704,136 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
 // kappa = 8w + 4e + i for coordinate 8w + 2i + e (the dequant's byte order).
 // corr[b] = [sigma_h] then [sigma_h * 8 * sum_g (128 a_g + b_g)]: the score is
 // sigma (128 S_a + S_b) - offset, the offset removing the +8 of the bytes.
-template <int G, int NQ>
-__global__ void absorb_query_tc(const uint16_t *__restrict__ q, const uint16_t *__restrict__ W_kv, int n_kv,
-                                float c, uint8_t *__restrict__ qphys, float *__restrict__ corr, uint32_t *err) {
+// Threads: KPAD coordinates x NDQ slices of the head dimension, so that every
+// thread has at most 32 rows of W_k^(j) to load (all issued at once); the
+// slices are summed in shared memory.
+template <int GRP>
+struct AbsorbShape {
+  static constexpr int NDQ = GRP <= 4 ? 4 : (GRP == 8 ? 2 : 1);
+};
+
+template <int G, int NQ, int GRP>
+__global__ void __launch_bounds__(Cfg<G, NQ>::KPAD * AbsorbShape<GRP>::NDQ)
+    absorb_query_tc(const uint16_t *__restrict__ q, const uint16_t *__restrict__ W_kv, float c,
+                    uint8_t *__restrict__ qphys, float *__restrict__ corr, uint32_t *err) {
+  // one CTA per (kv head j, batch row b): the group's heads share W_k^(j), read once
   using C = Cfg<G, NQ>;
   constexpr int D = FSQ_HEAD_DIM;
-  __shared__ float qs[D];
-  __shared__ float qv[C::KPAD];
-  __shared__ float red[8];
-  __shared__ int ired[8];
-  const int h = blockIdx.x, b = blockIdx.y;
-  const int j = h / (NQ / n_kv);
-  if (h == 0 && b == 0 && threadIdx.x == 0) *err = 0u;
-  for (int d = threadIdx.x; d < D; d += blockDim.x) qs[d] = bf16_to_f32(q[((int64_t)b * NQ + h) * D + d]);
+  constexpr int NDQ = AbsorbShape<GRP>::NDQ;
+  constexpr int GS = C::KPAD;       // threads per slice (one per padded coordinate)
+  constexpr int DS = D / NDQ;       // head-dimension rows per thread
+  constexpr int kBatch = DS < 32 ? DS : 32;
+  constexpr int NW = GS / 32;       // warps of slice 0
+  __shared__ __align__(16) float qs[GRP][D];  // read as float4
+  __shared__ float part[NDQ > 1 ? NDQ - 1 : 1][GRP][GS];
+  __shared__ float red[GRP][NW];
+  __shared__ int ired[GRP][NW];
+  __shared__ float sig_s[GRP];
+  const int j = blockIdx.x, b = blockIdx.y;
+  const int g = threadIdx.x % GS, dq = threadIdx.x / GS;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (j == 0 && b == 0 && threadIdx.x == 0) *err = 0u;
+  for (int i = threadIdx.x; i < GRP * D; i += blockDim.x)
+    qs[i / D][i % D] = bf16_to_f32(q[((int64_t)b * NQ + j * GRP) * D + i]);
   __syncthreads();
-  float amax = 0.f;
-  for (int g = threadIdx.x; g < C::KPAD; g += blockDim.x) {
-    float v = 0.f;
-    if (g < G) {
-      const uint16_t *wk = W_kv + (int64_t)j * D * G + g;
-      for (int d = 0; d < D; ++d) v = fmaf(bf16_to_f32(wk[(int64_t)d * G]), qs[d], v);
-      v *= c;
+  float v[GRP];
+#pragma unroll
+  for (int hh = 0; hh < GRP; ++hh) v[hh] = 0.f;
+  if (g < G) {
+    const uint16_t *wk = W_kv + ((int64_t)j * D + dq * DS) * G + g;
+#pragma unroll 1
+    for (int d0 = 0; d0 < DS; d0 += kBatch) {
+      float w[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) w[u] = bf16_to_f32(wk[(int64_t)(d0 + u) * G]);
+#pragma unroll
+      for (int u = 0; u < kBatch; u += 4)
+#pragma unroll
+        for (int hh = 0; hh < GRP; ++hh) {
+          const float4 qv = *reinterpret_cast<const float4 *>(&qs[hh][dq * DS + d0 + u]);
+          v[hh] = fmaf(w[u], qv.x, fmaf(w[u + 1], qv.y, fmaf(w[u + 2], qv.z, fmaf(w[u + 3], qv.w, v[hh]))));
+        }
     }
-    qv[g] = v;
-    amax = fmaxf(amax, fabsf(v));
   }
-  for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
+  if (NDQ > 1) {
+    if (dq > 0) {
+#pragma unroll
+      for (int hh = 0; hh < GRP; ++hh) part[dq - 1][hh][g] = v[hh];
+    }
+    __syncthreads();
+    if (dq == 0) {
+#pragma unroll
+      for (int i = 0; i < NDQ - 1; ++i)
+#pragma unroll
+        for (int hh = 0; hh < GRP; ++hh) v[hh] += part[i][hh][g];
+    }
+  }
+  if (dq == 0) {
+#pragma unroll
+    for (int hh = 0; hh < GRP; ++hh) {
+      v[hh] *= c;
+      float am = fabsf(v[hh]);
+#pragma unroll
+      for (int o = 16; o; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+      if (lane == 0) red[hh][warp] = am;
+    }
+  }
   __syncthreads();
-  float am = 0.f;
-  for (int i = 0; i < (int)(blockDim.x >> 5); ++i) am = fmaxf(am, red[i]);
-  const float sigma = am > 0.f ? am / (127.f * 128.f) : 1.f;
-  int isum = 0;
-  uint8_t *dst = qphys + (size_t)b * C::Q_BYTES;
-  for (int kap = threadIdx.x; kap < C::KPAD; kap += blockDim.x) {
-    const int w = kap >> 3, e = (kap >> 2) & 1, i4 = kap & 3;
-    const int g = 8 * w + 2 * i4 + e;
-    const float t = qv[g] / sigma;
-    int a = __float2int_rn(t / 128.f);
-    a = max(-127, min(127, a));
-    int bt = __float2int_rn(t - 128.f * (float)a);
-    bt = max(-127, min(127, bt));
-    isum += 128 * a + bt;
-    // K-major no swizzle, 8-bit: 16-byte K chunk kappa/16, 8-row group n/8, row n%8, byte kappa%16
+  if (threadIdx.x < GRP) {
+    float am = 0.f;
+    for (int i = 0; i < NW; ++i) am = fmaxf(am, red[threadIdx.x][i]);
+    sig_s[threadIdx.x] = am > 0.f ? am / (127.f * 128.f) : 1.f;
+  }
+  __syncthreads();
+  if (dq == 0) {
+    // coordinate g = 8w + 2i + e sits at K position kappa = 8w + 4e + i
+    const int kap = (g & ~7) | ((g & 1) << 2) | ((g >> 1) & 3);
+    uint8_t *dst = qphys + (size_t)b * C::Q_BYTES;
     const int base = (kap >> 4) * C::LBO_Q + (kap & 15);
-    dst[base + (h >> 3) * 128 + (h & 7) * 16] = (uint8_t)(int8_t)a;
-    dst[base + ((NQ + h) >> 3) * 128 + ((NQ + h) & 7) * 16] = (uint8_t)(int8_t)bt;
+#pragma unroll
+    for (int hh = 0; hh < GRP; ++hh) {
+      const int h = j * GRP + hh;
+      const float t = v[hh] / sig_s[hh];
+      const int a = max(-127, min(127, __float2int_rn(t / 128.f)));
+      const int bt = max(-127, min(127, __float2int_rn(t - 128.f * (float)a)));
+      int isum = 128 * a + bt;
+      dst[base + (h >> 3) * 128 + (h & 7) * 16] = (uint8_t)(int8_t)a;
+      dst[base + ((NQ + h) >> 3) * 128 + ((NQ + h) & 7) * 16] = (uint8_t)(int8_t)bt;
+#pragma unroll
+      for (int o = 16; o; o >>= 1) isum += __shfl_xor_sync(0xffffffffu, isum, o);
+      if (lane == 0) ired[hh][warp] = isum;
+    }
   }
-  for (int o = 16; o; o >>= 1) isum += __shfl_xor_sync(0xffffffffu, isum, o);
-  if ((threadIdx.x & 31) == 0) ired[threadIdx.x >> 5] = isum;
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (threadIdx.x < GRP) {
     long long tot = 0;
-    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) tot += ired[i];
-    corr[(size_t)b * 2 * NQ + h] = sigma;
-    corr[(size_t)b * 2 * NQ + NQ + h] = (float)((double)sigma * 8.0 * (double)tot);
+    for (int i = 0; i < NW; ++i) tot += ired[threadIdx.x][i];
+    const int h = j * GRP + threadIdx.x;
+    corr[(size_t)b * 2 * NQ + h] = sig_s[threadIdx.x];
+    corr[(size_t)b * 2 * NQ + NQ + h] = (float)((double)sig_s[threadIdx.x] * 8.0 * (double)tot);
   }
+}
+
+template <int G, int NQ, int GRP>
+void absorb_query_launch(const dim3 &grid, const uint16_t *q, const uint16_t *W_kv, float c, uint8_t *qphys,
+                         float *corr, uint32_t *err, cudaStream_t st) {
+  absorb_query_tc<G, NQ, GRP><<<grid, Cfg<G, NQ>::KPAD * AbsorbShape<GRP>::NDQ, 0, st>>>(q, W_kv, c, qphys, corr,
+                                                                                        err);
+}
+
+template <int G, int NQ>
+cudaError_t launch_absorb_query(const uint16_t *q, int64_t B, int n_kv, const uint16_t *W_kv, float c,
+                                uint8_t *qphys, float *corr, uint32_t *err, cudaStream_t st) {
+  const dim3 grid(n_kv, (unsigned)B);
+  switch (NQ / n_kv) {
+    case 1: absorb_query_launch<G, NQ, 1>(grid, q, W_kv, c, qphys, corr, err, st); break;
+    case 2: absorb_query_launch<G, NQ, 2>(grid, q, W_kv, c, qphys, corr, err, st); break;
+    case 4: absorb_query_launch<G, NQ, 4>(grid, q, W_kv, c, qphys, corr, err, st); break;
+    case 8: absorb_query_launch<G, NQ, 8>(grid, q, W_kv, c, qphys, corr, err, st); break;
+    case 16: absorb_query_launch<G, NQ, 16>(grid, q, W_kv, c, qphys, corr, err, st); break;
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
 }
 
 // Tensor map of the code cache as a 3-D byte tensor [B][T][row bytes]: the
@@ -797,8 +871,7 @@ cudaError_t launch(const uint16_t *q, const uint8_t *codes, int64_t bstride, int
                    const uint16_t *W_kv, float scale, int S, int64_t tps, uint8_t *qphys, float *corr, float *part,
                    uint32_t *err, void *const *prof, cudaStream_t st) {
   using C = Cfg<G, NQ>;
-  absorb_query_tc<G, NQ><<<dim3(NQ, (unsigned)B), 256, 0, st>>>(q, W_kv, n_kv, scale * kLog2e, qphys, corr, err);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_absorb_query<G, NQ>(q, B, n_kv, W_kv, scale * kLog2e, qphys, corr, err, st);
   if (e != cudaSuccess) return e;
   // one CTA per SM: ask for more shared memory than two CTAs could share
   const int smem = C::SM_TOTAL > 120 * 1024 ? C::SM_TOTAL : 120 * 1024;
@@ -820,7 +893,9 @@ cudaError_t launch(const uint16_t *q, const uint8_t *codes, int64_t bstride, int
 
 }  // namespace tc
 
-bool absorbed_tc_supported(int n_q, int G) { return (n_q == 16 || n_q == 32) && (G == 256 || G == 84); }
+bool absorbed_tc_supported(int n_q, int n_kv, int G) {
+  return (n_q == 16 || n_q == 32) && (G == 256 || G == 84) && n_kv > 0 && n_q % n_kv == 0 && n_q / n_kv <= 16;
+}
 
 size_t absorbed_tc_qphys_bytes(int n_q, int G) {
   const int kpad = (G + 31) / 32 * 32;

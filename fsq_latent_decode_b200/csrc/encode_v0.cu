@@ -97,6 +97,70 @@ __global__ void __launch_bounds__(256) encode_pack_rows(const uint16_t *__restri
   if (lane == 0) codes[t * ldc + by] = (uint8_t)(fsq_nibble(a0, th) | (fsq_nibble(a1, th) << 4));
 }
 
+// Decode-step append (up to 16 tokens): one CTA per coordinate pair (2i, 2i+1).
+// Its 512 threads take interleaved 16-byte chunks of C, so for C <= 4096 every
+// load of the kernel is issued at once; E's two rows are read once for all
+// tokens.  The 32 per-thread sums (16 tokens x 2 coordinates) are reduced
+// across the warp by a transposing butterfly (31 shuffles, lane l ends with
+// sum l), then across the 16 warps in shared memory.
+constexpr int kFewTok = 16;
+constexpr int kFewWarps = 16;
+__global__ void __launch_bounds__(kFewWarps * 32, 1)
+    encode_pack_few(const uint16_t *__restrict__ x, int n_tok, int64_t ldx, int64_t C,
+                    const uint16_t *__restrict__ E, int G, Thresholds th, uint8_t *__restrict__ codes, int64_t ldc) {
+  __shared__ float red[kFewWarps][2 * kFewTok];
+  const int by = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint4 *e0 = reinterpret_cast<const uint4 *>(E + (int64_t)(2 * by) * C);
+  const uint4 *e1 = reinterpret_cast<const uint4 *>(E + (int64_t)(2 * by + 1) * C);
+  float v[2 * kFewTok];  // v[t]: coordinate 2i of token t; v[16 + t]: coordinate 2i+1
+#pragma unroll
+  for (int i = 0; i < 2 * kFewTok; ++i) v[i] = 0.f;
+  for (int64_t k = threadIdx.x; k < C / 8; k += kFewWarps * 32) {
+    const uint4 w0 = e0[k], w1 = e1[k];
+    uint4 xv[kFewTok];
+#pragma unroll
+    for (int t = 0; t < kFewTok; ++t)
+      xv[t] = t < n_tok ? reinterpret_cast<const uint4 *>(x + (int64_t)t * ldx)[k] : make_uint4(0u, 0u, 0u, 0u);
+    const uint32_t s0[4] = {w0.x, w0.y, w0.z, w0.w}, s1[4] = {w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+    for (int t = 0; t < kFewTok; ++t) {
+      const uint32_t xs[4] = {xv[t].x, xv[t].y, xv[t].z, xv[t].w};
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const float xl = __uint_as_float(xs[jj] << 16), xh = __uint_as_float(xs[jj] & 0xFFFF0000u);
+        v[t] = fmaf(xl, __uint_as_float(s0[jj] << 16), fmaf(xh, __uint_as_float(s0[jj] & 0xFFFF0000u), v[t]));
+        v[kFewTok + t] =
+            fmaf(xl, __uint_as_float(s1[jj] << 16), fmaf(xh, __uint_as_float(s1[jj] & 0xFFFF0000u), v[kFewTok + t]));
+      }
+    }
+  }
+  // butterfly: at offset o a lane keeps the half of its values selected by
+  // (lane & o) and adds the partner's copy of that half
+#pragma unroll
+  for (int o = 16, n = 16; o; o >>= 1, n >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < n; ++i) {
+      const float send = up ? v[i] : v[i + n];
+      const float keep = up ? v[i + n] : v[i];
+      v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  red[warp][lane] = v[0];
+  __syncthreads();
+  if (threadIdx.x < n_tok) {
+    const int t = threadIdx.x;
+    float u0 = 0.f, u1 = 0.f;
+#pragma unroll
+    for (int w = 0; w < kFewWarps; ++w) {
+      u0 += red[w][t];
+      u1 += red[w][kFewTok + t];
+    }
+    codes[(int64_t)t * ldc + by] = (uint8_t)(fsq_nibble(u0, th) | (fsq_nibble(u1, th) << 4));
+  }
+}
+
 __global__ void quantize_pack_f32_kernel(const float *__restrict__ u, int64_t n_tok, int G, Thresholds th,
                                          uint8_t *__restrict__ codes, int64_t ldc) {
   const int half = G / 2;
@@ -113,6 +177,10 @@ __global__ void quantize_pack_f32_kernel(const float *__restrict__ u, int64_t n_
 cudaError_t launch_encode_pack_simt(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C,
                                     const uint16_t *E, int G, const Thresholds &th, uint8_t *codes,
                                     int64_t ldc, cudaStream_t s) {
+  if (n_tok <= kFewTok) {
+    encode_pack_few<<<(unsigned)(G / 2), kFewWarps * 32, 0, s>>>(x, (int)n_tok, ldx, C, E, G, th, codes, ldc);
+    return cudaGetLastError();
+  }
   if (n_tok <= 64) {
     const int64_t warps = n_tok * (G / 2);
     encode_pack_rows<<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(x, n_tok, ldx, C, E, G, th, codes, ldc);

@@ -52,7 +52,8 @@ def test_quantize_pack_bit_exact(G, h, n_tok):
 
 # ---------------------------------------------------------------- encoder + FSQ + pack
 @pytest.mark.parametrize("n_tok,C,G", [(1024, 1024, 256), (4096, 2048, 256), (4096, 4096, 256), (4096, 4096, 84),
-                                       (1, 1024, 84), (37, 2048, 256), (129, 4096, 84)])
+                                       (1, 1024, 84), (16, 4096, 256), (17, 2048, 84), (37, 2048, 256),
+                                       (129, 4096, 84)])
 def test_encode_pack_parity(n_tok, C, G):
     gen = synth._gen(synth.workload_seed(21, n_tok, C, G))
     x, E = synth.encoder_inputs(n_tok, C, G, gen)
