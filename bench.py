@@ -226,23 +226,29 @@ def run_gpu(args, wl_name, B, T, torch, F, synth, dist, rank, world, device, tim
         step(i)
     torch.cuda.synchronize()
     K = args.steps
-    evs = RawEvents(K)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(torch.cuda.current_device()) if (timed and rank == 0) else None
     if clocks:
         clocks.start()
+    # throughput: K steps exactly as a user issues them (no profiling events)
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
     t0.record(stream)
     for i in range(K):
-        step(i, evs.pair(i))
+        step(i)
     t1.record(stream)
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
-    clk = clocks.stop() if clocks else None
     ms = t0.elapsed_time(t1) / K
+    # main-kernel duration: K more steps with events recorded by the library
+    # around the split kernel on its own stream
+    evs = RawEvents(K)
+    for i in range(K):
+        step(i, evs.pair(i))
+    torch.cuda.synchronize()
+    clk = clocks.stop() if clocks else None
     kern_ms = sum(evs.elapsed_ms(i) for i in range(K)) / K
     evs.close()
     if dist is not None:
@@ -452,7 +458,8 @@ def main():
         line = {"metric": "FSQ decode-attn context tok/s & code GB/s, Qwen3-8B G=256/84; % roofline",
                 "value": value, "unit": "context tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": res["ms"], "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "f32",
+                "vs_baseline": None,
+                "dtype": "u4 codes; s8 x u8 score MMA (s32), f16 pooling MMA (f32), f32 softmax/merge, bf16 in/out",
                 "data": "synthetic (seeded; cache = FSQ codes of u ~ N(0,4), the law of E x; new token x ~ N(0,1) appended each step)",
                 "config": config, "code_gbs": world * res["code_bytes"] / (res["ms"] * 1e-3) / 1e9,
                 "roofline": rf, "cpu_baseline": cb, "e2e": res["e2e"], "clocks": res["clocks"],

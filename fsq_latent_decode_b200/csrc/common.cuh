@@ -5,6 +5,10 @@
 #include <cuda_fp16.h>
 #include <stdint.h>
 
+#include <map>
+#include <mutex>
+#include <utility>
+
 #include "../../include/fsq.h"
 
 namespace fsq {
@@ -45,5 +49,60 @@ __device__ __forceinline__ void record_error(uint32_t *err, int status) {
 }
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Raise a kernel's dynamic shared-memory limit on the current device, once:
+// the attribute is per function and device and stays set, so later calls
+// needing no more than the largest limit set so far skip the driver call.
+inline cudaError_t ensure_smem_limit(const void *fn, size_t bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static std::mutex mu;
+  static std::map<std::pair<const void *, int>, size_t> done;
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = done.find({fn, dev});
+  if (it != done.end() && it->second >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+  if (e == cudaSuccess) done[{fn, dev}] = bytes;
+  return e;
+}
+
+// Programmatic dependent launch.  Kernels launched with launch_pdl may start
+// while the previous kernel of the stream is still running, once every CTA of
+// that kernel has called pdl_trigger (or exited).  A kernel reads nothing that
+// the previous kernels write before pdl_wait, which returns when they have
+// completed and their writes are visible.  Each of these kernels calls
+// pdl_trigger only after its own pdl_wait, so a kernel that starts early
+// still sees every kernel before its predecessor complete.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// Profiling events around the main kernel.  While the stream is being
+// captured into a graph they are recorded as external events (event nodes of
+// the graph); otherwise as plain records.
+inline void record_prof_event(void *ev, cudaStream_t st) {
+  if (!ev) return;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(st, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags((cudaEvent_t)ev, st, cudaEventRecordExternal);
+  else
+    cudaEventRecord((cudaEvent_t)ev, st);
+}
 
 }  // namespace fsq

@@ -15,9 +15,10 @@
 //   -> score-dequant warps unpack each token's nibbles in registers into
 //      token-major Z in TMEM (A of the score MMA, double-buffered)
 //   -> pool-dequant warps build coordinate-major Z^T in TMEM (A of the pooling
-//      MMA, in two 64-token chunks): an 8x8 register transpose (movmatrix) of
-//      the still-packed 16-bit groups of four nibbles, then the nibbles are
-//      unpacked, so one transpose serves four coordinates
+//      MMA, in two 64-token chunks): the still-packed 16-bit groups of four
+//      nibbles are read transposed in 8x8 blocks (ldmatrix.trans; movmatrix
+//      when rows are not 16-byte aligned), then unpacked, so one transpose
+//      serves four coordinates
 //   -> three issuer threads (score MMAs; pooling MMAs of each 128-row half or
 //      chunk) keep the tensor core fed: a single issuing thread cannot issue
 //      small-N MMAs as fast as the tensor core retires them
@@ -28,10 +29,11 @@
 // LOP3 or SHF+LOP3 per four nibbles), and Q' is split per head into two int8
 // terms, Q' ~ sigma (128 a + b), stacked along N (2 n_q columns), so the score
 // is exact integer arithmetic on a 15-bit Q': s = sigma (128 S_a + S_b) minus a
-// per-head offset for the -8 level shift.  Pooling MMA (kind::f16): a shift
-// and a LOP3 per pair give the fp16 values 16 + n; ACC is corrected by 24 l
-// per head at the end (16 for the bias, 8 for the level offset), keeping the
-// split-long fp32 accumulation well conditioned.
+// per-head offset for the -8 level shift.  Pooling MMA (kind::f16): one LOP3
+// per pair (plus a shift shared by two pairs) leaves each nibble in place in
+// the mantissa of an fp16 subnormal, n 2^-24 or n 2^-20; the products with the
+// fp16 weights are exact, the pooled sums carry no bias, and the epilogue
+// scales them back and removes the level offset (8 l per head).
 //
 // Warps (24): 0 loads code tiles and owns TMEM; 1 issues score MMAs; 2-3 issue
 // pooling MMAs; 4-7 score dequant; 12-15 and 16-19 pooling dequant for the
@@ -147,12 +149,15 @@ __device__ __forceinline__ void mma_ts_i8(uint32_t d_tmem, uint32_t a_tmem, uint
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-// Nibble J (bits 4J..4J+3) of both half-words moved to mantissa bits 6..9 of
-// the pattern of 16.0: the fp16 pair (16 + n_lo, 16 + n_hi), exact.
-template <int J>
-__device__ __forceinline__ uint32_t nib16(uint32_t w) {
-  const uint32_t x = (J == 0) ? (w << 6) : (J == 1) ? (w << 2) : (J == 2) ? (w >> 2) : (w >> 6);
-  return (x & 0x03C003C0u) | 0x4C004C00u;
+// Pooling operand values as fp16 subnormals, no bias: nibble J of both
+// half-words left in place in mantissa bits 0..3 (value n 2^-24) or bits 4..7
+// (value n 2^-20).  w holds, per half-word, the four nibbles of one token.
+__device__ __forceinline__ void nib_sub4(uint32_t w, uint32_t &j0, uint32_t &j1, uint32_t &j2, uint32_t &j3) {
+  const uint32_t ws = w >> 8;
+  j0 = w & 0x000F000Fu;   // n 2^-24
+  j1 = w & 0x00F000F0u;   // n 2^-20
+  j2 = ws & 0x000F000Fu;  // n 2^-24
+  j3 = ws & 0x00F000F0u;  // n 2^-20
 }
 
 // Physical K position of token r in the pooling operand (see the 16x256b store below).
@@ -184,9 +189,10 @@ __device__ __forceinline__ uint32_t lds_u32_a2(const uint8_t *p) {
   return (uint32_t)h[0] | ((uint32_t)h[1] << 16);
 }
 
-// Bounded barrier wait: non-blocking probes with a short sleep between them,
-// so that a waiting warp neither spins on the issue port nor oversleeps the
-// phase flip.  Gives up after `limit_ns` or once *abort is set.
+// Bounded barrier wait.  mbarrier.try_wait with a suspend-time hint parks the
+// warp in hardware until the phase completes (or the hint expires), so a
+// waiting warp takes no issue slots from the working warps of its scheduler.
+// Gives up after `limit_ns` or once *abort is set.
 __device__ __forceinline__ bool bar_test(uint32_t a, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -198,18 +204,38 @@ __device__ __forceinline__ bool bar_test(uint32_t a, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-__device__ __forceinline__ bool wait_bar(uint64_t *b, uint32_t parity, volatile uint32_t *abort, uint64_t limit_ns,
-                                         uint32_t sleep_ns = 20) {
+__device__ __forceinline__ bool bar_try(uint32_t a, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(a), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool wait_bar(uint64_t *b, uint32_t parity, volatile uint32_t *abort, uint64_t limit_ns) {
   const uint32_t a = smem_u32(b);
   if (bar_test(a, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (sleep_ns) __nanosleep(sleep_ns);
-    if (bar_test(a, parity)) return true;
-    if ((it & 255u) == 0u) {
+    if (bar_try(a, parity, 1000u)) return true;
+    if ((it & 7u) == 0u) {
       if (*abort) return false;
       if (globaltimer_ns() - t0 > limit_ns) return false;
     }
+  }
+}
+
+// Error path: wait (time-bounded, ignoring the abort flag) for an async copy
+// already issued into this CTA's shared memory, so none lands after exit.
+__device__ __forceinline__ void drain_bar(uint64_t *b, uint32_t parity, uint64_t limit_ns) {
+  const uint32_t a = smem_u32(b);
+  const uint64_t t0 = globaltimer_ns();
+  while (!bar_test(a, parity)) {
+    __nanosleep(100);
+    if (globaltimer_ns() - t0 > limit_ns) return;
   }
 }
 
@@ -295,6 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = ms.tmem_base;
+  pdl_trigger();  // the merge kernel may start staging W_v
 
   auto fail = [&]() {
     record_error(p.err, FSQ_ERR_TIMEOUT);
@@ -304,15 +331,25 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     uint8_t *ring = smem + C::SM_CODES;
-    if (lane == 0) {
-      mbar_arrive_expect_tx(&ms.q_full, C::Q_BYTES);
-      bulk_g2s(smem + C::SM_Q, p.qphys + (size_t)b * C::Q_BYTES, C::Q_BYTES, &ms.q_full);
-    }
+    // The codes were written before the query prologue kernel started, so the
+    // first ring-full of tiles is requested before waiting for that kernel;
+    // Q' (its output) right after, before the first wait for a free stage.
+    auto load_q = [&]() {
+      if (lane == 0) {
+        pdl_wait();
+        mbar_arrive_expect_tx(&ms.q_full, C::Q_BYTES);
+        bulk_g2s(smem + C::SM_Q, p.qphys + (size_t)b * C::Q_BYTES, C::Q_BYTES, &ms.q_full);
+      }
+    };
     int issued = 0;
-    bool ok = true;
+    bool ok = true, q_loaded = false;
     for (int i = 0; i < n_tiles; ++i) {
       const int st = i % kStages;
       const uint32_t ph = (uint32_t)(i / kStages) & 1u;
+      if (i == kStages) {
+        load_q();
+        q_loaded = true;
+      }
       if (!wait_bar(&ms.empty[st], ph ^ 1u, abort, p.wait_ns)) {
         ok = false;
         break;
@@ -340,11 +377,13 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
       }
       issued = i + 1;
     }
+    if (!q_loaded) load_q();
     if (!ok) {
       if (lane == 0) fail();
       // let the copies still in flight land before the CTA exits
       for (int i = max(0, issued - kStages); i < issued; ++i)
-        wait_bar(&ms.full[i % kStages], (uint32_t)(i / kStages) & 1u, abort, p.wait_ns / 4 + 1);
+        drain_bar(&ms.full[i % kStages], (uint32_t)(i / kStages) & 1u, p.wait_ns / 4 + 1);
+      drain_bar(&ms.q_full, 0, p.wait_ns / 4 + 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ score-MMA issuer
@@ -485,23 +524,32 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
         const int byte0 = 64 * h + 16 * q;  // first byte of this warp's 32 coordinates
         if (byte0 >= C::HALF) continue;
         uint32_t lo[16], hi[16];
+        // y[2j + e]: the 8x8 block of 16-bit groups (four nibbles of one token)
+        // of tokens 8 tb .. 8 tb + 7, tb = 8c + 2j + e, transposed, so this
+        // thread holds one group (four coordinates) of two tokens
+        uint32_t y[8];
+        if constexpr (C::TMA) {
+          const uint32_t t0a = smem_u32(tile);
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const int rr = 8 * (8 * c + 4 * hf + (lane >> 3)) + (lane & 7);
+            uint32_t r4[4];
+            ldmatrix_x4_trans(t0a + (uint32_t)swz(rr, byte0 >> 4), r4);
+#pragma unroll
+            for (int m = 0; m < 4; ++m) y[4 * hf + m] = r4[m];
+          }
+        } else {
+#pragma unroll
+          for (int m = 0; m < 8; ++m) {
+            const int rr = 8 * (8 * c + m) + (lane >> 2);
+            y[m] = movmatrix_trans(lds_u32_a2(tile + rr * C::HALF + byte0 + 4 * (lane & 3)));
+          }
+        }
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
 #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int tb = 8 * c + 2 * j + e;  // 8-token block within the tile
-            const int rr = 8 * tb + (lane >> 2);
-            uint32_t x;
-            if constexpr (C::TMA) x = *reinterpret_cast<const uint32_t *>(tile + swz(rr, byte0 >> 4) + 4 * (lane & 3));
-            else x = lds_u32_a2(tile + rr * C::HALF + byte0 + 4 * (lane & 3));
-            // transpose 16-bit groups of four nibbles: this thread now holds one
-            // group (four coordinates) of two tokens, then unpack each coordinate
-            const uint32_t y = movmatrix_trans(x);
-            lo[4 * j + e] = nib16<0>(y);
-            lo[4 * j + 2 + e] = nib16<1>(y);
-            hi[4 * j + e] = nib16<2>(y);
-            hi[4 * j + 2 + e] = nib16<3>(y);
-          }
+          for (int e = 0; e < 2; ++e)
+            nib_sub4(y[2 * j + e], lo[4 * j + e], lo[4 * j + 2 + e], hi[4 * j + e], hi[4 * j + 2 + e]);
         }
         const uint32_t cbase = tm + lane_base + C::OFF_CP + cb * C::CP_CHUNK + h * 32;
         tmem_st_16x256b_x4(cbase, lo);
@@ -527,6 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
     const int barid = 1 + hh;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     if (gtid < HQ) {
+      pdl_wait();  // corr comes from the query prologue kernel
       ms.sig[h0 + gtid] = p.corr[(size_t)b * 2 * NQ + h0 + gtid];
       ms.corr[h0 + gtid] = p.corr[(size_t)b * 2 * NQ + NQ + h0 + gtid];
     }
@@ -661,9 +710,11 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
         out[(size_t)(h0 + gtid) * (2 + G) + 1] = Lt[h0 + gtid];
       }
       // TMEM lane L of sub-partition q in half h holds coordinate
-      // 128h + 32q + 8((L%8)/2) + 4(L%2) + L/8 (see the pooling dequant); values
-      // are 16 + nibble.  NH=1 keeps one ACC copy per 64-token chunk: add them.
+      // 128h + 32q + 8((L%8)/2) + 4(L%2) + L/8 (see the pooling dequant); the
+      // pooled values are n 2^-24 (L/8 even) or n 2^-20 (L/8 odd), n = level + 8.
+      // NH=1 keeps one ACC copy per 64-token chunk: add them.
       const int jn = lane >> 3, sl = lane & 7;
+      const float vscale = (jn & 1) ? 1048576.f : 16777216.f;
       uint32_t a0[HQ], a1[HQ];
       tmem_ld_hq<HQ>(tm + lane_base + C::OFF_ACC + h0, a0);
       tmem_ld_hq<HQ>(tm + lane_base + C::OFF_ACC + NQ + h0, a1);
@@ -674,7 +725,8 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
           const int g = 128 * h + 32 * q + 8 * (sl >> 1) + 4 * (sl & 1) + jn;
 #pragma unroll
           for (int n = 0; n < HQ; ++n)
-            out[(size_t)(h0 + n) * (2 + G) + 2 + g] = __uint_as_float(h ? a1[n] : a0[n]) - 24.f * Lt[h0 + n];
+            out[(size_t)(h0 + n) * (2 + G) + 2 + g] =
+                fmaf(__uint_as_float(h ? a1[n] : a0[n]), vscale, -8.f * Lt[h0 + n]);
         }
       } else {
         const int g = 32 * q + 8 * (sl >> 1) + 4 * (sl & 1) + jn;
@@ -682,7 +734,7 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
 #pragma unroll
           for (int n = 0; n < HQ; ++n) {
             const float d = __uint_as_float(a0[n]) + __uint_as_float(a1[n]);
-            out[(size_t)(h0 + n) * (2 + G) + 2 + g] = d - 24.f * Lt[h0 + n];
+            out[(size_t)(h0 + n) * (2 + G) + 2 + g] = fmaf(d, vscale, -8.f * Lt[h0 + n]);
           }
         }
       }
@@ -732,7 +784,9 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::KPAD * AbsorbShape<GRP>::NDQ)
   const int j = blockIdx.x, b = blockIdx.y;
   const int g = threadIdx.x % GS, dq = threadIdx.x / GS;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();
   if (j == 0 && b == 0 && threadIdx.x == 0) *err = 0u;
+  pdl_trigger();  // the split kernel may start its prologue and code loads
   for (int i = threadIdx.x; i < GRP * D; i += blockDim.x)
     qs[i / D][i % D] = bf16_to_f32(q[((int64_t)b * NQ + j * GRP) * D + i]);
   __syncthreads();
@@ -815,10 +869,10 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::KPAD * AbsorbShape<GRP>::NDQ)
 }
 
 template <int G, int NQ, int GRP>
-void absorb_query_launch(const dim3 &grid, const uint16_t *q, const uint16_t *W_kv, float c, uint8_t *qphys,
-                         float *corr, uint32_t *err, cudaStream_t st) {
-  absorb_query_tc<G, NQ, GRP><<<grid, Cfg<G, NQ>::KPAD * AbsorbShape<GRP>::NDQ, 0, st>>>(q, W_kv, c, qphys, corr,
-                                                                                        err);
+cudaError_t absorb_query_launch(const dim3 &grid, const uint16_t *q, const uint16_t *W_kv, float c, uint8_t *qphys,
+                                float *corr, uint32_t *err, cudaStream_t st) {
+  return launch_pdl(absorb_query_tc<G, NQ, GRP>, grid, dim3(Cfg<G, NQ>::KPAD * AbsorbShape<GRP>::NDQ), 0, st, q, W_kv,
+                    c, qphys, corr, err);
 }
 
 template <int G, int NQ>
@@ -826,14 +880,13 @@ cudaError_t launch_absorb_query(const uint16_t *q, int64_t B, int n_kv, const ui
                                 uint8_t *qphys, float *corr, uint32_t *err, cudaStream_t st) {
   const dim3 grid(n_kv, (unsigned)B);
   switch (NQ / n_kv) {
-    case 1: absorb_query_launch<G, NQ, 1>(grid, q, W_kv, c, qphys, corr, err, st); break;
-    case 2: absorb_query_launch<G, NQ, 2>(grid, q, W_kv, c, qphys, corr, err, st); break;
-    case 4: absorb_query_launch<G, NQ, 4>(grid, q, W_kv, c, qphys, corr, err, st); break;
-    case 8: absorb_query_launch<G, NQ, 8>(grid, q, W_kv, c, qphys, corr, err, st); break;
-    case 16: absorb_query_launch<G, NQ, 16>(grid, q, W_kv, c, qphys, corr, err, st); break;
+    case 1: return absorb_query_launch<G, NQ, 1>(grid, q, W_kv, c, qphys, corr, err, st);
+    case 2: return absorb_query_launch<G, NQ, 2>(grid, q, W_kv, c, qphys, corr, err, st);
+    case 4: return absorb_query_launch<G, NQ, 4>(grid, q, W_kv, c, qphys, corr, err, st);
+    case 8: return absorb_query_launch<G, NQ, 8>(grid, q, W_kv, c, qphys, corr, err, st);
+    case 16: return absorb_query_launch<G, NQ, 16>(grid, q, W_kv, c, qphys, corr, err, st);
     default: return cudaErrorInvalidValue;
   }
-  return cudaGetLastError();
 }
 
 // Tensor map of the code cache as a 3-D byte tensor [B][T][row bytes]: the
@@ -875,7 +928,7 @@ cudaError_t launch(const uint16_t *q, const uint8_t *codes, int64_t bstride, int
   if (e != cudaSuccess) return e;
   // one CTA per SM: ask for more shared memory than two CTAs could share
   const int smem = C::SM_TOTAL > 120 * 1024 ? C::SM_TOTAL : 120 * 1024;
-  e = cudaFuncSetAttribute(absorbed_split_tc<G, NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  e = ensure_smem_limit((const void *)absorbed_split_tc<G, NQ>, (size_t)smem);
   if (e != cudaSuccess) return e;
   Params p{codes, bstride, T, tps, S, qphys, corr, part, err, kWaitLimitNs};
   CUtensorMap tmap;
@@ -884,10 +937,9 @@ cudaError_t launch(const uint16_t *q, const uint8_t *codes, int64_t bstride, int
     e = make_code_tensor_map(&tmap, codes, bstride, T, B, C::HALF);
     if (e != cudaSuccess) return e;
   }
-  if (prof[0]) cudaEventRecord((cudaEvent_t)prof[0], st);
-  absorbed_split_tc<G, NQ><<<dim3(S, (unsigned)B), kThreads, smem, st>>>(tmap, p);
-  e = cudaGetLastError();
-  if (prof[1]) cudaEventRecord((cudaEvent_t)prof[1], st);
+  record_prof_event(prof[0], st);
+  e = launch_pdl(absorbed_split_tc<G, NQ>, dim3(S, (unsigned)B), dim3(kThreads), (size_t)smem, st, tmap, p);
+  record_prof_event(prof[1], st);
   return e;
 }
 

@@ -402,6 +402,8 @@ __global__ void __launch_bounds__(MergeThreads<GRP>::NT)
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
   }
+  pdl_wait();  // the partials come from the split kernel
+  pdl_trigger();
   const int64_t sstride = (int64_t)n_q * (2 + G);
   const float *pbase = part + ((int64_t)b * S * n_q + j * GRP) * (2 + G);
   if (warp < GRP) {  // split weights for head `warp`, 1/l folded in
@@ -481,12 +483,10 @@ template <int GRP>
 cudaError_t merge_group_launch(const float *part, int S, int64_t B, int n_q, int n_kv, int d_h, int G,
                                const uint16_t *W_kv, void *o, int out_fp32, cudaStream_t st) {
   const MergeShape ms = merge_shape(G, d_h, GRP, S);
-  cudaError_t e = cudaFuncSetAttribute(merge_absorbed_group_kernel<GRP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)ms.bytes);
+  cudaError_t e = ensure_smem_limit((const void *)merge_absorbed_group_kernel<GRP>, ms.bytes);
   if (e != cudaSuccess) return e;
-  merge_absorbed_group_kernel<GRP><<<dim3(n_kv, (unsigned)B), MergeThreads<GRP>::NT, ms.bytes, st>>>(
-      part, S, n_q, n_kv, G, W_kv, o, out_fp32, ms);
-  return cudaGetLastError();
+  return launch_pdl(merge_absorbed_group_kernel<GRP>, dim3(n_kv, (unsigned)B), dim3(MergeThreads<GRP>::NT), ms.bytes,
+                    st, part, S, n_q, n_kv, G, W_kv, o, out_fp32, ms);
 }
 
 }  // namespace
@@ -525,12 +525,12 @@ cudaError_t launch_absorbed_simt(const uint16_t *q, const uint8_t *codes, int64_
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   size_t smem = absorbed_simt_smem(n_q, G);
-  e = cudaFuncSetAttribute(absorbed_split_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = ensure_smem_limit((const void *)absorbed_split_simt, smem);
   if (e != cudaSuccess) return e;
-  if (prof[0]) cudaEventRecord((cudaEvent_t)prof[0], st);
+  record_prof_event(prof[0], st);
   absorbed_split_simt<<<dim3(S, (unsigned)B), 256, smem, st>>>(qa, codes, bstride, T, G, n_q, tps, part);
   e = cudaGetLastError();
-  if (prof[1]) cudaEventRecord((cudaEvent_t)prof[1], st);
+  record_prof_event(prof[1], st);
   if (e != cudaSuccess) return e;
   return merge_absorbed_launch(part, S, B, n_q, n_kv, d_h, G, W_kv, o, out_fp32, st);
 }
@@ -544,13 +544,13 @@ cudaError_t launch_expand_simt(const uint16_t *q, const uint8_t *codes, int64_t 
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   size_t smem = expand_simt_smem(G);
-  e = cudaFuncSetAttribute(expand_split_simt, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  e = ensure_smem_limit((const void *)expand_split_simt, smem);
   if (e != cudaSuccess) return e;
-  if (prof[0]) cudaEventRecord((cudaEvent_t)prof[0], st);
+  record_prof_event(prof[0], st);
   expand_split_simt<<<dim3(S, (unsigned)B, n_kv), FSQ_HEAD_DIM, smem, st>>>(
       q, codes, bstride, T, G, n_q, n_kv, W_kv, scale * kLog2e, tps, rope_knorm, rope_base, gain, eps, part);
   e = cudaGetLastError();
-  if (prof[1]) cudaEventRecord((cudaEvent_t)prof[1], st);
+  record_prof_event(prof[1], st);
   if (e != cudaSuccess) return e;
   merge_expand_kernel<<<dim3(n_q, (unsigned)B), d_h, 0, st>>>(part, S, n_q, d_h, o, out_fp32);
   return cudaGetLastError();

@@ -113,6 +113,8 @@ __global__ void __launch_bounds__(kFewWarps * 32, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint4 *e0 = reinterpret_cast<const uint4 *>(E + (int64_t)(2 * by) * C);
   const uint4 *e1 = reinterpret_cast<const uint4 *>(E + (int64_t)(2 * by + 1) * C);
+  pdl_wait();
+  pdl_trigger();
   float v[2 * kFewTok];  // v[t]: coordinate 2i of token t; v[16 + t]: coordinate 2i+1
 #pragma unroll
   for (int i = 0; i < 2 * kFewTok; ++i) v[i] = 0.f;
@@ -178,8 +180,8 @@ cudaError_t launch_encode_pack_simt(const uint16_t *x, int64_t n_tok, int64_t ld
                                     const uint16_t *E, int G, const Thresholds &th, uint8_t *codes,
                                     int64_t ldc, cudaStream_t s) {
   if (n_tok <= kFewTok) {
-    encode_pack_few<<<(unsigned)(G / 2), kFewWarps * 32, 0, s>>>(x, (int)n_tok, ldx, C, E, G, th, codes, ldc);
-    return cudaGetLastError();
+    return launch_pdl(encode_pack_few, dim3((unsigned)(G / 2)), dim3(kFewWarps * 32), 0, s, x, (int)n_tok, ldx, C, E,
+                      G, th, codes, ldc);
   }
   if (n_tok <= 64) {
     const int64_t warps = n_tok * (G / 2);

@@ -177,6 +177,15 @@ __device__ __forceinline__ void tmem_st_16x256b(uint32_t taddr, uint32_t r0, uin
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // 8x8 transpose of 16-bit elements held one pair per thread (mma fragment layout).
+// Four 8x8 matrices of 16-bit elements loaded transposed: threads 8m..8m+7
+// give the addresses of the eight 16-byte rows of matrix m; register m of
+// every thread receives its fragment of the transpose of matrix m.
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr)
+               : "memory");
+}
 __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t a) {
   uint32_t d;
   asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(a));
