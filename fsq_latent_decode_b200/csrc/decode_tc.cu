@@ -77,14 +77,16 @@ struct Cfg {
   static constexpr int STAGE_BYTES = TMA ? TILE_BYTES : (TILE_BYTES + 16 + 127) / 128 * 128;
   static constexpr int Q_BYTES = NS * KPAD;          // int8 Q' terms in the K-major no-swizzle layout
   static constexpr int P_BYTES = kTile * NQ * 2;     // P in the MN-major no-swizzle layout
-  // TMEM columns: Z (score A) x2 | Z^T 64-token chunks (pool A) x4 | S | ACC
+  // TMEM columns: Z (score A) x2 | Z^T 64-token chunks (pool A) x NCP | S x2 | ACC
   static constexpr int CS_COLS = (SCOLS + 15) / 16 * 16;
   static constexpr int CP_CHUNK = NH * 32;           // one 64-token chunk of Z^T
   static constexpr int OFF_CS = 0;
-  static constexpr int OFF_CP = 2 * CS_COLS;
-  static constexpr int OFF_S = OFF_CP + 4 * CP_CHUNK;
-  static constexpr int OFF_ACC = OFF_S + NS;
   static constexpr int ACC_COLS = 2 * NQ;            // NH=2: one per half; NH=1: one per chunk
+  // Z^T chunk ring: four chunks (two tiles) when TMEM allows, else three
+  static constexpr int NCP = (2 * CS_COLS + 4 * CP_CHUNK + 2 * NS + ACC_COLS) <= 512 ? 4 : 3;
+  static constexpr int OFF_CP = 2 * CS_COLS;
+  static constexpr int OFF_S = OFF_CP + NCP * CP_CHUNK;  // two S buffers
+  static constexpr int OFF_ACC = OFF_S + 2 * NS;
   static constexpr int TMEM_USED = OFF_ACC + ACC_COLS;
   static constexpr int TMEM_COLS = TMEM_USED <= 256 ? 256 : 512;
   static_assert(TMEM_USED <= 512, "TMEM plan exceeds 512 columns");
@@ -115,19 +117,18 @@ struct Misc {
   uint64_t full[kStages], empty[kStages];
   uint64_t cs_ready[2], cs_free[2];
   uint64_t cp_ready[4], cp_free[4];
-  uint64_t s_full, s_free;
+  uint64_t s_full[2], s_free[2];
   uint64_t p_full[2], p_free[2];
   uint64_t acc_full, q_full, done[5];
   uint32_t tmem_base;
   uint32_t abort;
-  uint32_t vote[2][2][4];
   float red[4][64];
   float fac[8][64];
   float m[64];
   float lt[64];
-  float cm[8][64];   // per softmax warp: score offset + running max, per head
+  __align__(16) float cm[8][64];  // per softmax warp: score offset + running max, per head
   float corr[64];
-  float sig[64];
+  __align__(16) float sig[64];
 };
 
 // Score operand bytes from one packed word: even coordinates, then odd ones.
@@ -228,6 +229,20 @@ __device__ __forceinline__ bool wait_bar(uint64_t *b, uint32_t parity, volatile 
   }
 }
 
+// Named barrier over `nthreads` threads that returns the OR of `pred` over them.
+__device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0u;
+}
+
 // Error path: wait (time-bounded, ignoring the abort flag) for an async copy
 // already issued into this CTA's shared memory, so none lands after exit.
 __device__ __forceinline__ void drain_bar(uint64_t *b, uint32_t parity, uint64_t limit_ns) {
@@ -305,8 +320,10 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
       mbar_init(&ms.cp_ready[i], 4);
       mbar_init(&ms.cp_free[i], C::NH == 2 ? 2 : 1);
     }
-    mbar_init(&ms.s_full, 1);
-    mbar_init(&ms.s_free, 8);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&ms.s_full[i], 1);
+      mbar_init(&ms.s_free[i], 8);
+    }
     mbar_init(&ms.acc_full, kPoolIssuers);
     mbar_init(&ms.q_full, 1);
     for (int i = 0; i < 5; ++i) mbar_init(&ms.done[i], 1);
@@ -394,15 +411,15 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
       for (int i = 0; i < n_tiles && ok; ++i) {
         const int sb = i & 1;
         ok = wait_bar(&ms.cs_ready[sb], (uint32_t)(i >> 1) & 1u, abort, p.wait_ns) &&
-             wait_bar(&ms.s_free, ((uint32_t)i & 1u) ^ 1u, abort, p.wait_ns);
+             wait_bar(&ms.s_free[sb], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort, p.wait_ns);
         if (!ok) break;
         tc_fence_after();
         const uint32_t a0 = tm + C::OFF_CS + sb * C::CS_COLS;
-        const uint32_t d = tm + C::OFF_S;
+        const uint32_t d = tm + C::OFF_S + sb * C::NS;
 #pragma unroll
         for (int k = 0; k < C::KPAD / 32; ++k)
           mma_ts_i8(d, a0 + k * 8, qd0 + (uint64_t)((k * 2 * C::LBO_Q) >> 4), id_s, k > 0 ? 1u : 0u);
-        tc_commit(&ms.s_full);
+        tc_commit(&ms.s_full[sb]);
         tc_commit(&ms.cs_free[sb]);
       }
       if (!ok) fail();
@@ -423,8 +440,9 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           if (C::NH == 1 && c != k_iss) continue;
-          const int cb = 2 * pb + c;  // chunk buffer
-          if (!wait_bar(&ms.cp_ready[cb], (uint32_t)(i >> 1) & 1u, abort, p.wait_ns)) { ok = false; break; }
+          const int kc = 2 * i + c;  // chunk index; ring buffer kc % NCP, use kc / NCP
+          const int cb = kc % C::NCP;
+          if (!wait_bar(&ms.cp_ready[cb], (uint32_t)(kc / C::NCP) & 1u, abort, p.wait_ns)) { ok = false; break; }
           tc_fence_after();
           const int h = C::NH == 2 ? k_iss : 0;
           const uint32_t d = tm + C::OFF_ACC + k_iss * NQ;
@@ -504,17 +522,18 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
     if (!ok && lane == 0) fail();
   } else if (warp >= 12 && warp < 20) {
     // ------------------------------------------------------------ pooling dequant: coordinates -> TMEM lanes
-    // group c = 0 / 1 builds 64-token chunk c of every tile into chunk buffer 2 (i % 2) + c
+    // group c = 0 / 1 builds 64-token chunk c of every tile (chunk index 2i + c) into ring buffer (2i + c) % NCP
     const int q = warp & 3;
     const int c = (warp - 12) >> 2;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     bool ok = true;
     for (int i = 0; i < n_tiles && ok; ++i) {
       const int st = i % kStages;
-      const int cb = 2 * (i & 1) + c;
+      const int kc = 2 * i + c;
+      const int cb = kc % C::NCP;
       const uint8_t *tile = smem + C::SM_CODES + st * C::STAGE_BYTES;
       if (!wait_bar(&ms.full[st], (uint32_t)(i / kStages) & 1u, abort, p.wait_ns) ||
-          !wait_bar(&ms.cp_free[cb], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort, p.wait_ns)) {
+          !wait_bar(&ms.cp_free[cb], ((uint32_t)(kc / C::NCP) & 1u) ^ 1u, abort, p.wait_ns)) {
         ok = false;
         break;
       }
@@ -592,31 +611,45 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
     bool ok = true;
     for (int i = 0; i < n_tiles && ok; ++i) {
       const uint32_t par = (uint32_t)(i >> 1) & 1u;
-      if (!wait_bar(&ms.s_full, (uint32_t)i & 1u, abort, p.wait_ns)) { ok = false; break; }
+      const int sb = i & 1;
+      if (!wait_bar(&ms.s_full[sb], par, abort, p.wait_ns)) { ok = false; break; }
       tc_fence_after();
-      const bool valid = (t0 + (int64_t)i * kTile + r) < t1;
       float x[HQ];  // score - m
-      bool need = (i == 0);
+      float xmax = -INFINITY;
       {
         uint32_t ra[HQ], rb[HQ];
-        tmem_ld_hq<HQ>(tm + lane_base + C::OFF_S + h0, ra);       // a terms
-        tmem_ld_hq<HQ>(tm + lane_base + C::OFF_S + NQ + h0, rb);  // b terms
+        const uint32_t sbase = tm + lane_base + C::OFF_S + sb * C::NS;
+        tmem_ld_hq<HQ>(sbase + h0, ra);       // a terms
+        tmem_ld_hq<HQ>(sbase + NQ + h0, rb);  // b terms
         tmem_ld_wait();
+        // S is in registers: the next score MMA may overwrite it
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ms.s_free[sb]);
+        const float4 *sg4 = reinterpret_cast<const float4 *>(ms.sig + h0);
+        const float4 *cm4 = reinterpret_cast<const float4 *>(cm);
 #pragma unroll
-        for (int n = 0; n < HQ; ++n) {
-          const int y = (int)ra[n] * 128 + (int)rb[n];  // exact: |y| < 2^27
-          x[n] = valid ? fmaf((float)y, ms.sig[h0 + n], -cm[n]) : -INFINITY;
-          need |= x[n] > kTau;
+        for (int n4 = 0; n4 < HQ / 4; ++n4) {
+          const float4 sg = sg4[n4], cc = cm4[n4];
+          const float sv[4] = {sg.x, sg.y, sg.z, sg.w}, cv[4] = {cc.x, cc.y, cc.z, cc.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int n = 4 * n4 + e;
+            const int y = (int)ra[n] * 128 + (int)rb[n];  // exact: |y| < 2^27
+            x[n] = fmaf((float)y, sv[e], -cv[e]);
+            xmax = fmaxf(xmax, x[n]);
+          }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ms.s_free);
-      const uint32_t wneed = __any_sync(0xffffffffu, need) ? 1u : 0u;
-      if (lane == 0) ms.vote[hh][i & 1][q] = wneed;
-      named_bar(barid, 128);
-      const uint32_t *vt = ms.vote[hh][i & 1];
-      const bool any = (vt[0] | vt[1] | vt[2] | vt[3]) != 0u;
+      // rows past the split's end (ragged last tile only) take no weight
+      if ((t0 + (int64_t)i * kTile + r) >= t1) {
+        xmax = -INFINITY;
+#pragma unroll
+        for (int n = 0; n < HQ; ++n) x[n] = -INFINITY;
+      }
+      const bool need = (i == 0) || xmax > kTau;
+      // one barrier over the group's four warps that also ORs their votes
+      const bool any = named_bar_or(barid, 128, need);
       if (any) {
         // raise the running max: m <- m + max(0, tile max of x) (the first tile: m <- its max)
 #pragma unroll
@@ -669,10 +702,10 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
         uint32_t h2[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const __half2 hv = __floats2half2_rn(ex2_approx(x[8 * g8 + 2 * k]), ex2_approx(x[8 * g8 + 2 * k + 1]));
-          const float2 back = __half22float2(hv);
-          lsum[8 * g8 + 2 * k] += back.x;
-          lsum[8 * g8 + 2 * k + 1] += back.y;
+          const float p0 = ex2_approx(x[8 * g8 + 2 * k]), p1 = ex2_approx(x[8 * g8 + 2 * k + 1]);
+          const __half2 hv = __floats2half2_rn(p0, p1);
+          lsum[8 * g8 + 2 * k] += p0;
+          lsum[8 * g8 + 2 * k + 1] += p1;
           h2[k] = *reinterpret_cast<const uint32_t *>(&hv);
         }
         *reinterpret_cast<uint4 *>(prow + g8 * C::SBO_P) = make_uint4(h2[0], h2[1], h2[2], h2[3]);
@@ -688,7 +721,8 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
       if (lane == 0) fail();
     } else {
       tc_fence_after();
-      // L~ = sum over the CTA's tokens of the fp16 weights actually pooled
+      // L = sum over the CTA's tokens of the softmax weights (fp32; the pooled
+      // copies are their fp16 roundings, relative difference <= 2^-11 each)
 #pragma unroll
       for (int n = 0; n < HQ; ++n) {
         float v = lsum[n];
