@@ -57,13 +57,18 @@ using namespace ptx;
 
 constexpr int kTile = 128;
 constexpr int kStages = 4;
-constexpr int kThreads = 24 * 32;
 constexpr float kTau = 8.f;                        // rescale when a score exceeds the running max by 2^8
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s per wait
+constexpr int kMiscBytes = 12288;                  // shared-memory reservation for the Misc block
 
 template <int G, int NQ>
 struct Cfg {
   static constexpr int HALF = G / 2;                 // bytes per token row
+  // softmax: NSG groups of four warps, each group owning HQ = 8 heads
+  static constexpr int NSG = NQ / 8;
+  static constexpr int HQ = NQ / NSG;
+  static constexpr int NSMX = 4 * NSG;               // softmax warps
+  static constexpr int THREADS = (16 + NSMX) * 32;
   static constexpr int KPAD = (G + 31) / 32 * 32;    // K of the score MMA (32 per kind::i8 step)
   static constexpr int KW = KPAD / 8;                // 32-bit code words (8 coordinates) per padded row
   static constexpr int SCOLS = KPAD / 4;             // TMEM columns of token-major Z (4 bytes per column)
@@ -95,7 +100,7 @@ struct Cfg {
   static constexpr int SM_Q = SM_CODES + kStages * STAGE_BYTES;
   static constexpr int SM_P = SM_Q + Q_BYTES;
   static constexpr int SM_MISC = SM_P + 2 * P_BYTES;
-  static constexpr int SM_TOTAL = SM_MISC + 8192;  // >= sizeof(Misc), checked below
+  static constexpr int SM_TOTAL = SM_MISC + kMiscBytes;
   static constexpr int LBO_Q = (NS / 8) * 128;       // 16-byte K-chunk stride of Q'
   static constexpr int SBO_P = (kTile / 8) * 128;    // N-group stride of P
 };
@@ -123,16 +128,16 @@ struct Misc {
   uint32_t tmem_base;
   uint32_t abort;
   float red[4][64];
-  float fac[8][64];
+  float fac[16][64];
   float m[64];
   float lt[64];
-  __align__(16) float cm[8][64];  // per softmax warp: score offset + running max, per head
+  __align__(16) float cm[16][64];  // per softmax warp: score offset + running max, per head
   float corr[64];
   __align__(16) float sig[64];
 };
 
 // Score operand bytes from one packed word: even coordinates, then odd ones.
-static_assert(sizeof(Misc) <= 8192, "Misc block exceeds its shared-memory reservation");
+static_assert(sizeof(Misc) <= kMiscBytes, "Misc block exceeds its shared-memory reservation");
 
 __device__ __forceinline__ uint32_t nib_even(uint32_t w) { return w & 0x0F0F0F0Fu; }
 __device__ __forceinline__ uint32_t nib_odd(uint32_t w) { return (w >> 4) & 0x0F0F0F0Fu; }
@@ -150,6 +155,36 @@ __device__ __forceinline__ void mma_ts_i8(uint32_t d_tmem, uint32_t a_tmem, uint
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// The same instructions issued by one elected lane of a converged warp, so
+// that the whole warp runs the issue loop on warp-uniform operands.
+__device__ __forceinline__ void mma_ts_i8_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts_f16_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred e, p;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void tc_commit_elect(uint64_t *bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
+      : "memory");
+}
+
 // Pooling operand values as fp16 subnormals, no bias: nibble J of both
 // half-words left in place in mantissa bits 0..3 (value n 2^-24) or bits 4..7
 // (value n 2^-20).  w holds, per half-word, the four nibbles of one token.
@@ -292,7 +327,7 @@ __device__ __forceinline__ void tmem_st_nq(uint32_t ta, const uint32_t *r) {
 }
 
 template <int G, int NQ>
-__global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_constant__ CUtensorMap tmap, Params p) {
+__global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(const __grid_constant__ CUtensorMap tmap, Params p) {
   using C = Cfg<G, NQ>;
   extern __shared__ __align__(1024) uint8_t smem[];
   Misc &ms = *reinterpret_cast<Misc *>(smem + C::SM_MISC);
@@ -313,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ms.cs_ready[i], 4);
       mbar_init(&ms.cs_free[i], 1);
-      mbar_init(&ms.p_full[i], 8);
+      mbar_init(&ms.p_full[i], C::NSMX);
       mbar_init(&ms.p_free[i], kPoolIssuers);
     }
     for (int i = 0; i < 4; ++i) {
@@ -322,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ms.s_full[i], 1);
-      mbar_init(&ms.s_free[i], 8);
+      mbar_init(&ms.s_free[i], C::NSMX);
     }
     mbar_init(&ms.acc_full, kPoolIssuers);
     mbar_init(&ms.q_full, 1);
@@ -403,66 +438,62 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
       drain_bar(&ms.q_full, 0, p.wait_ns / 4 + 1);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ score-MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t id_s = idesc_i8(128, C::NS);
-      const uint64_t qd0 = smem_desc(smem_u32(smem + C::SM_Q), C::LBO_Q, 128);
-      bool ok = wait_bar(&ms.q_full, 0, abort, p.wait_ns);
-      for (int i = 0; i < n_tiles && ok; ++i) {
-        const int sb = i & 1;
-        ok = wait_bar(&ms.cs_ready[sb], (uint32_t)(i >> 1) & 1u, abort, p.wait_ns) &&
-             wait_bar(&ms.s_free[sb], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort, p.wait_ns);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t a0 = tm + C::OFF_CS + sb * C::CS_COLS;
-        const uint32_t d = tm + C::OFF_S + sb * C::NS;
+    // ------------------------------------------------------------ score-MMA issuer (whole warp, one lane issues)
+    constexpr uint32_t id_s = idesc_i8(128, C::NS);
+    const uint64_t qd0 = smem_desc(smem_u32(smem + C::SM_Q), C::LBO_Q, 128);
+    bool ok = wait_bar(&ms.q_full, 0, abort, p.wait_ns);
+    for (int i = 0; i < n_tiles && ok; ++i) {
+      const int sb = i & 1;
+      ok = wait_bar(&ms.cs_ready[sb], (uint32_t)(i >> 1) & 1u, abort, p.wait_ns) &&
+           wait_bar(&ms.s_free[sb], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort, p.wait_ns);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t a0 = tm + C::OFF_CS + sb * C::CS_COLS;
+      const uint32_t d = tm + C::OFF_S + sb * C::NS;
 #pragma unroll
-        for (int k = 0; k < C::KPAD / 32; ++k)
-          mma_ts_i8(d, a0 + k * 8, qd0 + (uint64_t)((k * 2 * C::LBO_Q) >> 4), id_s, k > 0 ? 1u : 0u);
-        tc_commit(&ms.s_full[sb]);
-        tc_commit(&ms.cs_free[sb]);
-      }
-      if (!ok) fail();
-      tc_commit(&ms.done[0]);
-      wait_bar(&ms.done[0], 0, abort, p.wait_ns);
+      for (int k = 0; k < C::KPAD / 32; ++k)
+        mma_ts_i8_elect(d, a0 + k * 8, qd0 + (uint64_t)((k * 2 * C::LBO_Q) >> 4), id_s, k > 0 ? 1u : 0u);
+      tc_commit_elect(&ms.s_full[sb]);
+      tc_commit_elect(&ms.cs_free[sb]);
     }
+    if (!ok && lane == 0) fail();
+    tc_commit_elect(&ms.done[0]);
+    wait_bar(&ms.done[0], 0, abort, p.wait_ns);
   } else if (warp == 2 || warp == 3) {
-    // ------------------------------------------------------------ pooling-MMA issuers
-    if (lane == 0) {
-      const int k_iss = warp - 2;  // NH=2: half k_iss, both chunks; NH=1: chunk k_iss
-      constexpr uint32_t id_p = idesc_f16(128, NQ, 0, 1);
-      const uint64_t pd0 = smem_desc(smem_u32(smem + C::SM_P), 128, C::SBO_P);
-      bool ok = true;
-      for (int i = 0; i < n_tiles && ok; ++i) {
-        const int pb = i & 1;
-        ok = wait_bar(&ms.p_full[pb], (uint32_t)(i >> 1) & 1u, abort, p.wait_ns);
-        if (!ok) break;
+    // ------------------------------------------------------------ pooling-MMA issuers (whole warp, one lane issues)
+    const int k_iss = warp - 2;  // NH=2: half k_iss, both chunks; NH=1: chunk k_iss
+    constexpr uint32_t id_p = idesc_f16(128, NQ, 0, 1);
+    const uint64_t pd0 = smem_desc(smem_u32(smem + C::SM_P), 128, C::SBO_P);
+    const int h = C::NH == 2 ? k_iss : 0;
+    const uint32_t d = tm + C::OFF_ACC + k_iss * NQ;
+    bool ok = true;
+    for (int i = 0; i < n_tiles && ok; ++i) {
+      const int pb = i & 1;
+      ok = wait_bar(&ms.p_full[pb], (uint32_t)(i >> 1) & 1u, abort, p.wait_ns);
+      if (!ok) break;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          if (C::NH == 1 && c != k_iss) continue;
-          const int kc = 2 * i + c;  // chunk index; ring buffer kc % NCP, use kc / NCP
-          const int cb = kc % C::NCP;
-          if (!wait_bar(&ms.cp_ready[cb], (uint32_t)(kc / C::NCP) & 1u, abort, p.wait_ns)) { ok = false; break; }
-          tc_fence_after();
-          const int h = C::NH == 2 ? k_iss : 0;
-          const uint32_t d = tm + C::OFF_ACC + k_iss * NQ;
-          const uint32_t a0 = tm + C::OFF_CP + cb * C::CP_CHUNK + h * 32;
+      for (int c = 0; c < 2; ++c) {
+        if (C::NH == 1 && c != k_iss) continue;
+        const int kc = 2 * i + c;  // chunk index; ring buffer kc % NCP, use kc / NCP
+        const int cb = kc % C::NCP;
+        if (!wait_bar(&ms.cp_ready[cb], (uint32_t)(kc / C::NCP) & 1u, abort, p.wait_ns)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a0 = tm + C::OFF_CP + cb * C::CP_CHUNK + h * 32;
+        const uint64_t bd0 = pd0 + (uint64_t)((pb * C::P_BYTES + 4 * c * 256) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t bd = pd0 + (uint64_t)((pb * C::P_BYTES + (4 * c + kk) * 256) >> 4);
-            const bool first = (i == 0) && (C::NH == 1 ? kk == 0 : (c == 0 && kk == 0));
-            mma_ts(d, a0 + kk * 8, bd, id_p, first ? 0u : 1u);
-          }
-          tc_commit(&ms.cp_free[cb]);
+        for (int kk = 0; kk < 4; ++kk) {
+          const bool first = (i == 0) && (C::NH == 1 ? kk == 0 : (c == 0 && kk == 0));
+          mma_ts_f16_elect(d, a0 + kk * 8, bd0 + (uint64_t)(kk * 16), id_p, first ? 0u : 1u);
         }
-        if (!ok) break;
-        tc_commit(&ms.p_free[pb]);
+        tc_commit_elect(&ms.cp_free[cb]);
       }
-      if (ok) tc_commit(&ms.acc_full);
-      else fail();
-      tc_commit(&ms.done[2 + k_iss]);
-      wait_bar(&ms.done[2 + k_iss], 0, abort, p.wait_ns);
+      if (!ok) break;
+      tc_commit_elect(&ms.p_free[pb]);
     }
+    if (ok) tc_commit_elect(&ms.acc_full);
+    else if (lane == 0) fail();
+    tc_commit_elect(&ms.done[2 + k_iss]);
+    wait_bar(&ms.done[2 + k_iss], 0, abort, p.wait_ns);
   } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ score dequant: token row -> TMEM lane
     const int q = warp - 4;
@@ -584,12 +615,13 @@ __global__ void __launch_bounds__(kThreads, 1) absorbed_split_tc(const __grid_co
     if (!ok && lane == 0) fail();
   } else if ((warp >= 8 && warp < 12) || warp >= 20) {
     // ------------------------------------------------------------ softmax
-    // two groups of four warps (8-11, 20-23); each group owns half the heads
-    constexpr int HQ = NQ / 2;
+    // NSG groups of four warps (8-11, then 20-23, 24-27, ...); group hh owns
+    // heads hh*HQ .. hh*HQ+HQ-1, warp q of a group TMEM lanes 32q .. 32q+31
+    constexpr int HQ = C::HQ;
     const int q = warp & 3;
-    const int hh = warp >= 20 ? 1 : 0;  // head half
+    const int hh = warp < 12 ? 0 : 1 + ((warp - 20) >> 2);  // head group
     const int h0 = hh * HQ;             // first head of this warp
-    const int sw = 4 * hh + q;          // softmax warp index 0..7
+    const int sw = 4 * hh + q;          // softmax warp index
     const int gtid = 32 * q + lane;     // thread index within the group
     const int barid = 1 + hh;
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
@@ -972,7 +1004,7 @@ cudaError_t launch(const uint16_t *q, const uint8_t *codes, int64_t bstride, int
     if (e != cudaSuccess) return e;
   }
   record_prof_event(prof[0], st);
-  e = launch_pdl(absorbed_split_tc<G, NQ>, dim3(S, (unsigned)B), dim3(kThreads), (size_t)smem, st, tmap, p);
+  e = launch_pdl(absorbed_split_tc<G, NQ>, dim3(S, (unsigned)B), dim3(C::THREADS), (size_t)smem, st, tmap, p);
   record_prof_event(prof[1], st);
   return e;
 }
