@@ -60,6 +60,7 @@ constexpr int kStages = 4;
 constexpr float kTau = 8.f;                        // rescale when a score exceeds the running max by 2^8
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s per wait
 constexpr int kMiscBytes = 12288;                  // shared-memory reservation for the Misc block
+constexpr int kPBufs = 4;                          // ring of softmax-weight (P) tiles in shared memory
 
 template <int G, int NQ>
 struct Cfg {
@@ -99,7 +100,7 @@ struct Cfg {
   static constexpr int SM_CODES = 0;
   static constexpr int SM_Q = SM_CODES + kStages * STAGE_BYTES;
   static constexpr int SM_P = SM_Q + Q_BYTES;
-  static constexpr int SM_MISC = SM_P + 2 * P_BYTES;
+  static constexpr int SM_MISC = SM_P + kPBufs * P_BYTES;
   static constexpr int SM_TOTAL = SM_MISC + kMiscBytes;
   static constexpr int LBO_Q = (NS / 8) * 128;       // 16-byte K-chunk stride of Q'
   static constexpr int SBO_P = (kTile / 8) * 128;    // N-group stride of P
@@ -123,7 +124,7 @@ struct Misc {
   uint64_t cs_ready[2], cs_free[2];
   uint64_t cp_ready[4], cp_free[4];
   uint64_t s_full[2], s_free[2];
-  uint64_t p_full[2], p_free[2];
+  uint64_t p_full[kPBufs], p_free[kPBufs];
   uint64_t acc_full, q_full, done[5];
   uint32_t tmem_base;
   uint32_t abort;
@@ -348,6 +349,8 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
     for (int i = 0; i < 2; ++i) {
       mbar_init(&ms.cs_ready[i], 4);
       mbar_init(&ms.cs_free[i], 1);
+    }
+    for (int i = 0; i < kPBufs; ++i) {
       mbar_init(&ms.p_full[i], C::NSMX);
       mbar_init(&ms.p_free[i], kPoolIssuers);
     }
@@ -444,8 +447,11 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
     bool ok = wait_bar(&ms.q_full, 0, abort, p.wait_ns);
     for (int i = 0; i < n_tiles && ok; ++i) {
       const int sb = i & 1;
+      // S(i) is released to the softmax only once P buffer i % kPBufs is free
+      // again (pooling of tile i - kPBufs done), so the softmax never waits for it
       ok = wait_bar(&ms.cs_ready[sb], (uint32_t)(i >> 1) & 1u, abort, p.wait_ns) &&
-           wait_bar(&ms.s_free[sb], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort, p.wait_ns);
+           wait_bar(&ms.s_free[sb], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort, p.wait_ns) &&
+           wait_bar(&ms.p_free[i % kPBufs], ((uint32_t)(i / kPBufs) & 1u) ^ 1u, abort, p.wait_ns);
       if (!ok) break;
       tc_fence_after();
       const uint32_t a0 = tm + C::OFF_CS + sb * C::CS_COLS;
@@ -468,8 +474,8 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
     const uint32_t d = tm + C::OFF_ACC + k_iss * NQ;
     bool ok = true;
     for (int i = 0; i < n_tiles && ok; ++i) {
-      const int pb = i & 1;
-      ok = wait_bar(&ms.p_full[pb], (uint32_t)(i >> 1) & 1u, abort, p.wait_ns);
+      const int pb = i % kPBufs;
+      ok = wait_bar(&ms.p_full[pb], (uint32_t)(i / kPBufs) & 1u, abort, p.wait_ns);
       if (!ok) break;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
@@ -709,8 +715,8 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
         __syncwarp();
         if (i > 0) {
           // ACC must hold every earlier tile before it is rescaled
-          const int pj = (i - 1) & 1;
-          if (!wait_bar(&ms.p_free[pj], (uint32_t)((i - 1) >> 1) & 1u, abort, p.wait_ns)) { ok = false; break; }
+          const int pj = (i - 1) % kPBufs;
+          if (!wait_bar(&ms.p_free[pj], (uint32_t)((i - 1) / kPBufs) & 1u, abort, p.wait_ns)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll 1
           for (int blk = 0; blk < 2; ++blk) {  // both ACC blocks, this warp's head columns
@@ -726,8 +732,7 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
         }
       }
       // P row of this token (fp16) for this warp's heads, MN-major: HQ/8 chunks of 8 heads
-      const int pb = i & 1;
-      if (!wait_bar(&ms.p_free[pb], par ^ 1u, abort, p.wait_ns)) { ok = false; break; }
+      const int pb = i % kPBufs;  // free: the score MMA of tile i waited for it
       uint8_t *prow = smem + C::SM_P + pb * C::P_BYTES + (kap >> 3) * 128 + (kap & 7) * 16 + (h0 / 8) * C::SBO_P;
 #pragma unroll
       for (int g8 = 0; g8 < HQ / 8; ++g8) {
