@@ -14,8 +14,8 @@ cudaError_t launch_quantize_pack_f32(const float *u, int64_t n_tok, int G, const
                                      int64_t ldc, cudaStream_t s);
 cudaError_t launch_absorbed_simt(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
                                  int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv, float scale, int S,
-                                 int64_t tps, float *qa, float *part, uint32_t *err, void *o, int out_fp32,
-                                 void *const *prof, cudaStream_t st);
+                                 int64_t tps, float *qa, float *part, uint32_t *err, MergeScratch ms, void *o,
+                                 int out_fp32, void *const *prof, cudaStream_t st);
 cudaError_t launch_expand_simt(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
                                int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv, float scale, int S,
                                int64_t tps, int rope_knorm, float rope_base, const uint16_t *gain, float eps,
@@ -27,8 +27,8 @@ bool absorbed_tc_supported(int n_q, int n_kv, int G);
 size_t absorbed_tc_qphys_bytes(int n_q, int G);
 cudaError_t launch_absorbed_tc(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
                                int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv, float scale, int S,
-                               int64_t tps, uint8_t *qphys, float *corr, float *part, uint32_t *err, void *o,
-                               int out_fp32, void *const *prof, cudaStream_t st);
+                               int64_t tps, uint8_t *qphys, float *corr, float *part, uint32_t *err,
+                               MergeScratch ms, void *o, int out_fp32, void *const *prof, cudaStream_t st);
 
 namespace {
 
@@ -67,7 +67,8 @@ struct Plan {
   bool tc;        // tensor-core kernel (absorbed form)
   int S;          // splits per batch row
   int64_t tps;    // tokens per split
-  size_t off_qa, off_corr, off_part, total;
+  MergePlan mp;   // split merge of the absorbed form
+  size_t off_qa, off_corr, off_part, off_mslab, off_mcnt, total;
 };
 
 fsq_status plan_decode(int64_t B, int64_t T, int n_q, int n_kv, int d_h, int G, const fsq_attn_opts &op, Plan *p) {
@@ -120,6 +121,11 @@ fsq_status plan_decode(int64_t B, int64_t T, int n_q, int n_kv, int d_h, int G, 
   if (tc) off = align_up(off + 2 * sizeof(float) * (size_t)Bc * n_q, 256);
   p->off_part = off;
   off = align_up(off + sizeof(float) * (size_t)Bc * S * n_q * (2 + acc_len), 256);
+  if (variant == FSQ_VARIANT_ABSORBED) p->mp = merge_plan((int)S, Bc, n_q, n_kv, G);
+  p->off_mslab = off;
+  off = align_up(off + p->mp.slab_bytes, 256);
+  p->off_mcnt = off;
+  off = align_up(off + p->mp.cnt_bytes, 256);
   p->total = off;
   return FSQ_OK;
 }
@@ -217,14 +223,16 @@ fsq_status fsq_decode_attn(const uint16_t *q, int64_t B, int n_q, int d_h, const
   uint32_t *err = (uint32_t *)ws;
   float *part = (float *)(ws + p.off_part);
   cudaStream_t s = (cudaStream_t)stream;
+  MergeScratch ms{nullptr, nullptr, 0};
+  if (p.mp.cnt_bytes) ms = {(float *)(ws + p.off_mslab), (uint32_t *)(ws + p.off_mcnt), (int)(B * n_kv)};
   cudaError_t e;
   if (p.tc) {
     e = launch_absorbed_tc(q, codes, code_batch_stride_bytes, B, T, n_q, n_kv, d_h, G, W_kv, scale, p.S, p.tps,
-                           (uint8_t *)(ws + p.off_qa), (float *)(ws + p.off_corr), part, err, o, op.out_fp32,
+                           (uint8_t *)(ws + p.off_qa), (float *)(ws + p.off_corr), part, err, ms, o, op.out_fp32,
                            op.prof_events, s);
   } else if (p.variant == FSQ_VARIANT_ABSORBED) {
     e = launch_absorbed_simt(q, codes, code_batch_stride_bytes, B, T, n_q, n_kv, d_h, G, W_kv, scale, p.S, p.tps,
-                             (float *)(ws + p.off_qa), part, err, o, op.out_fp32, op.prof_events, s);
+                             (float *)(ws + p.off_qa), part, err, ms, o, op.out_fp32, op.prof_events, s);
   } else {
     e = launch_expand_simt(q, codes, code_batch_stride_bytes, B, T, n_q, n_kv, d_h, G, W_kv, scale, p.S, p.tps,
                            op.rope_knorm, op.rope_base, op.knorm_gain, op.knorm_eps, part, err, o, op.out_fp32,

@@ -41,6 +41,23 @@ __device__ __forceinline__ uint32_t fsq_nibble(float u, const Thresholds &t) {
   return n;
 }
 
+// Split-merge plan of the absorbed form (merge.cu): CTAs per (kv head, batch
+// row) as G slices x split chunks, and the workspace its sliced mode needs.
+struct MergePlan {
+  int ngq = 1, nsq = 1;
+  size_t slab_bytes = 0, cnt_bytes = 0;
+};
+MergePlan merge_plan(int S, int64_t B, int n_q, int n_kv, int G);
+
+// Workspace of the sliced merge: per-chunk shares of the pooled latents and
+// one arrival count per (batch row, kv head), which the query prologue of the
+// same call zeroes (ncnt counts; slab and cnt are null in direct mode).
+struct MergeScratch {
+  float *slab;
+  uint32_t *cnt;
+  int ncnt;
+};
+
 // Workspace header: the device error word lives in the first 4 bytes.
 constexpr size_t kWsHeader = 256;
 
@@ -71,9 +88,12 @@ inline cudaError_t ensure_smem_limit(const void *fn, size_t bytes) {
 // while the previous kernel of the stream is still running, once every CTA of
 // that kernel has called pdl_trigger (or exited).  A kernel reads nothing that
 // the previous kernels write before pdl_wait, which returns when they have
-// completed and their writes are visible.  Each of these kernels calls
-// pdl_trigger only after its own pdl_wait, so a kernel that starts early
-// still sees every kernel before its predecessor complete.
+// completed and their writes are visible.  Every kernel here completes only
+// after its own pdl_wait, so waiting for the immediate predecessor also covers
+// all kernels before it.  The query prologue triggers only after its wait, so
+// the split kernel, which requests code tiles before its own wait, starts
+// after the codes are complete; the merge never triggers early, so work after
+// a decode call starts once its output is written.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 

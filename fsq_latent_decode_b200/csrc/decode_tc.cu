@@ -838,7 +838,7 @@ struct AbsorbShape {
 template <int G, int NQ, int GRP>
 __global__ void __launch_bounds__(Cfg<G, NQ>::KPAD * AbsorbShape<GRP>::NDQ)
     absorb_query_tc(const uint16_t *__restrict__ q, const uint16_t *__restrict__ W_kv, float c,
-                    uint8_t *__restrict__ qphys, float *__restrict__ corr, uint32_t *err) {
+                    uint8_t *__restrict__ qphys, float *__restrict__ corr, uint32_t *err, MergeScratch ms) {
   // one CTA per (kv head j, batch row b): the group's heads share W_k^(j), read once
   using C = Cfg<G, NQ>;
   constexpr int D = FSQ_HEAD_DIM;
@@ -855,9 +855,17 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::KPAD * AbsorbShape<GRP>::NDQ)
   const int j = blockIdx.x, b = blockIdx.y;
   const int g = threadIdx.x % GS, dq = threadIdx.x / GS;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  pdl_wait();
-  if (j == 0 && b == 0 && threadIdx.x == 0) *err = 0u;
-  pdl_trigger();  // the split kernel may start its prologue and code loads
+  // Nothing here depends on the kernel before this one (q and W_kv are inputs
+  // of the call; no kernel of this library that may still run writes them,
+  // and the workspace is no longer read by the previous call's kernels, which
+  // have completed), so the whole prologue overlaps with it - with the append
+  // of the step's new tokens in a decode step.  It waits for that kernel only
+  // at the end, before releasing the split kernel, whose first code loads
+  // precede its own wait.
+  if (j == 0 && b == 0) {
+    if (threadIdx.x == 0) *err = 0u;
+    for (int i = threadIdx.x; i < ms.ncnt; i += blockDim.x) ms.cnt[i] = 0u;  // the merge's arrival counts
+  }
   for (int i = threadIdx.x; i < GRP * D; i += blockDim.x)
     qs[i / D][i % D] = bf16_to_f32(q[((int64_t)b * NQ + j * GRP) * D + i]);
   __syncthreads();
@@ -937,25 +945,27 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::KPAD * AbsorbShape<GRP>::NDQ)
     corr[(size_t)b * 2 * NQ + h] = sig_s[threadIdx.x];
     corr[(size_t)b * 2 * NQ + NQ + h] = (float)((double)sig_s[threadIdx.x] * 8.0 * (double)tot);
   }
+  pdl_wait();
+  pdl_trigger();  // the split kernel may start its prologue and code loads
 }
 
 template <int G, int NQ, int GRP>
 cudaError_t absorb_query_launch(const dim3 &grid, const uint16_t *q, const uint16_t *W_kv, float c, uint8_t *qphys,
-                                float *corr, uint32_t *err, cudaStream_t st) {
+                                float *corr, uint32_t *err, MergeScratch ms, cudaStream_t st) {
   return launch_pdl(absorb_query_tc<G, NQ, GRP>, grid, dim3(Cfg<G, NQ>::KPAD * AbsorbShape<GRP>::NDQ), 0, st, q, W_kv,
-                    c, qphys, corr, err);
+                    c, qphys, corr, err, ms);
 }
 
 template <int G, int NQ>
 cudaError_t launch_absorb_query(const uint16_t *q, int64_t B, int n_kv, const uint16_t *W_kv, float c,
-                                uint8_t *qphys, float *corr, uint32_t *err, cudaStream_t st) {
+                                uint8_t *qphys, float *corr, uint32_t *err, MergeScratch ms, cudaStream_t st) {
   const dim3 grid(n_kv, (unsigned)B);
   switch (NQ / n_kv) {
-    case 1: return absorb_query_launch<G, NQ, 1>(grid, q, W_kv, c, qphys, corr, err, st);
-    case 2: return absorb_query_launch<G, NQ, 2>(grid, q, W_kv, c, qphys, corr, err, st);
-    case 4: return absorb_query_launch<G, NQ, 4>(grid, q, W_kv, c, qphys, corr, err, st);
-    case 8: return absorb_query_launch<G, NQ, 8>(grid, q, W_kv, c, qphys, corr, err, st);
-    case 16: return absorb_query_launch<G, NQ, 16>(grid, q, W_kv, c, qphys, corr, err, st);
+    case 1: return absorb_query_launch<G, NQ, 1>(grid, q, W_kv, c, qphys, corr, err, ms, st);
+    case 2: return absorb_query_launch<G, NQ, 2>(grid, q, W_kv, c, qphys, corr, err, ms, st);
+    case 4: return absorb_query_launch<G, NQ, 4>(grid, q, W_kv, c, qphys, corr, err, ms, st);
+    case 8: return absorb_query_launch<G, NQ, 8>(grid, q, W_kv, c, qphys, corr, err, ms, st);
+    case 16: return absorb_query_launch<G, NQ, 16>(grid, q, W_kv, c, qphys, corr, err, ms, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -993,9 +1003,9 @@ cudaError_t make_code_tensor_map(CUtensorMap *map, const uint8_t *codes, int64_t
 template <int G, int NQ>
 cudaError_t launch(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T, int n_kv,
                    const uint16_t *W_kv, float scale, int S, int64_t tps, uint8_t *qphys, float *corr, float *part,
-                   uint32_t *err, void *const *prof, cudaStream_t st) {
+                   uint32_t *err, MergeScratch ms, void *const *prof, cudaStream_t st) {
   using C = Cfg<G, NQ>;
-  cudaError_t e = launch_absorb_query<G, NQ>(q, B, n_kv, W_kv, scale * kLog2e, qphys, corr, err, st);
+  cudaError_t e = launch_absorb_query<G, NQ>(q, B, n_kv, W_kv, scale * kLog2e, qphys, corr, err, ms, st);
   if (e != cudaSuccess) return e;
   // one CTA per SM: ask for more shared memory than two CTAs could share
   const int smem = C::SM_TOTAL > 120 * 1024 ? C::SM_TOTAL : 120 * 1024;
@@ -1026,20 +1036,20 @@ size_t absorbed_tc_qphys_bytes(int n_q, int G) {
 }
 
 cudaError_t merge_absorbed_launch(const float *part, int S, int64_t B, int n_q, int n_kv, int d_h, int G,
-                                  const uint16_t *W_kv, void *o, int out_fp32, cudaStream_t st);
+                                  const uint16_t *W_kv, void *o, int out_fp32, MergeScratch ms, cudaStream_t st);
 
 cudaError_t launch_absorbed_tc(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
                                int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv, float scale, int S,
-                               int64_t tps, uint8_t *qphys, float *corr, float *part, uint32_t *err, void *o,
-                               int out_fp32, void *const *prof, cudaStream_t st) {
+                               int64_t tps, uint8_t *qphys, float *corr, float *part, uint32_t *err,
+                               MergeScratch ms, void *o, int out_fp32, void *const *prof, cudaStream_t st) {
   cudaError_t e;
-  if (G == 256 && n_q == 32) e = tc::launch<256, 32>(q, codes, bstride, B, T, n_kv, W_kv, scale, S, tps, qphys, corr, part, err, prof, st);
-  else if (G == 256 && n_q == 16) e = tc::launch<256, 16>(q, codes, bstride, B, T, n_kv, W_kv, scale, S, tps, qphys, corr, part, err, prof, st);
-  else if (G == 84 && n_q == 32) e = tc::launch<84, 32>(q, codes, bstride, B, T, n_kv, W_kv, scale, S, tps, qphys, corr, part, err, prof, st);
-  else if (G == 84 && n_q == 16) e = tc::launch<84, 16>(q, codes, bstride, B, T, n_kv, W_kv, scale, S, tps, qphys, corr, part, err, prof, st);
+  if (G == 256 && n_q == 32) e = tc::launch<256, 32>(q, codes, bstride, B, T, n_kv, W_kv, scale, S, tps, qphys, corr, part, err, ms, prof, st);
+  else if (G == 256 && n_q == 16) e = tc::launch<256, 16>(q, codes, bstride, B, T, n_kv, W_kv, scale, S, tps, qphys, corr, part, err, ms, prof, st);
+  else if (G == 84 && n_q == 32) e = tc::launch<84, 32>(q, codes, bstride, B, T, n_kv, W_kv, scale, S, tps, qphys, corr, part, err, ms, prof, st);
+  else if (G == 84 && n_q == 16) e = tc::launch<84, 16>(q, codes, bstride, B, T, n_kv, W_kv, scale, S, tps, qphys, corr, part, err, ms, prof, st);
   else return cudaErrorInvalidValue;
   if (e != cudaSuccess) return e;
-  return merge_absorbed_launch(part, S, B, n_q, n_kv, d_h, G, W_kv, o, out_fp32, st);
+  return merge_absorbed_launch(part, S, B, n_q, n_kv, d_h, G, W_kv, o, out_fp32, ms, st);
 }
 
 }  // namespace fsq

@@ -27,11 +27,14 @@ constexpr int kMaxGrp = 16;    // query heads per kv head supported here
 // qa[b][h][g] = c * sum_d W_k[j*d_h + d][g] * q[b][h][d],  c = scale*log2(e)
 __global__ void absorb_query_kernel(const uint16_t *__restrict__ q, const uint16_t *__restrict__ W_kv,
                                     int n_q, int n_kv, int d_h, int G, float c, float *__restrict__ qa,
-                                    uint32_t *err) {
+                                    uint32_t *err, MergeScratch ms) {
   __shared__ float qs[FSQ_HEAD_DIM];
   const int h = blockIdx.x, b = blockIdx.y;
   const int j = h / (n_q / n_kv);
-  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *err = 0u;
+  if (blockIdx.x == 0 && blockIdx.y == 0) {
+    if (threadIdx.x == 0) *err = 0u;
+    for (int i = threadIdx.x; i < ms.ncnt; i += blockDim.x) ms.cnt[i] = 0u;
+  }
   for (int d = threadIdx.x; d < d_h; d += blockDim.x) qs[d] = bf16_to_f32(q[((int64_t)b * n_q + h) * d_h + d]);
   __syncthreads();
   for (int g = threadIdx.x; g < G; g += blockDim.x) {
@@ -332,175 +335,19 @@ __global__ void merge_expand_kernel(const float *__restrict__ part, int S, int n
 
 __global__ void clear_err_kernel(uint32_t *err) { *err = 0u; }
 
-// Split merge + W_v for one GQA group, one CTA per (kv head j, batch row b).
-// The group's heads share W_v^(j): it is staged once in shared memory by
-// cp.async, issued first so the copy overlaps the partial reads, in rows of
-// WS = 8 x odd elements so that a warp's 16-byte reads of 32 consecutive rows
-// fall on distinct bank groups.  Then abar_h = sum_s w_s acc_s / l over the
-// splits, and one thread per output (d, heads) forms o_h[d] = W_v[d] . abar_h
-// with 16-byte shared reads (abar is a broadcast).
-__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
-  const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
-}
-__device__ __forceinline__ void cp_async4(void *smem, const void *gmem) {
-  const uint32_t s = (uint32_t)__cvta_generic_to_shared(smem);
-  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(s), "l"(gmem) : "memory");
-}
-
-struct MergeShape {
-  int GP;   // G rounded up to 8 (abar row, zero tail)
-  int WS;   // W_v row stride in shared memory: 8 x odd >= GP
-  size_t off_abar, off_w, bytes;
-};
-
-inline MergeShape merge_shape(int G, int d_h, int grp, int S) {
-  MergeShape m;
-  m.GP = (G + 7) / 8 * 8;
-  m.WS = m.GP % 16 ? m.GP : m.GP + 8;
-  m.off_abar = sizeof(uint16_t) * (size_t)d_h * m.WS;
-  m.off_w = m.off_abar + sizeof(float) * (size_t)grp * m.GP;
-  m.bytes = m.off_w + sizeof(float) * (size_t)grp * S;
-  return m;
-}
-
-template <int GRP>
-struct MergeThreads {
-  static constexpr int HT = GRP < 4 ? GRP : 4;   // head slices, one thread per (d, slice)
-  static constexpr int H = GRP / HT;             // heads per thread
-  static constexpr int NT = FSQ_HEAD_DIM * HT;
-};
-
-template <int GRP>
-__global__ void __launch_bounds__(MergeThreads<GRP>::NT)
-    merge_absorbed_group_kernel(const float *__restrict__ part, int S, int n_q, int n_kv, int G,
-                                const uint16_t *__restrict__ W_kv, void *o, int out_fp32, MergeShape ms) {
-  constexpr int D = FSQ_HEAD_DIM;
-  constexpr int H = MergeThreads<GRP>::H;
-  extern __shared__ __align__(16) unsigned char msm[];
-  uint16_t *wv = reinterpret_cast<uint16_t *>(msm);                     // [D][WS]
-  float *abar = reinterpret_cast<float *>(msm + ms.off_abar);           // [GRP][GP]
-  float *wts = reinterpret_cast<float *>(msm + ms.off_w);               // [GRP][S]
-  const int j = blockIdx.x, b = blockIdx.y;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int GP = ms.GP, WS = ms.WS;
-  {  // W_v^(j): D contiguous rows of G bf16 starting at row (n_kv + j) D
-    const uint16_t *src = W_kv + (int64_t)(n_kv + j) * D * G;
-    if (G % 8 == 0) {
-      const int cpr = G / 8;
-      for (int i = threadIdx.x; i < D * cpr; i += blockDim.x) {
-        const int r = i / cpr, c8 = i % cpr;
-        cp_async16(wv + r * WS + 8 * c8, src + (int64_t)r * G + 8 * c8);
-      }
-    } else {
-      const int cpr = G / 2;
-      for (int i = threadIdx.x; i < D * cpr; i += blockDim.x) {
-        const int r = i / cpr, c2 = i % cpr;
-        cp_async4(wv + r * WS + 2 * c2, src + (int64_t)r * G + 2 * c2);
-      }
-      for (int i = threadIdx.x; i < D * (GP - G); i += blockDim.x) wv[(i / (GP - G)) * WS + G + i % (GP - G)] = 0;
-    }
-    asm volatile("cp.async.commit_group;" ::: "memory");
-  }
-  pdl_wait();  // the partials come from the split kernel
-  pdl_trigger();
-  const int64_t sstride = (int64_t)n_q * (2 + G);
-  const float *pbase = part + ((int64_t)b * S * n_q + j * GRP) * (2 + G);
-  if (warp < GRP) {  // split weights for head `warp`, 1/l folded in
-    const float *pb = pbase + (int64_t)warp * (2 + G);
-    float m = -INFINITY;
-    for (int s = lane; s < S; s += 32) m = fmaxf(m, pb[s * sstride]);
-#pragma unroll
-    for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-    float l = 0.f;
-    for (int s = lane; s < S; s += 32) {
-      const float w = exp2f(pb[s * sstride] - m);
-      wts[warp * S + s] = w;
-      l = fmaf(w, pb[s * sstride + 1], l);
-    }
-#pragma unroll
-    for (int off = 16; off; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
-    const float inv = 1.f / l;
-    __syncwarp();
-    for (int s = lane; s < S; s += 32) wts[warp * S + s] *= inv;
-  }
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < GRP * GP; idx += blockDim.x) {
-    const int hh = idx / GP, g = idx % GP;
-    float a0 = 0.f, a1 = 0.f;
-    if (g < G) {
-      const float *pb = pbase + (int64_t)hh * (2 + G) + 2 + g;
-      const float *ws = wts + hh * S;
-      int s = 0;
-      for (; s + 8 <= S; s += 8) {  // eight independent loads in flight
-        float pv[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) pv[u] = pb[(s + u) * sstride];
-#pragma unroll
-        for (int u = 0; u < 8; u += 2) {
-          a0 = fmaf(ws[s + u], pv[u], a0);
-          a1 = fmaf(ws[s + u + 1], pv[u + 1], a1);
-        }
-      }
-      for (; s < S; ++s) a0 = fmaf(ws[s], pb[s * sstride], a0);
-    }
-    abar[idx] = a0 + a1;
-  }
-  asm volatile("cp.async.wait_all;" ::: "memory");
-  __syncthreads();
-  const int d = threadIdx.x % D, h0 = (threadIdx.x / D) * H;
-  const uint16_t *wr = wv + d * WS;
-  float acc[H];
-#pragma unroll
-  for (int i = 0; i < H; ++i) acc[i] = 0.f;
-#pragma unroll 2
-  for (int g0 = 0; g0 < GP; g0 += 8) {
-    const uint4 wq = *reinterpret_cast<const uint4 *>(wr + g0);
-    const uint32_t wp[4] = {wq.x, wq.y, wq.z, wq.w};
-    float wf[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      wf[2 * i] = __uint_as_float(wp[i] << 16);
-      wf[2 * i + 1] = __uint_as_float(wp[i] & 0xFFFF0000u);
-    }
-#pragma unroll
-    for (int i = 0; i < H; ++i) {
-      const float4 lo = *reinterpret_cast<const float4 *>(abar + (h0 + i) * GP + g0);
-      const float4 hi = *reinterpret_cast<const float4 *>(abar + (h0 + i) * GP + g0 + 4);
-      acc[i] = fmaf(wf[0], lo.x, fmaf(wf[1], lo.y, fmaf(wf[2], lo.z, fmaf(wf[3], lo.w, acc[i]))));
-      acc[i] = fmaf(wf[4], hi.x, fmaf(wf[5], hi.y, fmaf(wf[6], hi.z, fmaf(wf[7], hi.w, acc[i]))));
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < H; ++i) {
-    const int64_t oi = ((int64_t)b * n_q + j * GRP + h0 + i) * D + d;
-    if (out_fp32) reinterpret_cast<float *>(o)[oi] = acc[i];
-    else reinterpret_cast<uint16_t *>(o)[oi] = f32_to_bf16_rn(acc[i]);
-  }
-}
-
-template <int GRP>
-cudaError_t merge_group_launch(const float *part, int S, int64_t B, int n_q, int n_kv, int d_h, int G,
-                               const uint16_t *W_kv, void *o, int out_fp32, cudaStream_t st) {
-  const MergeShape ms = merge_shape(G, d_h, GRP, S);
-  cudaError_t e = ensure_smem_limit((const void *)merge_absorbed_group_kernel<GRP>, ms.bytes);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(merge_absorbed_group_kernel<GRP>, dim3(n_kv, (unsigned)B), dim3(MergeThreads<GRP>::NT), ms.bytes,
-                    st, part, S, n_q, n_kv, G, W_kv, o, out_fp32, ms);
-}
-
 }  // namespace
 
+bool merge_grouped_supported(int n_q, int n_kv);
+cudaError_t merge_grouped_launch(const float *part, int S, int64_t B, int n_q, int n_kv, int G,
+                                 const uint16_t *W_kv, void *o, int out_fp32, float *slab, uint32_t *cnt,
+                                 cudaStream_t st);
+
+// Group sizes 1, 2, 4, 8, 16 share W_v^(j) reads across the group (merge.cu);
+// others take one CTA per query head.
 cudaError_t merge_absorbed_launch(const float *part, int S, int64_t B, int n_q, int n_kv, int d_h, int G,
-                                  const uint16_t *W_kv, void *o, int out_fp32, cudaStream_t st) {
-  switch (n_q / n_kv) {
-    case 1: return merge_group_launch<1>(part, S, B, n_q, n_kv, d_h, G, W_kv, o, out_fp32, st);
-    case 2: return merge_group_launch<2>(part, S, B, n_q, n_kv, d_h, G, W_kv, o, out_fp32, st);
-    case 4: return merge_group_launch<4>(part, S, B, n_q, n_kv, d_h, G, W_kv, o, out_fp32, st);
-    case 8: return merge_group_launch<8>(part, S, B, n_q, n_kv, d_h, G, W_kv, o, out_fp32, st);
-    case 16: return merge_group_launch<16>(part, S, B, n_q, n_kv, d_h, G, W_kv, o, out_fp32, st);
-    default: break;
-  }
+                                  const uint16_t *W_kv, void *o, int out_fp32, MergeScratch ms, cudaStream_t st) {
+  if (merge_grouped_supported(n_q, n_kv))
+    return merge_grouped_launch(part, S, B, n_q, n_kv, G, W_kv, o, out_fp32, ms.slab, ms.cnt, st);
   merge_absorbed_kernel<<<dim3(n_q, (unsigned)B), 256, 0, st>>>(part, S, n_q, n_kv, d_h, G, W_kv, o, out_fp32);
   return cudaGetLastError();
 }
@@ -519,9 +366,10 @@ int simt_max_grp() { return kMaxGrp; }
 
 cudaError_t launch_absorbed_simt(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
                                  int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv, float scale,
-                                 int S, int64_t tps, float *qa, float *part, uint32_t *err, void *o,
+                                 int S, int64_t tps, float *qa, float *part, uint32_t *err, MergeScratch ms, void *o,
                                  int out_fp32, void *const *prof, cudaStream_t st) {
-  absorb_query_kernel<<<dim3(n_q, (unsigned)B), 256, 0, st>>>(q, W_kv, n_q, n_kv, d_h, G, scale * kLog2e, qa, err);
+  absorb_query_kernel<<<dim3(n_q, (unsigned)B), 256, 0, st>>>(q, W_kv, n_q, n_kv, d_h, G, scale * kLog2e, qa, err,
+                                                              ms);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   size_t smem = absorbed_simt_smem(n_q, G);
@@ -532,7 +380,7 @@ cudaError_t launch_absorbed_simt(const uint16_t *q, const uint8_t *codes, int64_
   e = cudaGetLastError();
   record_prof_event(prof[1], st);
   if (e != cudaSuccess) return e;
-  return merge_absorbed_launch(part, S, B, n_q, n_kv, d_h, G, W_kv, o, out_fp32, st);
+  return merge_absorbed_launch(part, S, B, n_q, n_kv, d_h, G, W_kv, o, out_fp32, ms, st);
 }
 
 cudaError_t launch_expand_simt(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
