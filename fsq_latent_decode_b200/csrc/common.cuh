@@ -42,15 +42,15 @@ __device__ __forceinline__ uint32_t fsq_nibble(float u, const Thresholds &t) {
 }
 
 // Split-merge plan of the absorbed form (merge.cu): CTAs per (kv head, batch
-// row) as G slices x split chunks, and the workspace its sliced mode needs.
+// row), one per slice of G, and the workspace its sliced mode needs.
 struct MergePlan {
-  int ngq = 1, nsq = 1;
+  int ngq = 1;
   size_t slab_bytes = 0, cnt_bytes = 0;
 };
 MergePlan merge_plan(int S, int64_t B, int n_q, int n_kv, int G);
 
-// Workspace of the sliced merge: per-chunk shares of the pooled latents and
-// one arrival count per (batch row, kv head), which the query prologue of the
+// Workspace of the sliced merge: the merged latents of every slice and one
+// arrival count per (batch row, kv head), which the query prologue of the
 // same call zeroes (ncnt counts; slab and cnt are null in direct mode).
 struct MergeScratch {
   float *slab;

@@ -5,48 +5,58 @@
 // sum_t 2^(x_t - m_s) z_t[g].  The merge forms ([S] eq. (6); slide deck frame
 // "The kernel reads codes and never writes reconstructed K/V": merge partials
 // and apply W_v once)
-//   m = max_s m_s,  w_s = 2^(m_s - m) / sum_s' 2^(m_s' - m) l_s'
-//   abar_h[g] = sum_s w_s acc_s[g]
+//   m = max_s m_s,  L = sum_s 2^(m_s - m) l_s,  abar_h = sum_s 2^(m_s - m) acc_s / L
 //   o_h = W_v^(j) abar_h
-// for the GRP query heads of kv head j, per batch row b.
+// for the GRP query heads of kv head j, per batch row b.  Each thread owns a
+// pair of coordinates of one head and folds the splits into a running
+// (max, sum, pair) by log-sum-exp, so all of its loads - the (m_s, l_s)
+// records and the accumulator pairs - are independent of each other and are
+// issued sixteen splits at a time.
+//
+// When a CTA has more threads than pairs, its threads also split the range of
+// splits (interleaved) and their running states are combined, by the same
+// log-sum-exp, in shared memory.
 //
 // Direct mode (few splits): one CTA per (j, b) does all of it, with W_v^(j)
-// staged in shared memory before the wait for the split kernel.  Sliced mode
-// (long contexts, many splits): the CTAs of a (j, b) pair cut the G
-// coordinates into 32-wide slices and the splits into chunks; each writes its
-// share of abar to a slab in the workspace, and the last of them to finish
-// (an atomic count, zeroed by the query prologue of the same call) adds the
-// shares and applies W_v.
+// staged in shared memory (cp.async) before the wait for the split kernel.
+// Sliced mode (long contexts, many splits): the CTAs of a (j, b) pair take
+// 32-coordinate slices of G over all splits, write their slices of abar to a
+// slab in the workspace, and the last to finish (an arrival count, zeroed by
+// the query prologue of the same call) applies W_v.
 #include <algorithm>
 
 #include "common.cuh"
 
 namespace fsq {
-
 namespace {
 
-constexpr int kMT = 256;           // threads per CTA: two per output row d of W_v
-constexpr int kGsl = 32;           // G coordinates per slice (sliced mode)
-constexpr int kSplitsPerCta = 32;  // splits per chunk (sliced mode)
-constexpr size_t kDirectBytes = 48 * 1024;  // partial bytes of a (j, b) pair that one CTA reads
-static_assert(kMT == 2 * FSQ_HEAD_DIM, "the W_v pass maps (half, d) to threads");
+constexpr int kMT = 512;                    // threads per CTA
+constexpr int kParts = kMT / FSQ_HEAD_DIM;  // W_v pass: threads per output row d
+constexpr int kGsl = 32;                    // G coordinates per slice (sliced mode)
+constexpr int kBatch = 16;                  // splits whose loads a thread issues at once
+constexpr int kMaxSub = 16;                 // threads sharing one pair (split ranges)
+constexpr size_t kDirectBytes = 64 * 1024;  // partial bytes of a (j, b) pair that one CTA reads
+static_assert(kMT % FSQ_HEAD_DIM == 0, "the W_v pass maps (part, d) to threads");
 
-__host__ __device__ inline int g_pad(int G) { return (G + 31) / 32 * 32; }
+// Padded G: a multiple of 8 * kParts, so that each part of the W_v pass
+// covers whole 8-element pieces.
+__host__ __device__ inline int g_pad(int G) { return (G + 8 * kParts - 1) / (8 * kParts) * (8 * kParts); }
 __host__ __device__ inline int w_stride(int G) { return g_pad(G) + 8; }  // bf16: 16-byte rows, odd x 16 B
 
 struct MergeSmem {
-  size_t off_abar, off_wts, off_scr, bytes;
+  size_t off_abar, off_scr, off_lse, bytes;
 };
 
-inline MergeSmem merge_smem(int G, int grp, int S) {
+inline MergeSmem merge_smem(int G, int grp) {
   MergeSmem m;
   size_t off = sizeof(uint16_t) * (size_t)FSQ_HEAD_DIM * w_stride(G);  // W_v^(j), bf16
   m.off_abar = off;
   off += sizeof(float) * (size_t)grp * g_pad(G);
-  m.off_wts = off;
-  off += sizeof(float) * (size_t)grp * S;
-  m.off_scr = off;  // l_s scratch, then the halves of the W_v pass
-  off += sizeof(float) * std::max((size_t)grp * S, (size_t)grp * FSQ_HEAD_DIM);
+  m.off_scr = off;  // partial outputs of parts 1.. of the W_v pass
+  off += sizeof(float) * (size_t)(kParts - 1) * grp * FSQ_HEAD_DIM;
+  off = align_up(off, 16);
+  m.off_lse = off;  // running states of the threads of a pair: [sub][pair] x (m, l, a.x, a.y)
+  off += sizeof(float4) * (size_t)kMT;
   m.bytes = align_up(off, 16);
   return m;
 }
@@ -85,20 +95,21 @@ __device__ __forceinline__ void stage_wv(uint16_t *wv, const uint16_t *__restric
   for (int i = threadIdx.x; i < D * (GP - G); i += kMT) wv[(i / (GP - G)) * WS + G + i % (GP - G)] = 0;
 }
 
-// o_h[d] = W_v[d, :] . abar_h for the GRP heads; thread (half, d) covers half
-// of the coordinates for every head, so each W_v value read serves GRP heads
+// o_h[d] = W_v[d, :] . abar_h for the GRP heads; thread (part, d) covers a
+// kParts-th of the coordinates for every head, so each W_v value read serves
+// GRP heads (the abar reads are broadcasts)
 template <int GRP>
 __device__ __forceinline__ void apply_wv(const uint16_t *wv, const float *abar, float *scr, int G, int64_t obase,
                                          void *o, int out_fp32) {
   constexpr int D = FSQ_HEAD_DIM;
   const int GP = g_pad(G), WS = w_stride(G);
-  const int d = threadIdx.x % D, half = threadIdx.x / D;
-  const int gh = GP / 2;  // a multiple of 16
-  const uint16_t *wr = wv + d * WS + half * gh;
+  const int d = threadIdx.x % D, part = threadIdx.x / D;
+  const int gq = GP / kParts;  // a multiple of 8
+  const uint16_t *wr = wv + d * WS + part * gq;
   float acc[GRP];
 #pragma unroll
   for (int h = 0; h < GRP; ++h) acc[h] = 0.f;
-  for (int g8 = 0; g8 < gh; g8 += 8) {
+  for (int g8 = 0; g8 < gq; g8 += 8) {
     const uint4 wq = *reinterpret_cast<const uint4 *>(wr + g8);
     const uint32_t wp[4] = {wq.x, wq.y, wq.z, wq.w};
     float wf[8];
@@ -109,21 +120,23 @@ __device__ __forceinline__ void apply_wv(const uint16_t *wv, const float *abar, 
     }
 #pragma unroll
     for (int h = 0; h < GRP; ++h) {
-      const float4 lo = *reinterpret_cast<const float4 *>(abar + h * GP + half * gh + g8);
-      const float4 hi = *reinterpret_cast<const float4 *>(abar + h * GP + half * gh + g8 + 4);
+      const float4 lo = *reinterpret_cast<const float4 *>(abar + h * GP + part * gq + g8);
+      const float4 hi = *reinterpret_cast<const float4 *>(abar + h * GP + part * gq + g8 + 4);
       acc[h] = fmaf(wf[0], lo.x, fmaf(wf[1], lo.y, fmaf(wf[2], lo.z, fmaf(wf[3], lo.w, acc[h]))));
       acc[h] = fmaf(wf[4], hi.x, fmaf(wf[5], hi.y, fmaf(wf[6], hi.z, fmaf(wf[7], hi.w, acc[h]))));
     }
   }
-  if (half == 1) {
+  if (part > 0) {
 #pragma unroll
-    for (int h = 0; h < GRP; ++h) scr[h * D + d] = acc[h];
+    for (int h = 0; h < GRP; ++h) scr[((part - 1) * GRP + h) * D + d] = acc[h];
   }
   __syncthreads();
-  if (half == 0) {
+  if (part == 0) {
 #pragma unroll
     for (int h = 0; h < GRP; ++h) {
-      const float v = acc[h] + scr[h * D + d];
+      float v = acc[h];
+#pragma unroll
+      for (int p = 1; p < kParts; ++p) v += scr[((p - 1) * GRP + h) * D + d];
       const int64_t oi = obase + (int64_t)h * D + d;
       if (out_fp32) reinterpret_cast<float *>(o)[oi] = v;
       else reinterpret_cast<uint16_t *>(o)[oi] = f32_to_bf16_rn(v);
@@ -131,23 +144,65 @@ __device__ __forceinline__ void apply_wv(const uint16_t *wv, const float *abar, 
   }
 }
 
+// Running log-sum-exp state of one coordinate pair: max m, weight sum l, pair a.
+struct Lse {
+  float m, l;
+  float2 a;
+};
+
+// Fold splits s0, s0 + ds, ... below S of one head's records (rec: the
+// head's record in split 0; sstride: floats between splits; gi: the pair's
+// offset) into st.
+__device__ __forceinline__ void fold_splits(Lse &st, const float *__restrict__ rec, int64_t sstride, int gi, int s0,
+                                            int ds, int S) {
+  for (int s = s0; s < S; s += kBatch * ds) {
+    float2 ml[kBatch], av[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const bool in = s + u * ds < S;
+      const float *r = rec + (int64_t)(s + u * ds) * sstride;
+      ml[u] = in ? *reinterpret_cast<const float2 *>(r) : make_float2(-INFINITY, 0.f);
+      av[u] = in ? *reinterpret_cast<const float2 *>(r + 2 + gi) : make_float2(0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const float mn = fmaxf(st.m, ml[u].x);
+      if (mn == -INFINITY) continue;  // nothing folded yet and an empty slot
+      const float co = exp2f(st.m - mn), cs = exp2f(ml[u].x - mn);
+      st.l = fmaf(st.l, co, ml[u].y * cs);
+      st.a.x = fmaf(st.a.x, co, av[u].x * cs);
+      st.a.y = fmaf(st.a.y, co, av[u].y * cs);
+      st.m = mn;
+    }
+  }
+}
+
+__device__ __forceinline__ void fold_state(Lse &st, const float4 &o) {
+  const float mn = fmaxf(st.m, o.x);
+  if (mn == -INFINITY) return;
+  const float co = exp2f(st.m - mn), cs = exp2f(o.x - mn);
+  st.l = fmaf(st.l, co, o.y * cs);
+  st.a.x = fmaf(st.a.x, co, o.z * cs);
+  st.a.y = fmaf(st.a.y, co, o.w * cs);
+  st.m = mn;
+}
+
 template <int GRP>
 __global__ void __launch_bounds__(kMT) merge_absorbed_grouped(const float *__restrict__ part, int S, int n_q,
                                                               int n_kv, int G, const uint16_t *__restrict__ W_kv,
-                                                              void *o, int out_fp32, int ngq, int nsq,
+                                                              void *o, int out_fp32, int ngq,
                                                               float *__restrict__ slab, uint32_t *__restrict__ cnt,
                                                               MergeSmem L) {
   constexpr int D = FSQ_HEAD_DIM;
   extern __shared__ __align__(16) unsigned char msm[];
   uint16_t *wv = reinterpret_cast<uint16_t *>(msm);           // [D][WS] bf16
   float *abar = reinterpret_cast<float *>(msm + L.off_abar);  // [GRP][GP]
-  float *wts = reinterpret_cast<float *>(msm + L.off_wts);    // [GRP][S]
   float *scr = reinterpret_cast<float *>(msm + L.off_scr);
   __shared__ uint32_t last;
-  const int gq = blockIdx.x % ngq, sq = blockIdx.x / ngq;
+  const int gq = blockIdx.x;
   const int j = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool direct = ngq * nsq == 1;
+  const int tid = threadIdx.x;
+  const bool direct = ngq == 1;
   const int GP = g_pad(G);
   const uint16_t *wsrc = W_kv + (int64_t)(n_kv + j) * D * G;
   if (direct) stage_wv(wv, wsrc, G);  // W_v is not written by the split kernel
@@ -158,99 +213,44 @@ __global__ void __launch_bounds__(kMT) merge_absorbed_grouped(const float *__res
   const int64_t hstride = 2 + (int64_t)G;          // floats per (split, head) record
   const int64_t sstride = (int64_t)n_q * hstride;  // floats per split
   const float *pbase = part + ((int64_t)b * S * n_q + (int64_t)j * GRP) * hstride;
-
-  // split weights of each head, 1/l folded in; (m_s, l_s) is one 8-byte
-  // load, eight of them in flight per lane
-  for (int h = warp; h < GRP; h += kMT / 32) {
-    const float *ph = pbase + (int64_t)h * hstride;
-    float m = -INFINITY;
-    for (int s8 = 0; s8 < S; s8 += 256) {
-      float2 ml[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int s = s8 + 32 * u + lane;
-        ml[u] = s < S ? *reinterpret_cast<const float2 *>(ph + (int64_t)s * sstride) : make_float2(-INFINITY, 0.f);
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int s = s8 + 32 * u + lane;
-        if (s < S) {
-          wts[h * S + s] = ml[u].x;
-          scr[h * S + s] = ml[u].y;
-        }
-        m = fmaxf(m, ml[u].x);
-      }
-    }
-#pragma unroll
-    for (int off = 16; off; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-    float l = 0.f;
-    for (int s = lane; s < S; s += 32) {
-      const float w = exp2f(wts[h * S + s] - m);
-      wts[h * S + s] = w;
-      l = fmaf(w, scr[h * S + s], l);
-    }
-#pragma unroll
-    for (int off = 16; off; off >>= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
-    const float inv = 1.f / l;
-    __syncwarp();
-    for (int s = lane; s < S; s += 32) wts[h * S + s] *= inv;
-  }
-  __syncthreads();
-
-  // this CTA's coordinates and splits; a pair of coordinates per 8-byte load
-  // (records start 8-byte aligned), up to eight loads in flight per thread
+  // sliced mode: slab[b][j][h][GP] holds abar; CTA gq writes coordinates gq*32 ..
+  float *sl = slab + ((int64_t)b * n_kv + j) * GRP * GP;
   const int gc0 = direct ? 0 : gq * kGsl, gcn = direct ? G : min(kGsl, G - gc0);
-  const int s0 = direct ? 0 : sq * kSplitsPerCta, s1 = direct ? S : min(S, s0 + kSplitsPerCta);
   const int npair = gcn / 2;  // G is even, so are gc0 and gcn
-  for (int t = tid; t < GRP * npair; t += kMT) {
-    const int h = t / npair, gi = 2 * (t % npair);
-    const float *pg = pbase + (int64_t)h * hstride + 2 + gc0 + gi;
-    const float *w = wts + h * S;
-    float2 a = make_float2(0.f, 0.f);
-    for (int s = s0; s < s1; s += 8) {
-      float2 pv[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        pv[u] = s + u < s1 ? *reinterpret_cast<const float2 *>(pg + (int64_t)(s + u) * sstride) : make_float2(0.f, 0.f);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const float wu = s + u < s1 ? w[s + u] : 0.f;
-        a.x = fmaf(wu, pv[u].x, a.x);
-        a.y = fmaf(wu, pv[u].y, a.y);
-      }
+  const int items = GRP * npair;
+  const int nsub = items >= kMT ? 1 : min(kMaxSub, kMT / items);  // threads per pair
+  float4 *lse = reinterpret_cast<float4 *>(msm + L.off_lse);       // [nsub][items]
+  for (int t0 = 0; t0 < items * nsub; t0 += kMT) {
+    const int t = t0 + tid;
+    const int it = t % items, sub = t / items;
+    const int h = it / npair, gi = gc0 + 2 * (it % npair);
+    Lse st{-INFINITY, 0.f, make_float2(0.f, 0.f)};
+    if (t < items * nsub) fold_splits(st, pbase + (int64_t)h * hstride, sstride, gi, sub, nsub, S);
+    if (nsub > 1) {  // combine the sub-ranges of a pair (all of them lie in this round)
+      lse[tid] = make_float4(st.m, st.l, st.a.x, st.a.y);
+      __syncthreads();
+      if (sub == 0 && t < items)
+        for (int k = 1; k < nsub; ++k) fold_state(st, lse[k * items + it]);
     }
-    if (direct) {
-      abar[h * GP + gi] = a.x;
-      abar[h * GP + gi + 1] = a.y;
-    } else {  // slab[b][j][sq][h][g]
-      float *dst = slab + ((((int64_t)b * n_kv + j) * nsq + sq) * GRP + h) * GP + gc0 + gi;
-      *reinterpret_cast<float2 *>(dst) = a;
+    if (sub == 0 && t < items) {
+      const float inv = 1.f / st.l;
+      const float2 v = make_float2(st.a.x * inv, st.a.y * inv);
+      if (direct) *reinterpret_cast<float2 *>(abar + h * GP + gi) = v;
+      else *reinterpret_cast<float2 *>(sl + h * GP + gi) = v;
     }
   }
   if (direct) {
     for (int i = tid; i < GRP * (GP - G); i += kMT) abar[(i / (GP - G)) * GP + G + i % (GP - G)] = 0.f;
   } else {
-    // the last CTA of the (j, b) pair adds the shares of all chunks
+    // the last CTA of the (j, b) pair gathers abar and applies W_v
     __threadfence();
     __syncthreads();
-    if (tid == 0) last = atomicAdd(cnt + (int64_t)b * n_kv + j, 1u) == (uint32_t)(ngq * nsq - 1) ? 1u : 0u;
+    if (tid == 0) last = atomicAdd(cnt + (int64_t)b * n_kv + j, 1u) == (uint32_t)(ngq - 1) ? 1u : 0u;
     __syncthreads();
     if (!last) return;
     __threadfence();
     stage_wv(wv, wsrc, G);
-    const float *sl = slab + ((int64_t)b * n_kv + j) * nsq * GRP * GP;
-    for (int i = tid; i < GRP * GP; i += kMT) {
-      float a = 0.f;
-      if (i % GP < G)
-        for (int c0 = 0; c0 < nsq; c0 += 8) {  // eight loads in flight
-          float v[8];
-#pragma unroll
-          for (int u = 0; u < 8; ++u) v[u] = c0 + u < nsq ? __ldcg(sl + (int64_t)(c0 + u) * GRP * GP + i) : 0.f;
-#pragma unroll
-          for (int u = 0; u < 8; ++u) a += v[u];
-        }
-      abar[i] = a;
-    }
+    for (int i = tid; i < GRP * GP; i += kMT) abar[i] = i % GP < G ? __ldcg(sl + i) : 0.f;
   }
   cp_async_wait_all();
   __syncthreads();
@@ -260,12 +260,12 @@ __global__ void __launch_bounds__(kMT) merge_absorbed_grouped(const float *__res
 template <int GRP>
 cudaError_t merge_launch(const float *part, int S, int64_t B, int n_q, int n_kv, int G, const uint16_t *W_kv, void *o,
                          int out_fp32, const MergePlan &mp, float *slab, uint32_t *cnt, cudaStream_t st) {
-  const MergeSmem L = merge_smem(G, GRP, S);
+  const MergeSmem L = merge_smem(G, GRP);
   auto kern = merge_absorbed_grouped<GRP>;
   cudaError_t e = ensure_smem_limit((const void *)kern, L.bytes);
   if (e != cudaSuccess) return e;
-  return launch_pdl(kern, dim3((unsigned)(mp.ngq * mp.nsq), (unsigned)n_kv, (unsigned)B), dim3(kMT), L.bytes, st,
-                    part, S, n_q, n_kv, G, W_kv, o, out_fp32, mp.ngq, mp.nsq, slab, cnt, L);
+  return launch_pdl(kern, dim3((unsigned)mp.ngq, (unsigned)n_kv, (unsigned)B), dim3(kMT), L.bytes, st, part, S, n_q,
+                    n_kv, G, W_kv, o, out_fp32, mp.ngq, slab, cnt, L);
 }
 
 }  // namespace
@@ -275,16 +275,14 @@ bool merge_grouped_supported(int n_q, int n_kv) {
   return grp == 1 || grp == 2 || grp == 4 || grp == 8 || grp == 16;
 }
 
-// Direct mode when one CTA's share of partials is small; else G slices of 32
-// and split chunks of kSplitsPerCta.
+// Direct mode when one CTA's share of partials is small; else G slices of 32.
 MergePlan merge_plan(int S, int64_t B, int n_q, int n_kv, int G) {
   MergePlan mp;
   const int grp = n_q / n_kv;
   const size_t bytes = sizeof(float) * (size_t)S * grp * (2 + G);
   if (merge_grouped_supported(n_q, n_kv) && bytes > kDirectBytes) {
     mp.ngq = (G + kGsl - 1) / kGsl;
-    mp.nsq = (S + kSplitsPerCta - 1) / kSplitsPerCta;
-    mp.slab_bytes = sizeof(float) * (size_t)B * n_q * mp.nsq * g_pad(G);
+    mp.slab_bytes = sizeof(float) * (size_t)B * n_q * g_pad(G);
     mp.cnt_bytes = sizeof(uint32_t) * (size_t)B * n_kv;
   }
   return mp;
@@ -295,7 +293,7 @@ cudaError_t merge_grouped_launch(const float *part, int S, int64_t B, int n_q, i
                                  cudaStream_t st) {
   if (B > 65535 || n_kv > 65535 || G > FSQ_MAX_G) return cudaErrorInvalidValue;
   const MergePlan mp = merge_plan(S, B, n_q, n_kv, G);
-  if (mp.ngq * mp.nsq > 1 && (!slab || !cnt)) return cudaErrorInvalidValue;
+  if (mp.ngq > 1 && (!slab || !cnt)) return cudaErrorInvalidValue;
   switch (n_q / n_kv) {
     case 1: return merge_launch<1>(part, S, B, n_q, n_kv, G, W_kv, o, out_fp32, mp, slab, cnt, st);
     case 2: return merge_launch<2>(part, S, B, n_q, n_kv, G, W_kv, o, out_fp32, mp, slab, cnt, st);
