@@ -56,7 +56,9 @@ namespace tc {
 using namespace ptx;
 
 constexpr int kTile = 128;
-constexpr int kStages = 4;
+constexpr int kMaxStages = 16;                     // code-tile ring depth bound (barrier arrays)
+constexpr int kSmemBudget = 200 * 1024;            // shared memory a CTA plans for
+constexpr int kQAfterTiles = 4;                    // code tiles requested before Q' (and its wait)
 constexpr float kTau = 8.f;                        // rescale when a score exceeds the running max by 2^8
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s per wait
 constexpr int kMiscBytes = 12288;                  // shared-memory reservation for the Misc block
@@ -98,7 +100,13 @@ struct Cfg {
   static_assert(TMEM_USED <= 512, "TMEM plan exceeds 512 columns");
   // shared memory
   static constexpr int SM_CODES = 0;
-  static constexpr int SM_Q = SM_CODES + kStages * STAGE_BYTES;
+  // Code-tile ring: as deep as the shared memory left over allows (bytes in
+  // flight per SM hide the load latency), at most kMaxStages
+  static constexpr int OTHER_BYTES = Q_BYTES + kPBufs * P_BYTES + kMiscBytes;
+  static constexpr int STAGES_FIT = (kSmemBudget - OTHER_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT < kMaxStages ? STAGES_FIT : kMaxStages;
+  static_assert(STAGES >= 4, "code-tile ring too shallow");
+  static constexpr int SM_Q = SM_CODES + STAGES * STAGE_BYTES;
   static constexpr int SM_P = SM_Q + Q_BYTES;
   static constexpr int SM_MISC = SM_P + kPBufs * P_BYTES;
   static constexpr int SM_TOTAL = SM_MISC + kMiscBytes;
@@ -120,7 +128,7 @@ struct Params {
 };
 
 struct Misc {
-  uint64_t full[kStages], empty[kStages];
+  uint64_t full[kMaxStages], empty[kMaxStages];
   uint64_t cs_ready[2], cs_free[2];
   uint64_t cp_ready[4], cp_free[4];
   uint64_t s_full[2], s_free[2];
@@ -342,7 +350,7 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
   constexpr uint32_t kPoolIssuers = 2;
 
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(&ms.full[s], 1);
       mbar_init(&ms.empty[s], 12);
     }
@@ -399,9 +407,9 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
     int issued = 0;
     bool ok = true, q_loaded = false;
     for (int i = 0; i < n_tiles; ++i) {
-      const int st = i % kStages;
-      const uint32_t ph = (uint32_t)(i / kStages) & 1u;
-      if (i == kStages) {
+      const int st = i % C::STAGES;
+      const uint32_t ph = (uint32_t)(i / C::STAGES) & 1u;
+      if (i == kQAfterTiles) {
         load_q();
         q_loaded = true;
       }
@@ -436,8 +444,8 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
     if (!ok) {
       if (lane == 0) fail();
       // let the copies still in flight land before the CTA exits
-      for (int i = max(0, issued - kStages); i < issued; ++i)
-        drain_bar(&ms.full[i % kStages], (uint32_t)(i / kStages) & 1u, p.wait_ns / 4 + 1);
+      for (int i = max(0, issued - C::STAGES); i < issued; ++i)
+        drain_bar(&ms.full[i % C::STAGES], (uint32_t)(i / C::STAGES) & 1u, p.wait_ns / 4 + 1);
       drain_bar(&ms.q_full, 0, p.wait_ns / 4 + 1);
     }
   } else if (warp == 1) {
@@ -506,9 +514,9 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     bool ok = true;
     for (int i = 0; i < n_tiles; ++i) {
-      const int st = i % kStages, sb = i & 1;
+      const int st = i % C::STAGES, sb = i & 1;
       const uint8_t *tile = smem + C::SM_CODES + st * C::STAGE_BYTES;
-      if (!wait_bar(&ms.full[st], (uint32_t)(i / kStages) & 1u, abort, p.wait_ns) ||
+      if (!wait_bar(&ms.full[st], (uint32_t)(i / C::STAGES) & 1u, abort, p.wait_ns) ||
           !wait_bar(&ms.cs_free[sb], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort, p.wait_ns)) {
         ok = false;
         break;
@@ -565,11 +573,11 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     bool ok = true;
     for (int i = 0; i < n_tiles && ok; ++i) {
-      const int st = i % kStages;
+      const int st = i % C::STAGES;
       const int kc = 2 * i + c;
       const int cb = kc % C::NCP;
       const uint8_t *tile = smem + C::SM_CODES + st * C::STAGE_BYTES;
-      if (!wait_bar(&ms.full[st], (uint32_t)(i / kStages) & 1u, abort, p.wait_ns) ||
+      if (!wait_bar(&ms.full[st], (uint32_t)(i / C::STAGES) & 1u, abort, p.wait_ns) ||
           !wait_bar(&ms.cp_free[cb], ((uint32_t)(kc / C::NCP) & 1u) ^ 1u, abort, p.wait_ns)) {
         ok = false;
         break;
@@ -646,53 +654,93 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
     for (int n = 0; n < HQ; ++n) lsum[n] = 0.f;
     const int r = 32 * q + lane;        // token row within the tile
     const int kap = kappa_of_token(r);  // its K position in the pooling operand
-    bool ok = true;
-    for (int i = 0; i < n_tiles && ok; ++i) {
-      const uint32_t par = (uint32_t)(i >> 1) & 1u;
-      const int sb = i & 1;
-      if (!wait_bar(&ms.s_full[sb], par, abort, p.wait_ns)) { ok = false; break; }
-      tc_fence_after();
-      float x[HQ];  // score - m
-      float xmax = -INFINITY;
-      {
-        uint32_t ra[HQ], rb[HQ];
-        const uint32_t sbase = tm + lane_base + C::OFF_S + sb * C::NS;
-        tmem_ld_hq<HQ>(sbase + h0, ra);       // a terms
-        tmem_ld_hq<HQ>(sbase + NQ + h0, rb);  // b terms
-        tmem_ld_wait();
-        // S is in registers: the next score MMA may overwrite it
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ms.s_free[sb]);
-        const float4 *sg4 = reinterpret_cast<const float4 *>(ms.sig + h0);
-        const float4 *cm4 = reinterpret_cast<const float4 *>(cm);
+    static_assert(HQ == 8, "softmax warps own eight heads");
+    // x <- score - m of one tile from its raw S (a, b terms); rows past the
+    // split's end (ragged last tile only) take no weight; returns the row max
+    auto scores = [&](int i, const uint32_t (&ra)[HQ], const uint32_t (&rb)[HQ], float (&x)[HQ]) -> float {
+      const float4 *sg4 = reinterpret_cast<const float4 *>(ms.sig + h0);
+      const float4 *cm4 = reinterpret_cast<const float4 *>(cm);
+      float lm = -INFINITY;
 #pragma unroll
-        for (int n4 = 0; n4 < HQ / 4; ++n4) {
-          const float4 sg = sg4[n4], cc = cm4[n4];
-          const float sv[4] = {sg.x, sg.y, sg.z, sg.w}, cv[4] = {cc.x, cc.y, cc.z, cc.w};
+      for (int n4 = 0; n4 < HQ / 4; ++n4) {
+        const float4 sg = sg4[n4], cc = cm4[n4];
+        const float sv[4] = {sg.x, sg.y, sg.z, sg.w}, cv[4] = {cc.x, cc.y, cc.z, cc.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int n = 4 * n4 + e;
-            const int y = (int)ra[n] * 128 + (int)rb[n];  // exact: |y| < 2^27
-            x[n] = fmaf((float)y, sv[e], -cv[e]);
-            xmax = fmaxf(xmax, x[n]);
-          }
+        for (int e = 0; e < 4; ++e) {
+          const int n = 4 * n4 + e;
+          const int y = (int)ra[n] * 128 + (int)rb[n];  // exact: |y| < 2^27
+          x[n] = fmaf((float)y, sv[e], -cv[e]);
+          lm = fmaxf(lm, x[n]);
         }
       }
-      // rows past the split's end (ragged last tile only) take no weight
       if ((t0 + (int64_t)i * kTile + r) >= t1) {
-        xmax = -INFINITY;
+        lm = -INFINITY;
 #pragma unroll
         for (int n = 0; n < HQ; ++n) x[n] = -INFINITY;
       }
-      const bool need = (i == 0) || xmax > kTau;
+      return lm;
+    };
+    // P row of this token (fp16) for this warp's heads into P buffer i % kPBufs, MN-major
+    auto write_p = [&](int i, const float (&x)[HQ]) {
+      uint8_t *prow = smem + C::SM_P + (i % kPBufs) * C::P_BYTES + (kap >> 3) * 128 + (kap & 7) * 16 +
+                      (h0 / 8) * C::SBO_P;
+      uint32_t h2[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float p0 = ex2_approx(x[2 * k]), p1 = ex2_approx(x[2 * k + 1]);
+        const __half2 hv = __floats2half2_rn(p0, p1);
+        lsum[2 * k] += p0;
+        lsum[2 * k + 1] += p1;
+        h2[k] = *reinterpret_cast<const uint32_t *>(&hv);
+      }
+      *reinterpret_cast<uint4 *>(prow) = make_uint4(h2[0], h2[1], h2[2], h2[3]);
+    };
+    // Tiles go in pairs (2j in S buffer 0, 2j+1 in S buffer 1): both tiles'
+    // scores are loaded together and share one vote, one fence and one pass
+    // through the loop.  P buffers stay per tile (the score MMA of tile i
+    // waited for P buffer i % kPBufs to be free).
+    const int n_pairs = (n_tiles + 1) >> 1;
+    bool ok = true;
+    for (int j = 0; j < n_pairs && ok; ++j) {
+      const int i0 = 2 * j;
+      const bool two = i0 + 1 < n_tiles;
+      const uint32_t par = (uint32_t)j & 1u;  // use j of each S buffer
+      float x0[HQ], x1[HQ];
+      float xmax;
+      {  // tile 2j from S buffer 0, then tile 2j+1 from S buffer 1 (one buffer's raw terms live at a time)
+        uint32_t ra[HQ], rb[HQ];
+        if (!wait_bar(&ms.s_full[0], par, abort, p.wait_ns)) { ok = false; break; }
+        tc_fence_after();
+        tmem_ld8(tm + lane_base + C::OFF_S + h0, ra);
+        tmem_ld8(tm + lane_base + C::OFF_S + NQ + h0, rb);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ms.s_free[0]);  // the next score MMA may overwrite it
+        xmax = scores(i0, ra, rb, x0);
+        if (two) {
+          if (!wait_bar(&ms.s_full[1], par, abort, p.wait_ns)) { ok = false; break; }
+          tc_fence_after();
+          tmem_ld8(tm + lane_base + C::OFF_S + C::NS + h0, ra);
+          tmem_ld8(tm + lane_base + C::OFF_S + C::NS + NQ + h0, rb);
+          tmem_ld_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ms.s_free[1]);
+          xmax = fmaxf(xmax, scores(i0 + 1, ra, rb, x1));
+        } else {
+#pragma unroll
+          for (int n = 0; n < HQ; ++n) x1[n] = -INFINITY;
+        }
+      }
+      const bool need = (j == 0) || xmax > kTau;
       // one barrier over the group's four warps that also ORs their votes
       const bool any = named_bar_or(barid, 128, need);
       if (any) {
-        // raise the running max: m <- m + max(0, tile max of x) (the first tile: m <- its max)
+        // raise the running max: m <- m + max(0, pair max of x) (the first pair: m <- its max)
 #pragma unroll
         for (int n = 0; n < HQ; ++n) {
-          float v = x[n];
+          float v = fmaxf(x0[n], x1[n]);
 #pragma unroll
           for (int off = 16; off; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
           if (lane == 0) ms.red[q][h0 + n] = v;
@@ -703,9 +751,10 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
         for (int n = 0; n < HQ; ++n) {
           const int hn = h0 + n;
           const float d = fmaxf(fmaxf(ms.red[0][hn], ms.red[1][hn]), fmaxf(ms.red[2][hn], ms.red[3][hn]));
-          const float sh = (i == 0) ? d : fmaxf(d, 0.f);
-          const float fn = (i == 0) ? 0.f : exp2f(-sh);
-          x[n] -= sh;
+          const float sh = (j == 0) ? d : fmaxf(d, 0.f);
+          const float fn = (j == 0) ? 0.f : exp2f(-sh);
+          x0[n] -= sh;
+          x1[n] -= sh;
           lsum[n] *= fn;
           if (lane == 0) {
             f[n] = fn;
@@ -713,10 +762,10 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
           }
         }
         __syncwarp();
-        if (i > 0) {
+        if (j > 0) {
           // ACC must hold every earlier tile before it is rescaled
-          const int pj = (i - 1) % kPBufs;
-          if (!wait_bar(&ms.p_free[pj], (uint32_t)((i - 1) / kPBufs) & 1u, abort, p.wait_ns)) { ok = false; break; }
+          const int pi = i0 - 1;
+          if (!wait_bar(&ms.p_free[pi % kPBufs], (uint32_t)(pi / kPBufs) & 1u, abort, p.wait_ns)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll 1
           for (int blk = 0; blk < 2; ++blk) {  // both ACC blocks, this warp's head columns
@@ -731,26 +780,15 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
           tmem_st_wait();
         }
       }
-      // P row of this token (fp16) for this warp's heads, MN-major: HQ/8 chunks of 8 heads
-      const int pb = i % kPBufs;  // free: the score MMA of tile i waited for it
-      uint8_t *prow = smem + C::SM_P + pb * C::P_BYTES + (kap >> 3) * 128 + (kap & 7) * 16 + (h0 / 8) * C::SBO_P;
-#pragma unroll
-      for (int g8 = 0; g8 < HQ / 8; ++g8) {
-        uint32_t h2[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const float p0 = ex2_approx(x[8 * g8 + 2 * k]), p1 = ex2_approx(x[8 * g8 + 2 * k + 1]);
-          const __half2 hv = __floats2half2_rn(p0, p1);
-          lsum[8 * g8 + 2 * k] += p0;
-          lsum[8 * g8 + 2 * k + 1] += p1;
-          h2[k] = *reinterpret_cast<const uint32_t *>(&hv);
-        }
-        *reinterpret_cast<uint4 *>(prow + g8 * C::SBO_P) = make_uint4(h2[0], h2[1], h2[2], h2[3]);
-      }
+      write_p(i0, x0);
+      if (two) write_p(i0 + 1, x1);
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&ms.p_full[pb]);
+      if (lane == 0) {
+        mbar_arrive(&ms.p_full[i0 % kPBufs]);
+        if (two) mbar_arrive(&ms.p_full[(i0 + 1) % kPBufs]);
+      }
     }
     // ------------------------------------------------------------ epilogue: ACC -> partials
     if (ok) ok = wait_bar(&ms.acc_full, 0, abort, p.wait_ns);
