@@ -347,6 +347,42 @@ def _blas_threads():
         return os.cpu_count() or 1
 
 
+PAPER_SDPA_RATIOS = {  # decode tokens/s of the full model vs native SDPA, Qwen3-8B-Base, NVIDIA L40S
+    256: {"ratio": 1.01, "ci95": [0.98, 1.05], "compression": "32x"},
+    84: {"ratio": 1.54, "ci95": [1.16, 1.88], "compression": "97.5x"},
+}
+
+
+def sdpa_context(torch, B, T, n_q, n_kv, d_h, device, steps=20, warmup=3):
+    """torch scaled_dot_product_attention (default dispatch, bf16, enable_gqa)
+    for one decode query per row over an uncompressed [B, n_kv, T, d_h] K/V
+    cache of the same shape: context tokens/s, for comparison only."""
+    F_ = torch.nn.functional
+    g = torch.Generator(device=device)
+    g.manual_seed(0)
+    k = torch.randn((B, n_kv, T, d_h), generator=g, device=device, dtype=torch.bfloat16)
+    v = torch.randn((B, n_kv, T, d_h), generator=g, device=device, dtype=torch.bfloat16)
+    q = torch.randn((B, n_q, 1, d_h), generator=g, device=device, dtype=torch.bfloat16)
+    for _ in range(warmup):
+        F_.scaled_dot_product_attention(q, k, v, enable_gqa=True)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        F_.scaled_dot_product_attention(q, k, v, enable_gqa=True)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    kv_bytes = 2 * B * n_kv * T * d_h * 2
+    del k, v, q
+    torch.cuda.empty_cache()
+    return {"value": B * T / (ms * 1e-3), "unit": "context tokens/s", "ms_per_call": ms,
+            "kv_cache_bytes": kv_bytes, "kv_gbs": kv_bytes / (ms * 1e-3) / 1e9,
+            "what": f"torch.nn.functional.scaled_dot_product_attention (default dispatch, torch {torch.__version__}), "
+                    f"bf16 K,V [{B}, {n_kv}, {T}, {d_h}] ({kv_bytes // (B * T)} B/token), q [{B}, {n_q}, 1, {d_h}], "
+                    "enable_gqa=True; inputs larger than L2"}
+
+
 def cpu_baseline_oracle(wl_name, T, budget_s=20.0):
     """The fp64 oracle as it stands, timed on one batch row of the workload."""
     Ts = min(T, 8192)
@@ -398,6 +434,7 @@ def main():
     ap.add_argument("--variant", default="absorbed", choices=["absorbed", "expand"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-second", action="store_true", help="skip the G=84 companion measurement")
+    ap.add_argument("--no-sdpa", action="store_true", help="skip the uncompressed-cache SDPA context measurement")
     args = ap.parse_args()
     rank, world, local = dist_env()
     wl_name = args.workload
@@ -450,6 +487,18 @@ def main():
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline_oracle(wl_name, T)
+    sdpa = None
+    if rank == 0 and not args.no_sdpa:
+        sdpa = sdpa_context(torch, B, T, wl.n_q, wl.n_kv, wl.d_h, device)
+        fsq_ctx = B * T / (res["ms"] * 1e-3)
+        sdpa["fsq_step_over_sdpa"] = fsq_ctx / sdpa["value"]
+        pr = PAPER_SDPA_RATIOS.get(wl.G)
+        if pr:
+            sdpa["paper"] = dict(pr, what="full-model decode tokens/s vs native SDPA, Qwen3-8B-Base, NVIDIA L40S "
+                                          "(context only: another scope and GPU)")
+        if also is not None:
+            also["fsq_step_over_sdpa"] = also["value"] / world / sdpa["value"]
+            also["paper"] = dict(PAPER_SDPA_RATIOS[84], what=sdpa["paper"]["what"]) if "paper" in sdpa else None
     if rank == 0:
         rf = roofline(res, peaks, kernel_name)
         value = world * B * T / (res["ms"] * 1e-3)
@@ -463,7 +512,7 @@ def main():
                 "data": "synthetic (seeded; cache = FSQ codes of u ~ N(0,4), the law of E x; new token x ~ N(0,1) appended each step)",
                 "config": config, "code_gbs": world * res["code_bytes"] / (res["ms"] * 1e-3) / 1e9,
                 "roofline": rf, "cpu_baseline": cb, "e2e": res["e2e"], "clocks": res["clocks"],
-                "gpu_launches": args.steps * 4, "also": also}
+                "gpu_launches": args.steps * 4, "also": also, "sdpa_context": sdpa}
         print(json.dumps(line))
     if dist is not None:
         dist.barrier()
