@@ -9,7 +9,7 @@ memory and streams.
 from ._abi import (  # noqa: F401
     EXPORTED, FSQ_OK, FSQ_ERR_CUDA, FSQ_ERR_INVALID_ARG, FSQ_ERR_MISALIGNED, FSQ_ERR_TIMEOUT,
     FSQ_ERR_UNSUPPORTED, FSQ_ERR_WORKSPACE, AttnOpts, FsqError, QuantParams, Workspace, attn_opts,
-    decode_attn, decode_attn_raw, encode_pack, encode_pack_raw, lib, quant_params, quantize_pack_f32,
+    decode_attn, decode_attn_raw, encode_pack, encode_pack_raw, encode_status, lib, quant_params, quantize_pack_f32,
     quantize_pack_f32_raw, status_string, thresholds, workspace_size, workspace_status,
 )
 

@@ -27,7 +27,7 @@ VARIANTS = {"auto": VARIANT_AUTO, "absorbed": VARIANT_ABSORBED, "expand": VARIAN
 # Every symbol include/fsq.h declares.
 EXPORTED = ("fsq_attn_opts_default", "fsq_thresholds", "fsq_encode_pack", "fsq_quantize_pack_f32",
             "fsq_decode_attn_workspace_size", "fsq_decode_attn", "fsq_workspace_status",
-            "fsq_status_string", "fsq_format_version", "fsq_decode_attn_noalloc")
+            "fsq_status_string", "fsq_format_version", "fsq_decode_attn_noalloc", "fsq_encode_status")
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -59,6 +59,8 @@ def _load() -> C.CDLL:
     lib.fsq_thresholds.restype = i32
     lib.fsq_encode_pack.argtypes = [vp, i64, i64, i64, vp, i32, QuantParams, vp, i64, vp]
     lib.fsq_encode_pack.restype = i32
+    lib.fsq_encode_status.argtypes = [vp]
+    lib.fsq_encode_status.restype = i32
     lib.fsq_quantize_pack_f32.argtypes = [vp, i64, i32, QuantParams, vp, i64, vp]
     lib.fsq_quantize_pack_f32.restype = i32
     lib.fsq_decode_attn_workspace_size.argtypes = [i64, i64, i32, i32, i32, i32, C.POINTER(AttnOpts)]
@@ -152,6 +154,11 @@ def decode_attn_noalloc_raw(q_ptr, B, n_q, d_h, codes_ptr, bstride, T, G, wkv_pt
                             stream_ptr) -> int:
     return lib.fsq_decode_attn_noalloc(q_ptr, B, n_q, d_h, codes_ptr, bstride, T, G, wkv_ptr, n_kv,
                                        None if opts is None else C.byref(opts), o_ptr, stream_ptr)
+
+
+def encode_status(stream=None) -> int:
+    """Reads and clears the append path's device error word (blocking)."""
+    return lib.fsq_encode_status(_stream_ptr(stream))
 
 
 def workspace_status(ws, stream=None) -> int:

@@ -10,6 +10,7 @@
 namespace fsq {
 cudaError_t launch_encode_pack_simt(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C, const uint16_t *E,
                                     int G, const Thresholds &th, uint8_t *codes, int64_t ldc, cudaStream_t s);
+cudaError_t encode_status(uint32_t *out, cudaStream_t s);
 cudaError_t launch_quantize_pack_f32(const float *u, int64_t n_tok, int G, const Thresholds &th, uint8_t *codes,
                                      int64_t ldc, cudaStream_t s);
 cudaError_t launch_absorbed_simt(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
@@ -174,6 +175,12 @@ fsq_status fsq_encode_pack(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_
   Thresholds th;
   make_thresholds(qp, th.th);
   return from_cuda(launch_encode_pack_simt(x, n_tok, ldx, C, E, G, th, codes, ldc_bytes, (cudaStream_t)stream));
+}
+
+fsq_status fsq_encode_status(fsq_stream_t stream) {
+  uint32_t v = 0;
+  if (encode_status(&v, (cudaStream_t)stream) != cudaSuccess) return FSQ_ERR_CUDA;
+  return v == 0 ? FSQ_OK : (fsq_status)(-(int)v);
 }
 
 fsq_status fsq_quantize_pack_f32(const float *u, int64_t n_tok, int G, fsq_quant_params qp, uint8_t *codes,

@@ -1,5 +1,5 @@
-// Append path, portable SIMT kernels: u = E x (fp32), FSQ threshold count,
-// nibble packing.  Transformer-FSQ summary, Methodology/Architecture eq. (4);
+// Append path for decode-step token counts (CUDA cores): u = E x (fp32), FSQ
+// threshold count, nibble packing.  Transformer-FSQ summary, Methodology/Architecture eq. (4);
 // Theoretical Basis eq. (2); slide deck frame "A wide product code uses four
 // bits per coordinate" (ceil(G*b/8) bytes per token).
 #include "common.cuh"
@@ -7,57 +7,6 @@
 namespace fsq {
 
 namespace {
-
-constexpr int kEncTok = 32;  // tokens per CTA
-constexpr int kEncK = 32;    // K (= C) chunk
-
-__global__ void __launch_bounds__(256) encode_pack_simt(const uint16_t *__restrict__ x, int64_t n_tok,
-                                                        int64_t ldx, int64_t C,
-                                                        const uint16_t *__restrict__ E, int G,
-                                                        Thresholds th, uint8_t *__restrict__ codes,
-                                                        int64_t ldc) {
-  __shared__ float xs[kEncTok][kEncK + 1];
-  __shared__ float es[kEncK][FSQ_MAX_G];
-  __shared__ uint8_t nib[kEncTok][FSQ_MAX_G];
-  const int tid = threadIdx.x;
-  const int64_t tok0 = (int64_t)blockIdx.x * kEncTok;
-  float acc[kEncTok];
-#pragma unroll
-  for (int i = 0; i < kEncTok; ++i) acc[i] = 0.f;
-
-  for (int64_t k0 = 0; k0 < C; k0 += kEncK) {
-    for (int i = tid; i < kEncTok * kEncK; i += blockDim.x) {
-      int t = i / kEncK, k = i % kEncK;
-      int64_t tt = tok0 + t;
-      xs[t][k] = (tt < n_tok) ? bf16_to_f32(x[tt * ldx + k0 + k]) : 0.f;
-    }
-    for (int i = tid; i < kEncK * G; i += blockDim.x) {
-      int g = i / kEncK, k = i % kEncK;
-      es[k][g] = bf16_to_f32(E[(int64_t)g * C + k0 + k]);
-    }
-    __syncthreads();
-    if (tid < G) {
-#pragma unroll 4
-      for (int k = 0; k < kEncK; ++k) {
-        float e = es[k][tid];
-#pragma unroll
-        for (int t = 0; t < kEncTok; ++t) acc[t] = fmaf(xs[t][k], e, acc[t]);
-      }
-    }
-    __syncthreads();
-  }
-  if (tid < G) {
-#pragma unroll
-    for (int t = 0; t < kEncTok; ++t) nib[t][tid] = (uint8_t)fsq_nibble(acc[t], th);
-  }
-  __syncthreads();
-  const int half = G / 2;
-  for (int i = tid; i < kEncTok * half; i += blockDim.x) {
-    int t = i / half, b = i % half;
-    int64_t tt = tok0 + t;
-    if (tt < n_tok) codes[tt * ldc + b] = (uint8_t)(nib[t][2 * b] | (nib[t][2 * b + 1] << 4));
-  }
-}
 
 // Few-token append (a decode step appends one token per batch row): one warp
 // per (token, byte), i.e. per pair of coordinates (2i, 2i+1); 16-byte loads of
@@ -176,6 +125,11 @@ __global__ void quantize_pack_f32_kernel(const float *__restrict__ u, int64_t n_
 
 }  // namespace
 
+cudaError_t launch_encode_pack_tc(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C, const uint16_t *E, int G,
+                                  const Thresholds &th, uint8_t *codes, int64_t ldc, cudaStream_t s);
+
+// Decode-step appends (up to 64 tokens) on CUDA cores; prefill-sized ones on
+// the tensor cores (encode_tc.cu).
 cudaError_t launch_encode_pack_simt(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C,
                                     const uint16_t *E, int G, const Thresholds &th, uint8_t *codes,
                                     int64_t ldc, cudaStream_t s) {
@@ -188,9 +142,7 @@ cudaError_t launch_encode_pack_simt(const uint16_t *x, int64_t n_tok, int64_t ld
     encode_pack_rows<<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(x, n_tok, ldx, C, E, G, th, codes, ldc);
     return cudaGetLastError();
   }
-  dim3 grid((unsigned)((n_tok + kEncTok - 1) / kEncTok));
-  encode_pack_simt<<<grid, 256, 0, s>>>(x, n_tok, ldx, C, E, G, th, codes, ldc);
-  return cudaGetLastError();
+  return launch_encode_pack_tc(x, n_tok, ldx, C, E, G, th, codes, ldc, s);
 }
 
 cudaError_t launch_quantize_pack_f32(const float *u, int64_t n_tok, int G, const Thresholds &th,

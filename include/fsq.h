@@ -18,14 +18,22 @@
  *
  * Conventions shared by every call
  *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
- *    never allocates device memory, never synchronises the host (except
- *    fsq_workspace_status, which says so) and keeps no global state.
+ *    never allocates device memory at run time and never synchronises the
+ *    host (except fsq_workspace_status and fsq_encode_status, which say so).
+ *    Its only device state is the error word of the append path and the
+ *    scratch of fsq_decode_attn_noalloc (file-scope arrays of the library).
  *  - bf16 means IEEE bfloat16 stored as uint16; row-major throughout.
  *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default).
  *  - Argument errors are returned synchronously, before anything is
  *    launched.  A failed launch returns FSQ_ERR_CUDA.  A bounded device-side
- *    wait that gives up records FSQ_ERR_TIMEOUT in the workspace's error word
- *    (see fsq_workspace_status) instead of hanging or trapping.
+ *    wait that gives up records FSQ_ERR_TIMEOUT (in the workspace's error
+ *    word, see fsq_workspace_status; for the append path see
+ *    fsq_encode_status) instead of hanging or trapping.
+ *  - The decode kernels use programmatic dependent launch: the first of
+ *    them may start before the kernel preceding the call on the stream has
+ *    finished, and reads q and W_kv early.  If that kernel is itself a
+ *    programmatic-launch primary (it executes griddepcontrol.launch_dependents)
+ *    it must not write q or W_kv.  Ordinary kernels are unaffected.
  *
  * Cache format (FSQ_FORMAT_VERSION 1)
  *  - A token's G levels z_i in {-8..7} are stored as nibbles n_i = z_i + 8.
@@ -122,6 +130,13 @@ FSQ_API fsq_status fsq_thresholds(fsq_quant_params qp, float theta_out[15]);
 FSQ_API fsq_status fsq_encode_pack(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C,
                            const uint16_t *E, int G, fsq_quant_params qp,
                            uint8_t *codes, int64_t ldc_bytes, fsq_stream_t stream);
+
+/* Reads and clears the device error word of the append path's tensor-core
+ * kernel (used by fsq_encode_pack for more than 64 tokens) on the current
+ * device.  Returns FSQ_OK, the recorded device status (FSQ_ERR_TIMEOUT: a
+ * bounded wait gave up, the codes of that call are incomplete), or
+ * FSQ_ERR_CUDA.  Blocking: synchronises with `stream` first. */
+FSQ_API fsq_status fsq_encode_status(fsq_stream_t stream);
 
 /* Quantiser + packing alone on given fp32 pre-activations u [n_tok, G]
  * (row-major, contiguous).  Same codes as fsq_encode_pack would write for

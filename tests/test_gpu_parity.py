@@ -203,6 +203,7 @@ def test_workload_append_leg(name):
     F.encode_pack(_dev(x), _dev(E), out=cache[T0:T0 + wl.n_new])
     got = cache.cpu().numpy()
     assert (got[:T0] == 0).all() and (got[T0 + wl.n_new:] == 0).all()
+    assert F.encode_status() == F.FSQ_OK  # no device wait gave up
     lv_r, u = O.encode(x.float().numpy(), E.float().numpy())
     bad = O.unpack(got[T0:T0 + wl.n_new], wl.G) != lv_r
     assert bad.sum() <= max(2, lv_r.size // 2000)
