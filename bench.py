@@ -383,6 +383,36 @@ def sdpa_context(torch, B, T, n_q, n_kv, d_h, device, steps=20, warmup=3):
                     "enable_gqa=True; inputs larger than L2"}
 
 
+def append_prefill(torch, F, synth, wl, device, peaks, n_new=4096, reps=20):
+    """The append leg of a chunked prefill: fsq_encode_pack of n_new tokens
+    (encoder GEMM -> FSQ -> pack) into a cache slice; x rotates over copies
+    larger than L2 in total."""
+    C, G = wl.C, wl.G
+    gen = torch.Generator(device=device)
+    gen.manual_seed(synth.workload_seed(0, n_new, C, G))
+    E = synth.normal((G, C), (4.0 / C) ** 0.5, gen, device=device)
+    xb = n_new * C * 2
+    ncop = max(2, min(8, math.ceil(2 * L2_BYTES / xb)))
+    xs = [synth.normal((n_new, C), 1.0, gen, device=device) for _ in range(ncop)]
+    out = torch.empty((n_new, G // 2), dtype=torch.uint8, device=device)
+    for i in range(3):
+        F.encode_pack(xs[i % ncop], E, out=out)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(reps):
+        F.encode_pack(xs[i % ncop], E, out=out)
+    b.record()
+    torch.cuda.synchronize()
+    t = a.elapsed_time(b) / reps * 1e-3
+    flops = 2.0 * n_new * C * G
+    nbytes = xb + G * C * 2 + n_new * G // 2
+    t_roof = max(flops / (peaks["bf16_tflops"] * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9))
+    return {"what": f"fsq_encode_pack of {n_new} tokens, C={C}, G={G} (bf16 x bf16 -> fp32 on tcgen05, FSQ, pack)",
+            "us_per_call": t * 1e6, "tokens_per_s": n_new / t, "tflops": flops / t / 1e12, "gbs": nbytes / t / 1e9,
+            "frac_of_roofline": t_roof / t, "l2": f"{ncop} rotating x copies"}
+
+
 def cpu_baseline_oracle(wl_name, T, budget_s=20.0):
     """The fp64 oracle as it stands, timed on one batch row of the workload."""
     Ts = min(T, 8192)
@@ -435,6 +465,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-second", action="store_true", help="skip the G=84 companion measurement")
     ap.add_argument("--no-sdpa", action="store_true", help="skip the uncompressed-cache SDPA context measurement")
+    ap.add_argument("--no-append", action="store_true", help="skip the 4096-token prefill append measurement")
     args = ap.parse_args()
     rank, world, local = dist_env()
     wl_name = args.workload
@@ -487,6 +518,9 @@ def main():
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = cpu_baseline_oracle(wl_name, T)
+    appf = None
+    if rank == 0 and not args.no_append:
+        appf = append_prefill(torch, F, synth, wl, device, peaks)
     sdpa = None
     if rank == 0 and not args.no_sdpa:
         sdpa = sdpa_context(torch, B, T, wl.n_q, wl.n_kv, wl.d_h, device)
@@ -512,7 +546,7 @@ def main():
                 "data": "synthetic (seeded; cache = FSQ codes of u ~ N(0,4), the law of E x; new token x ~ N(0,1) appended each step)",
                 "config": config, "code_gbs": world * res["code_bytes"] / (res["ms"] * 1e-3) / 1e9,
                 "roofline": rf, "cpu_baseline": cb, "e2e": res["e2e"], "clocks": res["clocks"],
-                "gpu_launches": args.steps * 4, "also": also, "sdpa_context": sdpa}
+                "gpu_launches": args.steps * 4, "also": also, "sdpa_context": sdpa, "append_prefill": appf}
         print(json.dumps(line))
     if dist is not None:
         dist.barrier()
