@@ -62,7 +62,7 @@ constexpr int kQAfterTiles = 4;                    // code tiles requested befor
 constexpr float kTau = 8.f;                        // rescale when a score exceeds the running max by 2^8
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s per wait
 constexpr int kMiscBytes = 12288;                  // shared-memory reservation for the Misc block
-constexpr int kPBufs = 4;                          // ring of softmax-weight (P) tiles in shared memory
+constexpr int kPBufs = 8;                          // ring of softmax-weight (P) tiles in shared memory
 
 template <int G, int NQ>
 struct Cfg {
