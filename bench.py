@@ -153,6 +153,27 @@ class RawEvents:
             self.rt.cudaEventDestroy(self.ct.c_void_p(b))
 
 
+def max_over_ranks(torch, dist, values, device):
+    """Element-wise maximum of per-rank timings (ms) over all ranks; the
+    values unchanged when there is no process group."""
+    if dist is None:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput(world, B, T, ms):
+    """Whole-job context tokens/s: every rank owns B rows of T tokens and a
+    step takes ms (the slowest rank's time)."""
+    return world * B * T / (ms * 1e-3)
+
+
+def rank_seed(synth, rank, B, T, G):
+    """Seed of a rank's inputs: each rank draws its own batch rows."""
+    return synth.workload_seed(0, rank, B, T, G)
+
+
 def dist_env():
     return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
 
@@ -169,7 +190,7 @@ def build_state(torch, F, synth, wl, B, T, rank, device, n_copies):
     T_max = T
     while (T_max * half) % 16:
         T_max += 1
-    seed = synth.workload_seed(0, rank, B, T, G)
+    seed = rank_seed(synth, rank, B, T, G)
     gen = torch.Generator(device=device)
     gen.manual_seed(seed)
     E = synth.normal((G, C), (4.0 / C) ** 0.5, gen, device=device)
@@ -251,10 +272,7 @@ def run_gpu(args, wl_name, B, T, torch, F, synth, dist, rank, world, device, tim
     clk = clocks.stop() if clocks else None
     kern_ms = sum(evs.elapsed_ms(i) for i in range(K)) / K
     evs.close()
-    if dist is not None:
-        t = torch.tensor([ms, kern_ms], device=device, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, kern_ms = float(t[0]), float(t[1])
+    ms, kern_ms = max_over_ranks(torch, dist, [ms, kern_ms], device)
 
     # end to end through the public API with host buffers
     e2e = None
@@ -292,11 +310,8 @@ def run_gpu(args, wl_name, B, T, torch, F, synth, dist, rank, world, device, tim
         b.record(stream)
         torch.cuda.synchronize()
         e_ms = a.elapsed_time(b) / K
-        if dist is not None:
-            t = torch.tensor([e_ms], device=device, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t[0])
-        e2e = {"value": world * B * T / (e_ms * 1e-3), "unit": "context tokens/s",
+        (e_ms,) = max_over_ranks(torch, dist, [e_ms], device)
+        e2e = {"value": job_throughput(world, B, T, e_ms), "unit": "context tokens/s",
                "h2d_bytes_per_step": q_h.numel() * 2 + x_h.numel() * 2, "d2h_bytes_per_step": o_h.numel() * 2,
                "ms_per_step": e_ms}
     return dict(ms=ms, kern_ms=kern_ms, clocks=clk, e2e=e2e, n_copies=n_copies, wl=wl, B=B, T=T,
@@ -512,7 +527,7 @@ def main():
                      world, device, timed=False)
         rf2 = roofline(r2, peaks, kernel_name)
         also = {"workload": f"{SECOND_WORKLOAD[0]} B={SECOND_WORKLOAD[1]} T={SECOND_WORKLOAD[2]} G=84",
-                "value": world * r2["B"] * r2["T"] / (r2["ms"] * 1e-3), "unit": "context tokens/s",
+                "value": job_throughput(world, r2["B"], r2["T"], r2["ms"]), "unit": "context tokens/s",
                 "ms_per_step": r2["ms"], "code_gbs": rf2["code_gbs"], "roofline": rf2,
                 "l2": f"{r2['n_copies']} rotating caches"}
     cb = None
@@ -535,7 +550,7 @@ def main():
             also["paper"] = dict(PAPER_SDPA_RATIOS[84], what=sdpa["paper"]["what"]) if "paper" in sdpa else None
     if rank == 0:
         rf = roofline(res, peaks, kernel_name)
-        value = world * B * T / (res["ms"] * 1e-3)
+        value = job_throughput(world, B, T, res["ms"])
         config["l2"] = ("codes larger than L2 (%.0f MB per cache)" % (res["code_bytes"] / 1e6) if res["n_copies"] == 1
                         else f"{res['n_copies']} rotating caches > 2x L2")
         line = {"metric": "FSQ decode-attn context tok/s & code GB/s, Qwen3-8B G=256/84; % roofline",
