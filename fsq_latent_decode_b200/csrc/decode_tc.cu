@@ -164,28 +164,17 @@ __device__ __forceinline__ void mma_ts_i8(uint32_t d_tmem, uint32_t a_tmem, uint
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-// The same instructions issued by one elected lane of a converged warp, so
-// that the whole warp runs the issue loop on warp-uniform operands.
-__device__ __forceinline__ void mma_ts_i8_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                                uint32_t accumulate) {
+// One lane of a converged warp (elect.sync)
+__device__ __forceinline__ bool elect_one() {
+  uint32_t e;
   asm volatile(
-      "{\n\t.reg .pred e, p;\n\t"
+      "{\n\t.reg .pred e;\n\t"
       "elect.sync _|e, 0xffffffff;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
+      "selp.u32 %0, 1, 0, e;\n\t}"
+      : "=r"(e));
+  return e != 0;
 }
-__device__ __forceinline__ void mma_ts_f16_elect(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                                 uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred e, p;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
+// A commit issued by one elected lane of a converged warp
 __device__ __forceinline__ void tc_commit_elect(uint64_t *bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"
@@ -260,6 +249,37 @@ __device__ __forceinline__ bool bar_try(uint32_t a, uint32_t parity, uint32_t hi
       : "memory");
   return ok != 0;
 }
+// Tests of two or three phases at once: the tests are independent, so their
+// shared-memory round trips overlap (a completed hand-off costs one of them)
+__device__ __forceinline__ bool bar_test2(uint32_t a0, uint32_t p0, uint32_t a1, uint32_t p1) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 q, [%3], %4;\n\t"
+      "and.pred p, p, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(a0), "r"(p0), "r"(a1), "r"(p1)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool bar_test3(uint32_t a0, uint32_t p0, uint32_t a1, uint32_t p1, uint32_t a2,
+                                          uint32_t p2) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p, q, r;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 q, [%3], %4;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 r, [%5], %6;\n\t"
+      "and.pred p, p, q;\n\t"
+      "and.pred p, p, r;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(a0), "r"(p0), "r"(a1), "r"(p1), "r"(a2), "r"(p2)
+      : "memory");
+  return ok != 0;
+}
 __device__ __forceinline__ bool wait_bar(uint64_t *b, uint32_t parity, volatile uint32_t *abort, uint64_t limit_ns) {
   const uint32_t a = smem_u32(b);
   if (bar_test(a, parity)) return true;
@@ -271,6 +291,17 @@ __device__ __forceinline__ bool wait_bar(uint64_t *b, uint32_t parity, volatile 
       if (globaltimer_ns() - t0 > limit_ns) return false;
     }
   }
+}
+// Waits for two (three) phases: one combined test, then each in turn
+__device__ __forceinline__ bool wait_bars(uint64_t *b0, uint32_t p0, uint64_t *b1, uint32_t p1,
+                                          volatile uint32_t *abort, uint64_t limit_ns) {
+  if (bar_test2(smem_u32(b0), p0, smem_u32(b1), p1)) return true;
+  return wait_bar(b0, p0, abort, limit_ns) && wait_bar(b1, p1, abort, limit_ns);
+}
+__device__ __forceinline__ bool wait_bars(uint64_t *b0, uint32_t p0, uint64_t *b1, uint32_t p1, uint64_t *b2,
+                                          uint32_t p2, volatile uint32_t *abort, uint64_t limit_ns) {
+  if (bar_test3(smem_u32(b0), p0, smem_u32(b1), p1, smem_u32(b2), p2)) return true;
+  return wait_bar(b0, p0, abort, limit_ns) && wait_bar(b1, p1, abort, limit_ns) && wait_bar(b2, p2, abort, limit_ns);
 }
 
 // Named barrier over `nthreads` threads that returns the OR of `pred` over them.
@@ -457,18 +488,20 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
       const int sb = i & 1;
       // S(i) is released to the softmax only once P buffer i % kPBufs is free
       // again (pooling of tile i - kPBufs done), so the softmax never waits for it
-      ok = wait_bar(&ms.cs_ready[sb], (uint32_t)(i >> 1) & 1u, abort, p.wait_ns) &&
-           wait_bar(&ms.s_free[sb], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort, p.wait_ns) &&
-           wait_bar(&ms.p_free[i % kPBufs], ((uint32_t)(i / kPBufs) & 1u) ^ 1u, abort, p.wait_ns);
+      ok = wait_bars(&ms.cs_ready[sb], (uint32_t)(i >> 1) & 1u, &ms.s_free[sb], ((uint32_t)(i >> 1) & 1u) ^ 1u,
+                     &ms.p_free[i % kPBufs], ((uint32_t)(i / kPBufs) & 1u) ^ 1u, abort, p.wait_ns);
       if (!ok) break;
       tc_fence_after();
       const uint32_t a0 = tm + C::OFF_CS + sb * C::CS_COLS;
       const uint32_t d = tm + C::OFF_S + sb * C::NS;
+      if (elect_one()) {  // one lane issues the tile's MMAs and both commits
 #pragma unroll
-      for (int k = 0; k < C::KPAD / 32; ++k)
-        mma_ts_i8_elect(d, a0 + k * 8, qd0 + (uint64_t)((k * 2 * C::LBO_Q) >> 4), id_s, k > 0 ? 1u : 0u);
-      tc_commit_elect(&ms.s_full[sb]);
-      tc_commit_elect(&ms.cs_free[sb]);
+        for (int k = 0; k < C::KPAD / 32; ++k)
+          mma_ts_i8(d, a0 + k * 8, qd0 + (uint64_t)((k * 2 * C::LBO_Q) >> 4), id_s, k > 0 ? 1u : 0u);
+        tc_commit(&ms.s_full[sb]);
+        tc_commit(&ms.cs_free[sb]);
+      }
+      __syncwarp();
     }
     if (!ok && lane == 0) fail();
     tc_commit_elect(&ms.done[0]);
@@ -494,12 +527,15 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
         tc_fence_after();
         const uint32_t a0 = tm + C::OFF_CP + cb * C::CP_CHUNK + h * 32;
         const uint64_t bd0 = pd0 + (uint64_t)((pb * C::P_BYTES + 4 * c * 256) >> 4);
+        if (elect_one()) {  // one lane issues the chunk's MMAs and its commit
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const bool first = (i == 0) && (C::NH == 1 ? kk == 0 : (c == 0 && kk == 0));
-          mma_ts_f16_elect(d, a0 + kk * 8, bd0 + (uint64_t)(kk * 16), id_p, first ? 0u : 1u);
+          for (int kk = 0; kk < 4; ++kk) {
+            const bool first = (i == 0) && (C::NH == 1 ? kk == 0 : (c == 0 && kk == 0));
+            mma_ts(d, a0 + kk * 8, bd0 + (uint64_t)(kk * 16), id_p, first ? 0u : 1u);
+          }
+          tc_commit(&ms.cp_free[cb]);
         }
-        tc_commit_elect(&ms.cp_free[cb]);
+        __syncwarp();
       }
       if (!ok) break;
       tc_commit_elect(&ms.p_free[pb]);
@@ -516,8 +552,8 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
     for (int i = 0; i < n_tiles; ++i) {
       const int st = i % C::STAGES, sb = i & 1;
       const uint8_t *tile = smem + C::SM_CODES + st * C::STAGE_BYTES;
-      if (!wait_bar(&ms.full[st], (uint32_t)(i / C::STAGES) & 1u, abort, p.wait_ns) ||
-          !wait_bar(&ms.cs_free[sb], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort, p.wait_ns)) {
+      if (!wait_bars(&ms.full[st], (uint32_t)(i / C::STAGES) & 1u, &ms.cs_free[sb], ((uint32_t)(i >> 1) & 1u) ^ 1u,
+                     abort, p.wait_ns)) {
         ok = false;
         break;
       }
@@ -577,8 +613,8 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
       const int kc = 2 * i + c;
       const int cb = kc % C::NCP;
       const uint8_t *tile = smem + C::SM_CODES + st * C::STAGE_BYTES;
-      if (!wait_bar(&ms.full[st], (uint32_t)(i / C::STAGES) & 1u, abort, p.wait_ns) ||
-          !wait_bar(&ms.cp_free[cb], ((uint32_t)(kc / C::NCP) & 1u) ^ 1u, abort, p.wait_ns)) {
+      if (!wait_bars(&ms.full[st], (uint32_t)(i / C::STAGES) & 1u, &ms.cp_free[cb], ((uint32_t)(kc / C::NCP) & 1u) ^ 1u,
+                     abort, p.wait_ns)) {
         ok = false;
         break;
       }
