@@ -209,11 +209,28 @@ __device__ __forceinline__ float ex2_approx(float x) {
 // 128-byte-swizzle layout of a TMA tile: 16-byte chunk c of row r sits at chunk c ^ (r % 8).
 __device__ __forceinline__ int swz(int r, int chunk) { return r * 128 + ((chunk ^ (r & 7)) << 4); }
 
-__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int c0, int c1, int c2, uint64_t *bar) {
+// L2 policy for the code stream, which every call reads once: evict it
+// first, so that it does not push out of L2 the small operands each call
+// re-reads (E, W_kv, the partials)
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int c0, int c1, int c2, uint64_t *bar,
+                                            uint64_t pol) {
   asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
-      "[%5];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar)), "l"(pol)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_g2s_hint(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
+                                              uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
       : "memory");
 }
 
@@ -428,6 +445,7 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
     // The codes were written before the query prologue kernel started, so the
     // first ring-full of tiles is requested before waiting for that kernel;
     // Q' (its output) right after, before the first wait for a free stage.
+    const uint64_t pol = l2_evict_first();
     auto load_q = [&]() {
       if (lane == 0) {
         pdl_wait();
@@ -455,12 +473,12 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
         // rows past T arrive as zeros; rows past this split's end are masked by the softmax
         if (lane == 0) {
           mbar_arrive_expect_tx(&ms.full[st], C::TILE_BYTES);
-          tma_load_3d(dst, &tmap, 0, (int)(t0 + (int64_t)i * kTile), b, &ms.full[st]);
+          tma_load_3d(dst, &tmap, 0, (int)(t0 + (int64_t)i * kTile), b, &ms.full[st], pol);
         }
       } else if (rows == kTile) {
         if (lane == 0) {
           mbar_arrive_expect_tx(&ms.full[st], C::TILE_BYTES);
-          bulk_g2s(dst, src, C::TILE_BYTES, &ms.full[st]);
+          bulk_g2s_hint(dst, src, C::TILE_BYTES, &ms.full[st], pol);
         }
       } else {
         // ragged tail: plain bounded loads, zero fill
@@ -702,11 +720,16 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
         const float4 sg = sg4[n4], cc = cm4[n4];
         const float sv[4] = {sg.x, sg.y, sg.z, sg.w}, cv[4] = {cc.x, cc.y, cc.z, cc.w};
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
+        for (int e = 0; e < 4; e += 2) {
           const int n = 4 * n4 + e;
-          const int y = (int)ra[n] * 128 + (int)rb[n];  // exact: |y| < 2^27
-          x[n] = fmaf((float)y, sv[e], -cv[e]);
-          lm = fmaxf(lm, x[n]);
+          const int y0 = (int)ra[n] * 128 + (int)rb[n];  // exact: |y| < 2^27
+          const int y1 = (int)ra[n + 1] * 128 + (int)rb[n + 1];
+          // two heads per packed FMA (each element rounded once, as fmaf)
+          const float2 xv = __ffma2_rn(make_float2((float)y0, (float)y1), make_float2(sv[e], sv[e + 1]),
+                                       make_float2(-cv[e], -cv[e + 1]));
+          x[n] = xv.x;
+          x[n + 1] = xv.y;
+          lm = fmaxf(lm, fmaxf(xv.x, xv.y));
         }
       }
       if ((t0 + (int64_t)i * kTile + r) >= t1) {
@@ -725,8 +748,9 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
       for (int k = 0; k < 4; ++k) {
         const float p0 = ex2_approx(x[2 * k]), p1 = ex2_approx(x[2 * k + 1]);
         const __half2 hv = __floats2half2_rn(p0, p1);
-        lsum[2 * k] += p0;
-        lsum[2 * k + 1] += p1;
+        const float2 ls = __fadd2_rn(make_float2(lsum[2 * k], lsum[2 * k + 1]), make_float2(p0, p1));
+        lsum[2 * k] = ls.x;
+        lsum[2 * k + 1] = ls.y;
         h2[k] = *reinterpret_cast<const uint32_t *>(&hv);
       }
       *reinterpret_cast<uint4 *>(prow) = make_uint4(h2[0], h2[1], h2[2], h2[3]);
@@ -940,6 +964,12 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::KPAD * AbsorbShape<GRP>::NDQ)
     if (threadIdx.x == 0) *err = 0u;
     for (int i = threadIdx.x; i < ms.ncnt; i += blockDim.x) ms.cnt[i] = 0u;  // the merge's arrival counts
   }
+  // the first batch of W_k rows is requested before q, so that the two
+  // loads' latencies overlap
+  const uint16_t *wk = W_kv + ((int64_t)j * D + dq * DS) * G + min(g, G - 1);
+  uint16_t wraw[kBatch];
+#pragma unroll
+  for (int u = 0; u < kBatch; ++u) wraw[u] = wk[(int64_t)u * G];
   for (int i = threadIdx.x; i < GRP * D; i += blockDim.x)
     qs[i / D][i % D] = bf16_to_f32(q[((int64_t)b * NQ + j * GRP) * D + i]);
   __syncthreads();
@@ -947,12 +977,15 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::KPAD * AbsorbShape<GRP>::NDQ)
 #pragma unroll
   for (int hh = 0; hh < GRP; ++hh) v[hh] = 0.f;
   if (g < G) {
-    const uint16_t *wk = W_kv + ((int64_t)j * D + dq * DS) * G + g;
 #pragma unroll 1
     for (int d0 = 0; d0 < DS; d0 += kBatch) {
       float w[kBatch];
+      if (d0 > 0) {
 #pragma unroll
-      for (int u = 0; u < kBatch; ++u) w[u] = bf16_to_f32(wk[(int64_t)(d0 + u) * G]);
+        for (int u = 0; u < kBatch; ++u) wraw[u] = wk[(int64_t)(d0 + u) * G];
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) w[u] = bf16_to_f32(wraw[u]);
 #pragma unroll
       for (int u = 0; u < kBatch; u += 4)
 #pragma unroll

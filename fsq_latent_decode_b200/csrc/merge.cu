@@ -106,26 +106,29 @@ __device__ __forceinline__ void apply_wv(const uint16_t *wv, const float *abar, 
   const int d = threadIdx.x % D, part = threadIdx.x / D;
   const int gq = GP / kParts;  // a multiple of 8
   const uint16_t *wr = wv + d * WS + part * gq;
-  float acc[GRP];
+  // even and odd coordinates accumulate in the two lanes of packed fp32x2 FMAs
+  float2 acc2[GRP];
 #pragma unroll
-  for (int h = 0; h < GRP; ++h) acc[h] = 0.f;
+  for (int h = 0; h < GRP; ++h) acc2[h] = make_float2(0.f, 0.f);
   for (int g8 = 0; g8 < gq; g8 += 8) {
     const uint4 wq = *reinterpret_cast<const uint4 *>(wr + g8);
     const uint32_t wp[4] = {wq.x, wq.y, wq.z, wq.w};
-    float wf[8];
+    float2 wf[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      wf[2 * e] = __uint_as_float(wp[e] << 16);
-      wf[2 * e + 1] = __uint_as_float(wp[e] & 0xFFFF0000u);
-    }
+    for (int e = 0; e < 4; ++e) wf[e] = make_float2(__uint_as_float(wp[e] << 16), __uint_as_float(wp[e] & 0xFFFF0000u));
 #pragma unroll
     for (int h = 0; h < GRP; ++h) {
       const float4 lo = *reinterpret_cast<const float4 *>(abar + h * GP + part * gq + g8);
       const float4 hi = *reinterpret_cast<const float4 *>(abar + h * GP + part * gq + g8 + 4);
-      acc[h] = fmaf(wf[0], lo.x, fmaf(wf[1], lo.y, fmaf(wf[2], lo.z, fmaf(wf[3], lo.w, acc[h]))));
-      acc[h] = fmaf(wf[4], hi.x, fmaf(wf[5], hi.y, fmaf(wf[6], hi.z, fmaf(wf[7], hi.w, acc[h]))));
+      acc2[h] = __ffma2_rn(wf[0], make_float2(lo.x, lo.y), acc2[h]);
+      acc2[h] = __ffma2_rn(wf[1], make_float2(lo.z, lo.w), acc2[h]);
+      acc2[h] = __ffma2_rn(wf[2], make_float2(hi.x, hi.y), acc2[h]);
+      acc2[h] = __ffma2_rn(wf[3], make_float2(hi.z, hi.w), acc2[h]);
     }
   }
+  float acc[GRP];
+#pragma unroll
+  for (int h = 0; h < GRP; ++h) acc[h] = acc2[h].x + acc2[h].y;
   if (part > 0) {
 #pragma unroll
     for (int h = 0; h < GRP; ++h) scr[((part - 1) * GRP + h) * D + d] = acc[h];
@@ -150,37 +153,62 @@ struct Lse {
   float2 a;
 };
 
+// 2^x on the special-function unit (x <= 0 here; -inf gives 0)
+__device__ __forceinline__ float ex2_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // Fold splits s0, s0 + ds, ... below S of one head's records (rec: the
 // head's record in split 0; sstride: floats between splits; gi: the pair's
-// offset) into st.
+// offset) into st.  A batch of up to kBatch splits is folded at once: its
+// maximum first, then one exponential per split, so the weighted sums of the
+// batch do not wait on one another.
+template <int NB>
+__device__ __forceinline__ void fold_batch(Lse &st, const float *__restrict__ rec, int64_t sstride, int gi, int s,
+                                           int ds, int S) {
+  float2 ml[NB], av[NB];
+#pragma unroll
+  for (int u = 0; u < NB; ++u) {
+    const bool in = s + u * ds < S;
+    const float *r = rec + (int64_t)(s + u * ds) * sstride;
+    ml[u] = in ? *reinterpret_cast<const float2 *>(r) : make_float2(-INFINITY, 0.f);
+    av[u] = in ? *reinterpret_cast<const float2 *>(r + 2 + gi) : make_float2(0.f, 0.f);
+  }
+  float mn = st.m;
+#pragma unroll
+  for (int u = 0; u < NB; ++u) mn = fmaxf(mn, ml[u].x);
+  if (mn == -INFINITY) return;  // nothing folded yet and only empty splits
+  const float co = ex2_fast(st.m - mn);
+  float l = st.l * co, ax = st.a.x * co, ay = st.a.y * co;
+#pragma unroll
+  for (int u = 0; u < NB; ++u) {
+    const float cs = ex2_fast(ml[u].x - mn);  // 0 for an empty slot
+    l = fmaf(ml[u].y, cs, l);
+    ax = fmaf(av[u].x, cs, ax);
+    ay = fmaf(av[u].y, cs, ay);
+  }
+  st.m = mn;
+  st.l = l;
+  st.a = make_float2(ax, ay);
+}
 __device__ __forceinline__ void fold_splits(Lse &st, const float *__restrict__ rec, int64_t sstride, int gi, int s0,
                                             int ds, int S) {
-  for (int s = s0; s < S; s += kBatch * ds) {
-    float2 ml[kBatch], av[kBatch];
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const bool in = s + u * ds < S;
-      const float *r = rec + (int64_t)(s + u * ds) * sstride;
-      ml[u] = in ? *reinterpret_cast<const float2 *>(r) : make_float2(-INFINITY, 0.f);
-      av[u] = in ? *reinterpret_cast<const float2 *>(r + 2 + gi) : make_float2(0.f, 0.f);
-    }
-#pragma unroll
-    for (int u = 0; u < kBatch; ++u) {
-      const float mn = fmaxf(st.m, ml[u].x);
-      if (mn == -INFINITY) continue;  // nothing folded yet and an empty slot
-      const float co = exp2f(st.m - mn), cs = exp2f(ml[u].x - mn);
-      st.l = fmaf(st.l, co, ml[u].y * cs);
-      st.a.x = fmaf(st.a.x, co, av[u].x * cs);
-      st.a.y = fmaf(st.a.y, co, av[u].y * cs);
-      st.m = mn;
-    }
+  const int n = (S - s0 + ds - 1) / ds;  // splits this thread folds
+  if (n <= 4) {
+    fold_batch<4>(st, rec, sstride, gi, s0, ds, S);
+  } else if (n <= 8) {
+    fold_batch<8>(st, rec, sstride, gi, s0, ds, S);
+  } else {
+    for (int s = s0; s < S; s += kBatch * ds) fold_batch<kBatch>(st, rec, sstride, gi, s, ds, S);
   }
 }
 
 __device__ __forceinline__ void fold_state(Lse &st, const float4 &o) {
   const float mn = fmaxf(st.m, o.x);
   if (mn == -INFINITY) return;
-  const float co = exp2f(st.m - mn), cs = exp2f(o.x - mn);
+  const float co = ex2_fast(st.m - mn), cs = ex2_fast(o.x - mn);
   st.l = fmaf(st.l, co, o.y * cs);
   st.a.x = fmaf(st.a.x, co, o.z * cs);
   st.a.y = fmaf(st.a.y, co, o.w * cs);
