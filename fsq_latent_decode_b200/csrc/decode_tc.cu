@@ -925,13 +925,27 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
 // kappa = 8w + 4e + i for coordinate 8w + 2i + e (the dequant's byte order).
 // corr[b] = [sigma_h] then [sigma_h * 8 * sum_g (128 a_g + b_g)]: the score is
 // sigma (128 S_a + S_b) - offset, the offset removing the +8 of the bytes.
-// Threads: KPAD coordinates x NDQ slices of the head dimension, so that every
-// thread has at most 32 rows of W_k^(j) to load (all issued at once); the
-// slices are summed in shared memory.
+// Threads: KPAD coordinates x NDQ slices of the head dimension.  W_k^(j)
+// is staged in shared memory by 16-byte asynchronous copies (requested before
+// q, so the two latencies overlap); thread (dq, g) sums its slice of the head
+// dimension for coordinate g, and after one exchange of the slices' sums
+// slice dq finishes heads dq, dq + NDQ, ... (scale, split into two int8 terms).
 template <int GRP>
 struct AbsorbShape {
   static constexpr int NDQ = GRP <= 4 ? 4 : (GRP == 8 ? 2 : 1);
 };
+template <int G, int NQ, int GRP>
+struct AbsorbSmem {
+  static constexpr int GS = Cfg<G, NQ>::KPAD;
+  static constexpr int NDQ = AbsorbShape<GRP>::NDQ;
+  static constexpr int W_BYTES = FSQ_HEAD_DIM * G * 2;          // W_k^(j), bf16 [D][G]
+  static constexpr int PART_OFF = (W_BYTES + 15) / 16 * 16;
+  static constexpr int BYTES = PART_OFF + NDQ * GRP * GS * 4;  // slice sums, fp32 [NDQ][GRP][GS]
+};
+
+__device__ __forceinline__ void cp_async16_g2s(void *smem_dst, const void *gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
 
 template <int G, int NQ, int GRP>
 __global__ void __launch_bounds__(Cfg<G, NQ>::KPAD * AbsorbShape<GRP>::NDQ)
@@ -939,20 +953,23 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::KPAD * AbsorbShape<GRP>::NDQ)
                     uint8_t *__restrict__ qphys, float *__restrict__ corr, uint32_t *err, MergeScratch ms) {
   // one CTA per (kv head j, batch row b): the group's heads share W_k^(j), read once
   using C = Cfg<G, NQ>;
+  using SM = AbsorbSmem<G, NQ, GRP>;
   constexpr int D = FSQ_HEAD_DIM;
-  constexpr int NDQ = AbsorbShape<GRP>::NDQ;
-  constexpr int GS = C::KPAD;       // threads per slice (one per padded coordinate)
+  constexpr int NDQ = SM::NDQ;
+  constexpr int GS = SM::GS;        // threads per slice (one per padded coordinate)
   constexpr int DS = D / NDQ;       // head-dimension rows per thread
-  constexpr int kBatch = DS < 32 ? DS : 32;
-  constexpr int NW = GS / 32;       // warps of slice 0
+  constexpr int NW = GS / 32;       // warps per slice
+  constexpr int NT = GS * NDQ;
+  extern __shared__ __align__(16) uint8_t asmem[];
+  const uint16_t *wks = reinterpret_cast<const uint16_t *>(asmem);
+  float *part = reinterpret_cast<float *>(asmem + SM::PART_OFF);
   __shared__ __align__(16) float qs[GRP][D];  // read as float4
-  __shared__ float part[NDQ > 1 ? NDQ - 1 : 1][GRP][GS];
   __shared__ float red[GRP][NW];
   __shared__ int ired[GRP][NW];
-  __shared__ float sig_s[GRP];
+  __shared__ float sig_s[GRP], inv_s[GRP];
   const int j = blockIdx.x, b = blockIdx.y;
   const int g = threadIdx.x % GS, dq = threadIdx.x / GS;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int wis = g >> 5, lane = threadIdx.x & 31;  // warp within the slice
   // Nothing here depends on the kernel before this one (q and W_kv are inputs
   // of the call; no kernel of this library that may still run writes them,
   // and the workspace is no longer read by the previous call's kernels, which
@@ -960,89 +977,82 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::KPAD * AbsorbShape<GRP>::NDQ)
   // of the step's new tokens in a decode step.  It waits for that kernel only
   // at the end, before releasing the split kernel, whose first code loads
   // precede its own wait.
+  {
+    const uint8_t *src = reinterpret_cast<const uint8_t *>(W_kv + (int64_t)j * D * G);
+    for (int k = threadIdx.x; k < SM::W_BYTES / 16; k += NT) cp_async16_g2s(asmem + 16 * k, src + 16 * k);
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
   if (j == 0 && b == 0) {
     if (threadIdx.x == 0) *err = 0u;
-    for (int i = threadIdx.x; i < ms.ncnt; i += blockDim.x) ms.cnt[i] = 0u;  // the merge's arrival counts
+    for (int i = threadIdx.x; i < ms.ncnt; i += NT) ms.cnt[i] = 0u;  // the merge's arrival counts
   }
-  // the first batch of W_k rows is requested before q, so that the two
-  // loads' latencies overlap
-  const uint16_t *wk = W_kv + ((int64_t)j * D + dq * DS) * G + min(g, G - 1);
-  uint16_t wraw[kBatch];
-#pragma unroll
-  for (int u = 0; u < kBatch; ++u) wraw[u] = wk[(int64_t)u * G];
-  for (int i = threadIdx.x; i < GRP * D; i += blockDim.x)
+  for (int i = threadIdx.x; i < GRP * D; i += NT)
     qs[i / D][i % D] = bf16_to_f32(q[((int64_t)b * NQ + j * GRP) * D + i]);
+  asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
   float v[GRP];
 #pragma unroll
   for (int hh = 0; hh < GRP; ++hh) v[hh] = 0.f;
   if (g < G) {
-#pragma unroll 1
-    for (int d0 = 0; d0 < DS; d0 += kBatch) {
-      float w[kBatch];
-      if (d0 > 0) {
+    const uint16_t *wk = wks + (dq * DS) * G + g;
+#pragma unroll 8
+    for (int u = 0; u < DS; u += 4) {
+      const float w0 = bf16_to_f32(wk[(u + 0) * G]), w1 = bf16_to_f32(wk[(u + 1) * G]);
+      const float w2 = bf16_to_f32(wk[(u + 2) * G]), w3 = bf16_to_f32(wk[(u + 3) * G]);
 #pragma unroll
-        for (int u = 0; u < kBatch; ++u) wraw[u] = wk[(int64_t)(d0 + u) * G];
+      for (int hh = 0; hh < GRP; ++hh) {
+        const float4 qv = *reinterpret_cast<const float4 *>(&qs[hh][dq * DS + u]);
+        v[hh] = fmaf(w0, qv.x, fmaf(w1, qv.y, fmaf(w2, qv.z, fmaf(w3, qv.w, v[hh]))));
       }
-#pragma unroll
-      for (int u = 0; u < kBatch; ++u) w[u] = bf16_to_f32(wraw[u]);
-#pragma unroll
-      for (int u = 0; u < kBatch; u += 4)
-#pragma unroll
-        for (int hh = 0; hh < GRP; ++hh) {
-          const float4 qv = *reinterpret_cast<const float4 *>(&qs[hh][dq * DS + d0 + u]);
-          v[hh] = fmaf(w[u], qv.x, fmaf(w[u + 1], qv.y, fmaf(w[u + 2], qv.z, fmaf(w[u + 3], qv.w, v[hh]))));
-        }
     }
   }
-  if (NDQ > 1) {
-    if (dq > 0) {
 #pragma unroll
-      for (int hh = 0; hh < GRP; ++hh) part[dq - 1][hh][g] = v[hh];
+  for (int hh = 0; hh < GRP; ++hh) part[(dq * GRP + hh) * GS + g] = v[hh];
+  __syncthreads();
+  // slice dq finishes heads dq, dq + NDQ, ...
+  constexpr int HPS = (GRP + NDQ - 1) / NDQ;  // heads per slice
+  float vf[HPS];
+#pragma unroll
+  for (int k = 0; k < HPS; ++k) {
+    const int hh = dq + k * NDQ;
+    float t = 0.f;
+    if (hh < GRP) {
+#pragma unroll
+      for (int i = 0; i < NDQ; ++i) t += part[(i * GRP + hh) * GS + g];
     }
-    __syncthreads();
-    if (dq == 0) {
+    vf[k] = t * c;
+    float am = fabsf(vf[k]);
 #pragma unroll
-      for (int i = 0; i < NDQ - 1; ++i)
-#pragma unroll
-        for (int hh = 0; hh < GRP; ++hh) v[hh] += part[i][hh][g];
-    }
-  }
-  if (dq == 0) {
-#pragma unroll
-    for (int hh = 0; hh < GRP; ++hh) {
-      v[hh] *= c;
-      float am = fabsf(v[hh]);
-#pragma unroll
-      for (int o = 16; o; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-      if (lane == 0) red[hh][warp] = am;
-    }
+    for (int o = 16; o; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+    if (lane == 0 && hh < GRP) red[hh][wis] = am;
   }
   __syncthreads();
   if (threadIdx.x < GRP) {
     float am = 0.f;
     for (int i = 0; i < NW; ++i) am = fmaxf(am, red[threadIdx.x][i]);
-    sig_s[threadIdx.x] = am > 0.f ? am / (127.f * 128.f) : 1.f;
+    const float sg = am > 0.f ? am / (127.f * 128.f) : 1.f;
+    sig_s[threadIdx.x] = sg;
+    inv_s[threadIdx.x] = 1.f / sg;
   }
   __syncthreads();
-  if (dq == 0) {
-    // coordinate g = 8w + 2i + e sits at K position kappa = 8w + 4e + i
-    const int kap = (g & ~7) | ((g & 1) << 2) | ((g >> 1) & 3);
-    uint8_t *dst = qphys + (size_t)b * C::Q_BYTES;
-    const int base = (kap >> 4) * C::LBO_Q + (kap & 15);
+  // coordinate g = 8w + 2i + e sits at K position kappa = 8w + 4e + i
+  const int kap = (g & ~7) | ((g & 1) << 2) | ((g >> 1) & 3);
+  uint8_t *dst = qphys + (size_t)b * C::Q_BYTES;
+  const int base = (kap >> 4) * C::LBO_Q + (kap & 15);
 #pragma unroll
-    for (int hh = 0; hh < GRP; ++hh) {
-      const int h = j * GRP + hh;
-      const float t = v[hh] / sig_s[hh];
-      const int a = max(-127, min(127, __float2int_rn(t / 128.f)));
-      const int bt = max(-127, min(127, __float2int_rn(t - 128.f * (float)a)));
-      int isum = 128 * a + bt;
-      dst[base + (h >> 3) * 128 + (h & 7) * 16] = (uint8_t)(int8_t)a;
-      dst[base + ((NQ + h) >> 3) * 128 + ((NQ + h) & 7) * 16] = (uint8_t)(int8_t)bt;
+  for (int k = 0; k < HPS; ++k) {
+    const int hh = dq + k * NDQ;
+    if (hh >= GRP) break;
+    const int h = j * GRP + hh;
+    const float t = vf[k] * inv_s[hh];
+    const int a = max(-127, min(127, __float2int_rn(t * (1.f / 128.f))));
+    const int bt = max(-127, min(127, __float2int_rn(t - 128.f * (float)a)));
+    int isum = 128 * a + bt;
+    dst[base + (h >> 3) * 128 + (h & 7) * 16] = (uint8_t)(int8_t)a;
+    dst[base + ((NQ + h) >> 3) * 128 + ((NQ + h) & 7) * 16] = (uint8_t)(int8_t)bt;
 #pragma unroll
-      for (int o = 16; o; o >>= 1) isum += __shfl_xor_sync(0xffffffffu, isum, o);
-      if (lane == 0) ired[hh][warp] = isum;
-    }
+    for (int o = 16; o; o >>= 1) isum += __shfl_xor_sync(0xffffffffu, isum, o);
+    if (lane == 0) ired[hh][wis] = isum;
   }
   __syncthreads();
   if (threadIdx.x < GRP) {
@@ -1059,8 +1069,11 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::KPAD * AbsorbShape<GRP>::NDQ)
 template <int G, int NQ, int GRP>
 cudaError_t absorb_query_launch(const dim3 &grid, const uint16_t *q, const uint16_t *W_kv, float c, uint8_t *qphys,
                                 float *corr, uint32_t *err, MergeScratch ms, cudaStream_t st) {
-  return launch_pdl(absorb_query_tc<G, NQ, GRP>, grid, dim3(Cfg<G, NQ>::KPAD * AbsorbShape<GRP>::NDQ), 0, st, q, W_kv,
-                    c, qphys, corr, err, ms);
+  using SM = AbsorbSmem<G, NQ, GRP>;
+  cudaError_t e = ensure_smem_limit((const void *)absorb_query_tc<G, NQ, GRP>, (size_t)SM::BYTES);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(absorb_query_tc<G, NQ, GRP>, grid, dim3(Cfg<G, NQ>::KPAD * AbsorbShape<GRP>::NDQ),
+                    (size_t)SM::BYTES, st, q, W_kv, c, qphys, corr, err, ms);
 }
 
 template <int G, int NQ>
