@@ -199,6 +199,13 @@ __device__ __forceinline__ int kappa_of_token(int r) {
   return (r & ~15) | (((r >> 1) & 3) << 2) | (((r >> 3) & 1) << 1) | (r & 1);
 }
 
+// max(a, b, c) in one instruction (three-input max.f32, sm_100)
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // 2^x on the special-function unit (inputs <= 8 here; -inf gives 0).
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
@@ -708,6 +715,10 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
     for (int n = 0; n < HQ; ++n) lsum[n] = 0.f;
     const int r = 32 * q + lane;        // token row within the tile
     const int kap = kappa_of_token(r);  // its K position in the pooling operand
+    // tiles i >= ilim hold this row past the split's end; only the last tile
+    // can, when the range is not a whole number of tiles (-1: none)
+    const int ilim = (int)min((int64_t)n_tiles, (t1 - t0 - r + kTile - 1) / kTile);
+    const int last_ragged = ((t1 - t0) % kTile) != 0 ? n_tiles - 1 : -1;
     static_assert(HQ == 8, "softmax warps own eight heads");
     // x <- score - m of one tile from its raw S (a, b terms); rows past the
     // split's end (ragged last tile only) take no weight; returns the row max
@@ -729,10 +740,10 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
                                        make_float2(-cv[e], -cv[e + 1]));
           x[n] = xv.x;
           x[n + 1] = xv.y;
-          lm = fmaxf(lm, fmaxf(xv.x, xv.y));
+          lm = fmax3f(lm, xv.x, xv.y);
         }
       }
-      if ((t0 + (int64_t)i * kTile + r) >= t1) {
+      if (i == last_ragged && i >= ilim) {  // only the last tile of a ragged range has such rows
         lm = -INFINITY;
 #pragma unroll
         for (int n = 0; n < HQ; ++n) x[n] = -INFINITY;
