@@ -140,7 +140,7 @@ struct Misc {
   float fac[16][64];
   float m[64];
   float lt[64];
-  __align__(16) float cm[16][64];  // per softmax warp: score offset + running max, per head
+  __align__(16) float cm[16][64];  // per softmax warp: -(score offset + running max), per head
   float corr[64];
   __align__(16) float sig[64];
 };
@@ -706,10 +706,11 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
       ms.corr[h0 + gtid] = p.corr[(size_t)b * 2 * NQ + NQ + h0 + gtid];
     }
     named_bar(barid, 128);
-    float *cm = ms.cm[sw];  // score offset + running max m, per head (this warp's copy)
+    float *cm = ms.cm[sw];  // -(score offset + running max m), per head (this warp's copy), negated
+                            // so that the score FMA adds it
     float lsum[HQ];
     if (lane == 0)
-      for (int n = 0; n < HQ; ++n) cm[n] = ms.corr[h0 + n];  // provisional m = 0; the first tile rescales
+      for (int n = 0; n < HQ; ++n) cm[n] = -ms.corr[h0 + n];  // provisional m = 0; the first tile rescales
     __syncwarp();
 #pragma unroll
     for (int n = 0; n < HQ; ++n) lsum[n] = 0.f;
@@ -737,7 +738,7 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
           const int y1 = (int)ra[n + 1] * 128 + (int)rb[n + 1];
           // two heads per packed FMA (each element rounded once, as fmaf)
           const float2 xv = __ffma2_rn(make_float2((float)y0, (float)y1), make_float2(sv[e], sv[e + 1]),
-                                       make_float2(-cv[e], -cv[e + 1]));
+                                       make_float2(cv[e], cv[e + 1]));
           x[n] = xv.x;
           x[n + 1] = xv.y;
           lm = fmax3f(lm, xv.x, xv.y);
@@ -829,7 +830,7 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
           lsum[n] *= fn;
           if (lane == 0) {
             f[n] = fn;
-            cm[n] += sh;
+            cm[n] -= sh;
           }
         }
         __syncwarp();
@@ -880,7 +881,7 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
       if (gtid < HQ) {
         const int hn = h0 + gtid;
         ms.lt[hn] = (ms.red[0][hn] + ms.red[1][hn]) + (ms.red[2][hn] + ms.red[3][hn]);
-        ms.m[hn] = ms.cm[4 * hh][gtid] - ms.corr[hn];
+        ms.m[hn] = -ms.cm[4 * hh][gtid] - ms.corr[hn];
       }
       named_bar(barid, 128);
       const float *Lt = ms.lt;
