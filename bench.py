@@ -373,6 +373,71 @@ def roofline(res, peaks, kernel_name):
     return r
 
 
+POINT_WORKLOADS = ("tiny_0p6b", "qwen3_1p7b_32x", "qwen3_8b_32x", "qwen3_8b_97x", "long_8b_97x")
+
+
+def points(args, torch, F, synth, peaks):
+    """Every (workload, batch, length) point of the five configurations: one
+    JSON line each with the decode step's time (append + decode call), the
+    split kernel's time and its roofline fraction.  Each step is timed alone
+    with CUDA events, after a write of twice L2 that evicts the codes, so
+    small caches are read from HBM as large ones are."""
+    device = torch.device("cuda", 0)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    sptr = stream.cuda_stream
+    qp = F.quant_params()
+    rows = []
+    for wl_name in POINT_WORKLOADS:
+        wl = synth.WORKLOADS[wl_name]
+        G, half = wl.G, wl.G // 2
+        for B in wl.batches:
+            for T in wl.lengths:
+                st = build_state(torch, F, synth, wl, B, T, 0, device, 1)
+                bstride = st["T_max"] * half
+                out = torch.empty((B, wl.n_q, wl.d_h), dtype=torch.bfloat16, device=device)
+                ws = F.Workspace(device)
+                wbuf = ws.get(F.workspace_size(B, T, wl.n_q, wl.n_kv, wl.d_h, G, F.attn_opts(variant="absorbed")))
+                cache = st["caches"][0]
+
+                def step(prof=None):
+                    rc = F.encode_pack_raw(st["x_new"].data_ptr(), B, wl.C, wl.C, st["E"].data_ptr(), G, qp,
+                                           cache.data_ptr() + (T - 1) * half, bstride, sptr)
+                    if rc:
+                        raise F.FsqError(rc, "fsq_encode_pack")
+                    rc = F.decode_attn_raw(st["q"].data_ptr(), B, wl.n_q, wl.d_h, cache.data_ptr(), bstride, T, G,
+                                           st["W_kv"].data_ptr(), wl.n_kv,
+                                           F.attn_opts(variant="absorbed", prof_events=prof), wbuf.data_ptr(),
+                                           wbuf.numel(), out.data_ptr(), sptr)
+                    if rc:
+                        raise F.FsqError(rc, "fsq_decode_attn")
+
+                for _ in range(max(3, args.warmup)):
+                    step()
+                K = max(5, args.steps)
+                evs = RawEvents(K)
+                ab = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+                for i in range(K):
+                    flush.zero_()
+                    ab[i][0].record(stream)
+                    step(evs.pair(i))
+                    ab[i][1].record(stream)
+                torch.cuda.synchronize()
+                step_ms = sorted(a.elapsed_time(b) for a, b in ab)[K // 2]
+                kern_ms = sorted(evs.elapsed_ms(i) for i in range(K))[K // 2]
+                evs.close()
+                rf = roofline(dict(wl=wl, B=B, T=T, kern_ms=kern_ms), peaks, "absorbed_split")
+                row = {"point": wl_name, "G": G, "n_q": wl.n_q, "C": wl.C, "B": B, "T": T,
+                       "step_us": step_ms * 1e3, "kernel_us": kern_ms * 1e3,
+                       "ctx_tok_s": B * T / (step_ms * 1e-3), "code_gbs": rf["code_gbs"],
+                       "roofline_bound": rf["bound"], "roofline_frac": rf["frac_of_roofline"]}
+                print(json.dumps(row), flush=True)
+                rows.append(row)
+                del st, out, ws, wbuf, cache
+                torch.cuda.empty_cache()
+    return rows
+
+
 def _oracle_setup(wl_name, Ts):
     from fsq_latent_decode_b200 import synth
     from oracle import fsq_oracle as O
@@ -512,7 +577,15 @@ def main():
     ap.add_argument("--no-second", action="store_true", help="skip the G=84 companion measurement")
     ap.add_argument("--no-sdpa", action="store_true", help="skip the uncompressed-cache SDPA context measurement")
     ap.add_argument("--no-append", action="store_true", help="skip the 4096-token prefill append measurement")
+    ap.add_argument("--points", action="store_true",
+                    help="time every (workload, batch, length) point of the five configurations, one JSON line each")
     args = ap.parse_args()
+    if args.points:
+        import torch
+        import fsq_latent_decode_b200 as F
+        from fsq_latent_decode_b200 import synth
+        points(args, torch, F, synth, load_peaks())
+        return
     rank, world, local = dist_env()
     wl_name = args.workload
     from fsq_latent_decode_b200 import synth
