@@ -108,6 +108,19 @@ def test_decode_split_counts_agree(splits):
         assert rel_err(got, ref) <= TOL
 
 
+@pytest.mark.parametrize("splits", [5, 7, 12, 20])
+def test_decode_split_counts_agree_g256(splits):
+    """G=256 with four heads per kv head: one merge thread per coordinate pair,
+    so the fold takes the 8-split batch (5, 7), one 16-split batch (12) and two
+    (20)."""
+    B, n_q, n_kv, G, T = 2, 32, 8, 256, 20 * 128 + 77
+    codes = oracle_cache(B, T, G, seed=43)
+    W, q = decoder_weights(n_q, n_kv, G, B, seed=44)
+    ref = O.decode_attn(q.float().numpy(), codes[:, :T], W.float().numpy(), n_kv, G)
+    got = _decode(q, codes, W, T, n_kv, G, variant="absorbed", num_splits=splits, out_fp32=True).cpu().numpy()
+    assert rel_err(got, ref) <= TOL
+
+
 def test_decode_bf16_output_and_scale():
     B, n_q, n_kv, G, T = 2, 32, 8, 256, 513
     codes = oracle_cache(B, T, G, seed=51)
