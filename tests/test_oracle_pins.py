@@ -73,6 +73,17 @@ def test_threshold_values_at_h7p5():
         assert hi == lo + 1
 
 
+def test_threshold_endpoints_at_deck_h():
+    # The slide deck's h = 7.5075 (four-bit product-code frame): the first and
+    # last boundaries, atanh(-7/h) - atanh(0.5/h) and atanh(7/h) - atanh(0.5/h),
+    # hand-evaluated to 5 places; the oracle steps across both.
+    th = _closed_form_thresholds(7.5075, 0.5)
+    assert abs(th[0] - (-1.74316)) < 6e-6 and abs(th[-1] - 1.60976) < 6e-6
+    for t in (th[0], th[-1]):
+        lo, hi = O.fsq_quantize(np.array([t - 1e-7, t + 1e-7]), 7.5075, 0.5)
+        assert hi == lo + 1
+
+
 @pytest.mark.parametrize("h", [7.5, 7.5075])
 def test_odd_symmetry_about_minus_a(h):
     # u~(u) + delta = h tanh(u + a) is odd about u = -a, so
