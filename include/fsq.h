@@ -167,7 +167,9 @@ FSQ_API size_t fsq_decode_attn_workspace_size(int64_t B, int64_t T, int n_q, int
  * Needs: d_h == 128, n_q % n_kv == 0, G even, 2 <= G <= 256, T >= 1; codes
  * and code_batch_stride_bytes 16-byte aligned, code_batch_stride_bytes >=
  * T*G/2; q, W_kv, o 16-byte aligned.  B == 0 is a no-op.  opts may be NULL
- * (defaults). */
+ * (defaults).  The absorbed form on the tensor cores reads each code tile once
+ * with an L2 evict-first hint, so the call's code stream does not displace
+ * other data from L2 (the weights, the workspace, the caller's tensors). */
 FSQ_API fsq_status fsq_decode_attn(const uint16_t *q, int64_t B, int n_q, int d_h,
                            const uint8_t *codes, int64_t code_batch_stride_bytes, int64_t T, int G,
                            const uint16_t *W_kv, int n_kv, const fsq_attn_opts *opts,
