@@ -4,14 +4,21 @@ run single-token GQA attention directly over the codes.
 
 The compute lives in libfsq.so (C ABI, include/fsq.h); this package is its
 ctypes binding plus seeded synthetic inputs.  PyTorch only provides device
-memory and streams.
+memory and streams.  The library is loaded on first use.
 """
 from ._abi import (  # noqa: F401
     EXPORTED, FSQ_OK, FSQ_ERR_CUDA, FSQ_ERR_INVALID_ARG, FSQ_ERR_MISALIGNED, FSQ_ERR_TIMEOUT,
-    FSQ_ERR_UNSUPPORTED, FSQ_ERR_WORKSPACE, AttnOpts, FsqError, QuantParams, Workspace, attn_opts,
-    decode_attn, decode_attn_raw, encode_pack, encode_pack_raw, encode_status, lib, quant_params, quantize_pack_f32,
-    quantize_pack_f32_raw, status_string, thresholds, workspace_size, workspace_status,
+    FSQ_ERR_UNSUPPORTED, FSQ_ERR_WORKSPACE, AttnOpts, EncodeOpts, FsqError, QuantParams, Workspace, attn_opts,
+    decode_attn, decode_attn_noalloc_status, decode_attn_raw, encode_opts, encode_pack, encode_pack_raw, quant_params,
+    quantize_pack_f32, quantize_pack_f32_raw, status_string, thresholds, workspace_size, workspace_status,
 )
+
+
+def __getattr__(name):  # `lib` (the loaded libfsq.so) is mapped on first access
+    if name == "lib":
+        from . import _abi
+        return _abi.lib
+    raise AttributeError(name)
 
 __all__ = ["encode_pack", "quantize_pack_f32", "decode_attn", "attn_opts", "thresholds", "workspace_size",
            "Workspace", "FsqError"]

@@ -1,8 +1,10 @@
 """ctypes binding of libfsq.so (declared in include/fsq.h).
 
 Argument marshalling only: every step of the path runs in the library's CUDA
-kernels.  If the shared library is missing the import fails loudly; there is
-no fallback implementation.
+kernels.  The shared library is loaded on first use (the first call, or the
+first access to `lib`), so that importing the package for its seeded input
+generators maps no native code.  If the library is missing, that first use
+fails loudly; there is no fallback implementation.
 """
 from __future__ import annotations
 
@@ -27,7 +29,9 @@ VARIANTS = {"auto": VARIANT_AUTO, "absorbed": VARIANT_ABSORBED, "expand": VARIAN
 # Every symbol include/fsq.h declares.
 EXPORTED = ("fsq_attn_opts_default", "fsq_thresholds", "fsq_encode_pack", "fsq_quantize_pack_f32",
             "fsq_decode_attn_workspace_size", "fsq_decode_attn", "fsq_workspace_status",
-            "fsq_status_string", "fsq_format_version", "fsq_decode_attn_noalloc", "fsq_encode_status")
+            "fsq_status_string", "fsq_format_version", "fsq_decode_attn_noalloc",
+            "fsq_decode_attn_noalloc_status")
+# FSQ_NOALLOC_SCRATCH_BYTES of include/fsq.h (a host test checks the two agree)
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
@@ -38,7 +42,12 @@ class QuantParams(C.Structure):
 class AttnOpts(C.Structure):
     _fields_ = [("variant", C.c_int), ("scale", C.c_float), ("num_splits", C.c_int),
                 ("rope_knorm", C.c_int), ("rope_base", C.c_float), ("knorm_gain", C.c_void_p),
-                ("knorm_eps", C.c_float), ("out_fp32", C.c_int), ("prof_events", C.c_void_p * 2)]
+                ("knorm_eps", C.c_float), ("out_fp32", C.c_int), ("prof_events", C.c_void_p * 2),
+                ("seq_lens", C.c_void_p), ("debug_stall_ns", C.c_uint32)]
+
+
+class EncodeOpts(C.Structure):
+    _fields_ = [("status_word", C.c_void_p), ("debug_stall_ns", C.c_uint32)]
 
 
 class FsqError(RuntimeError):
@@ -57,10 +66,8 @@ def _load() -> C.CDLL:
     lib.fsq_attn_opts_default.restype = None
     lib.fsq_thresholds.argtypes = [QuantParams, C.POINTER(C.c_float)]
     lib.fsq_thresholds.restype = i32
-    lib.fsq_encode_pack.argtypes = [vp, i64, i64, i64, vp, i32, QuantParams, vp, i64, vp]
+    lib.fsq_encode_pack.argtypes = [vp, i64, i64, i64, vp, i32, QuantParams, vp, i64, C.POINTER(EncodeOpts), vp]
     lib.fsq_encode_pack.restype = i32
-    lib.fsq_encode_status.argtypes = [vp]
-    lib.fsq_encode_status.restype = i32
     lib.fsq_quantize_pack_f32.argtypes = [vp, i64, i32, QuantParams, vp, i64, vp]
     lib.fsq_quantize_pack_f32.restype = i32
     lib.fsq_decode_attn_workspace_size.argtypes = [i64, i64, i32, i32, i32, i32, C.POINTER(AttnOpts)]
@@ -71,6 +78,8 @@ def _load() -> C.CDLL:
     lib.fsq_decode_attn_noalloc.argtypes = [vp, i64, i32, i32, vp, i64, i64, i32, vp, i32, C.POINTER(AttnOpts),
                                             vp, vp]
     lib.fsq_decode_attn_noalloc.restype = i32
+    lib.fsq_decode_attn_noalloc_status.argtypes = [vp]
+    lib.fsq_decode_attn_noalloc_status.restype = i32
     lib.fsq_workspace_status.argtypes = [vp, C.c_size_t, vp]
     lib.fsq_workspace_status.restype = i32
     lib.fsq_status_string.argtypes = [i32]
@@ -80,11 +89,24 @@ def _load() -> C.CDLL:
     return lib
 
 
-lib = _load()
+_LIB = None
+
+
+def _lib() -> C.CDLL:
+    global _LIB
+    if _LIB is None:
+        _LIB = _load()
+    return _LIB
+
+
+def __getattr__(name):  # `_abi.lib` loads the library on first access
+    if name == "lib":
+        return _lib()
+    raise AttributeError(name)
 
 
 def status_string(s: int) -> str:
-    return lib.fsq_status_string(int(s)).decode()
+    return _lib().fsq_status_string(int(s)).decode()
 
 
 def _check(st: int, what: str):
@@ -98,14 +120,15 @@ def quant_params(h: float = 7.5, delta: float = 0.5) -> QuantParams:
 
 def thresholds(h: float = 7.5, delta: float = 0.5):
     buf = (C.c_float * 15)()
-    _check(lib.fsq_thresholds(quant_params(h, delta), buf), "fsq_thresholds")
+    _check(_lib().fsq_thresholds(quant_params(h, delta), buf), "fsq_thresholds")
     return [buf[i] for i in range(15)]
 
 
 def attn_opts(variant="auto", scale=0.0, num_splits=0, rope_knorm=False, rope_base=1.0e6,
-              knorm_gain=None, knorm_eps=1e-6, out_fp32=False, prof_events=None) -> AttnOpts:
+              knorm_gain=None, knorm_eps=1e-6, out_fp32=False, prof_events=None, seq_lens=None,
+              debug_stall_ns=0) -> AttnOpts:
     o = AttnOpts()
-    lib.fsq_attn_opts_default(C.byref(o))
+    _lib().fsq_attn_opts_default(C.byref(o))
     o.variant = VARIANTS[variant] if isinstance(variant, str) else int(variant)
     o.scale = float(scale)
     o.num_splits = int(num_splits)
@@ -117,7 +140,14 @@ def attn_opts(variant="auto", scale=0.0, num_splits=0, rope_knorm=False, rope_ba
     if prof_events is not None:  # a pair of objects exposing a raw cudaEvent_t as .cuda_event
         o.prof_events[0] = int(prof_events[0].cuda_event)
         o.prof_events[1] = int(prof_events[1].cuda_event)
+    o.seq_lens = None if seq_lens is None else int(seq_lens.data_ptr())  # device int32 [B]
+    o.debug_stall_ns = int(debug_stall_ns)
     return o
+
+
+def encode_opts(status_word=None, debug_stall_ns=0) -> EncodeOpts:
+    """status_word: a device tensor whose first 4 bytes are the caller's status word."""
+    return EncodeOpts(None if status_word is None else int(status_word.data_ptr()), int(debug_stall_ns))
 
 
 def _stream_ptr(stream) -> int:
@@ -131,43 +161,48 @@ def _ptr(t) -> int:
 
 
 # ---------------------------------------------------------------- raw C-ABI calls (pointers in, status out)
-def encode_pack_raw(x_ptr, n_tok, ldx, C_, E_ptr, G, qp, codes_ptr, ldc, stream_ptr) -> int:
-    return lib.fsq_encode_pack(x_ptr, n_tok, ldx, C_, E_ptr, G, qp, codes_ptr, ldc, stream_ptr)
+def encode_pack_raw(x_ptr, n_tok, ldx, C_, E_ptr, G, qp, codes_ptr, ldc, stream_ptr, opts=None) -> int:
+    return _lib().fsq_encode_pack(x_ptr, n_tok, ldx, C_, E_ptr, G, qp, codes_ptr, ldc,
+                                  None if opts is None else C.byref(opts), stream_ptr)
 
 
 def quantize_pack_f32_raw(u_ptr, n_tok, G, qp, codes_ptr, ldc, stream_ptr) -> int:
-    return lib.fsq_quantize_pack_f32(u_ptr, n_tok, G, qp, codes_ptr, ldc, stream_ptr)
+    return _lib().fsq_quantize_pack_f32(u_ptr, n_tok, G, qp, codes_ptr, ldc, stream_ptr)
 
 
 def workspace_size(B, T, n_q, n_kv, d_h, G, opts: AttnOpts | None = None) -> int:
-    return int(lib.fsq_decode_attn_workspace_size(B, T, n_q, n_kv, d_h, G,
-                                                  None if opts is None else C.byref(opts)))
+    return int(_lib().fsq_decode_attn_workspace_size(B, T, n_q, n_kv, d_h, G,
+                                                     None if opts is None else C.byref(opts)))
 
 
 def decode_attn_raw(q_ptr, B, n_q, d_h, codes_ptr, bstride, T, G, wkv_ptr, n_kv, opts, ws_ptr, ws_bytes,
                     o_ptr, stream_ptr) -> int:
-    return lib.fsq_decode_attn(q_ptr, B, n_q, d_h, codes_ptr, bstride, T, G, wkv_ptr, n_kv,
-                               None if opts is None else C.byref(opts), ws_ptr, ws_bytes, o_ptr, stream_ptr)
+    return _lib().fsq_decode_attn(q_ptr, B, n_q, d_h, codes_ptr, bstride, T, G, wkv_ptr, n_kv,
+                                  None if opts is None else C.byref(opts), ws_ptr, ws_bytes, o_ptr, stream_ptr)
 
 
 def decode_attn_noalloc_raw(q_ptr, B, n_q, d_h, codes_ptr, bstride, T, G, wkv_ptr, n_kv, opts, o_ptr,
                             stream_ptr) -> int:
-    return lib.fsq_decode_attn_noalloc(q_ptr, B, n_q, d_h, codes_ptr, bstride, T, G, wkv_ptr, n_kv,
-                                       None if opts is None else C.byref(opts), o_ptr, stream_ptr)
+    return _lib().fsq_decode_attn_noalloc(q_ptr, B, n_q, d_h, codes_ptr, bstride, T, G, wkv_ptr, n_kv,
+                                          None if opts is None else C.byref(opts), o_ptr, stream_ptr)
 
 
-def encode_status(stream=None) -> int:
-    """Reads and clears the append path's device error word (blocking)."""
-    return lib.fsq_encode_status(_stream_ptr(stream))
+def decode_attn_noalloc_status(stream=None) -> int:
+    """Device status of the last allocation-free decode call on this device (blocking)."""
+    return _lib().fsq_decode_attn_noalloc_status(_stream_ptr(stream))
 
 
 def workspace_status(ws, stream=None) -> int:
-    return lib.fsq_workspace_status(_ptr(ws), ws.numel() * ws.element_size(), _stream_ptr(stream))
+    """Reads a device status word: a decode workspace's error word, or an
+    append status word (a device tensor of at least 4 bytes).  Blocking."""
+    return _lib().fsq_workspace_status(_ptr(ws), ws.numel() * ws.element_size(), _stream_ptr(stream))
 
 
 # ---------------------------------------------------------------- tensor-level wrappers (torch for memory only)
-def encode_pack(x, E, h=7.5, delta=0.5, out=None, stream=None):
-    """codes[n_tok, G/2] (uint8) for bf16 rows x[n_tok, C] through E[G, C]."""
+def encode_pack(x, E, h=7.5, delta=0.5, out=None, stream=None, status_word=None):
+    """codes[n_tok, G/2] (uint8) for bf16 rows x[n_tok, C] through E[G, C].
+    status_word: optional device tensor (>= 4 bytes, zeroed by the caller)
+    that receives a device-detected failure (read it with workspace_status)."""
     import torch
     n_tok, C_ = x.shape
     G = E.shape[0]
@@ -175,7 +210,7 @@ def encode_pack(x, E, h=7.5, delta=0.5, out=None, stream=None):
         out = torch.empty((n_tok, G // 2), dtype=torch.uint8, device=x.device)
     ldc = out.stride(0) if out.dim() == 2 else G // 2
     st = encode_pack_raw(_ptr(x), n_tok, x.stride(0), C_, _ptr(E), G, quant_params(h, delta), _ptr(out), ldc,
-                         _stream_ptr(stream))
+                         _stream_ptr(stream), encode_opts(status_word))
     _check(st, "fsq_encode_pack")
     return out
 

@@ -9,27 +9,28 @@
 
 namespace fsq {
 cudaError_t launch_encode_pack_simt(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C, const uint16_t *E,
-                                    int G, const Thresholds &th, uint8_t *codes, int64_t ldc, cudaStream_t s);
-cudaError_t encode_status(uint32_t *out, cudaStream_t s);
+                                    int G, const Thresholds &th, uint8_t *codes, int64_t ldc, uint32_t *status,
+                                    uint32_t stall_ns, cudaStream_t s);
 cudaError_t launch_quantize_pack_f32(const float *u, int64_t n_tok, int G, const Thresholds &th, uint8_t *codes,
                                      int64_t ldc, cudaStream_t s);
 cudaError_t launch_absorbed_simt(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
-                                 int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv, float scale, int S,
-                                 int64_t tps, float *qa, float *part, uint32_t *err, MergeScratch ms, void *o,
-                                 int out_fp32, void *const *prof, cudaStream_t st);
+                                 const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv,
+                                 float scale, int S, int64_t tps, float *qa, float *part, uint32_t *err,
+                                 MergeScratch ms, void *o, int out_fp32, void *const *prof, cudaStream_t st);
 cudaError_t launch_expand_simt(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
-                               int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv, float scale, int S,
-                               int64_t tps, int rope_knorm, float rope_base, const uint16_t *gain, float eps,
-                               float *part, uint32_t *err, void *o, int out_fp32, void *const *prof,
-                               cudaStream_t st);
+                               const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv,
+                               float scale, int S, int64_t tps, int rope_knorm, float rope_base,
+                               const uint16_t *gain, float eps, float *part, uint32_t *err, void *o, int out_fp32,
+                               void *const *prof, cudaStream_t st);
 int simt_max_nq();
 int simt_max_grp();
 bool absorbed_tc_supported(int n_q, int n_kv, int G);
 size_t absorbed_tc_qphys_bytes(int n_q, int G);
 cudaError_t launch_absorbed_tc(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
-                               int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv, float scale, int S,
-                               int64_t tps, uint8_t *qphys, float *corr, float *part, uint32_t *err,
-                               MergeScratch ms, void *o, int out_fp32, void *const *prof, cudaStream_t st);
+                               const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv,
+                               float scale, int S, int64_t tps, uint8_t *qphys, float *corr, float *part,
+                               uint32_t *err, MergeScratch ms, void *o, int out_fp32, uint32_t stall_ns,
+                               void *const *prof, cudaStream_t st);
 
 namespace {
 
@@ -152,6 +153,8 @@ void fsq_attn_opts_default(fsq_attn_opts *opts) {
   opts->knorm_eps = 1.0e-6f;
   opts->out_fp32 = 0;
   opts->prof_events[0] = opts->prof_events[1] = nullptr;
+  opts->seq_lens = nullptr;
+  opts->debug_stall_ns = 0;
 }
 
 fsq_status fsq_thresholds(fsq_quant_params qp, float theta_out[15]) {
@@ -163,7 +166,8 @@ fsq_status fsq_thresholds(fsq_quant_params qp, float theta_out[15]) {
 }
 
 fsq_status fsq_encode_pack(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C, const uint16_t *E, int G,
-                           fsq_quant_params qp, uint8_t *codes, int64_t ldc_bytes, fsq_stream_t stream) {
+                           fsq_quant_params qp, uint8_t *codes, int64_t ldc_bytes, const fsq_encode_opts *opts,
+                           fsq_stream_t stream) {
   if (n_tok < 0 || C < 1 || G < 2) return FSQ_ERR_INVALID_ARG;
   if (G % 2 || G > FSQ_MAX_G || C % 64) return FSQ_ERR_UNSUPPORTED;
   if (ldx < C || ldc_bytes < G / 2) return FSQ_ERR_INVALID_ARG;
@@ -172,15 +176,12 @@ fsq_status fsq_encode_pack(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_
   if (n_tok == 0) return FSQ_OK;
   if (!x || !E || !codes) return FSQ_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(E) || ldx % 8) return FSQ_ERR_MISALIGNED;
+  uint32_t *status = opts ? opts->status_word : nullptr;
+  if ((uintptr_t)status & 3u) return FSQ_ERR_MISALIGNED;
   Thresholds th;
   make_thresholds(qp, th.th);
-  return from_cuda(launch_encode_pack_simt(x, n_tok, ldx, C, E, G, th, codes, ldc_bytes, (cudaStream_t)stream));
-}
-
-fsq_status fsq_encode_status(fsq_stream_t stream) {
-  uint32_t v = 0;
-  if (encode_status(&v, (cudaStream_t)stream) != cudaSuccess) return FSQ_ERR_CUDA;
-  return v == 0 ? FSQ_OK : (fsq_status)(-(int)v);
+  return from_cuda(launch_encode_pack_simt(x, n_tok, ldx, C, E, G, th, codes, ldc_bytes, status,
+                                           opts ? opts->debug_stall_ns : 0u, (cudaStream_t)stream));
 }
 
 fsq_status fsq_quantize_pack_f32(const float *u, int64_t n_tok, int G, fsq_quant_params qp, uint8_t *codes,
@@ -223,6 +224,7 @@ fsq_status fsq_decode_attn(const uint16_t *q, int64_t B, int n_q, int d_h, const
   if (code_batch_stride_bytes < T * (G / 2)) return FSQ_ERR_INVALID_ARG;
   if (!aligned16(codes) || code_batch_stride_bytes % 16) return FSQ_ERR_MISALIGNED;
   if (!aligned16(q) || !aligned16(W_kv) || !aligned16(o)) return FSQ_ERR_MISALIGNED;
+  if ((uintptr_t)op.seq_lens & 3u) return FSQ_ERR_MISALIGNED;
   if (!workspace || workspace_bytes < p.total) return FSQ_ERR_WORKSPACE;
   if ((uintptr_t)workspace & 255u) return FSQ_ERR_MISALIGNED;
   const float scale = op.scale > 0.f ? op.scale : 1.f / sqrtf((float)d_h);
@@ -234,22 +236,23 @@ fsq_status fsq_decode_attn(const uint16_t *q, int64_t B, int n_q, int d_h, const
   if (p.mp.cnt_bytes) ms = {(float *)(ws + p.off_mslab), (uint32_t *)(ws + p.off_mcnt), (int)(B * n_kv)};
   cudaError_t e;
   if (p.tc) {
-    e = launch_absorbed_tc(q, codes, code_batch_stride_bytes, B, T, n_q, n_kv, d_h, G, W_kv, scale, p.S, p.tps,
-                           (uint8_t *)(ws + p.off_qa), (float *)(ws + p.off_corr), part, err, ms, o, op.out_fp32,
-                           op.prof_events, s);
+    e = launch_absorbed_tc(q, codes, code_batch_stride_bytes, B, T, op.seq_lens, n_q, n_kv, d_h, G, W_kv, scale,
+                           p.S, p.tps, (uint8_t *)(ws + p.off_qa), (float *)(ws + p.off_corr), part, err, ms, o,
+                           op.out_fp32, op.debug_stall_ns, op.prof_events, s);
   } else if (p.variant == FSQ_VARIANT_ABSORBED) {
-    e = launch_absorbed_simt(q, codes, code_batch_stride_bytes, B, T, n_q, n_kv, d_h, G, W_kv, scale, p.S, p.tps,
-                             (float *)(ws + p.off_qa), part, err, ms, o, op.out_fp32, op.prof_events, s);
+    e = launch_absorbed_simt(q, codes, code_batch_stride_bytes, B, T, op.seq_lens, n_q, n_kv, d_h, G, W_kv, scale,
+                             p.S, p.tps, (float *)(ws + p.off_qa), part, err, ms, o, op.out_fp32, op.prof_events, s);
   } else {
-    e = launch_expand_simt(q, codes, code_batch_stride_bytes, B, T, n_q, n_kv, d_h, G, W_kv, scale, p.S, p.tps,
-                           op.rope_knorm, op.rope_base, op.knorm_gain, op.knorm_eps, part, err, o, op.out_fp32,
-                           op.prof_events, s);
+    e = launch_expand_simt(q, codes, code_batch_stride_bytes, B, T, op.seq_lens, n_q, n_kv, d_h, G, W_kv, scale,
+                           p.S, p.tps, op.rope_knorm, op.rope_base, op.knorm_gain, op.knorm_eps, part, err, o,
+                           op.out_fp32, op.prof_events, s);
   }
   return from_cuda(e);
 }
 
 fsq_status fsq_workspace_status(const void *workspace, size_t workspace_bytes, fsq_stream_t stream) {
-  if (!workspace || workspace_bytes < kWsHeader) return FSQ_ERR_INVALID_ARG;
+  if (!workspace || workspace_bytes < sizeof(uint32_t)) return FSQ_ERR_INVALID_ARG;
+  if ((uintptr_t)workspace & 3u) return FSQ_ERR_MISALIGNED;
   uint32_t v = 0;
   cudaError_t e = cudaMemcpyAsync(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost, (cudaStream_t)stream);
   if (e == cudaSuccess) e = cudaStreamSynchronize((cudaStream_t)stream);

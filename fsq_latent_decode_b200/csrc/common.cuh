@@ -65,6 +65,18 @@ __device__ __forceinline__ void record_error(uint32_t *err, int status) {
   atomicCAS(err, 0u, (uint32_t)(-status));
 }
 
+// Cached tokens of batch row b: T, or seq_lens[b] for a ragged batch, clamped
+// into [1, T]; a value outside records FSQ_ERR_INVALID_ARG when `report`
+// (one thread per row reports, after the call's error word was cleared).
+__device__ __forceinline__ int64_t row_len(const int32_t *seq_lens, int64_t b, int64_t T, uint32_t *err,
+                                           bool report) {
+  if (seq_lens == nullptr) return T;
+  const int64_t v = seq_lens[b];
+  if (v >= 1 && v <= T) return v;
+  if (report) record_error(err, FSQ_ERR_INVALID_ARG);
+  return v < 1 ? 1 : T;
+}
+
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Raise a kernel's dynamic shared-memory limit on the current device, once:

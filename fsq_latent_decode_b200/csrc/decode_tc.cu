@@ -60,7 +60,8 @@ constexpr int kMaxStages = 16;                     // code-tile ring depth bound
 constexpr int kSmemBudget = 200 * 1024;            // shared memory a CTA plans for
 constexpr int kQAfterTiles = 4;                    // code tiles requested before Q' (and its wait)
 constexpr float kTau = 8.f;                        // rescale when a score exceeds the running max by 2^8
-constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s per wait
+constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s per hand-off wait
+constexpr uint64_t kDrainNs = 1000000000ull;       // 1 s for in-flight copies and MMAs on the error path
 constexpr int kMiscBytes = 12288;                  // shared-memory reservation for the Misc block
 constexpr int kPBufs = 8;                          // ring of softmax-weight (P) tiles in shared memory
 
@@ -124,7 +125,9 @@ struct Params {
   const float *corr;     // per batch row: [NQ] sigma, then [NQ] score offsets
   float *part;           // [B][S][NQ][2 + G]
   uint32_t *err;
-  uint64_t wait_ns;
+  uint64_t wait_ns;      // limit of every hand-off wait
+  const int32_t *seq_lens;  // per-row lengths (ragged batch) or null
+  uint32_t stall_ns;     // test-only: > 0 makes the softmax wait on `never` first
 };
 
 struct Misc {
@@ -133,7 +136,7 @@ struct Misc {
   uint64_t cp_ready[4], cp_free[4];
   uint64_t s_full[2], s_free[2];
   uint64_t p_full[kPBufs], p_free[kPBufs];
-  uint64_t acc_full, q_full, done[5];
+  uint64_t acc_full, q_full, done[5], never;
   uint32_t tmem_base;
   uint32_t abort;
   float red[4][64];
@@ -398,7 +401,15 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int split = blockIdx.x, b = blockIdx.y;
   const int64_t t0 = (int64_t)split * p.tps;
-  const int64_t t1 = min(p.T, t0 + p.tps);
+  const int64_t t1 = min(row_len(p.seq_lens, b, p.T, p.err, false), t0 + p.tps);
+  if (t1 <= t0) {
+    // this split lies wholly past its row's length (ragged batch): an empty
+    // partial, which the merge weighs by 2^-inf = 0
+    pdl_wait();
+    float *out = p.part + (((size_t)b * p.S + split) * NQ) * (2 + G);
+    for (int i = tid; i < NQ * (2 + G); i += C::THREADS) out[i] = (i % (2 + G)) == 0 ? -INFINITY : 0.f;
+    return;
+  }
   const int n_tiles = (int)((t1 - t0 + kTile - 1) / kTile);
   const uint8_t *gcodes = p.codes + (int64_t)b * p.bstride + t0 * C::HALF;
   volatile uint32_t *abort = &ms.abort;
@@ -428,6 +439,7 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
     mbar_init(&ms.acc_full, kPoolIssuers);
     mbar_init(&ms.q_full, 1);
     for (int i = 0; i < 5; ++i) mbar_init(&ms.done[i], 1);
+    mbar_init(&ms.never, 1);  // completed by nothing: the test-only stall waits on it
     ms.abort = 0;
     fence_mbar_init();
   }
@@ -501,8 +513,8 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
       if (lane == 0) fail();
       // let the copies still in flight land before the CTA exits
       for (int i = max(0, issued - C::STAGES); i < issued; ++i)
-        drain_bar(&ms.full[i % C::STAGES], (uint32_t)(i / C::STAGES) & 1u, p.wait_ns / 4 + 1);
-      drain_bar(&ms.q_full, 0, p.wait_ns / 4 + 1);
+        drain_bar(&ms.full[i % C::STAGES], (uint32_t)(i / C::STAGES) & 1u, kDrainNs);
+      drain_bar(&ms.q_full, 0, kDrainNs);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ score-MMA issuer (whole warp, one lane issues)
@@ -529,8 +541,9 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
       __syncwarp();
     }
     if (!ok && lane == 0) fail();
+    // every MMA of this warp completes before TMEM is freed, error or not
     tc_commit_elect(&ms.done[0]);
-    wait_bar(&ms.done[0], 0, abort, p.wait_ns);
+    drain_bar(&ms.done[0], 0, kDrainNs);
   } else if (warp == 2 || warp == 3) {
     // ------------------------------------------------------------ pooling-MMA issuers (whole warp, one lane issues)
     const int k_iss = warp - 2;  // NH=2: half k_iss, both chunks; NH=1: chunk k_iss
@@ -568,7 +581,7 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
     if (ok) tc_commit_elect(&ms.acc_full);
     else if (lane == 0) fail();
     tc_commit_elect(&ms.done[2 + k_iss]);
-    wait_bar(&ms.done[2 + k_iss], 0, abort, p.wait_ns);
+    drain_bar(&ms.done[2 + k_iss], 0, kDrainNs);
   } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------------------------ score dequant: token row -> TMEM lane
     const int q = warp - 4;
@@ -704,8 +717,14 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
       pdl_wait();  // corr comes from the query prologue kernel
       ms.sig[h0 + gtid] = p.corr[(size_t)b * 2 * NQ + h0 + gtid];
       ms.corr[h0 + gtid] = p.corr[(size_t)b * 2 * NQ + NQ + h0 + gtid];
+      // a bad per-row length is reported once, after the prologue cleared the error word
+      if (split == 0 && hh == 0 && gtid == 0) row_len(p.seq_lens, b, p.T, p.err, true);
     }
     named_bar(barid, 128);
+    bool ok = true;
+    // test-only stall: every softmax warp waits on a barrier that nothing
+    // completes, so the bounded wait runs out and the failure path runs
+    if (p.stall_ns != 0u && !wait_bar(&ms.never, 0, abort, p.stall_ns)) ok = false;
     float *cm = ms.cm[sw];  // -(score offset + running max m), per head (this warp's copy), negated
                             // so that the score FMA adds it
     float lsum[HQ];
@@ -772,7 +791,6 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
     // through the loop.  P buffers stay per tile (the score MMA of tile i
     // waited for P buffer i % kPBufs to be free).
     const int n_pairs = (n_tiles + 1) >> 1;
-    bool ok = true;
     for (int j = 0; j < n_pairs && ok; ++j) {
       const int i0 = 2 * j;
       const bool two = i0 + 1 < n_tiles;
@@ -1133,9 +1151,10 @@ cudaError_t make_code_tensor_map(CUtensorMap *map, const uint8_t *codes, int64_t
 }
 
 template <int G, int NQ>
-cudaError_t launch(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T, int n_kv,
-                   const uint16_t *W_kv, float scale, int S, int64_t tps, uint8_t *qphys, float *corr, float *part,
-                   uint32_t *err, MergeScratch ms, void *const *prof, cudaStream_t st) {
+cudaError_t launch(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
+                   const int32_t *seq_lens, int n_kv, const uint16_t *W_kv, float scale, int S, int64_t tps,
+                   uint8_t *qphys, float *corr, float *part, uint32_t *err, MergeScratch ms, uint32_t stall_ns,
+                   void *const *prof, cudaStream_t st) {
   using C = Cfg<G, NQ>;
   cudaError_t e = launch_absorb_query<G, NQ>(q, B, n_kv, W_kv, scale * kLog2e, qphys, corr, err, ms, st);
   if (e != cudaSuccess) return e;
@@ -1143,7 +1162,7 @@ cudaError_t launch(const uint16_t *q, const uint8_t *codes, int64_t bstride, int
   const int smem = C::SM_TOTAL > 120 * 1024 ? C::SM_TOTAL : 120 * 1024;
   e = ensure_smem_limit((const void *)absorbed_split_tc<G, NQ>, (size_t)smem);
   if (e != cudaSuccess) return e;
-  Params p{codes, bstride, T, tps, S, qphys, corr, part, err, kWaitLimitNs};
+  Params p{codes, bstride, T, tps, S, qphys, corr, part, err, kWaitLimitNs, seq_lens, stall_ns};
   CUtensorMap tmap;
   memset(&tmap, 0, sizeof(tmap));
   if constexpr (C::TMA) {
@@ -1171,15 +1190,20 @@ cudaError_t merge_absorbed_launch(const float *part, int S, int64_t B, int n_q, 
                                   const uint16_t *W_kv, void *o, int out_fp32, MergeScratch ms, cudaStream_t st);
 
 cudaError_t launch_absorbed_tc(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
-                               int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv, float scale, int S,
-                               int64_t tps, uint8_t *qphys, float *corr, float *part, uint32_t *err,
-                               MergeScratch ms, void *o, int out_fp32, void *const *prof, cudaStream_t st) {
+                               const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv,
+                               float scale, int S, int64_t tps, uint8_t *qphys, float *corr, float *part,
+                               uint32_t *err, MergeScratch ms, void *o, int out_fp32, uint32_t stall_ns,
+                               void *const *prof, cudaStream_t st) {
   cudaError_t e;
-  if (G == 256 && n_q == 32) e = tc::launch<256, 32>(q, codes, bstride, B, T, n_kv, W_kv, scale, S, tps, qphys, corr, part, err, ms, prof, st);
-  else if (G == 256 && n_q == 16) e = tc::launch<256, 16>(q, codes, bstride, B, T, n_kv, W_kv, scale, S, tps, qphys, corr, part, err, ms, prof, st);
-  else if (G == 84 && n_q == 32) e = tc::launch<84, 32>(q, codes, bstride, B, T, n_kv, W_kv, scale, S, tps, qphys, corr, part, err, ms, prof, st);
-  else if (G == 84 && n_q == 16) e = tc::launch<84, 16>(q, codes, bstride, B, T, n_kv, W_kv, scale, S, tps, qphys, corr, part, err, ms, prof, st);
+#define FSQ_TC_LAUNCH(GG, NN)                                                                                  \
+  tc::launch<GG, NN>(q, codes, bstride, B, T, seq_lens, n_kv, W_kv, scale, S, tps, qphys, corr, part, err, ms, \
+                     stall_ns, prof, st)
+  if (G == 256 && n_q == 32) e = FSQ_TC_LAUNCH(256, 32);
+  else if (G == 256 && n_q == 16) e = FSQ_TC_LAUNCH(256, 16);
+  else if (G == 84 && n_q == 32) e = FSQ_TC_LAUNCH(84, 32);
+  else if (G == 84 && n_q == 16) e = FSQ_TC_LAUNCH(84, 16);
   else return cudaErrorInvalidValue;
+#undef FSQ_TC_LAUNCH
   if (e != cudaSuccess) return e;
   return merge_absorbed_launch(part, S, B, n_q, n_kv, d_h, G, W_kv, o, out_fp32, ms, st);
 }

@@ -49,8 +49,9 @@ __global__ void absorb_query_kernel(const uint16_t *__restrict__ q, const uint16
 // part layout: [B][S][n_q][2 + G]  (m, l, acc[G]), log2 domain.
 __global__ void __launch_bounds__(256) absorbed_split_simt(const float *__restrict__ qa,
                                                            const uint8_t *__restrict__ codes, int64_t bstride,
-                                                           int64_t T, int G, int n_q, int64_t tps,
-                                                           float *__restrict__ part) {
+                                                           int64_t T, const int32_t *__restrict__ seq_lens,
+                                                           int G, int n_q, int64_t tps, float *__restrict__ part,
+                                                           uint32_t *err) {
   extern __shared__ float sm[];
   float *qs = sm;                                   // [n_q][G]
   float *acc = qs + n_q * G;                        // [n_q][G]
@@ -62,7 +63,7 @@ __global__ void __launch_bounds__(256) absorbed_split_simt(const float *__restri
   const int tid = threadIdx.x, nth = blockDim.x;
   const int s = blockIdx.x, b = blockIdx.y, S = gridDim.x;
   const int64_t t0 = (int64_t)s * tps;
-  const int64_t t1 = min(T, t0 + tps);
+  const int64_t t1 = min(row_len(seq_lens, b, T, err, s == 0 && tid == 0), t0 + tps);  // empty past the row's end
   const int half = G / 2;
   const uint8_t *cb = codes + (int64_t)b * bstride;
 
@@ -180,11 +181,11 @@ __global__ void merge_absorbed_kernel(const float *__restrict__ part, int S, int
 // part layout: [B][S][n_q][2 + d_h].
 __global__ void __launch_bounds__(128) expand_split_simt(const uint16_t *__restrict__ q,
                                                          const uint8_t *__restrict__ codes, int64_t bstride,
-                                                         int64_t T, int G, int n_q, int n_kv,
-                                                         const uint16_t *__restrict__ W_kv, float c, int64_t tps,
-                                                         int rope_knorm, float rope_base,
+                                                         int64_t T, const int32_t *__restrict__ seq_lens, int G,
+                                                         int n_q, int n_kv, const uint16_t *__restrict__ W_kv,
+                                                         float c, int64_t tps, int rope_knorm, float rope_base,
                                                          const uint16_t *__restrict__ gain, float eps,
-                                                         float *__restrict__ part) {
+                                                         float *__restrict__ part, uint32_t *err) {
   constexpr int D = FSQ_HEAD_DIM;
   extern __shared__ float sm[];
   uint16_t *wk = reinterpret_cast<uint16_t *>(sm);          // [G][D]
@@ -197,7 +198,8 @@ __global__ void __launch_bounds__(128) expand_split_simt(const uint16_t *__restr
   const int d = threadIdx.x, warp = d / 32, lane = d % 32;
   const int s = blockIdx.x, b = blockIdx.y, j = blockIdx.z, S = gridDim.x;
   const int grp = n_q / n_kv;
-  const int64_t t0 = (int64_t)s * tps, t1 = min(T, t0 + tps);
+  const int64_t t0 = (int64_t)s * tps;
+  const int64_t t1 = min(row_len(seq_lens, b, T, err, s == 0 && j == 0 && d == 0), t0 + tps);
   const int half = G / 2;
   const uint8_t *cb = codes + (int64_t)b * bstride;
 
@@ -365,9 +367,9 @@ int simt_max_nq() { return kMaxNQ; }
 int simt_max_grp() { return kMaxGrp; }
 
 cudaError_t launch_absorbed_simt(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
-                                 int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv, float scale,
-                                 int S, int64_t tps, float *qa, float *part, uint32_t *err, MergeScratch ms, void *o,
-                                 int out_fp32, void *const *prof, cudaStream_t st) {
+                                 const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv,
+                                 float scale, int S, int64_t tps, float *qa, float *part, uint32_t *err,
+                                 MergeScratch ms, void *o, int out_fp32, void *const *prof, cudaStream_t st) {
   absorb_query_kernel<<<dim3(n_q, (unsigned)B), 256, 0, st>>>(q, W_kv, n_q, n_kv, d_h, G, scale * kLog2e, qa, err,
                                                               ms);
   cudaError_t e = cudaGetLastError();
@@ -376,7 +378,8 @@ cudaError_t launch_absorbed_simt(const uint16_t *q, const uint8_t *codes, int64_
   e = ensure_smem_limit((const void *)absorbed_split_simt, smem);
   if (e != cudaSuccess) return e;
   record_prof_event(prof[0], st);
-  absorbed_split_simt<<<dim3(S, (unsigned)B), 256, smem, st>>>(qa, codes, bstride, T, G, n_q, tps, part);
+  absorbed_split_simt<<<dim3(S, (unsigned)B), 256, smem, st>>>(qa, codes, bstride, T, seq_lens, G, n_q, tps, part,
+                                                                err);
   e = cudaGetLastError();
   record_prof_event(prof[1], st);
   if (e != cudaSuccess) return e;
@@ -384,10 +387,10 @@ cudaError_t launch_absorbed_simt(const uint16_t *q, const uint8_t *codes, int64_
 }
 
 cudaError_t launch_expand_simt(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
-                               int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv, float scale, int S,
-                               int64_t tps, int rope_knorm, float rope_base, const uint16_t *gain, float eps,
-                               float *part, uint32_t *err, void *o, int out_fp32, void *const *prof,
-                               cudaStream_t st) {
+                               const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv,
+                               float scale, int S, int64_t tps, int rope_knorm, float rope_base,
+                               const uint16_t *gain, float eps, float *part, uint32_t *err, void *o, int out_fp32,
+                               void *const *prof, cudaStream_t st) {
   clear_err_kernel<<<1, 1, 0, st>>>(err);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -396,7 +399,8 @@ cudaError_t launch_expand_simt(const uint16_t *q, const uint8_t *codes, int64_t 
   if (e != cudaSuccess) return e;
   record_prof_event(prof[0], st);
   expand_split_simt<<<dim3(S, (unsigned)B, n_kv), FSQ_HEAD_DIM, smem, st>>>(
-      q, codes, bstride, T, G, n_q, n_kv, W_kv, scale * kLog2e, tps, rope_knorm, rope_base, gain, eps, part);
+      q, codes, bstride, T, seq_lens, G, n_q, n_kv, W_kv, scale * kLog2e, tps, rope_knorm, rope_base, gain, eps,
+      part, err);
   e = cudaGetLastError();
   record_prof_event(prof[1], st);
   if (e != cudaSuccess) return e;

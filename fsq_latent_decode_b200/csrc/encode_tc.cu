@@ -11,8 +11,9 @@
 // with both operands K-major in that swizzled layout; after the last slice
 // all four warps read their 32 token rows of the accumulator from TMEM, count
 // thresholds and store the packed bytes.  Every wait is bounded; a wait that
-// gives up records FSQ_ERR_TIMEOUT in a per-device error word (read by
-// fsq_encode_status) and the CTA drains its copies and exits.
+// gives up records FSQ_ERR_TIMEOUT in the caller's status word (if any), and
+// the CTA lets its copies and MMAs finish (waits with their own fixed limit)
+// and exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -20,9 +21,6 @@
 
 #include "common.cuh"
 #include "tc_ptx.cuh"
-
-// Error word of the tensor-core append path on this device (0 = ok, else -status).
-__device__ uint32_t g_encode_error;
 
 namespace fsq {
 namespace enc {
@@ -34,6 +32,7 @@ constexpr int kKc = 64;             // C elements per stage: one 128-byte swizzl
 constexpr int kStages = 6;
 constexpr int kThreads = 128;
 constexpr uint64_t kWaitNs = 1000000000ull;  // 1 s per wait
+constexpr uint64_t kDrainNs = 1000000000ull; // 1 s for in-flight copies and MMAs on the error path
 constexpr int kABytes = kM * kKc * 2;        // x slice per stage
 
 template <int NC>
@@ -46,7 +45,7 @@ struct ECfg {
 };
 
 struct EncMisc {
-  uint64_t full[kStages], empty[kStages], done;
+  uint64_t full[kStages], empty[kStages], done, never;
   uint32_t tmem_base;
   uint32_t abort;
 };
@@ -77,18 +76,6 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
       : "memory");
 }
 
-__device__ __forceinline__ bool test_bar(uint64_t *b, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(b)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
 // Bounded wait (gives up after kWaitNs or once *abort is set).
 __device__ __forceinline__ bool wait_ok(uint64_t *b, uint32_t parity, volatile uint32_t *abort) {
   return mbar_wait(b, parity, abort, kWaitNs);
@@ -97,7 +84,8 @@ __device__ __forceinline__ bool wait_ok(uint64_t *b, uint32_t parity, volatile u
 template <int NC>
 __global__ void __launch_bounds__(kThreads, 1)
     encode_pack_tc(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap te, int64_t n_tok,
-                   int64_t C, int G, Thresholds th, uint8_t *__restrict__ codes, int64_t ldc) {
+                   int64_t C, int G, Thresholds th, uint8_t *__restrict__ codes, int64_t ldc, uint32_t *status,
+                   uint32_t stall_ns) {
   using EC = ECfg<NC>;
   extern __shared__ __align__(1024) uint8_t esm[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(esm) + 1023) & ~uintptr_t(1023));
@@ -114,6 +102,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&ms.empty[s], 1);
     }
     mbar_init(&ms.done, 1);
+    mbar_init(&ms.never, 1);  // completed by nothing: the test-only stall waits on it
     ms.abort = 0u;
     fence_mbar_init();
   }
@@ -126,7 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tm = ms.tmem_base;
   auto fail = [&]() {
-    atomicCAS(&g_encode_error, 0u, (uint32_t)(-FSQ_ERR_TIMEOUT));
+    if (status) atomicCAS(status, 0u, (uint32_t)(-FSQ_ERR_TIMEOUT));
     *abort = 1u;
   };
 
@@ -150,12 +139,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) {
         fail();
         // let the copies in flight land before the CTA exits
-        for (int c = max(0, issued - kStages); c < issued; ++c) {
-          const uint64_t t0 = globaltimer_ns();
-          while (!test_bar(&ms.full[c % kStages], (uint32_t)(c / kStages) & 1u) &&
-                 globaltimer_ns() - t0 < kWaitNs / 4) {
-          }
-        }
+        for (int c = max(0, issued - kStages); c < issued; ++c)
+          mbar_wait_fixed(&ms.full[c % kStages], (uint32_t)(c / kStages) & 1u, kDrainNs);
       }
     }
   } else if (warp == 1) {
@@ -183,7 +168,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   // ---------------------------------------------------------------- epilogue: all four warps
   __syncwarp();
-  const bool ok = wait_ok(&ms.done, 0, abort) && *abort == 0u;
+  // test-only stall: a wait that runs out on purpose (nothing completes `never`)
+  if (stall_ns != 0u && !mbar_wait(&ms.never, 0, abort, stall_ns) && lane == 0) fail();
+  __syncwarp();
+  // the MMAs must be complete before TMEM is read or freed, error or not: this
+  // wait ignores the abort flag and keeps its own limit
+  const bool ok = mbar_wait_fixed(&ms.done, 0, kDrainNs) && *abort == 0u;
   if (!ok) {
     if (lane == 0) fail();
   } else {
@@ -251,7 +241,8 @@ cudaError_t make_bf16_map(CUtensorMap *map, const uint16_t *base, int64_t rows, 
 
 template <int NC>
 cudaError_t launch_nc(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C, const uint16_t *E, int G,
-                      const Thresholds &th, uint8_t *codes, int64_t ldc, cudaStream_t s) {
+                      const Thresholds &th, uint8_t *codes, int64_t ldc, uint32_t *status, uint32_t stall_ns,
+                      cudaStream_t s) {
   using EC = ECfg<NC>;
   CUtensorMap tx, te;
   cudaError_t e = make_bf16_map(&tx, x, n_tok, C, ldx, kM);
@@ -262,7 +253,7 @@ cudaError_t launch_nc(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C, 
   if (e != cudaSuccess) return e;
   const int gp = (G + 15) / 16 * 16;
   const dim3 grid((unsigned)(gp / NC), (unsigned)((n_tok + kM - 1) / kM));
-  encode_pack_tc<NC><<<grid, kThreads, EC::SMEM, s>>>(tx, te, n_tok, C, G, th, codes, ldc);
+  encode_pack_tc<NC><<<grid, kThreads, EC::SMEM, s>>>(tx, te, n_tok, C, G, th, codes, ldc, status, stall_ns);
   return cudaGetLastError();
 }
 
@@ -270,24 +261,14 @@ cudaError_t launch_nc(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C, 
 
 // Tensor-core append for n_tok tokens; C a multiple of 64, G even <= 256.
 cudaError_t launch_encode_pack_tc(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C, const uint16_t *E, int G,
-                                  const Thresholds &th, uint8_t *codes, int64_t ldc, cudaStream_t s) {
+                                  const Thresholds &th, uint8_t *codes, int64_t ldc, uint32_t *status,
+                                  uint32_t stall_ns, cudaStream_t s) {
   if (n_tok > (int64_t)65535 * enc::kM || C > 0x7fffffffLL) return cudaErrorInvalidValue;
   const int gp = (G + 15) / 16 * 16;
-  if (gp % 64 == 0) return enc::launch_nc<64>(x, n_tok, ldx, C, E, G, th, codes, ldc, s);
-  if (gp % 48 == 0) return enc::launch_nc<48>(x, n_tok, ldx, C, E, G, th, codes, ldc, s);
-  if (gp % 32 == 0) return enc::launch_nc<32>(x, n_tok, ldx, C, E, G, th, codes, ldc, s);
-  return enc::launch_nc<16>(x, n_tok, ldx, C, E, G, th, codes, ldc, s);
-}
-
-// Reads and clears the error word of the tensor-core append path on the
-// current device (synchronises with the stream first).
-cudaError_t encode_status(uint32_t *out, cudaStream_t s) {
-  cudaError_t e = cudaStreamSynchronize(s);
-  if (e != cudaSuccess) return e;
-  e = cudaMemcpyFromSymbol(out, g_encode_error, sizeof(uint32_t));
-  if (e != cudaSuccess) return e;
-  const uint32_t zero = 0;
-  return cudaMemcpyToSymbol(g_encode_error, &zero, sizeof(uint32_t));
+  if (gp % 64 == 0) return enc::launch_nc<64>(x, n_tok, ldx, C, E, G, th, codes, ldc, status, stall_ns, s);
+  if (gp % 48 == 0) return enc::launch_nc<48>(x, n_tok, ldx, C, E, G, th, codes, ldc, status, stall_ns, s);
+  if (gp % 32 == 0) return enc::launch_nc<32>(x, n_tok, ldx, C, E, G, th, codes, ldc, status, stall_ns, s);
+  return enc::launch_nc<16>(x, n_tok, ldx, C, E, G, th, codes, ldc, status, stall_ns, s);
 }
 
 }  // namespace fsq

@@ -126,13 +126,14 @@ __global__ void quantize_pack_f32_kernel(const float *__restrict__ u, int64_t n_
 }  // namespace
 
 cudaError_t launch_encode_pack_tc(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C, const uint16_t *E, int G,
-                                  const Thresholds &th, uint8_t *codes, int64_t ldc, cudaStream_t s);
+                                  const Thresholds &th, uint8_t *codes, int64_t ldc, uint32_t *status,
+                                  uint32_t stall_ns, cudaStream_t s);
 
 // Decode-step appends (up to 64 tokens) on CUDA cores; prefill-sized ones on
 // the tensor cores (encode_tc.cu).
 cudaError_t launch_encode_pack_simt(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C,
                                     const uint16_t *E, int G, const Thresholds &th, uint8_t *codes,
-                                    int64_t ldc, cudaStream_t s) {
+                                    int64_t ldc, uint32_t *status, uint32_t stall_ns, cudaStream_t s) {
   if (n_tok <= kFewTok) {
     return launch_pdl(encode_pack_few, dim3((unsigned)(G / 2)), dim3(kFewWarps * 32), 0, s, x, (int)n_tok, ldx, C, E,
                       G, th, codes, ldc);
@@ -142,7 +143,7 @@ cudaError_t launch_encode_pack_simt(const uint16_t *x, int64_t n_tok, int64_t ld
     encode_pack_rows<<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(x, n_tok, ldx, C, E, G, th, codes, ldc);
     return cudaGetLastError();
   }
-  return launch_encode_pack_tc(x, n_tok, ldx, C, E, G, th, codes, ldc, s);
+  return launch_encode_pack_tc(x, n_tok, ldx, C, E, G, th, codes, ldc, status, stall_ns, s);
 }
 
 cudaError_t launch_quantize_pack_f32(const float *u, int64_t n_tok, int G, const Thresholds &th,

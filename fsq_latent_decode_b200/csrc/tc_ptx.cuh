@@ -50,6 +50,19 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *b, uint32_t parity, volatile
   }
 }
 
+// Waits for the phase with the given parity for up to `limit_ns`, whatever
+// any abort flag says: the error paths use it so that no copy or tensor-core
+// operation is still in flight when a CTA frees its memory and exits.
+__device__ __forceinline__ bool mbar_wait_fixed(uint64_t *b, uint32_t parity, uint64_t limit_ns) {
+  if (mbar_try_wait(b, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    for (int i = 0; i < 64; ++i)
+      if (mbar_try_wait(b, parity)) return true;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }

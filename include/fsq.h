@@ -19,16 +19,16 @@
  * Conventions shared by every call
  *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
  *    never allocates device memory at run time and never synchronises the
- *    host (except fsq_workspace_status and fsq_encode_status, which say so).
- *    Its only device state is the error word of the append path and the
- *    scratch of fsq_decode_attn_noalloc (file-scope arrays of the library).
+ *    host (except the status readers, which say so).  It keeps no state
+ *    between calls; its only device memory of its own is the scratch of
+ *    fsq_decode_attn_noalloc (a file-scope array of the library).
  *  - bf16 means IEEE bfloat16 stored as uint16; row-major throughout.
  *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default).
  *  - Argument errors are returned synchronously, before anything is
  *    launched.  A failed launch returns FSQ_ERR_CUDA.  A bounded device-side
- *    wait that gives up records FSQ_ERR_TIMEOUT (in the workspace's error
- *    word, see fsq_workspace_status; for the append path see
- *    fsq_encode_status) instead of hanging or trapping.
+ *    wait that gives up records FSQ_ERR_TIMEOUT in a caller-owned status word
+ *    (decode: the workspace's error word; append: fsq_encode_opts.status_word;
+ *    read either with fsq_workspace_status) instead of hanging or trapping.
  *  - The decode kernels use programmatic dependent launch: the first of
  *    them may start before the kernel preceding the call on the stream has
  *    finished, and reads q and W_kv early.  If that kernel is itself a
@@ -103,10 +103,25 @@ typedef struct {
   void *prof_events[2];   /* optional cudaEvent_t pair: recorded on `stream`
                              right before and right after the main attention
                              kernel (for timing it alone); NULL = none */
+  const int32_t *seq_lens; /* optional device int32 [B]: batch row b attends to
+                             its first seq_lens[b] cached tokens (a ragged
+                             batch; 1 <= seq_lens[b] <= T, where T is the call's
+                             argument, the longest row).  NULL = T for every
+                             row.  A value outside [1, T] is clamped into it and
+                             records FSQ_ERR_INVALID_ARG in the workspace's error
+                             word.  Read by the kernels like q and codes. */
+  uint32_t debug_stall_ns; /* test-only, 0 in normal use.  When > 0, the tensor-
+                             core attention kernel first waits, with this limit
+                             in nanoseconds, for a barrier that nothing
+                             completes, so that its bounded-wait failure path
+                             runs: the call records FSQ_ERR_TIMEOUT and its
+                             output is undefined.  Only that wait uses the
+                             limit; the waits that let in-flight copies and
+                             tensor-core operations finish keep their own. */
 } fsq_attn_opts;
 
 /* Fills *opts with {AUTO, 1/sqrt(d_h), auto splits, rope off, 1e6, NULL,
- * 1e-6, bf16 output, no profiling events}. */
+ * 1e-6, bf16 output, no profiling events, no per-row lengths, no stall}. */
 FSQ_API void fsq_attn_opts_default(fsq_attn_opts *opts);
 
 /* Host-side: the 15 ascending u-space decision thresholds the kernels
@@ -117,11 +132,30 @@ FSQ_API void fsq_attn_opts_default(fsq_attn_opts *opts);
  * boundaries are +/-infinity.  Returns FSQ_ERR_INVALID_ARG for bad params. */
 FSQ_API fsq_status fsq_thresholds(fsq_quant_params qp, float theta_out[15]);
 
+/* Options of the append path. */
+typedef struct {
+  uint32_t *status_word;   /* optional device pointer to a caller-owned 32-bit
+                             word.  When the tensor-core append kernel (used for
+                             more than 64 tokens) gives up a bounded wait, it
+                             records FSQ_ERR_TIMEOUT there and the codes of that
+                             call are incomplete.  The library only ever sets
+                             the word (the first error stays) and never clears
+                             it: zero it before use, read it with
+                             fsq_workspace_status(word, 4, stream).  NULL: such
+                             a failure is reported nowhere. */
+  uint32_t debug_stall_ns; /* test-only, 0 in normal use.  When > 0, the
+                             tensor-core append kernel's epilogue first waits,
+                             with this limit in nanoseconds, for a barrier that
+                             nothing completes, so that its bounded-wait failure
+                             path runs (FSQ_ERR_TIMEOUT in status_word). */
+} fsq_encode_opts;
+
 /* Append path ([S] eq. 4 then packing; [D] product-code frame):
  *   u = E x_t (bf16 operands, fp32 accumulation), level = eq. (2), packed.
  *  x      bf16 [n_tok, ldx], row t = x_t (C used entries)      — read
  *  E      bf16 [G, C] encoder                                    — read
  *  codes  uint8 [n_tok, ldc_bytes]; row t gets G/2 bytes          — written
+ *  opts   may be NULL (no status word, no stall)
  * To append at position T of a [T_max, G/2] cache pass codes + T*G/2 and
  * ldc_bytes = G/2.  Needs: G even, 2 <= G <= 256; C a positive multiple of
  * 64; ldx >= C and ldx % 8 == 0; x and E 16-byte aligned.  n_tok == 0 is a
@@ -129,14 +163,8 @@ FSQ_API fsq_status fsq_thresholds(fsq_quant_params qp, float theta_out[15]);
  * itself differs from exact arithmetic by the GEMM's rounding. */
 FSQ_API fsq_status fsq_encode_pack(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C,
                            const uint16_t *E, int G, fsq_quant_params qp,
-                           uint8_t *codes, int64_t ldc_bytes, fsq_stream_t stream);
-
-/* Reads and clears the device error word of the append path's tensor-core
- * kernel (used by fsq_encode_pack for more than 64 tokens) on the current
- * device.  Returns FSQ_OK, the recorded device status (FSQ_ERR_TIMEOUT: a
- * bounded wait gave up, the codes of that call are incomplete), or
- * FSQ_ERR_CUDA.  Blocking: synchronises with `stream` first. */
-FSQ_API fsq_status fsq_encode_status(fsq_stream_t stream);
+                           uint8_t *codes, int64_t ldc_bytes, const fsq_encode_opts *opts,
+                           fsq_stream_t stream);
 
 /* Quantiser + packing alone on given fp32 pre-activations u [n_tok, G]
  * (row-major, contiguous).  Same codes as fsq_encode_pack would write for
@@ -154,8 +182,9 @@ FSQ_API size_t fsq_decode_attn_workspace_size(int64_t B, int64_t T, int n_q, int
  * For batch row b and query head h, with kv head j = h / (n_q / n_kv):
  *   k_t = W_k^(j) z_t (RoPE_t(N_k(.)) when opts->rope_knorm), v_t = W_v^(j) z_t
  *   o_h = sum_t softmax_t(scale * q_h . k_t) v_t                 ([S] eq. 5)
- * over cached tokens t = 0..T-1 (the caller appends the current token first;
- * cached token t sits at position t).  ABSORBED evaluates the same sum as
+ * over cached tokens t = 0..T-1, or t = 0..seq_lens[b]-1 for a ragged batch
+ * (the caller appends the current token first; cached token t sits at
+ * position t).  ABSORBED evaluates the same sum as
  * (W_k^T q_h) . z_t and W_v (sum_t a_t z_t) ([S] eq. 6).
  *  q        bf16 [B, n_q, d_h], already projected/normed/rotated by the caller
  *  codes    uint8 cache, rows as in the format above
@@ -185,9 +214,10 @@ FSQ_API fsq_status fsq_decode_attn(const uint16_t *q, int64_t B, int n_q, int d_
  * FSQ_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads
  * the library holds until the process exits.  Nothing is allocated: no
  * cudaMalloc, cudaFree or allocating library routine is called.
- *  - The first call on a device looks up that array's device address
- *    (cudaGetSymbolAddress, with the device current); make that first call
- *    before any stream capture.
+ *  - The first call in a device's CUDA context looks up that array's device
+ *    address there (cudaGetSymbolAddress, with the device current) and keeps
+ *    it for that context; a reset device gets a new context and a new lookup.
+ *    Make the first call before any stream capture.
  *  - Requests whose fsq_decode_attn_workspace_size exceeds
  *    FSQ_NOALLOC_SCRATCH_BYTES return FSQ_ERR_WORKSPACE before any launch
  *    (use fsq_decode_attn with a workspace of your own for those).
@@ -201,9 +231,20 @@ FSQ_API fsq_status fsq_decode_attn_noalloc(const uint16_t *q, int64_t B, int n_q
                                            int G, const uint16_t *W_kv, int n_kv, const fsq_attn_opts *opts,
                                            void *o, fsq_stream_t stream);
 
-/* Reads the device error word of a workspace last used by fsq_decode_attn
- * (blocking copy: synchronises with `stream`).  Returns FSQ_OK or the
- * recorded device status (e.g. FSQ_ERR_TIMEOUT); clears nothing. */
+/* The device status of the last fsq_decode_attn_noalloc call on the current
+ * device: the error word of the built-in scratch, which each call clears
+ * first (the same word fsq_workspace_status reads in a caller's workspace).
+ * Returns FSQ_OK or the recorded status, e.g. FSQ_ERR_TIMEOUT when a
+ * bounded device wait of that call gave up and its output is undefined.
+ * Blocking: synchronises with `stream`.  A device with no call yet reads
+ * FSQ_OK. */
+FSQ_API fsq_status fsq_decode_attn_noalloc_status(fsq_stream_t stream);
+
+/* Reads a device status word: the error word at the start of a workspace
+ * last used by fsq_decode_attn (each decode call clears it first), or an
+ * append path's fsq_encode_opts.status_word (workspace_bytes >= 4).  Blocking
+ * copy: synchronises with `stream`.  Returns FSQ_OK or the recorded device
+ * status (e.g. FSQ_ERR_TIMEOUT); clears nothing. */
 FSQ_API fsq_status fsq_workspace_status(const void *workspace, size_t workspace_bytes, fsq_stream_t stream);
 
 FSQ_API const char *fsq_status_string(fsq_status s);

@@ -207,7 +207,7 @@ def softmax(s):
 # ---------------------------------------------------------------------------
 # Decode attention: expanded K/V, then standard GQA softmax attention
 # ---------------------------------------------------------------------------
-def decode_attn(q, codes, W_kv, n_kv, G, scale=None, rope_knorm=None, rows=None, heads=None):
+def decode_attn(q, codes, W_kv, n_kv, G, scale=None, rope_knorm=None, rows=None, heads=None, lengths=None):
     """Single-token GQA decode attention over a packed FSQ code cache.
 
     q: [B, n_q, d_h]; codes: [B, T, G/2] uint8; W_kv: [2*n_kv*d_h, G].
@@ -216,6 +216,8 @@ def decode_attn(q, codes, W_kv, n_kv, G, scale=None, rope_knorm=None, rows=None,
         o_h = sum_t a_t v_t.
     rows / heads optionally restrict the computation to a sample (others are
     left as NaN) so large caches can be checked one output at a time.
+    lengths: optional per-row token counts (a ragged batch): row b attends to
+    its first lengths[b] cached tokens only.
     Returns o [B, n_q, d_h] fp64.
     """
     q = np.asarray(q, dtype=np.float64)
@@ -229,7 +231,7 @@ def decode_attn(q, codes, W_kv, n_kv, G, scale=None, rope_knorm=None, rows=None,
     heads = range(n_q) if heads is None else heads
     o = np.full((B, n_q, d_h), np.nan)
     for b in rows:
-        lv = unpack(codes[b], G)
+        lv = unpack(codes[b] if lengths is None else codes[b][: int(lengths[b])], G)
         need_j = sorted({h // grp for h in heads})
         Wk, Wv = split_wkv(W_kv, n_kv, d_h)
         for j in need_j:

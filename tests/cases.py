@@ -57,9 +57,26 @@ def decoder_weights(n_q, n_kv, G, B, seed, d_h=128):
     return W_kv, q
 
 
-def gemm_error_bound(x, E):
-    """fp32 forward-error bound gamma_C * sum_c |E_ic x_tc| of the encoder GEMM."""
+def gemm_error_bound(x, E, unit_roundoff=2.0 ** -23):
+    """Forward-error bound gamma_C * sum_c |E_ic x_tc| of an fp32 dot product of
+    length C, gamma_C = C u / (1 - C u) (the classical bound for summation in any
+    order with unit roundoff u; Higham, Accuracy and Stability of Numerical
+    Algorithms, section 3.1).  The bf16 x bf16 products are exact in fp32, so
+    only the accumulation rounds.  u = 2^-23, one fp32 ulp rather than half of
+    one: the tensor core's fp32 accumulation is not specified to round to
+    nearest, and this value also covers truncating (round-toward-zero) adds."""
     Cdim = x.shape[1]
-    u = 2.0 ** -24
+    u = unit_roundoff
     gam = Cdim * u / (1 - Cdim * u)
     return gam * (np.abs(np.asarray(x, np.float64)) @ np.abs(np.asarray(E, np.float64)).T)
+
+
+def record(kind: str, **fields):
+    """Appends one JSON line to $FSQ_PARITY_RECORD (if set): counts that a GPU
+    run reports, such as code mismatches near a rounding boundary."""
+    import json
+    import os
+    path = os.environ.get("FSQ_PARITY_RECORD")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(dict(kind=kind, **fields)) + "\n")

@@ -29,6 +29,26 @@ def test_header_symbols_are_exported():
         assert hasattr(F.lib, n), n
 
 
+def test_noalloc_scratch_size_matches_header():
+    src = open(os.path.join(ROOT, "include", "fsq.h")).read()
+    m = re.search(r"#define\s+FSQ_NOALLOC_SCRATCH_BYTES\s+\((\d+)u\s*<<\s*(\d+)\)", src)
+    assert m, "FSQ_NOALLOC_SCRATCH_BYTES not found in include/fsq.h"
+    assert _abi.NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
+
+
+def test_struct_layouts_match_header():
+    """The ctypes mirrors of fsq_attn_opts and fsq_encode_opts list the header's fields in order."""
+    src = open(os.path.join(ROOT, "include", "fsq.h")).read()
+
+    def fields(struct):
+        body = re.search(r"typedef struct \{([^{}]*)\}\s*" + struct + ";", src).group(1)
+        body = re.sub(r"/\*.*?\*/", "", body, flags=re.S)
+        return [re.findall(r"(\w+)\s*(?:\[\d+\])?\s*$", d.strip())[0] for d in body.split(";") if d.strip()]
+
+    assert fields("fsq_attn_opts") == [f[0] for f in _abi.AttnOpts._fields_]
+    assert fields("fsq_encode_opts") == [f[0] for f in _abi.EncodeOpts._fields_]
+
+
 def test_format_version_and_status_strings():
     assert F.lib.fsq_format_version() == 1
     for s in range(0, -7, -1):
@@ -85,6 +105,9 @@ def test_invalid_arguments_return_before_launch():
     assert F.encode_pack_raw(16, 4, 68, 64, 16, 256, qp, 16, 128, null) == F.FSQ_ERR_MISALIGNED
     assert F.encode_pack_raw(16, 4, 64, 64, 16, 256, F.quant_params(9.0, 0.5), 16, 128, null) == F.FSQ_ERR_INVALID_ARG
     assert F.encode_pack_raw(null, 0, 64, 64, null, 256, qp, null, 128, null) == F.FSQ_OK  # empty: no-op
+    bad_word = F.encode_opts()
+    bad_word.status_word = 18  # a status word must be 4-byte aligned
+    assert F.encode_pack_raw(16, 4, 64, 64, 16, 256, qp, 16, 128, null, bad_word) == F.FSQ_ERR_MISALIGNED
     assert F.quantize_pack_f32_raw(null, 3, 256, qp, null, 128, null) == F.FSQ_ERR_INVALID_ARG
     assert F.quantize_pack_f32_raw(8, 3, 256, qp, 16, 128, null) == F.FSQ_ERR_MISALIGNED
     # decode
@@ -111,3 +134,10 @@ def test_invalid_arguments_return_before_launch():
     assert call(ws=None) == F.FSQ_ERR_WORKSPACE
     assert call(ws=272) == F.FSQ_ERR_MISALIGNED
     assert call(B=0, q=None, codes=None, w=None) == F.FSQ_OK  # empty batch: no-op
+    o.seq_lens = 18  # per-row lengths must be 4-byte aligned int32
+    assert call() == F.FSQ_ERR_MISALIGNED
+    o.seq_lens = None
+    # status words: null and misaligned pointers are refused before any copy
+    assert F.lib.fsq_workspace_status(None, 256, None) == F.FSQ_ERR_INVALID_ARG
+    assert F.lib.fsq_workspace_status(16, 2, None) == F.FSQ_ERR_INVALID_ARG
+    assert F.lib.fsq_workspace_status(18, 4, None) == F.FSQ_ERR_MISALIGNED

@@ -232,6 +232,27 @@ def test_reduces_to_torch_sdpa(shape):
     assert np.abs(o - ref).max() <= 1e-12 * max(1.0, np.abs(ref).max())
 
 
+def test_ragged_lengths_reduce_to_masked_sdpa():
+    """Per-row lengths (a ragged batch) equal torch SDPA with a key mask that
+    hides each row's tokens past its length; a row of length 1 returns that
+    token's value."""
+    B, n_q, n_kv, d_h, G, T = 3, 8, 2, 16, 12, 41
+    q, codes, W, n_kv, G = _rand_case(8, B, n_q, n_kv, d_h, G, T)
+    lengths = [1, 17, 41]
+    o = O.decode_attn(q, codes, W, n_kv, G, lengths=lengths)
+    K = np.stack([O.reconstruct_kv(O.unpack(codes[b], G), W, n_kv, d_h)[0] for b in range(B)])
+    V = np.stack([O.reconstruct_kv(O.unpack(codes[b], G), W, n_kv, d_h)[1] for b in range(B)])
+    keep = torch.arange(T)[None, :] < torch.tensor(lengths)[:, None]
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q)[:, :, None, :], torch.from_numpy(K), torch.from_numpy(V),
+        attn_mask=keep[:, None, None, :], enable_gqa=True)[:, :, 0, :].numpy()
+    assert np.abs(o - ref).max() <= 1e-12 * max(1.0, np.abs(ref).max())
+    grp = n_q // n_kv
+    for h in range(n_q):
+        assert np.allclose(o[0, h], V[0, h // grp, 0], atol=1e-12)
+    assert np.array_equal(O.decode_attn(q, codes, W, n_kv, G, lengths=[T] * B), O.decode_attn(q, codes, W, n_kv, G))
+
+
 def test_value_pooling_identity_eq6():
     for seed in range(3):
         q, codes, W, n_kv, G = _rand_case(10 + seed, B=2, n_q=32, n_kv=8, d_h=128, G=84, T=200)
