@@ -226,9 +226,19 @@ def run_gpu(args, wl_name, B, T, torch, F, synth, dist, rank, world, device, tim
     out = torch.empty((B, wl.n_q, wl.d_h), dtype=torch.bfloat16, device=device)
     stream = torch.cuda.current_stream()
     qp = F.quant_params()
-    nbytes_ws = F.workspace_size(B, T, wl.n_q, wl.n_kv, wl.d_h, G, F.attn_opts(variant=args.variant))
+    nbytes_ws = F.workspace_size(B, T, wl.n_q, wl.n_kv, wl.d_h, G,
+                                 F.attn_opts(variant=args.variant, rope_knorm=args.rope))
     wbuf = ws.get(nbytes_ws)
     sptr = stream.cuda_stream
+    gain = None
+    if args.rope:  # key RMS-norm gain ~ 1 + N(0, 0.1^2), seeded
+        g_gen = torch.Generator(device=device)
+        g_gen.manual_seed(rank_seed(synth, rank, B, T, G) + 17)
+        gain = (1.0 + 0.1 * torch.randn(wl.d_h, generator=g_gen, device=device)).to(torch.bfloat16)
+
+    def make_opts(prof=None):
+        return F.attn_opts(variant=args.variant, prof_events=prof, rope_knorm=args.rope, rope_base=1.0e6,
+                           knorm_gain=gain, knorm_eps=1e-6)
 
     def step(i, prof=None):
         cache = st["caches"][i % n_copies]
@@ -237,7 +247,7 @@ def run_gpu(args, wl_name, B, T, torch, F, synth, dist, rank, world, device, tim
                                cache.data_ptr() + (T - 1) * half, bstride, sptr)
         if rc:
             raise F.FsqError(rc, "fsq_encode_pack")
-        opts = F.attn_opts(variant=args.variant, prof_events=prof)
+        opts = make_opts(prof)
         rc = F.decode_attn_raw(q.data_ptr(), B, wl.n_q, wl.d_h, cache.data_ptr(), bstride, T, G,
                                W_kv.data_ptr(), wl.n_kv, opts, wbuf.data_ptr(), wbuf.numel(), out.data_ptr(), sptr)
         if rc:
@@ -315,7 +325,7 @@ def run_gpu(args, wl_name, B, T, torch, F, synth, dist, rank, world, device, tim
                 if rc:
                     raise F.FsqError(rc, "fsq_encode_pack")
                 rc = F.decode_attn_raw(q_d[s_].data_ptr(), B, wl.n_q, wl.d_h, cache.data_ptr(), bstride, T, G,
-                                       W_kv.data_ptr(), wl.n_kv, F.attn_opts(variant=args.variant), wbuf.data_ptr(),
+                                       W_kv.data_ptr(), wl.n_kv, make_opts(), wbuf.data_ptr(),
                                        wbuf.numel(), o_d[s_].data_ptr(), sptr)
                 if rc:
                     raise F.FsqError(rc, "fsq_decode_attn")
@@ -346,7 +356,7 @@ def run_gpu(args, wl_name, B, T, torch, F, synth, dist, rank, world, device, tim
                "copies": "pinned host buffers; a second stream carries step i+1's inputs up and step i's output "
                          "back while step i computes (double-buffered, event-ordered)"}
     return dict(ms=ms, kern_ms=kern_ms, clocks=clk, e2e=e2e, n_copies=n_copies, wl=wl, B=B, T=T,
-                code_bytes=code_bytes)
+                code_bytes=code_bytes, variant=args.variant, rope=args.rope)
 
 
 def roofline(res, peaks, kernel_name):
@@ -355,9 +365,21 @@ def roofline(res, peaks, kernel_name):
     step (append, query prologue, split kernel, merge) is reported beside it as
     `frac_of_roofline_step` when its device time is known."""
     wl, B, T = res["wl"], res["B"], res["T"]
-    G, n_q, d_h = wl.G, wl.n_q, wl.d_h
+    G, n_q, n_kv, d_h = wl.G, wl.n_q, wl.n_kv, wl.d_h
+    variant, rope = res.get("variant", "absorbed"), res.get("rope", False)
     bytes_alg = B * T * (G // 2)
-    flops_alg = B * T * 4 * n_q * G  # scores + latent pooling; per-query W_k^T q and W_v run outside this kernel
+    if rope:
+        # keys must be rebuilt per position (RoPE): key expansion + scores + latent pooling
+        flops_alg = B * T * (2 * n_kv * d_h * G + 2 * n_q * d_h + 2 * n_q * G)
+    else:
+        flops_alg = B * T * 4 * n_q * G  # scores + latent pooling; per-query W_k^T q and W_v run outside this kernel
+    # tensor-core work the variant actually issues per token (its own utilisation)
+    if variant == "expand":
+        flops_variant = B * T * (2 * 2 * n_kv * d_h * G + 2 * n_q * d_h * 2)
+    elif variant == "hybrid":
+        flops_variant = B * T * (2 * n_kv * d_h * G + 2 * n_q * d_h + 2 * n_q * G)
+    else:
+        flops_variant = flops_alg
     t = res["kern_ms"] * 1e-3
     t_b = bytes_alg / (peaks["hbm_gbs"] * 1e9)
     t_f = flops_alg / (peaks["bf16_tflops"] * 1e12)
@@ -370,6 +392,9 @@ def roofline(res, peaks, kernel_name):
     else:
         ach = bytes_alg / t / 1e9
         r = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": ach / peaks["hbm_gbs"]}
+    r["variant_flops"] = flops_variant
+    r["variant_tflops"] = flops_variant / t / 1e12
+    r["variant_frac_of_tensor_peak"] = flops_variant / t / 1e12 / peaks["bf16_tflops"]
     r.update({"traffic": traffic, "kernel": kernel_name, "kernel_ms": res["kern_ms"],
               "scope": "split (attention) kernel only; the step adds the append, the query prologue and the merge",
               "code_gbs": bytes_alg / t / 1e9, "frac_of_roofline": max(t_b, t_f) / t,
@@ -580,7 +605,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD[0])
     ap.add_argument("--B", type=int, default=None)
     ap.add_argument("--T", type=int, default=None)
-    ap.add_argument("--variant", default="absorbed", choices=["absorbed", "expand"])
+    ap.add_argument("--variant", default="absorbed", choices=["absorbed", "expand", "hybrid"])
+    ap.add_argument("--rope", action="store_true", help="key RMS-norm + RoPE on (the pages' full key path)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-second", action="store_true", help="skip the G=84 companion measurement")
     ap.add_argument("--no-sdpa", action="store_true", help="skip the uncompressed-cache SDPA context measurement")
@@ -603,7 +629,8 @@ def main():
     config = {"workload": f"{wl_name}: Qwen3-8B-shaped layer, n_q={wl.n_q} n_kv={wl.n_kv} d_h={wl.d_h} G={wl.G} "
                           f"({wl.G // 2} B/token), C={wl.C}, batch {B} per GPU, T={T}",
               "B_per_gpu": B, "T": T, "G": wl.G, "n_q": wl.n_q, "n_kv": wl.n_kv, "d_h": wl.d_h, "C": wl.C,
-              "variant": args.variant, "parallelism": f"replicas x{world} (batch rows sharded, no collective)"}
+              "variant": args.variant, "rope_knorm": args.rope,
+              "parallelism": f"replicas x{world} (batch rows sharded, no collective)"}
 
     if args.impl == "reference":
         if rank != 0:
@@ -631,7 +658,7 @@ def main():
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     peaks = load_peaks()
-    kernel_name = "absorbed_split" if args.variant == "absorbed" else "expand_split"
+    kernel_name = {"absorbed": "absorbed_split", "expand": "expand_split", "hybrid": "hybrid_split"}[args.variant]
     res = run_gpu(args, wl_name, B, T, torch, F, synth, dist, rank, world, device)
     also = None
     if not args.no_second and wl_name == DEFAULT_WORKLOAD[0] and args.B is None and args.T is None:
@@ -674,7 +701,12 @@ def main():
                 "value": value, "unit": "context tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": res["ms"], "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None,
-                "dtype": "u4 codes; s8 x u8 score MMA (s32), f16 pooling MMA (f32), f32 softmax/merge, bf16 in/out",
+                "dtype": {"absorbed": "u4 codes; s8 x u8 score MMA (s32), f16 pooling MMA (f32), f32 softmax/merge, "
+                                      "bf16 in/out",
+                          "hybrid": "u4 codes; f16 key, score and pooling MMAs (f32), f32 key norm/RoPE/softmax/merge, "
+                                    "bf16 in/out",
+                          "expand": "u4 codes; f16 key, value, score and output MMAs (f32), f32 softmax/merge, "
+                                    "bf16 in/out"}[args.variant],
                 "data": "synthetic (seeded; cache = FSQ codes of u ~ N(0,4), the law of E x; new token x ~ N(0,1) appended each step)",
                 "config": config, "l2": l2, "code_gbs": world * res["code_bytes"] / (res["ms"] * 1e-3) / 1e9,
                 "roofline": rf, "cpu_baseline": cb, "e2e": res["e2e"], "clocks": res["clocks"],

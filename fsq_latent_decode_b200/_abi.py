@@ -23,8 +23,8 @@ FSQ_ERR_WORKSPACE = -4
 FSQ_ERR_CUDA = -5
 FSQ_ERR_TIMEOUT = -6
 
-VARIANT_AUTO, VARIANT_ABSORBED, VARIANT_EXPAND = 0, 1, 2
-VARIANTS = {"auto": VARIANT_AUTO, "absorbed": VARIANT_ABSORBED, "expand": VARIANT_EXPAND}
+VARIANT_AUTO, VARIANT_ABSORBED, VARIANT_EXPAND, VARIANT_HYBRID = 0, 1, 2, 3
+VARIANTS = {"auto": VARIANT_AUTO, "absorbed": VARIANT_ABSORBED, "expand": VARIANT_EXPAND, "hybrid": VARIANT_HYBRID}
 
 # Every symbol include/fsq.h declares.
 EXPORTED = ("fsq_attn_opts_default", "fsq_thresholds", "fsq_encode_pack", "fsq_quantize_pack_f32",
@@ -142,12 +142,17 @@ def attn_opts(variant="auto", scale=0.0, num_splits=0, rope_knorm=False, rope_ba
         o.prof_events[1] = int(prof_events[1].cuda_event)
     o.seq_lens = None if seq_lens is None else int(seq_lens.data_ptr())  # device int32 [B]
     o.debug_stall_ns = int(debug_stall_ns)
+    # the struct holds raw device pointers: keep their tensors alive as long as it
+    # lives, or the allocator may hand their memory to the next buffer
+    o._tensors = (knorm_gain, seq_lens)
     return o
 
 
 def encode_opts(status_word=None, debug_stall_ns=0) -> EncodeOpts:
     """status_word: a device tensor whose first 4 bytes are the caller's status word."""
-    return EncodeOpts(None if status_word is None else int(status_word.data_ptr()), int(debug_stall_ns))
+    o = EncodeOpts(None if status_word is None else int(status_word.data_ptr()), int(debug_stall_ns))
+    o._tensors = (status_word,)  # keeps the word's memory alive with the struct
+    return o
 
 
 def _stream_ptr(stream) -> int:

@@ -22,6 +22,14 @@ cudaError_t launch_expand_simt(const uint16_t *q, const uint8_t *codes, int64_t 
                                float scale, int S, int64_t tps, int rope_knorm, float rope_base,
                                const uint16_t *gain, float eps, float *part, uint32_t *err, void *o, int out_fp32,
                                void *const *prof, cudaStream_t st);
+bool expand_tc_supported(int n_q, int n_kv, int G);
+size_t expand_tc_stage_bytes(int G, int variant_expand);
+cudaError_t launch_expand_tc(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
+                             const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv,
+                             float scale, int S, int64_t tps, int hybrid, int rope, float rope_base,
+                             const uint16_t *gain, float eps, uint8_t *wk, uint8_t *wv, float *ck, float *cv,
+                             uint8_t *qs, float *part, uint32_t *err, MergeScratch ms, void *o, int out_fp32,
+                             uint32_t stall_ns, void *const *prof, cudaStream_t st);
 int simt_max_nq();
 int simt_max_grp();
 bool absorbed_tc_supported(int n_q, int n_kv, int G);
@@ -66,11 +74,12 @@ void make_thresholds(fsq_quant_params qp, float out[15]) {
 
 struct Plan {
   int variant;
-  bool tc;        // tensor-core kernel (absorbed form)
+  bool tc;        // tensor-core kernel (absorbed, expand or hybrid form)
   int S;          // splits per batch row
   int64_t tps;    // tokens per split
-  MergePlan mp;   // split merge of the absorbed form
+  MergePlan mp;   // split merge of the absorbed and hybrid forms
   size_t off_qa, off_corr, off_part, off_mslab, off_mcnt, total;
+  size_t off_wk, off_wv, off_ck, off_cv;  // staged decoder slices of the tensor-core expand / hybrid forms
 };
 
 fsq_status plan_decode(int64_t B, int64_t T, int n_q, int n_kv, int d_h, int G, const fsq_attn_opts &op, Plan *p) {
@@ -78,24 +87,28 @@ fsq_status plan_decode(int64_t B, int64_t T, int n_q, int n_kv, int d_h, int G, 
   if (n_q % n_kv) return FSQ_ERR_INVALID_ARG;
   if (G % 2) return FSQ_ERR_UNSUPPORTED;
   if (G > FSQ_MAX_G || d_h != FSQ_HEAD_DIM) return FSQ_ERR_UNSUPPORTED;
-  if (op.variant < FSQ_VARIANT_AUTO || op.variant > FSQ_VARIANT_EXPAND) return FSQ_ERR_INVALID_ARG;
+  if (op.variant < FSQ_VARIANT_AUTO || op.variant > FSQ_VARIANT_HYBRID) return FSQ_ERR_INVALID_ARG;
   if (op.num_splits < 0) return FSQ_ERR_INVALID_ARG;
   if (op.rope_knorm != 0 && op.rope_knorm != 1) return FSQ_ERR_INVALID_ARG;
   int variant = op.variant;
-  if (variant == FSQ_VARIANT_AUTO) variant = op.rope_knorm ? FSQ_VARIANT_EXPAND : FSQ_VARIANT_ABSORBED;
+  const bool xtc_shape = kEnableTc && expand_tc_supported(n_q, n_kv, G);
+  if (variant == FSQ_VARIANT_AUTO)
+    variant = !op.rope_knorm ? FSQ_VARIANT_ABSORBED : (xtc_shape ? FSQ_VARIANT_HYBRID : FSQ_VARIANT_EXPAND);
   if (variant == FSQ_VARIANT_ABSORBED && op.rope_knorm) return FSQ_ERR_UNSUPPORTED;
   if (variant == FSQ_VARIANT_ABSORBED && n_q > simt_max_nq()) return FSQ_ERR_UNSUPPORTED;
-  if (variant == FSQ_VARIANT_EXPAND && n_q / n_kv > simt_max_grp()) return FSQ_ERR_UNSUPPORTED;
+  if (variant == FSQ_VARIANT_HYBRID && !xtc_shape) return FSQ_ERR_UNSUPPORTED;
+  if (variant == FSQ_VARIANT_EXPAND && !xtc_shape && n_q / n_kv > simt_max_grp()) return FSQ_ERR_UNSUPPORTED;
   if (op.rope_knorm && !(op.rope_base > 1.f && op.knorm_eps >= 0.f)) return FSQ_ERR_INVALID_ARG;
 
   const int64_t Bc = B > 0 ? B : 1;
-  const bool tc = kEnableTc && variant == FSQ_VARIANT_ABSORBED && absorbed_tc_supported(n_q, n_kv, G);
-  const int64_t ctas_per_row = variant == FSQ_VARIANT_EXPAND ? n_kv : 1;
+  const bool xtc = (variant == FSQ_VARIANT_EXPAND || variant == FSQ_VARIANT_HYBRID) && xtc_shape;
+  const bool tc = (kEnableTc && variant == FSQ_VARIANT_ABSORBED && absorbed_tc_supported(n_q, n_kv, G)) || xtc;
+  const int64_t ctas_per_row = (variant == FSQ_VARIANT_EXPAND || variant == FSQ_VARIANT_HYBRID) ? n_kv : 1;
   int64_t S = op.num_splits;
   if (S == 0) {
     if (tc) {
       // one CTA per SM (each holds all of TMEM): fill the 148 SMs in a single wave
-      S = kNumSMs / Bc;
+      S = kNumSMs / (Bc * ctas_per_row);
       if (S < 1) S = 1;
     } else {
       const int64_t target = 2 * kNumSMs;
@@ -117,13 +130,26 @@ fsq_status plan_decode(int64_t B, int64_t T, int n_q, int n_kv, int d_h, int G, 
   const int acc_len = variant == FSQ_VARIANT_EXPAND ? d_h : G;
   size_t off = kWsHeader;
   p->off_qa = off;
-  if (tc) off = align_up(off + absorbed_tc_qphys_bytes(n_q, G) * (size_t)Bc, 256);
+  if (xtc) off = align_up(off + (size_t)Bc * n_kv * 16 * d_h * 2, 256);  // staged queries
+  else if (tc) off = align_up(off + absorbed_tc_qphys_bytes(n_q, G) * (size_t)Bc, 256);
   else if (variant == FSQ_VARIANT_ABSORBED) off = align_up(off + sizeof(float) * (size_t)Bc * n_q * G, 256);
   p->off_corr = off;
-  if (tc) off = align_up(off + 2 * sizeof(float) * (size_t)Bc * n_q, 256);
+  if (tc && !xtc) off = align_up(off + 2 * sizeof(float) * (size_t)Bc * n_q, 256);
+  p->off_wk = p->off_wv = p->off_ck = p->off_cv = off;
+  if (xtc) {
+    const size_t slice = expand_tc_stage_bytes(G, 0);
+    p->off_wk = off;
+    off = align_up(off + slice * n_kv, 256);
+    p->off_wv = off;
+    if (variant == FSQ_VARIANT_EXPAND) off = align_up(off + slice * n_kv, 256);
+    p->off_ck = off;
+    off = align_up(off + sizeof(float) * d_h * n_kv, 256);
+    p->off_cv = off;
+    off = align_up(off + sizeof(float) * d_h * n_kv, 256);
+  }
   p->off_part = off;
   off = align_up(off + sizeof(float) * (size_t)Bc * S * n_q * (2 + acc_len), 256);
-  if (variant == FSQ_VARIANT_ABSORBED) p->mp = merge_plan((int)S, Bc, n_q, n_kv, G);
+  if (variant == FSQ_VARIANT_ABSORBED || variant == FSQ_VARIANT_HYBRID) p->mp = merge_plan((int)S, Bc, n_q, n_kv, G);
   p->off_mslab = off;
   off = align_up(off + p->mp.slab_bytes, 256);
   p->off_mcnt = off;
@@ -235,7 +261,13 @@ fsq_status fsq_decode_attn(const uint16_t *q, int64_t B, int n_q, int d_h, const
   MergeScratch ms{nullptr, nullptr, 0};
   if (p.mp.cnt_bytes) ms = {(float *)(ws + p.off_mslab), (uint32_t *)(ws + p.off_mcnt), (int)(B * n_kv)};
   cudaError_t e;
-  if (p.tc) {
+  if (p.tc && (p.variant == FSQ_VARIANT_EXPAND || p.variant == FSQ_VARIANT_HYBRID)) {
+    e = launch_expand_tc(q, codes, code_batch_stride_bytes, B, T, op.seq_lens, n_q, n_kv, d_h, G, W_kv, scale, p.S,
+                         p.tps, p.variant == FSQ_VARIANT_HYBRID, op.rope_knorm, op.rope_base, op.knorm_gain,
+                         op.knorm_eps, (uint8_t *)(ws + p.off_wk), (uint8_t *)(ws + p.off_wv),
+                         (float *)(ws + p.off_ck), (float *)(ws + p.off_cv), (uint8_t *)(ws + p.off_qa), part, err,
+                         ms, o, op.out_fp32, op.debug_stall_ns, op.prof_events, s);
+  } else if (p.tc) {
     e = launch_absorbed_tc(q, codes, code_batch_stride_bytes, B, T, op.seq_lens, n_q, n_kv, d_h, G, W_kv, scale,
                            p.S, p.tps, (uint8_t *)(ws + p.off_qa), (float *)(ws + p.off_corr), part, err, ms, o,
                            op.out_fp32, op.debug_stall_ns, op.prof_events, s);

@@ -48,6 +48,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "tc_decode.cuh"
 #include "tc_ptx.cuh"
 
 namespace fsq {
@@ -57,7 +58,15 @@ using namespace ptx;
 
 constexpr int kTile = 128;
 constexpr int kMaxStages = 16;                     // code-tile ring depth bound (barrier arrays)
-constexpr int kSmemBudget = 200 * 1024;            // shared memory a CTA plans for
+constexpr int kSmemBudget = 224 * 1024;            // shared memory a CTA plans for
+// Every kFlushTiles tiles the softmax warps fold the pooled latents of the
+// tensor-core accumulator into fp32 sums of their own, and the pooling MMAs
+// start a fresh accumulation.  The pooled products are all non-negative
+// (nibbles n = level + 8), and the tensor core's fp32 accumulation is not
+// round-to-nearest, so one chain over a whole long split drifts by a bias
+// that grows with its length; the epilogue's -8 l correction cancels most of
+// the sum and magnifies that drift.  Short chains keep it near one fp32 ulp.
+constexpr int kFlushTiles = 64;
 constexpr int kQAfterTiles = 4;                    // code tiles requested before Q' (and its wait)
 constexpr float kTau = 8.f;                        // rescale when a score exceeds the running max by 2^8
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s per hand-off wait
@@ -103,14 +112,16 @@ struct Cfg {
   static constexpr int SM_CODES = 0;
   // Code-tile ring: as deep as the shared memory left over allows (bytes in
   // flight per SM hide the load latency), at most kMaxStages
-  static constexpr int OTHER_BYTES = Q_BYTES + kPBufs * P_BYTES + kMiscBytes;
+  static constexpr int FL_BYTES = 16 * NSMX * 32 * 4;   // 16 flushed fp32 sums per softmax thread
+  static constexpr int OTHER_BYTES = Q_BYTES + kPBufs * P_BYTES + kMiscBytes + FL_BYTES;
   static constexpr int STAGES_FIT = (kSmemBudget - OTHER_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT < kMaxStages ? STAGES_FIT : kMaxStages;
   static_assert(STAGES >= 4, "code-tile ring too shallow");
   static constexpr int SM_Q = SM_CODES + STAGES * STAGE_BYTES;
   static constexpr int SM_P = SM_Q + Q_BYTES;
   static constexpr int SM_MISC = SM_P + kPBufs * P_BYTES;
-  static constexpr int SM_TOTAL = SM_MISC + kMiscBytes;
+  static constexpr int SM_FL = SM_MISC + kMiscBytes;
+  static constexpr int SM_TOTAL = SM_FL + FL_BYTES;
   static constexpr int LBO_Q = (NS / 8) * 128;       // 16-byte K-chunk stride of Q'
   static constexpr int SBO_P = (kTile / 8) * 128;    // N-group stride of P
 };
@@ -139,6 +150,7 @@ struct Misc {
   uint64_t acc_full, q_full, done[5], never;
   uint32_t tmem_base;
   uint32_t abort;
+  uint32_t gfail[4];  // per softmax group: a wait of one of its warps gave up (read after a group barrier)
   float red[4][64];
   float fac[16][64];
   float m[64];
@@ -167,232 +179,6 @@ __device__ __forceinline__ void mma_ts_i8(uint32_t d_tmem, uint32_t a_tmem, uint
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-// One lane of a converged warp (elect.sync)
-__device__ __forceinline__ bool elect_one() {
-  uint32_t e;
-  asm volatile(
-      "{\n\t.reg .pred e;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "selp.u32 %0, 1, 0, e;\n\t}"
-      : "=r"(e));
-  return e != 0;
-}
-// A commit issued by one elected lane of a converged warp
-__device__ __forceinline__ void tc_commit_elect(uint64_t *bar) {
-  asm volatile(
-      "{\n\t.reg .pred e;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(smem_u32(bar))
-      : "memory");
-}
-
-// Pooling operand values as fp16 subnormals, no bias: nibble J of both
-// half-words left in place in mantissa bits 0..3 (value n 2^-24) or bits 4..7
-// (value n 2^-20).  w holds, per half-word, the four nibbles of one token.
-__device__ __forceinline__ void nib_sub4(uint32_t w, uint32_t &j0, uint32_t &j1, uint32_t &j2, uint32_t &j3) {
-  const uint32_t ws = w >> 8;
-  j0 = w & 0x000F000Fu;   // n 2^-24
-  j1 = w & 0x00F000F0u;   // n 2^-20
-  j2 = ws & 0x000F000Fu;  // n 2^-24
-  j3 = ws & 0x00F000F0u;  // n 2^-20
-}
-
-// Physical K position of token r in the pooling operand (see the 16x256b store below).
-__device__ __forceinline__ int kappa_of_token(int r) {
-  return (r & ~15) | (((r >> 1) & 3) << 2) | (((r >> 3) & 1) << 1) | (r & 1);
-}
-
-// max(a, b, c) in one instruction (three-input max.f32, sm_100)
-__device__ __forceinline__ float fmax3f(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-
-// 2^x on the special-function unit (inputs <= 8 here; -inf gives 0).
-__device__ __forceinline__ float ex2_approx(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-// 128-byte-swizzle layout of a TMA tile: 16-byte chunk c of row r sits at chunk c ^ (r % 8).
-__device__ __forceinline__ int swz(int r, int chunk) { return r * 128 + ((chunk ^ (r & 7)) << 4); }
-
-// L2 policy for the code stream, which every call reads once: evict it
-// first, so that it does not push out of L2 the small operands each call
-// re-reads (E, W_kv, the partials)
-__device__ __forceinline__ uint64_t l2_evict_first() {
-  uint64_t pol;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-  return pol;
-}
-__device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int c0, int c1, int c2, uint64_t *bar,
-                                            uint64_t pol) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint "
-      "[%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar)), "l"(pol)
-      : "memory");
-}
-__device__ __forceinline__ void bulk_g2s_hint(void *dst, const void *src, uint32_t bytes, uint64_t *bar,
-                                              uint64_t pol) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
-          smem_u32(dst)),
-      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
-      : "memory");
-}
-
-// 32-bit little-endian load from a 2-byte aligned shared address
-__device__ __forceinline__ uint32_t lds_u32_a2(const uint8_t *p) {
-  const uint16_t *h = reinterpret_cast<const uint16_t *>(p);
-  return (uint32_t)h[0] | ((uint32_t)h[1] << 16);
-}
-
-// Bounded barrier wait.  mbarrier.try_wait with a suspend-time hint parks the
-// warp in hardware until the phase completes (or the hint expires), so a
-// waiting warp takes no issue slots from the working warps of its scheduler.
-// Gives up after `limit_ns` or once *abort is set.
-__device__ __forceinline__ bool bar_test(uint32_t a, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(a), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ bool bar_try(uint32_t a, uint32_t parity, uint32_t hint_ns) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(a), "r"(parity), "r"(hint_ns)
-      : "memory");
-  return ok != 0;
-}
-// Tests of two or three phases at once: the tests are independent, so their
-// shared-memory round trips overlap (a completed hand-off costs one of them)
-__device__ __forceinline__ bool bar_test2(uint32_t a0, uint32_t p0, uint32_t a1, uint32_t p1) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 q, [%3], %4;\n\t"
-      "and.pred p, p, q;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(a0), "r"(p0), "r"(a1), "r"(p1)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ bool bar_test3(uint32_t a0, uint32_t p0, uint32_t a1, uint32_t p1, uint32_t a2,
-                                          uint32_t p2) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p, q, r;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 q, [%3], %4;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 r, [%5], %6;\n\t"
-      "and.pred p, p, q;\n\t"
-      "and.pred p, p, r;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(a0), "r"(p0), "r"(a1), "r"(p1), "r"(a2), "r"(p2)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ bool wait_bar(uint64_t *b, uint32_t parity, volatile uint32_t *abort, uint64_t limit_ns) {
-  const uint32_t a = smem_u32(b);
-  if (bar_test(a, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (bar_try(a, parity, 1000u)) return true;
-    if ((it & 7u) == 0u) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > limit_ns) return false;
-    }
-  }
-}
-// Waits for two (three) phases: one combined test, then each in turn
-__device__ __forceinline__ bool wait_bars(uint64_t *b0, uint32_t p0, uint64_t *b1, uint32_t p1,
-                                          volatile uint32_t *abort, uint64_t limit_ns) {
-  if (bar_test2(smem_u32(b0), p0, smem_u32(b1), p1)) return true;
-  return wait_bar(b0, p0, abort, limit_ns) && wait_bar(b1, p1, abort, limit_ns);
-}
-__device__ __forceinline__ bool wait_bars(uint64_t *b0, uint32_t p0, uint64_t *b1, uint32_t p1, uint64_t *b2,
-                                          uint32_t p2, volatile uint32_t *abort, uint64_t limit_ns) {
-  if (bar_test3(smem_u32(b0), p0, smem_u32(b1), p1, smem_u32(b2), p2)) return true;
-  return wait_bar(b0, p0, abort, limit_ns) && wait_bar(b1, p1, abort, limit_ns) && wait_bar(b2, p2, abort, limit_ns);
-}
-
-// Named barrier over `nthreads` threads that returns the OR of `pred` over them.
-__device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, %2, %3, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
-      : "memory");
-  return r != 0u;
-}
-
-// Error path: wait (time-bounded, ignoring the abort flag) for an async copy
-// already issued into this CTA's shared memory, so none lands after exit.
-__device__ __forceinline__ void drain_bar(uint64_t *b, uint32_t parity, uint64_t limit_ns) {
-  const uint32_t a = smem_u32(b);
-  const uint64_t t0 = globaltimer_ns();
-  while (!bar_test(a, parity)) {
-    __nanosleep(100);
-    if (globaltimer_ns() - t0 > limit_ns) return;
-  }
-}
-
-__device__ __forceinline__ void tmem_st_16x256b_x4(uint32_t taddr, const uint32_t *r) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.16x256b.x4.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
-          taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
-      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
-}
-
-__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t *r) {
-  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
-               : "r"(taddr)
-               : "memory");
-}
-template <int HQ>
-__device__ __forceinline__ void tmem_ld_hq(uint32_t ta, uint32_t *r) {
-  if constexpr (HQ == 16) tmem_ld16(ta, r);
-  else tmem_ld8(ta, r);
-}
-template <int HQ>
-__device__ __forceinline__ void tmem_st_hq(uint32_t ta, const uint32_t *r) {
-  if constexpr (HQ == 16) tmem_st16(ta, r);
-  else tmem_st8(ta, r);
-}
-
-template <int NQ>
-__device__ __forceinline__ void tmem_ld_nq(uint32_t ta, uint32_t *r) {
-  if constexpr (NQ == 32) tmem_ld32(ta, r);
-  else tmem_ld16(ta, r);
-}
-template <int NQ>
-__device__ __forceinline__ void tmem_st_nq(uint32_t ta, const uint32_t *r) {
-  if constexpr (NQ == 32) tmem_st32(ta, r);
-  else tmem_st16(ta, r);
-}
-
 template <int G, int NQ>
 __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(const __grid_constant__ CUtensorMap tmap, Params p) {
   using C = Cfg<G, NQ>;
@@ -441,6 +227,7 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
     for (int i = 0; i < 5; ++i) mbar_init(&ms.done[i], 1);
     mbar_init(&ms.never, 1);  // completed by nothing: the test-only stall waits on it
     ms.abort = 0;
+    for (int g = 0; g < 4; ++g) ms.gfail[g] = 0u;
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -568,7 +355,7 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
         if (elect_one()) {  // one lane issues the chunk's MMAs and its commit
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const bool first = (i == 0) && (C::NH == 1 ? kk == 0 : (c == 0 && kk == 0));
+            const bool first = (i % kFlushTiles == 0) && (C::NH == 1 ? kk == 0 : (c == 0 && kk == 0));
             mma_ts(d, a0 + kk * 8, bd0 + (uint64_t)(kk * 16), id_p, first ? 0u : 1u);
           }
           tc_commit(&ms.cp_free[cb]);
@@ -733,6 +520,10 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
     __syncwarp();
 #pragma unroll
     for (int n = 0; n < HQ; ++n) lsum[n] = 0.f;
+    // this thread's flushed sums: slot k (ACC block k / 8, head k % 8) at fl[k * NSMX * 32]
+    float *fl = reinterpret_cast<float *>(smem + C::SM_FL) + (sw * 32 + lane);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) fl[k * C::NSMX * 32] = 0.f;
     const int r = 32 * q + lane;        // token row within the tile
     const int kap = kappa_of_token(r);  // its K position in the pooling operand
     // tiles i >= ilim hold this row past the split's end; only the last tile
@@ -790,43 +581,62 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
     // scores are loaded together and share one vote, one fence and one pass
     // through the loop.  P buffers stay per tile (the score MMA of tile i
     // waited for P buffer i % kPBufs to be free).
+    // A warp whose wait gives up does not leave on its own: it records the
+    // failure in its group's flag and attends the group's next vote, after
+    // which all four warps leave together (no warp is left at a named barrier).
     const int n_pairs = (n_tiles + 1) >> 1;
-    for (int j = 0; j < n_pairs && ok; ++j) {
+    for (int j = 0; j < n_pairs; ++j) {
       const int i0 = 2 * j;
       const bool two = i0 + 1 < n_tiles;
       const uint32_t par = (uint32_t)j & 1u;  // use j of each S buffer
       float x0[HQ], x1[HQ];
-      float xmax;
+      float xmax = -INFINITY;
+      bool good = ok;
       {  // tile 2j from S buffer 0, then tile 2j+1 from S buffer 1 (one buffer's raw terms live at a time)
         uint32_t ra[HQ], rb[HQ];
-        if (!wait_bar(&ms.s_full[0], par, abort, p.wait_ns)) { ok = false; break; }
-        tc_fence_after();
-        tmem_ld8(tm + lane_base + C::OFF_S + h0, ra);
-        tmem_ld8(tm + lane_base + C::OFF_S + NQ + h0, rb);
-        tmem_ld_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&ms.s_free[0]);  // the next score MMA may overwrite it
-        xmax = scores(i0, ra, rb, x0);
-        if (two) {
-          if (!wait_bar(&ms.s_full[1], par, abort, p.wait_ns)) { ok = false; break; }
+        if (good) good = wait_bar(&ms.s_full[0], par, abort, p.wait_ns);
+        if (good) {
           tc_fence_after();
-          tmem_ld8(tm + lane_base + C::OFF_S + C::NS + h0, ra);
-          tmem_ld8(tm + lane_base + C::OFF_S + C::NS + NQ + h0, rb);
+          tmem_ld8(tm + lane_base + C::OFF_S + h0, ra);
+          tmem_ld8(tm + lane_base + C::OFF_S + NQ + h0, rb);
           tmem_ld_wait();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&ms.s_free[1]);
-          xmax = fmaxf(xmax, scores(i0 + 1, ra, rb, x1));
-        } else {
+          if (lane == 0) mbar_arrive(&ms.s_free[0]);  // the next score MMA may overwrite it
+          xmax = scores(i0, ra, rb, x0);
+        }
+        if (good && two) {
+          good = wait_bar(&ms.s_full[1], par, abort, p.wait_ns);
+          if (good) {
+            tc_fence_after();
+            tmem_ld8(tm + lane_base + C::OFF_S + C::NS + h0, ra);
+            tmem_ld8(tm + lane_base + C::OFF_S + C::NS + NQ + h0, rb);
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ms.s_free[1]);
+            xmax = fmaxf(xmax, scores(i0 + 1, ra, rb, x1));
+          }
+        } else if (!two) {
 #pragma unroll
           for (int n = 0; n < HQ; ++n) x1[n] = -INFINITY;
         }
       }
+      if (!good && lane == 0) {
+        ms.gfail[hh] = 1u;
+        fail();
+      }
       const bool need = (j == 0) || xmax > kTau;
       // one barrier over the group's four warps that also ORs their votes
       const bool any = named_bar_or(barid, 128, need);
-      if (any) {
+      if (ms.gfail[hh]) {  // the same value in all four warps: written before the barrier
+        ok = false;
+        break;
+      }
+      const bool flush = (j > 0) && (i0 % kFlushTiles) == 0;  // the pooling MMAs restart at tile i0
+      if (any || flush) {
+        float *f = ms.fac[sw];
+        if (any) {
         // raise the running max: m <- m + max(0, pair max of x) (the first pair: m <- its max)
 #pragma unroll
         for (int n = 0; n < HQ; ++n) {
@@ -836,7 +646,6 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
           if (lane == 0) ms.red[q][h0 + n] = v;
         }
         named_bar(barid, 128);
-        float *f = ms.fac[sw];
 #pragma unroll
         for (int n = 0; n < HQ; ++n) {
           const int hn = h0 + n;
@@ -851,11 +660,23 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
             cm[n] -= sh;
           }
         }
+        } else if (lane == 0) {
+#pragma unroll
+          for (int n = 0; n < HQ; ++n) f[n] = 1.f;
+        }
         __syncwarp();
         if (j > 0) {
-          // ACC must hold every earlier tile before it is rescaled
+          // ACC must hold every earlier tile before it is rescaled or folded
           const int pi = i0 - 1;
-          if (!wait_bar(&ms.p_free[pi % kPBufs], (uint32_t)(pi / kPBufs) & 1u, abort, p.wait_ns)) { ok = false; break; }
+          good = wait_bar(&ms.p_free[pi % kPBufs], (uint32_t)(pi / kPBufs) & 1u, abort, p.wait_ns);
+          if (!good) {
+            ok = false;
+            if (lane == 0) {
+              ms.gfail[hh] = 1u;  // the group leaves at its next vote
+              fail();
+            }
+            continue;
+          }
           tc_fence_after();
 #pragma unroll 1
           for (int blk = 0; blk < 2; ++blk) {  // both ACC blocks, this warp's head columns
@@ -863,11 +684,24 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
             const uint32_t ta = tm + lane_base + C::OFF_ACC + blk * NQ + h0;
             tmem_ld_hq<HQ>(ta, a);
             tmem_ld_wait();
+            if (flush) {
+              // fold into this thread's fp32 sums (rescaled alike); tile i0's MMAs overwrite ACC
 #pragma unroll
-            for (int n = 0; n < HQ; ++n) a[n] = __float_as_uint(__uint_as_float(a[n]) * f[n]);
-            tmem_st_hq<HQ>(ta, a);
+              for (int n = 0; n < HQ; ++n) {
+                float *slot = fl + (blk * 8 + n) * C::NSMX * 32;
+                *slot = (*slot + __uint_as_float(a[n])) * f[n];
+              }
+            } else {
+              // rescale: ACC and the sums folded out of earlier runs (relative to the same max)
+#pragma unroll
+              for (int n = 0; n < HQ; ++n) {
+                a[n] = __float_as_uint(__uint_as_float(a[n]) * f[n]);
+                fl[(blk * 8 + n) * C::NSMX * 32] *= f[n];
+              }
+              tmem_st_hq<HQ>(ta, a);
+            }
           }
-          tmem_st_wait();
+          if (!flush) tmem_st_wait();
         }
       }
       write_p(i0, x0);
@@ -882,7 +716,7 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
     }
     // ------------------------------------------------------------ epilogue: ACC -> partials
     if (ok) ok = wait_bar(&ms.acc_full, 0, abort, p.wait_ns);
-    if (!ok) {
+    if (named_bar_or(barid, 128, !ok)) {  // the group leaves together if any of its waits gave up
       if (lane == 0) fail();
     } else {
       tc_fence_after();
@@ -918,6 +752,11 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
       tmem_ld_hq<HQ>(tm + lane_base + C::OFF_ACC + h0, a0);
       tmem_ld_hq<HQ>(tm + lane_base + C::OFF_ACC + NQ + h0, a1);
       tmem_ld_wait();
+#pragma unroll
+      for (int n = 0; n < HQ; ++n) {  // plus the sums folded out of earlier accumulation runs
+        a0[n] = __float_as_uint(__uint_as_float(a0[n]) + fl[n * C::NSMX * 32]);
+        a1[n] = __float_as_uint(__uint_as_float(a1[n]) + fl[(8 + n) * C::NSMX * 32]);
+      }
       if constexpr (C::NH == 2) {
 #pragma unroll
         for (int h = 0; h < 2; ++h) {

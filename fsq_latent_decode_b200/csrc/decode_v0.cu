@@ -354,6 +354,13 @@ cudaError_t merge_absorbed_launch(const float *part, int S, int64_t B, int n_q, 
   return cudaGetLastError();
 }
 
+// Log-sum-exp merge of expanded-value partials [B][S][n_q][2 + d_h].
+cudaError_t merge_expand_launch(const float *part, int S, int64_t B, int n_q, int d_h, void *o, int out_fp32,
+                                cudaStream_t st) {
+  merge_expand_kernel<<<dim3(n_q, (unsigned)B), d_h, 0, st>>>(part, S, n_q, d_h, o, out_fp32);
+  return cudaGetLastError();
+}
+
 size_t absorbed_simt_smem(int n_q, int G) {
   return sizeof(float) * (2 * (size_t)n_q * G + kNT * (G + 1) + kNT * n_q + 3 * n_q);
 }

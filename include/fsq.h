@@ -86,16 +86,21 @@ typedef struct {
 } fsq_quant_params;
 
 enum {
-  FSQ_VARIANT_AUTO = 0,     /* library picks (ABSORBED when rope_knorm == 0) */
+  FSQ_VARIANT_AUTO = 0,     /* library picks: ABSORBED when rope_knorm == 0, else
+                               HYBRID (EXPAND for shapes HYBRID does not cover) */
   FSQ_VARIANT_ABSORBED = 1, /* score with W_k^T q, pool codes, apply W_v once */
-  FSQ_VARIANT_EXPAND = 2    /* rebuild K and V per tile through W_kv, then GQA */
+  FSQ_VARIANT_EXPAND = 2,   /* rebuild K and V per tile through W_kv, then GQA */
+  FSQ_VARIANT_HYBRID = 3    /* rebuild K per tile through W_k (then N_k and RoPE_t
+                               when rope_knorm), pool codes with the weights and
+                               apply W_v once ([D] kernel frame, steps 1-4);
+                               tensor cores; G in {84, 256}, n_q / n_kv <= 8 */
 };
 
 typedef struct {
   int variant;            /* FSQ_VARIANT_* */
   float scale;            /* softmax scale; <= 0 selects 1/sqrt(d_h) */
   int num_splits;         /* token-range splits per batch row; 0 = automatic */
-  int rope_knorm;         /* 1: k_t = RoPE_t(N_k(W_k z_t)) ([S] eq. 5); EXPAND only */
+  int rope_knorm;         /* 1: k_t = RoPE_t(N_k(W_k z_t)) ([S] eq. 5); EXPAND or HYBRID */
   float rope_base;        /* RoPE base (rope_knorm == 1) */
   const uint16_t *knorm_gain; /* device bf16 [d_h] RMS-norm gain, NULL = ones */
   float knorm_eps;        /* RMS-norm epsilon */

@@ -80,3 +80,25 @@ def record(kind: str, **fields):
     if path:
         with open(path, "a") as f:
             f.write(json.dumps(dict(kind=kind, **fields)) + "\n")
+
+
+def fp16_key_floor(q, codes, W_kv, n_kv, G, ref):
+    """The error (max|delta|/max|ref| against the oracle's `ref`) of decode
+    attention computed exactly except that the rebuilt keys are rounded to fp16
+    before the score product: the floor any kernel holding its keys in fp16
+    reaches.  Built from the oracle's own functions (reconstruct_kv, softmax);
+    used only to bound the key-expanding forms where scores span hundreds of
+    log2 units (q x 30), where bf16 keys would be off by ~14 %."""
+    import math as _m
+    q = np.asarray(q, dtype=np.float64)
+    B, n_q, d_h = q.shape
+    grp = n_q // n_kv
+    out = np.zeros((B, n_q, d_h))
+    for b in range(B):
+        K, V = O.reconstruct_kv(O.unpack(codes[b], G), W_kv, n_kv, d_h)
+        K16 = K.astype(np.float16).astype(np.float64)
+        for h in range(n_q):
+            j = h // grp
+            out[b, h] = O.softmax((K16[j] @ q[b, h]) / _m.sqrt(d_h)) @ V[j]
+    return rel_err(out, ref)
+

@@ -13,7 +13,7 @@ import fsq_latent_decode_b200 as F
 from fsq_latent_decode_b200 import synth
 from oracle import fsq_oracle as O
 
-from cases import TOL, decoder_weights, gemm_error_bound, oracle_cache, padded_len, record, rel_err
+from cases import TOL, decoder_weights, fp16_key_floor, gemm_error_bound, oracle_cache, padded_len, record, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -284,9 +284,11 @@ def test_decode_softmax_edge_cases(case, n_q, G, splits):
 
 # ---------------------------------------------------------------- ragged batches (per-row lengths)
 @pytest.mark.parametrize("splits", [0, 23])
-@pytest.mark.parametrize("variant", ["absorbed", "expand"])
+@pytest.mark.parametrize("variant", ["absorbed", "expand", "hybrid"])
 @pytest.mark.parametrize("n_q,n_kv,G", [(32, 8, 256), (16, 8, 84), (8, 2, 12)])
 def test_decode_ragged_lengths(variant, n_q, n_kv, G, splits):
+    if variant == "hybrid" and G not in (84, 256):
+        pytest.skip("the hybrid form runs on the tensor cores only (G in {84, 256})")
     B, T = 4, 3000
     lengths = [1, 129, 1000, T]
     codes = oracle_cache(B, T, G, seed=81)
@@ -352,3 +354,128 @@ def test_encode_bounded_wait_gives_up_and_next_call_recovers():
     got = F.encode_pack(xd, Ed, out=out, status_word=word).cpu().numpy()
     assert F.workspace_status(word) == F.FSQ_OK
     check_codes(got, x.float().numpy(), E.float().numpy(), G, "after a stalled call")
+
+
+# ---------------------------------------------------------------- keys rebuilt per tile on the tensor cores
+def _rope_args(seed):
+    gen = synth._gen(seed)
+    gain = (1.0 + 0.1 * torch.randn(128, generator=gen)).to(torch.bfloat16)
+    return gain, dict(gain=gain.float().numpy(), eps=1e-6, base=1.0e6)
+
+
+XSHAPES = [
+    # B, n_q, n_kv, G, T
+    (1, 16, 8, 256, 1), (2, 32, 8, 256, 300), (1, 32, 8, 84, 129), (3, 16, 8, 84, 1000), (2, 32, 8, 256, 4099),
+    (1, 32, 4, 84, 777), (2, 8, 8, 256, 513),
+]
+
+
+@pytest.mark.parametrize("rope", [False, True])
+@pytest.mark.parametrize("variant", ["hybrid", "expand"])
+@pytest.mark.parametrize("B,n_q,n_kv,G,T", XSHAPES)
+def test_decode_keys_expanded_on_tensor_cores(variant, rope, B, n_q, n_kv, G, T):
+    """The pages' kernel design (keys rebuilt per tile through W_k, key norm and
+    RoPE on chip, values pooled in latent space) and the form that rebuilds the
+    values too, against the oracle's expanded K and V (summary eq. 5)."""
+    codes = oracle_cache(B, T, G, seed=401 + T)
+    W, q = decoder_weights(n_q, n_kv, G, B, seed=402 + T)
+    gain, rk = _rope_args(403)
+    ref = O.decode_attn(q.float().numpy(), codes[:, :T], W.float().numpy(), n_kv, G, rope_knorm=rk if rope else None)
+    ws = F.Workspace(DEV)
+    got = F.decode_attn(_dev(q), _dev(codes), _dev(W), T, n_kv, G, workspace=ws,
+                        opts=F.attn_opts(variant=variant, rope_knorm=rope, rope_base=1.0e6,
+                                         knorm_gain=_dev(gain) if rope else None, knorm_eps=1e-6, out_fp32=True))
+    assert F.workspace_status(ws.buf) == F.FSQ_OK
+    got = got.cpu().numpy()
+    assert np.isfinite(got).all()
+    assert rel_err(got, ref) <= TOL
+
+
+@pytest.mark.parametrize("splits", [1, 5, 64])
+@pytest.mark.parametrize("variant", ["hybrid", "expand"])
+def test_decode_keys_expanded_split_counts(variant, splits):
+    B, n_q, n_kv, G, T = 2, 32, 8, 84, 3001
+    codes = oracle_cache(B, T, G, seed=411)
+    W, q = decoder_weights(n_q, n_kv, G, B, seed=412)
+    gain, rk = _rope_args(413)
+    ref = O.decode_attn(q.float().numpy(), codes[:, :T], W.float().numpy(), n_kv, G, rope_knorm=rk)
+    got = F.decode_attn(_dev(q), _dev(codes), _dev(W), T, n_kv, G,
+                        opts=F.attn_opts(variant=variant, rope_knorm=True, rope_base=1.0e6, knorm_gain=_dev(gain),
+                                         knorm_eps=1e-6, out_fp32=True, num_splits=splits)).cpu().numpy()
+    assert rel_err(got, ref) <= TOL
+
+
+@pytest.mark.parametrize("case", ["q_zero", "q_x30", "ascending_fast", "saturated"])
+@pytest.mark.parametrize("variant", ["hybrid", "expand"])
+@pytest.mark.parametrize("n_q,G", [(32, 256), (16, 84)])
+def test_decode_keys_expanded_softmax_edge_cases(case, variant, n_q, G):
+    B, n_kv, T = 2, 8, 2048 + 77
+    q, codes, W = _edge_inputs(case, B, n_q, n_kv, G, T, seed=500 + n_q + G)
+    ref = O.decode_attn(q.float().numpy(), codes[:, :T], W.float().numpy(), n_kv, G)
+    got = _decode(q, codes, W, T, n_kv, G, variant=variant, num_splits=1, out_fp32=True).cpu().numpy()
+    assert np.isfinite(got).all()
+    tol = TOL
+    if case == "q_x30":
+        # scores span hundreds of log2 units: fp16 keys alone move the output by
+        # `floor` (bf16 keys by ~14 %), so the bound is that floor plus 10 %
+        tol = max(TOL, 1.1 * fp16_key_floor(q.float().numpy(), codes[:, :T], W.float().numpy(), n_kv, G, ref))
+    assert rel_err(got, ref) <= tol
+
+
+@pytest.mark.parametrize("variant", ["hybrid", "expand"])
+def test_decode_keys_expanded_bounded_wait_gives_up(variant):
+    B, n_q, n_kv, G, T = 2, 32, 8, 256, 3000
+    codes = oracle_cache(B, T, G, seed=421)
+    W, q = decoder_weights(n_q, n_kv, G, B, seed=422)
+    qd, cd, Wd = _dev(q), _dev(codes), _dev(W)
+    ws = F.Workspace(DEV)
+    F.decode_attn(qd, cd, Wd, T, n_kv, G, workspace=ws, opts=F.attn_opts(variant=variant, debug_stall_ns=2_000_000))
+    assert F.workspace_status(ws.buf) == F.FSQ_ERR_TIMEOUT
+    got = F.decode_attn(qd, cd, Wd, T, n_kv, G, workspace=ws, opts=F.attn_opts(variant=variant, out_fp32=True))
+    assert F.workspace_status(ws.buf) == F.FSQ_OK
+    ref = O.decode_attn(q.float().numpy(), codes[:, :T], W.float().numpy(), n_kv, G)
+    assert rel_err(got.cpu().numpy(), ref) <= TOL
+
+
+@pytest.mark.parametrize("name,B,T", FULL)
+def test_full_size_workloads_rope_on_sampled(name, B, T):
+    """Every workload shape with the key norm and RoPE on, through the pages'
+    design (the hybrid form), at the launch configuration the benchmark uses;
+    the oracle checks the first and last batch rows (a head sample per kv head
+    group for long caches)."""
+    wl = synth.WORKLOADS[name]
+    rows = sorted({0, B - 1})
+    codes = oracle_cache(B, T, wl.G, seed=3000 + B, rows=rows)
+    W, q = decoder_weights(wl.n_q, wl.n_kv, wl.G, B, seed=4000 + B)
+    gain, rk = _rope_args(4001)
+    heads = None if T <= 8192 else [0, wl.n_q // 2 - 1, wl.n_q - 1]
+    ref = O.decode_attn(q.float().numpy(), codes[:, :T], W.float().numpy(), wl.n_kv, wl.G, rows=rows, heads=heads,
+                        rope_knorm=rk)
+    got = _decode(q, codes, W, T, wl.n_kv, wl.G, variant="hybrid", rope_knorm=True, rope_base=1.0e6,
+                  knorm_gain=_dev(gain), knorm_eps=1e-6).float().cpu().numpy()
+    assert rel_err(got, ref) <= TOL
+    assert np.isfinite(got[rows]).all()
+
+
+# ---------------------------------------------------------------- long accumulation runs
+@pytest.mark.parametrize("variant,n_q,G,rope", [("absorbed", 32, 256, False), ("absorbed", 16, 256, False),
+                                                ("absorbed", 32, 84, False), ("absorbed", 16, 84, False),
+                                                ("hybrid", 32, 256, True), ("hybrid", 32, 84, True),
+                                                ("hybrid", 16, 256, False), ("expand", 32, 256, True)])
+def test_decode_flat_softmax_long_single_split(variant, n_q, G, rope):
+    """A nearly flat softmax (q x 0.05, or the key norm on) over ~20k tokens in
+    one split: every token weighs in, so the latent pooling sums ~20k
+    non-negative terms per coordinate.  Parity here needs the kernels to keep
+    their tensor-core accumulation runs short (they fold the accumulator into
+    fp32 sums every 64 tiles); one run over the whole split drifted by up to
+    1.5 % at 131k tokens."""
+    B, n_kv, T = 1, 8, 20000 + 77
+    codes = oracle_cache(B, T, G, seed=601 + G)
+    W, q = decoder_weights(n_q, n_kv, G, B, seed=602 + G)
+    if not rope:
+        q = (q.float() * 0.05).to(torch.bfloat16)
+    gain, rk = _rope_args(603)
+    ref = O.decode_attn(q.float().numpy(), codes[:, :T], W.float().numpy(), n_kv, G, rope_knorm=rk if rope else None)
+    got = _decode(q, codes, W, T, n_kv, G, variant=variant, num_splits=1, out_fp32=True, rope_knorm=rope,
+                  rope_base=1.0e6, knorm_gain=_dev(gain) if rope else None, knorm_eps=1e-6).cpu().numpy()
+    assert rel_err(got, ref) <= TOL
