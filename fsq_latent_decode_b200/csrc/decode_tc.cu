@@ -59,14 +59,18 @@ using namespace ptx;
 constexpr int kTile = 128;
 constexpr int kMaxStages = 16;                     // code-tile ring depth bound (barrier arrays)
 constexpr int kSmemBudget = 224 * 1024;            // shared memory a CTA plans for
-// Every kFlushTiles tiles the softmax warps fold the pooled latents of the
-// tensor-core accumulator into fp32 sums of their own, and the pooling MMAs
-// start a fresh accumulation.  The pooled products are all non-negative
-// (nibbles n = level + 8), and the tensor core's fp32 accumulation is not
-// round-to-nearest, so one chain over a whole long split drifts by a bias
-// that grows with its length; the epilogue's -8 l correction cancels most of
-// the sum and magnifies that drift.  Short chains keep it near one fp32 ulp.
+// The pooled products are all non-negative (nibbles n = level + 8) and the
+// tensor core's fp32 accumulation is not round-to-nearest, so one MMA chain
+// over a long split drifts by a bias that grows with its length; the
+// epilogue's -8 l correction cancels most of the sum and magnifies it (1.45 %
+// on a flat softmax over 131k tokens).  Splits of up to kFoldAbove tokens
+// (every one-wave plan of the benchmarked shapes) stay within 0.15 %; longer
+// ones run the FOLD instance, whose softmax warps move the accumulator into
+// fp32 sums of their own every kFlushTiles tiles while the pooling MMAs start
+// a fresh chain.  The folding code costs the hot loop about 10 %, so the
+// shorter splits run without it.
 constexpr int kFlushTiles = 64;
+constexpr int64_t kFoldAbove = 16384;
 constexpr int kQAfterTiles = 4;                    // code tiles requested before Q' (and its wait)
 constexpr float kTau = 8.f;                        // rescale when a score exceeds the running max by 2^8
 constexpr uint64_t kWaitLimitNs = 1000000000ull;   // 1 s per hand-off wait
@@ -150,7 +154,6 @@ struct Misc {
   uint64_t acc_full, q_full, done[5], never;
   uint32_t tmem_base;
   uint32_t abort;
-  uint32_t gfail[4];  // per softmax group: a wait of one of its warps gave up (read after a group barrier)
   float red[4][64];
   float fac[16][64];
   float m[64];
@@ -179,7 +182,7 @@ __device__ __forceinline__ void mma_ts_i8(uint32_t d_tmem, uint32_t a_tmem, uint
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-template <int G, int NQ>
+template <int G, int NQ, bool FOLD>
 __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(const __grid_constant__ CUtensorMap tmap, Params p) {
   using C = Cfg<G, NQ>;
   extern __shared__ __align__(1024) uint8_t smem[];
@@ -227,7 +230,6 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
     for (int i = 0; i < 5; ++i) mbar_init(&ms.done[i], 1);
     mbar_init(&ms.never, 1);  // completed by nothing: the test-only stall waits on it
     ms.abort = 0;
-    for (int g = 0; g < 4; ++g) ms.gfail[g] = 0u;
     fence_mbar_init();
   }
   if (warp == 0) {
@@ -355,7 +357,7 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
         if (elect_one()) {  // one lane issues the chunk's MMAs and its commit
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            const bool first = (i % kFlushTiles == 0) && (C::NH == 1 ? kk == 0 : (c == 0 && kk == 0));
+            const bool first = (FOLD ? i % kFlushTiles == 0 : i == 0) && (C::NH == 1 ? kk == 0 : (c == 0 && kk == 0));
             mma_ts(d, a0 + kk * 8, bd0 + (uint64_t)(kk * 16), id_p, first ? 0u : 1u);
           }
           tc_commit(&ms.cp_free[cb]);
@@ -520,10 +522,14 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
     __syncwarp();
 #pragma unroll
     for (int n = 0; n < HQ; ++n) lsum[n] = 0.f;
-    // this thread's flushed sums: slot k (ACC block k / 8, head k % 8) at fl[k * NSMX * 32]
-    float *fl = reinterpret_cast<float *>(smem + C::SM_FL) + (sw * 32 + lane);
+    // this thread's folded sums: slot k (ACC block k / 8, head k % 8), addressed on use
+    auto fl_slot = [&](int k) -> float * {
+      return reinterpret_cast<float *>(smem + C::SM_FL) + k * C::NSMX * 32 + sw * 32 + lane;
+    };
+    if constexpr (FOLD) {
 #pragma unroll
-    for (int k = 0; k < 16; ++k) fl[k * C::NSMX * 32] = 0.f;
+      for (int k = 0; k < 16; ++k) *fl_slot(k) = 0.f;
+    }
     const int r = 32 * q + lane;        // token row within the tile
     const int kap = kappa_of_token(r);  // its K position in the pooling operand
     // tiles i >= ilim hold this row past the split's end; only the last tile
@@ -581,85 +587,79 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
     // scores are loaded together and share one vote, one fence and one pass
     // through the loop.  P buffers stay per tile (the score MMA of tile i
     // waited for P buffer i % kPBufs to be free).
-    // A warp whose wait gives up does not leave on its own: it records the
-    // failure in its group's flag and attends the group's next vote, after
-    // which all four warps leave together (no warp is left at a named barrier).
+    // A wait that gives up does not end the loop: the warp records the failure
+    // (and the abort flag) and keeps running the same instructions without
+    // waiting, its data meaningless, so every warp of the group passes the same
+    // named barriers; the group decides together after the loop.
     const int n_pairs = (n_tiles + 1) >> 1;
     for (int j = 0; j < n_pairs; ++j) {
       const int i0 = 2 * j;
       const bool two = i0 + 1 < n_tiles;
       const uint32_t par = (uint32_t)j & 1u;  // use j of each S buffer
       float x0[HQ], x1[HQ];
-      float xmax = -INFINITY;
-      bool good = ok;
+      float xmax;
       {  // tile 2j from S buffer 0, then tile 2j+1 from S buffer 1 (one buffer's raw terms live at a time)
         uint32_t ra[HQ], rb[HQ];
-        if (good) good = wait_bar(&ms.s_full[0], par, abort, p.wait_ns);
-        if (good) {
+        if (ok && !wait_bar(&ms.s_full[0], par, abort, p.wait_ns)) {
+          ok = false;
+          fail();
+        }
+        tc_fence_after();
+        tmem_ld8(tm + lane_base + C::OFF_S + h0, ra);
+        tmem_ld8(tm + lane_base + C::OFF_S + NQ + h0, rb);
+        tmem_ld_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&ms.s_free[0]);  // the next score MMA may overwrite it
+        xmax = scores(i0, ra, rb, x0);
+        if (two) {
+          if (ok && !wait_bar(&ms.s_full[1], par, abort, p.wait_ns)) {
+            ok = false;
+            fail();
+          }
           tc_fence_after();
-          tmem_ld8(tm + lane_base + C::OFF_S + h0, ra);
-          tmem_ld8(tm + lane_base + C::OFF_S + NQ + h0, rb);
+          tmem_ld8(tm + lane_base + C::OFF_S + C::NS + h0, ra);
+          tmem_ld8(tm + lane_base + C::OFF_S + C::NS + NQ + h0, rb);
           tmem_ld_wait();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&ms.s_free[0]);  // the next score MMA may overwrite it
-          xmax = scores(i0, ra, rb, x0);
-        }
-        if (good && two) {
-          good = wait_bar(&ms.s_full[1], par, abort, p.wait_ns);
-          if (good) {
-            tc_fence_after();
-            tmem_ld8(tm + lane_base + C::OFF_S + C::NS + h0, ra);
-            tmem_ld8(tm + lane_base + C::OFF_S + C::NS + NQ + h0, rb);
-            tmem_ld_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&ms.s_free[1]);
-            xmax = fmaxf(xmax, scores(i0 + 1, ra, rb, x1));
-          }
-        } else if (!two) {
+          if (lane == 0) mbar_arrive(&ms.s_free[1]);
+          xmax = fmaxf(xmax, scores(i0 + 1, ra, rb, x1));
+        } else {
 #pragma unroll
           for (int n = 0; n < HQ; ++n) x1[n] = -INFINITY;
         }
       }
-      if (!good && lane == 0) {
-        ms.gfail[hh] = 1u;
-        fail();
-      }
       const bool need = (j == 0) || xmax > kTau;
       // one barrier over the group's four warps that also ORs their votes
       const bool any = named_bar_or(barid, 128, need);
-      if (ms.gfail[hh]) {  // the same value in all four warps: written before the barrier
-        ok = false;
-        break;
-      }
-      const bool flush = (j > 0) && (i0 % kFlushTiles) == 0;  // the pooling MMAs restart at tile i0
+      const bool flush = FOLD && (j > 0) && (i0 % kFlushTiles) == 0;  // the pooling MMAs restart at tile i0
       if (any || flush) {
         float *f = ms.fac[sw];
         if (any) {
-        // raise the running max: m <- m + max(0, pair max of x) (the first pair: m <- its max)
+          // raise the running max: m <- m + max(0, pair max of x) (the first pair: m <- its max)
 #pragma unroll
-        for (int n = 0; n < HQ; ++n) {
-          float v = fmaxf(x0[n], x1[n]);
+          for (int n = 0; n < HQ; ++n) {
+            float v = fmaxf(x0[n], x1[n]);
 #pragma unroll
-          for (int off = 16; off; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-          if (lane == 0) ms.red[q][h0 + n] = v;
-        }
-        named_bar(barid, 128);
-#pragma unroll
-        for (int n = 0; n < HQ; ++n) {
-          const int hn = h0 + n;
-          const float d = fmaxf(fmaxf(ms.red[0][hn], ms.red[1][hn]), fmaxf(ms.red[2][hn], ms.red[3][hn]));
-          const float sh = (j == 0) ? d : fmaxf(d, 0.f);
-          const float fn = (j == 0) ? 0.f : exp2f(-sh);
-          x0[n] -= sh;
-          x1[n] -= sh;
-          lsum[n] *= fn;
-          if (lane == 0) {
-            f[n] = fn;
-            cm[n] -= sh;
+            for (int off = 16; off; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+            if (lane == 0) ms.red[q][h0 + n] = v;
           }
-        }
+          named_bar(barid, 128);
+#pragma unroll
+          for (int n = 0; n < HQ; ++n) {
+            const int hn = h0 + n;
+            const float d = fmaxf(fmaxf(ms.red[0][hn], ms.red[1][hn]), fmaxf(ms.red[2][hn], ms.red[3][hn]));
+            const float sh = (j == 0) ? d : fmaxf(d, 0.f);
+            const float fn = (j == 0) ? 0.f : exp2f(-sh);
+            x0[n] -= sh;
+            x1[n] -= sh;
+            lsum[n] *= fn;
+            if (lane == 0) {
+              f[n] = fn;
+              cm[n] -= sh;
+            }
+          }
         } else if (lane == 0) {
 #pragma unroll
           for (int n = 0; n < HQ; ++n) f[n] = 1.f;
@@ -668,14 +668,9 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
         if (j > 0) {
           // ACC must hold every earlier tile before it is rescaled or folded
           const int pi = i0 - 1;
-          good = wait_bar(&ms.p_free[pi % kPBufs], (uint32_t)(pi / kPBufs) & 1u, abort, p.wait_ns);
-          if (!good) {
+          if (ok && !wait_bar(&ms.p_free[pi % kPBufs], (uint32_t)(pi / kPBufs) & 1u, abort, p.wait_ns)) {
             ok = false;
-            if (lane == 0) {
-              ms.gfail[hh] = 1u;  // the group leaves at its next vote
-              fail();
-            }
-            continue;
+            fail();
           }
           tc_fence_after();
 #pragma unroll 1
@@ -684,19 +679,17 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
             const uint32_t ta = tm + lane_base + C::OFF_ACC + blk * NQ + h0;
             tmem_ld_hq<HQ>(ta, a);
             tmem_ld_wait();
+            float *fl = fl_slot(blk * 8);
             if (flush) {
               // fold into this thread's fp32 sums (rescaled alike); tile i0's MMAs overwrite ACC
 #pragma unroll
-              for (int n = 0; n < HQ; ++n) {
-                float *slot = fl + (blk * 8 + n) * C::NSMX * 32;
-                *slot = (*slot + __uint_as_float(a[n])) * f[n];
-              }
+              for (int n = 0; n < HQ; ++n) fl[n * C::NSMX * 32] = (fl[n * C::NSMX * 32] + __uint_as_float(a[n])) * f[n];
             } else {
               // rescale: ACC and the sums folded out of earlier runs (relative to the same max)
 #pragma unroll
               for (int n = 0; n < HQ; ++n) {
                 a[n] = __float_as_uint(__uint_as_float(a[n]) * f[n]);
-                fl[(blk * 8 + n) * C::NSMX * 32] *= f[n];
+                if constexpr (FOLD) fl[n * C::NSMX * 32] *= f[n];
               }
               tmem_st_hq<HQ>(ta, a);
             }
@@ -752,10 +745,12 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
       tmem_ld_hq<HQ>(tm + lane_base + C::OFF_ACC + h0, a0);
       tmem_ld_hq<HQ>(tm + lane_base + C::OFF_ACC + NQ + h0, a1);
       tmem_ld_wait();
+      if constexpr (FOLD) {
 #pragma unroll
-      for (int n = 0; n < HQ; ++n) {  // plus the sums folded out of earlier accumulation runs
-        a0[n] = __float_as_uint(__uint_as_float(a0[n]) + fl[n * C::NSMX * 32]);
-        a1[n] = __float_as_uint(__uint_as_float(a1[n]) + fl[(8 + n) * C::NSMX * 32]);
+        for (int n = 0; n < HQ; ++n) {  // plus the sums folded out of earlier accumulation runs
+          a0[n] = __float_as_uint(__uint_as_float(a0[n]) + *fl_slot(n));
+          a1[n] = __float_as_uint(__uint_as_float(a1[n]) + *fl_slot(8 + n));
+        }
       }
       if constexpr (C::NH == 2) {
 #pragma unroll
@@ -999,7 +994,9 @@ cudaError_t launch(const uint16_t *q, const uint8_t *codes, int64_t bstride, int
   if (e != cudaSuccess) return e;
   // one CTA per SM: ask for more shared memory than two CTAs could share
   const int smem = C::SM_TOTAL > 120 * 1024 ? C::SM_TOTAL : 120 * 1024;
-  e = ensure_smem_limit((const void *)absorbed_split_tc<G, NQ>, (size_t)smem);
+  const bool fold = tps > kFoldAbove;  // long splits keep their accumulation runs short
+  auto kern = fold ? absorbed_split_tc<G, NQ, true> : absorbed_split_tc<G, NQ, false>;
+  e = ensure_smem_limit((const void *)kern, (size_t)smem);
   if (e != cudaSuccess) return e;
   Params p{codes, bstride, T, tps, S, qphys, corr, part, err, kWaitLimitNs, seq_lens, stall_ns};
   CUtensorMap tmap;
@@ -1009,7 +1006,7 @@ cudaError_t launch(const uint16_t *q, const uint8_t *codes, int64_t bstride, int
     if (e != cudaSuccess) return e;
   }
   record_prof_event(prof[0], st);
-  e = launch_pdl(absorbed_split_tc<G, NQ>, dim3(S, (unsigned)B), dim3(C::THREADS), (size_t)smem, st, tmap, p);
+  e = launch_pdl(kern, dim3(S, (unsigned)B), dim3(C::THREADS), (size_t)smem, st, tmap, p);
   record_prof_event(prof[1], st);
   return e;
 }

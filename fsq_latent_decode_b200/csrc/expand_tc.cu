@@ -454,6 +454,12 @@ __global__ void __launch_bounds__(XC<G, VEXP>::THREADS, 1)
     const uint32_t lane_base = (uint32_t)(32 * q) << 16;
     const int r = 32 * q + lane;               // token row within the tile
     const float rf = (float)r;
+    // threads r < 64 of warps 8-9 carry (tile start * theta_r) mod 2 pi and its per-tile step
+    double phd = 0.0, dphi = 0.0;
+    if (hv == 0 && r < 64) {
+      phd = fmod((double)t0 * ms.theta_d[r], 6.283185307179586);
+      dphi = fmod((double)kT * ms.theta_d[r], 6.283185307179586);
+    }
     const int gt = tid - 256;                  // 0..255 over the eight token warps
     pdl_wait();                                // the offset terms come from the prologue kernel
     // a bad per-row length is reported once, after the prologue cleared the error word
@@ -523,9 +529,10 @@ __global__ void __launch_bounds__(XC<G, VEXP>::THREADS, 1)
         tc_fence_before();
       }
       if (hv) ms.ss[r] = ss;
-      if (hv == 0 && r < 64) {  // base angles of the next tile
-        ms.phib[(i + 1) & 1][r] =
-            (float)fmod((double)(t0 + (int64_t)(i + 1) * kT) * ms.theta_d[r], 6.283185307179586);
+      if (hv == 0 && r < 64) {  // base angles of the next tile: advance by 128 theta_r, mod 2 pi, in fp64
+        phd += dphi;
+        if (phd >= 6.283185307179586) phd -= 6.283185307179586;
+        ms.phib[(i + 1) & 1][r] = (float)phd;
       }
       if (named_bar_or(2, 256, !good)) {
         if (lane == 0) fail();

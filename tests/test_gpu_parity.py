@@ -462,14 +462,14 @@ def test_full_size_workloads_rope_on_sampled(name, B, T):
                                                 ("absorbed", 32, 84, False), ("absorbed", 16, 84, False),
                                                 ("hybrid", 32, 256, True), ("hybrid", 32, 84, True),
                                                 ("hybrid", 16, 256, False), ("expand", 32, 256, True)])
-def test_decode_flat_softmax_long_single_split(variant, n_q, G, rope):
-    """A nearly flat softmax (q x 0.05, or the key norm on) over ~20k tokens in
-    one split: every token weighs in, so the latent pooling sums ~20k
-    non-negative terms per coordinate.  Parity here needs the kernels to keep
-    their tensor-core accumulation runs short (they fold the accumulator into
-    fp32 sums every 64 tiles); one run over the whole split drifted by up to
-    1.5 % at 131k tokens."""
-    B, n_kv, T = 1, 8, 20000 + 77
+@pytest.mark.parametrize("T", [16384 - 77, 20000 + 77])
+def test_decode_flat_softmax_long_single_split(variant, n_q, G, rope, T):
+    """A nearly flat softmax (q x 0.05, or the key norm on) over a whole split
+    of ~16k (one accumulation run) or ~20k tokens (runs folded into fp32 sums
+    every 64 tiles): every token weighs in, so the latent pooling sums that
+    many non-negative terms per coordinate.  One run over a 131k-token split
+    drifted by 1.5 %."""
+    B, n_kv = 1, 8
     codes = oracle_cache(B, T, G, seed=601 + G)
     W, q = decoder_weights(n_q, n_kv, G, B, seed=602 + G)
     if not rope:
