@@ -38,8 +38,24 @@ import math
 import numpy as np
 
 # L=16 levels -> b = ceil(log2 L) = 4 bits per coordinate ([D], product-code frame).
+# The deck's backup frame "the grid size is an allocation choice" (Table 8) also
+# compares L = 4 (2 bits) and L = 256 (8 bits) at fixed byte budgets; every
+# function below takes the level count L (default 16).
 LEVELS = 16
 BITS = 4
+SUPPORTED_LEVELS = (4, 16, 256)
+
+
+def bits_per_coordinate(levels=LEVELS):
+    """b = ceil(log2 L) ([D] product-code frame)."""
+    return int(math.ceil(math.log2(levels)))
+
+
+def default_h(levels=LEVELS):
+    """Reading for the bound h of eq. (2) at L levels (the deck gives only
+    L = 16, h = 7.5075 = 7.5 x 1.001; the acceptance spec uses 7.5): h = (L-1)/2,
+    so that with delta = 1/2 the rounded values are exactly -L/2 .. L/2 - 1."""
+    return (levels - 1) / 2.0
 # The deck prints h=7.5075, delta=0.5 for L=16 ([D]); the acceptance spec of
 # this library uses h=7.5.  Both are accepted as parameters.
 H_DEFAULT = 7.5
@@ -55,7 +71,7 @@ def fsq_bounded(u, h=H_DEFAULT, delta=DELTA_DEFAULT):
     return h * np.tanh(u + math.atanh(delta / h)) - delta
 
 
-def fsq_quantize(u, h=H_DEFAULT, delta=DELTA_DEFAULT):
+def fsq_quantize(u, h=H_DEFAULT, delta=DELTA_DEFAULT, levels=LEVELS):
     """Forward value of eq. (2): round(u~) as an integer level.
 
     The straight-through term sg(round(u~) - u~) only changes gradients; its
@@ -65,13 +81,13 @@ def fsq_quantize(u, h=H_DEFAULT, delta=DELTA_DEFAULT):
     """
     ut = fsq_bounded(u, h, delta)
     c = np.rint(ut)
-    lo, hi = -(LEVELS // 2), LEVELS // 2 - 1
+    lo, hi = -(levels // 2), levels // 2 - 1
     if c.size and (c.min() < lo or c.max() > hi):
-        raise AssertionError("FSQ level outside the 16-level grid")
+        raise AssertionError(f"FSQ level outside the {levels}-level grid")
     return c.astype(np.int64)
 
 
-def fsq_boundary_distance(u, h=H_DEFAULT, delta=DELTA_DEFAULT):
+def fsq_boundary_distance(u, h=H_DEFAULT, delta=DELTA_DEFAULT, levels=LEVELS):
     """Distance in u-space from u to the nearest rounding boundary of eq. (2).
 
     A boundary is a u whose u~ is a half-integer m + 1/2.  Inverting eq. (2)
@@ -80,7 +96,7 @@ def fsq_boundary_distance(u, h=H_DEFAULT, delta=DELTA_DEFAULT):
     """
     u = np.asarray(u, dtype=np.float64)
     a = math.atanh(delta / h)
-    halves = np.arange(-(LEVELS // 2), LEVELS // 2 - 1) + 0.5  # -7.5 .. 6.5
+    halves = np.arange(-(levels // 2), levels // 2 - 1) + 0.5  # -7.5 .. 6.5 at L = 16
     arg = (halves + delta) / h
     ok = np.abs(arg) < 1.0
     bounds = np.arctanh(arg[ok]) - a
@@ -91,7 +107,7 @@ def fsq_boundary_distance(u, h=H_DEFAULT, delta=DELTA_DEFAULT):
 # ---------------------------------------------------------------------------
 # eq. (4): linear encoder followed by FSQ; nibble packing
 # ---------------------------------------------------------------------------
-def encode(x, E, h=H_DEFAULT, delta=DELTA_DEFAULT):
+def encode(x, E, h=H_DEFAULT, delta=DELTA_DEFAULT, levels=LEVELS):
     """z_t = Q_FSQ(E x_t) for every row x_t of x  ([S] Architecture, eq. 4).
 
     x: [N, C], E: [G, C] (any real dtype; converted exactly to fp64).
@@ -100,49 +116,56 @@ def encode(x, E, h=H_DEFAULT, delta=DELTA_DEFAULT):
     x64 = np.asarray(x, dtype=np.float64)
     E64 = np.asarray(E, dtype=np.float64)
     u = x64 @ E64.T
-    return fsq_quantize(u, h, delta), u
+    return fsq_quantize(u, h, delta, levels), u
 
 
-def pack(levels):
-    """Nibble-pack integer levels [..., G] into bytes [..., G/2].
+def pack(levels, L=LEVELS):
+    """Pack integer levels [..., G] into bytes [..., G*b/8], b = log2 L.
 
-    Stored nibble n = level + 8 (0..15).  Byte i holds coordinate 2i in its low
-    nibble and 2i+1 in its high nibble.  No scale, zero point or norm is stored
-    ([S] Summary: "no per-token quantisation metadata"; [D] product-code frame:
-    ceil(G*b/8) bytes per token).
+    Stored code n = level + L/2 (0..L-1, b bits).  Byte k holds coordinates
+    k*(8/b) .. k*(8/b) + 8/b - 1, the first in its lowest b bits (at L = 16:
+    coordinate 2i in the low nibble of byte i, 2i+1 in the high nibble).  No
+    scale, zero point or norm is stored ([S] Summary: "no per-token
+    quantisation metadata"; [D] product-code frame: ceil(G*b/8) bytes per
+    token).
     """
     lv = np.asarray(levels, dtype=np.int64)
     G = lv.shape[-1]
-    if G % 2:
-        raise ValueError("G must be even")
-    n = lv + LEVELS // 2
-    if n.size and (n.min() < 0 or n.max() > LEVELS - 1):
-        raise ValueError("level outside the 16-level grid")
-    lo = n[..., 0::2]
-    hi = n[..., 1::2]
-    return (lo | (hi << 4)).astype(np.uint8)
+    b = bits_per_coordinate(L)
+    per = 8 // b
+    if G % per:
+        raise ValueError(f"G must be a multiple of {per} at {L} levels")
+    n = lv + L // 2
+    if n.size and (n.min() < 0 or n.max() > L - 1):
+        raise ValueError(f"level outside the {L}-level grid")
+    out = np.zeros(lv.shape[:-1] + (G // per,), dtype=np.int64)
+    for i in range(per):
+        out |= n[..., i::per] << (b * i)
+    return out.astype(np.uint8)
 
 
-def unpack(codes, G):
-    """Inverse of pack: bytes [..., G/2] -> integer levels [..., G] (nibble - 8)."""
-    b = np.asarray(codes, dtype=np.uint8).astype(np.int64)
-    if b.shape[-1] != G // 2:
-        raise ValueError("codes row length must be G/2")
-    out = np.empty(b.shape[:-1] + (G,), dtype=np.int64)
-    out[..., 0::2] = b & 0xF
-    out[..., 1::2] = b >> 4
-    return out - LEVELS // 2
+def unpack(codes, G, L=LEVELS):
+    """Inverse of pack: bytes [..., G*b/8] -> integer levels [..., G] (code - L/2)."""
+    b = bits_per_coordinate(L)
+    per = 8 // b
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    if c.shape[-1] != G // per:
+        raise ValueError("codes row length must be G*b/8")
+    out = np.empty(c.shape[:-1] + (G,), dtype=np.int64)
+    for i in range(per):
+        out[..., i::per] = (c >> (b * i)) & (L - 1)
+    return out - L // 2
 
 
-def encode_pack(x, E, h=H_DEFAULT, delta=DELTA_DEFAULT):
-    """Append path: packed codes [N, G/2] for rows of x (eq. 4 then packing)."""
-    lv, _ = encode(x, E, h, delta)
-    return pack(lv)
+def encode_pack(x, E, h=H_DEFAULT, delta=DELTA_DEFAULT, levels=LEVELS):
+    """Append path: packed codes [N, G*b/8] for rows of x (eq. 4 then packing)."""
+    lv, _ = encode(x, E, h, delta, levels)
+    return pack(lv, levels)
 
 
-def quantize_pack(u, h=H_DEFAULT, delta=DELTA_DEFAULT):
+def quantize_pack(u, h=H_DEFAULT, delta=DELTA_DEFAULT, levels=LEVELS):
     """Quantiser + packing alone, on given pre-activations u [N, G]."""
-    return pack(fsq_quantize(u, h, delta))
+    return pack(fsq_quantize(u, h, delta, levels), levels)
 
 
 # ---------------------------------------------------------------------------
@@ -207,7 +230,8 @@ def softmax(s):
 # ---------------------------------------------------------------------------
 # Decode attention: expanded K/V, then standard GQA softmax attention
 # ---------------------------------------------------------------------------
-def decode_attn(q, codes, W_kv, n_kv, G, scale=None, rope_knorm=None, rows=None, heads=None, lengths=None):
+def decode_attn(q, codes, W_kv, n_kv, G, scale=None, rope_knorm=None, rows=None, heads=None, lengths=None,
+                levels=LEVELS):
     """Single-token GQA decode attention over a packed FSQ code cache.
 
     q: [B, n_q, d_h]; codes: [B, T, G/2] uint8; W_kv: [2*n_kv*d_h, G].
@@ -217,7 +241,7 @@ def decode_attn(q, codes, W_kv, n_kv, G, scale=None, rope_knorm=None, rows=None,
     rows / heads optionally restrict the computation to a sample (others are
     left as NaN) so large caches can be checked one output at a time.
     lengths: optional per-row token counts (a ragged batch): row b attends to
-    its first lengths[b] cached tokens only.
+    its first lengths[b] cached tokens only.  levels: L of the code grid.
     Returns o [B, n_q, d_h] fp64.
     """
     q = np.asarray(q, dtype=np.float64)
@@ -231,7 +255,7 @@ def decode_attn(q, codes, W_kv, n_kv, G, scale=None, rope_knorm=None, rows=None,
     heads = range(n_q) if heads is None else heads
     o = np.full((B, n_q, d_h), np.nan)
     for b in rows:
-        lv = unpack(codes[b] if lengths is None else codes[b][: int(lengths[b])], G)
+        lv = unpack(codes[b] if lengths is None else codes[b][: int(lengths[b])], G, levels)
         need_j = sorted({h // grp for h in heads})
         Wk, Wv = split_wkv(W_kv, n_kv, d_h)
         for j in need_j:

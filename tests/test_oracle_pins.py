@@ -319,3 +319,94 @@ def test_rope_flag_breaks_pooled_keys():
     # which cannot change a single-token softmax
     q1, c1, W1, _, _ = _rand_case(12, B=1, n_q=4, n_kv=2, d_h=16, G=12, T=1)
     assert np.allclose(O.decode_attn(q1, c1, W1, 2, 12, rope_knorm=rk), O.decode_attn(q1, c1, W1, 2, 12), atol=1e-12)
+
+
+# ---------------------------------------------------------------- level-count variants (L = 4, 256)
+def _closed_form_thresholds_L(L, h, delta):
+    # Hand inversion of eq. (2) at L levels: the level steps from m to m+1 where
+    # u~ = m + 1/2, m = -L/2 .. L/2 - 2; a boundary past the tanh range is never reached.
+    a = math.atanh(delta / h)
+    out = []
+    for m in range(-(L // 2), L // 2 - 1):
+        arg = (m + 0.5 + delta) / h
+        out.append(math.atanh(arg) - a if abs(arg) < 1 else (math.inf if arg > 0 else -math.inf))
+    return np.array(out)
+
+
+@pytest.mark.parametrize("L", [4, 256])
+def test_level_variants_zero_saturation_and_grid(L):
+    h = O.default_h(L)
+    assert h == (L - 1) / 2
+    assert O.fsq_quantize(np.array([0.0]), h, 0.5, L)[0] == 0  # h tanh(atanh(delta/h)) - delta = 0
+    u = np.linspace(-200, 200, 400001)
+    c = O.fsq_quantize(u, h, 0.5, L)
+    assert c[0] == -(L // 2) and c[-1] == L // 2 - 1
+    assert np.all(np.diff(c) >= 0)
+    assert sorted(set(c.tolist())) == list(range(-(L // 2), L // 2))  # exactly L levels are reached
+
+
+@pytest.mark.parametrize("L", [4, 256])
+def test_level_variants_equal_threshold_count(L):
+    h = O.default_h(L)
+    th = _closed_form_thresholds_L(L, h, 0.5)
+    assert len(th) == L - 1 and np.all(np.diff(th) > 0)
+    u = np.linspace(-8.0, 8.0, 400_001)
+    c = O.fsq_quantize(u, h, 0.5, L)
+    n = (u[:, None] >= th[None, :]).sum(axis=1) - L // 2
+    d = np.abs(u[:, None] - th[None, :]).min(axis=1)
+    far = d > 1e-9
+    assert np.array_equal(c[far], n[far])
+    assert np.allclose(O.fsq_boundary_distance(u[::991], h, 0.5, L), d[::991], atol=1e-12)
+
+
+def test_level_variant_thresholds_hand_values():
+    # L = 4, h = 1.5, delta = 0.5: boundaries at u~ = -1.5, -0.5, 0.5 solve
+    # tanh(u + atanh(1/3)) = -2/3, 0, 2/3.  With atanh(x) = ln((1+x)/(1-x))/2,
+    # atanh(1/3) = ln(2)/2 and atanh(2/3) = ln(5)/2, so the three boundaries are
+    # -ln(10)/2, -ln(2)/2 and ln(5/2)/2.
+    hand = [-math.log(10) / 2, -math.log(2) / 2, math.log(2.5) / 2]
+    assert np.allclose(_closed_form_thresholds_L(4, 1.5, 0.5), hand, atol=1e-15)
+    assert O.fsq_quantize(np.array([hand[0] - 1e-6, hand[0] + 1e-6]), 1.5, 0.5, 4).tolist() == [-2, -1]
+
+
+def test_level_variant_packing_layout_and_budgets(golden_dir):
+    rng = np.random.default_rng(3)
+    for L, G in ((4, 320), (4, 576), (256, 80), (256, 144), (16, 160)):
+        lv = rng.integers(-(L // 2), L // 2, size=(9, G))
+        b = O.pack(lv, L)
+        assert b.shape == (9, G * O.bits_per_coordinate(L) // 8)
+        assert np.array_equal(O.unpack(b, G, L), lv)
+    # L = 4: byte k holds coordinates 4k .. 4k+3, the first in bits 0-1; code = level + 2
+    assert O.pack(np.array([[-2, -1, 0, 1]]), 4)[0, 0] == 0b11100100
+    assert O.pack(np.array([[1, 0, 0, 0]]), 4)[0, 0] == 0b00000011 | (0b10 << 2) | (0b10 << 4) | (0b10 << 6)
+    # L = 256: one byte per coordinate, code = level + 128
+    assert O.pack(np.array([[-128, 127, 0]]), 256).tolist() == [[0, 255, 128]]
+    with pytest.raises(ValueError):
+        O.pack(np.array([[2, 0, 0, 0]]), 4)
+    # Table 8: a fixed budget B bytes/token holds 8B/b coordinates at b bits
+    g = json.load(open(os.path.join(golden_dir, "paper_constants.json")))["level_grid_table8"]["value"]
+    for L, bits in zip(g["levels"], g["bits"]):
+        assert O.bits_per_coordinate(L) == bits
+        for budget in g["budgets_bytes_per_token"]:
+            G = 8 * budget // bits
+            assert O.code_bytes_per_token(G, bits) == budget
+    assert [8 * 80 // bb for bb in g["bits"]] == [320, 160, 80]
+    assert [8 * 144 // bb for bb in g["bits"]] == [576, 288, 144]
+
+
+def test_level_variant_attention_matches_sdpa():
+    # decode over L = 4 and L = 256 codes reduces to torch SDPA on the expanded K, V
+    for L, G in ((4, 32), (256, 12)):
+        rng = np.random.default_rng(L)
+        B, n_q, n_kv, d_h, T = 2, 8, 2, 16, 37
+        lv = rng.integers(-(L // 2), L // 2, size=(B, T, G))
+        codes = O.pack(lv, L)
+        W = rng.normal(size=(2 * n_kv * d_h, G)) / math.sqrt(G)
+        q = rng.normal(size=(B, n_q, d_h))
+        o = O.decode_attn(q, codes, W, n_kv, G, levels=L)
+        K = np.stack([O.reconstruct_kv(lv[b], W, n_kv, d_h)[0] for b in range(B)])
+        V = np.stack([O.reconstruct_kv(lv[b], W, n_kv, d_h)[1] for b in range(B)])
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(q)[:, :, None, :], torch.from_numpy(K), torch.from_numpy(V),
+            enable_gqa=True)[:, :, 0, :].numpy()
+        assert np.abs(o - ref).max() <= 1e-12 * max(1.0, np.abs(ref).max())
