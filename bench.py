@@ -186,7 +186,7 @@ def build_state(torch, F, synth, wl, B, T, rank, device, n_copies):
     not need x materialised); each step's new token goes through the whole
     append path (encoder GEMM, FSQ, pack)."""
     G, C = wl.G, wl.C
-    half = G // 2
+    half = F.row_bytes(G, wl.levels)  # bytes per cached token
     T_max = T
     while (T_max * half) % 16:
         T_max += 1
@@ -194,7 +194,7 @@ def build_state(torch, F, synth, wl, B, T, rank, device, n_copies):
     gen = torch.Generator(device=device)
     gen.manual_seed(seed)
     E = synth.normal((G, C), (4.0 / C) ** 0.5, gen, device=device)
-    W_kv, q = synth.decoder_inputs(B, wl.n_q, wl.n_kv, wl.d_h, G, gen, device=device)
+    W_kv, q = synth.decoder_inputs(B, wl.n_q, wl.n_kv, wl.d_h, G, gen, device=device, levels=wl.levels)
     caches = []
     chunk = 1 << 16
     for c in range(n_copies):
@@ -204,7 +204,7 @@ def build_state(torch, F, synth, wl, B, T, rank, device, n_copies):
             for t0 in range(0, T, chunk):
                 n = min(chunk, T - t0)
                 u = synth.preactivations(n, G, gen, device=device)
-                F.quantize_pack_f32(u, out=flat[b * T_max + t0: b * T_max + t0 + n])
+                F.quantize_pack_f32(u, out=flat[b * T_max + t0: b * T_max + t0 + n], levels=wl.levels)
         caches.append(cache)
     x_new = synth.normal((B, C), 1.0, gen, device=device)
     torch.cuda.synchronize()
@@ -214,7 +214,7 @@ def build_state(torch, F, synth, wl, B, T, rank, device, n_copies):
 def run_gpu(args, wl_name, B, T, torch, F, synth, dist, rank, world, device, timed=True):
     wl = synth.WORKLOADS[wl_name]
     G = wl.G
-    half = G // 2
+    half = F.row_bytes(G, wl.levels)
     code_bytes = B * T * half
     n_copies = max(1, math.ceil(2 * L2_BYTES / code_bytes)) if code_bytes < 2 * L2_BYTES else 1
     n_copies = min(n_copies, 8)
@@ -225,9 +225,9 @@ def run_gpu(args, wl_name, B, T, torch, F, synth, dist, rank, world, device, tim
     ws = F.Workspace(device)
     out = torch.empty((B, wl.n_q, wl.d_h), dtype=torch.bfloat16, device=device)
     stream = torch.cuda.current_stream()
-    qp = F.quant_params()
+    qp = F.quant_params(levels=wl.levels)
     nbytes_ws = F.workspace_size(B, T, wl.n_q, wl.n_kv, wl.d_h, G,
-                                 F.attn_opts(variant=args.variant, rope_knorm=args.rope))
+                                 F.attn_opts(variant=args.variant, rope_knorm=args.rope, levels=wl.levels))
     wbuf = ws.get(nbytes_ws)
     sptr = stream.cuda_stream
     gain = None
@@ -238,7 +238,7 @@ def run_gpu(args, wl_name, B, T, torch, F, synth, dist, rank, world, device, tim
 
     def make_opts(prof=None):
         return F.attn_opts(variant=args.variant, prof_events=prof, rope_knorm=args.rope, rope_base=1.0e6,
-                           knorm_gain=gain, knorm_eps=1e-6)
+                           knorm_gain=gain, knorm_eps=1e-6, levels=wl.levels)
 
     def step(i, prof=None):
         cache = st["caches"][i % n_copies]
@@ -367,7 +367,7 @@ def roofline(res, peaks, kernel_name):
     wl, B, T = res["wl"], res["B"], res["T"]
     G, n_q, n_kv, d_h = wl.G, wl.n_q, wl.n_kv, wl.d_h
     variant, rope = res.get("variant", "absorbed"), res.get("rope", False)
-    bytes_alg = B * T * (G // 2)
+    bytes_alg = B * T * (G * {4: 2, 16: 4, 256: 8}[wl.levels] // 8)
     if rope:
         # keys must be rebuilt per position (RoPE): key expansion + scores + latent pooling
         flops_alg = B * T * (2 * n_kv * d_h * G + 2 * n_q * d_h + 2 * n_q * G)
@@ -476,11 +476,11 @@ def _oracle_setup(wl_name, Ts):
     from oracle import fsq_oracle as O
     wl = synth.WORKLOADS[wl_name]
     gen = synth._gen(123)
-    W, q = synth.decoder_inputs(1, wl.n_q, wl.n_kv, wl.d_h, wl.G, gen)
+    W, q = synth.decoder_inputs(1, wl.n_q, wl.n_kv, wl.d_h, wl.G, gen, levels=wl.levels)
     u = synth.preactivations(Ts, wl.G, gen).numpy()
-    codes = O.quantize_pack(u)[None]
+    codes = O.quantize_pack(u, O.default_h(wl.levels), 0.5, wl.levels)[None]
     qn, Wn = q.float().numpy(), W.float().numpy()
-    return lambda: O.decode_attn(qn, codes, Wn, wl.n_kv, wl.G), wl
+    return lambda: O.decode_attn(qn, codes, Wn, wl.n_kv, wl.G, levels=wl.levels), wl
 
 
 def _blas_threads():
@@ -538,21 +538,23 @@ def append_prefill(torch, F, synth, wl, device, peaks, n_new=4096, reps=20):
     xb = n_new * C * 2
     ncop = max(2, min(8, math.ceil(2 * L2_BYTES / xb)))
     xs = [synth.normal((n_new, C), 1.0, gen, device=device) for _ in range(ncop)]
-    out = torch.empty((n_new, G // 2), dtype=torch.uint8, device=device)
+    rb = F.row_bytes(G, wl.levels)
+    out = torch.empty((n_new, rb), dtype=torch.uint8, device=device)
     for i in range(3):
-        F.encode_pack(xs[i % ncop], E, out=out)
+        F.encode_pack(xs[i % ncop], E, out=out, levels=wl.levels)
     torch.cuda.synchronize()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     a.record()
     for i in range(reps):
-        F.encode_pack(xs[i % ncop], E, out=out)
+        F.encode_pack(xs[i % ncop], E, out=out, levels=wl.levels)
     b.record()
     torch.cuda.synchronize()
     t = a.elapsed_time(b) / reps * 1e-3
     flops = 2.0 * n_new * C * G
-    nbytes = xb + G * C * 2 + n_new * G // 2
+    nbytes = xb + G * C * 2 + n_new * rb
     t_roof = max(flops / (peaks["bf16_tflops"] * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9))
-    return {"what": f"fsq_encode_pack of {n_new} tokens, C={C}, G={G} (bf16 x bf16 -> fp32 on tcgen05, FSQ, pack)",
+    return {"what": f"fsq_encode_pack of {n_new} tokens, C={C}, G={G}, {wl.levels} levels "
+                    "(bf16 x bf16 -> fp32 on tcgen05, FSQ, pack)",
             "us_per_call": t * 1e6, "tokens_per_s": n_new / t, "tflops": flops / t / 1e12, "gbs": nbytes / t / 1e9,
             "frac_of_roofline": t_roof / t, "l2": f"{ncop} rotating x copies"}
 
@@ -626,9 +628,11 @@ def main():
     wl = synth.WORKLOADS[wl_name]
     B = args.B if args.B is not None else (DEFAULT_WORKLOAD[1] if wl_name == DEFAULT_WORKLOAD[0] else wl.batches[-1])
     T = args.T if args.T is not None else (DEFAULT_WORKLOAD[2] if wl_name == DEFAULT_WORKLOAD[0] else wl.lengths[-1])
+    rbytes = wl.G * {4: 2, 16: 4, 256: 8}[wl.levels] // 8
     config = {"workload": f"{wl_name}: Qwen3-8B-shaped layer, n_q={wl.n_q} n_kv={wl.n_kv} d_h={wl.d_h} G={wl.G} "
-                          f"({wl.G // 2} B/token), C={wl.C}, batch {B} per GPU, T={T}",
-              "B_per_gpu": B, "T": T, "G": wl.G, "n_q": wl.n_q, "n_kv": wl.n_kv, "d_h": wl.d_h, "C": wl.C,
+                          f"L={wl.levels} ({rbytes} B/token), C={wl.C}, batch {B} per GPU, T={T}",
+              "B_per_gpu": B, "T": T, "G": wl.G, "levels": wl.levels, "n_q": wl.n_q, "n_kv": wl.n_kv,
+              "d_h": wl.d_h, "C": wl.C,
               "variant": args.variant, "rope_knorm": args.rope,
               "parallelism": f"replicas x{world} (batch rows sharded, no collective)"}
 
@@ -659,6 +663,8 @@ def main():
     torch.cuda.set_device(device)
     peaks = load_peaks()
     kernel_name = {"absorbed": "absorbed_split", "expand": "expand_split", "hybrid": "hybrid_split"}[args.variant]
+    if wl.levels != 16:  # the tensor-core kernels read 16-level codes; other level counts run on CUDA cores
+        kernel_name += "_simt"
     res = run_gpu(args, wl_name, B, T, torch, F, synth, dist, rank, world, device)
     also = None
     if not args.no_second and wl_name == DEFAULT_WORKLOAD[0] and args.B is None and args.T is None:
@@ -701,12 +707,13 @@ def main():
                 "value": value, "unit": "context tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": res["ms"], "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None,
-                "dtype": {"absorbed": "u4 codes; s8 x u8 score MMA (s32), f16 pooling MMA (f32), f32 softmax/merge, "
-                                      "bf16 in/out",
-                          "hybrid": "u4 codes; f16 key, score and pooling MMAs (f32), f32 key norm/RoPE/softmax/merge, "
-                                    "bf16 in/out",
-                          "expand": "u4 codes; f16 key, value, score and output MMAs (f32), f32 softmax/merge, "
-                                    "bf16 in/out"}[args.variant],
+                "dtype": ({"absorbed": "u4 codes; s8 x u8 score MMA (s32), f16 pooling MMA (f32), f32 "
+                                       "softmax/merge, bf16 in/out",
+                           "hybrid": "u4 codes; f16 key, score and pooling MMAs (f32), f32 key norm/RoPE/softmax/"
+                                     "merge, bf16 in/out",
+                           "expand": "u4 codes; f16 key, value, score and output MMAs (f32), f32 softmax/merge, "
+                                     "bf16 in/out"}[args.variant] if wl.levels == 16 else
+                          f"u{rbytes * 8 // wl.G} codes; f32 CUDA-core scores, pooling, softmax and merge, bf16 in/out"),
                 "data": "synthetic (seeded; cache = FSQ codes of u ~ N(0,4), the law of E x; new token x ~ N(0,1) appended each step)",
                 "config": config, "l2": l2, "code_gbs": world * res["code_bytes"] / (res["ms"] * 1e-3) / 1e9,
                 "roofline": rf, "cpu_baseline": cb, "e2e": res["e2e"], "clocks": res["clocks"],

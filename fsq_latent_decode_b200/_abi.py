@@ -36,14 +36,14 @@ NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 class QuantParams(C.Structure):
-    _fields_ = [("h", C.c_float), ("delta", C.c_float)]
+    _fields_ = [("h", C.c_float), ("delta", C.c_float), ("levels", C.c_int)]
 
 
 class AttnOpts(C.Structure):
     _fields_ = [("variant", C.c_int), ("scale", C.c_float), ("num_splits", C.c_int),
                 ("rope_knorm", C.c_int), ("rope_base", C.c_float), ("knorm_gain", C.c_void_p),
                 ("knorm_eps", C.c_float), ("out_fp32", C.c_int), ("prof_events", C.c_void_p * 2),
-                ("seq_lens", C.c_void_p), ("debug_stall_ns", C.c_uint32)]
+                ("seq_lens", C.c_void_p), ("debug_stall_ns", C.c_uint32), ("levels", C.c_int)]
 
 
 class EncodeOpts(C.Structure):
@@ -114,19 +114,33 @@ def _check(st: int, what: str):
         raise FsqError(st, what)
 
 
-def quant_params(h: float = 7.5, delta: float = 0.5) -> QuantParams:
-    return QuantParams(float(h), float(delta))
+def bits_of_levels(levels: int) -> int:
+    """b = log2 L bits per coordinate code (L = 4, 16 or 256)."""
+    return {4: 2, 16: 4, 256: 8}[int(levels)]
 
 
-def thresholds(h: float = 7.5, delta: float = 0.5):
-    buf = (C.c_float * 15)()
-    _check(_lib().fsq_thresholds(quant_params(h, delta), buf), "fsq_thresholds")
-    return [buf[i] for i in range(15)]
+def row_bytes(G: int, levels: int = 16) -> int:
+    """Bytes of one token's packed codes: G * b / 8."""
+    return G * bits_of_levels(levels) // 8
+
+
+def quant_params(h: float | None = None, delta: float = 0.5, levels: int = 16) -> QuantParams:
+    """eq. (2) parameters; h defaults to (L-1)/2 (7.5 at 16 levels)."""
+    if h is None:
+        h = (int(levels) - 1) / 2.0
+    return QuantParams(float(h), float(delta), int(levels))
+
+
+def thresholds(h: float | None = None, delta: float = 0.5, levels: int = 16):
+    n = max(int(levels), 16) - 1  # room for the table of a supported level count
+    buf = (C.c_float * n)()
+    _check(_lib().fsq_thresholds(quant_params(h, delta, levels), buf), "fsq_thresholds")
+    return [buf[i] for i in range(int(levels) - 1)]
 
 
 def attn_opts(variant="auto", scale=0.0, num_splits=0, rope_knorm=False, rope_base=1.0e6,
               knorm_gain=None, knorm_eps=1e-6, out_fp32=False, prof_events=None, seq_lens=None,
-              debug_stall_ns=0) -> AttnOpts:
+              debug_stall_ns=0, levels=16) -> AttnOpts:
     o = AttnOpts()
     _lib().fsq_attn_opts_default(C.byref(o))
     o.variant = VARIANTS[variant] if isinstance(variant, str) else int(variant)
@@ -142,6 +156,7 @@ def attn_opts(variant="auto", scale=0.0, num_splits=0, rope_knorm=False, rope_ba
         o.prof_events[1] = int(prof_events[1].cuda_event)
     o.seq_lens = None if seq_lens is None else int(seq_lens.data_ptr())  # device int32 [B]
     o.debug_stall_ns = int(debug_stall_ns)
+    o.levels = int(levels)
     # the struct holds raw device pointers: keep their tensors alive as long as it
     # lives, or the allocator may hand their memory to the next buffer
     o._tensors = (knorm_gain, seq_lens)
@@ -204,28 +219,29 @@ def workspace_status(ws, stream=None) -> int:
 
 
 # ---------------------------------------------------------------- tensor-level wrappers (torch for memory only)
-def encode_pack(x, E, h=7.5, delta=0.5, out=None, stream=None, status_word=None):
-    """codes[n_tok, G/2] (uint8) for bf16 rows x[n_tok, C] through E[G, C].
+def encode_pack(x, E, h=None, delta=0.5, out=None, stream=None, status_word=None, levels=16):
+    """codes[n_tok, G*b/8] (uint8) for bf16 rows x[n_tok, C] through E[G, C].
     status_word: optional device tensor (>= 4 bytes, zeroed by the caller)
     that receives a device-detected failure (read it with workspace_status)."""
     import torch
     n_tok, C_ = x.shape
     G = E.shape[0]
+    rb = row_bytes(G, levels)
     if out is None:
-        out = torch.empty((n_tok, G // 2), dtype=torch.uint8, device=x.device)
-    ldc = out.stride(0) if out.dim() == 2 else G // 2
-    st = encode_pack_raw(_ptr(x), n_tok, x.stride(0), C_, _ptr(E), G, quant_params(h, delta), _ptr(out), ldc,
-                         _stream_ptr(stream), encode_opts(status_word))
+        out = torch.empty((n_tok, rb), dtype=torch.uint8, device=x.device)
+    ldc = out.stride(0) if out.dim() == 2 else rb
+    st = encode_pack_raw(_ptr(x), n_tok, x.stride(0), C_, _ptr(E), G, quant_params(h, delta, levels), _ptr(out),
+                         ldc, _stream_ptr(stream), encode_opts(status_word))
     _check(st, "fsq_encode_pack")
     return out
 
 
-def quantize_pack_f32(u, h=7.5, delta=0.5, out=None, stream=None):
+def quantize_pack_f32(u, h=None, delta=0.5, out=None, stream=None, levels=16):
     import torch
     n_tok, G = u.shape
     if out is None:
-        out = torch.empty((n_tok, G // 2), dtype=torch.uint8, device=u.device)
-    st = quantize_pack_f32_raw(_ptr(u), n_tok, G, quant_params(h, delta), _ptr(out), out.stride(0),
+        out = torch.empty((n_tok, row_bytes(G, levels)), dtype=torch.uint8, device=u.device)
+    st = quantize_pack_f32_raw(_ptr(u), n_tok, G, quant_params(h, delta, levels), _ptr(out), out.stride(0),
                                _stream_ptr(stream))
     _check(st, "fsq_quantize_pack_f32")
     return out
@@ -247,7 +263,8 @@ class Workspace:
 
 def decode_attn(q, codes, W_kv, T, n_kv, G, code_batch_stride=None, opts=None, workspace=None, out=None,
                 stream=None):
-    """o[B, n_q, d_h] = GQA decode attention over codes[B, T_max, G/2] (first T rows)."""
+    """o[B, n_q, d_h] = GQA decode attention over codes[B, T_max, G*b/8] (first T rows);
+    the level count of the codes is opts.levels."""
     import torch
     B, n_q, d_h = q.shape
     if opts is None:
@@ -259,7 +276,7 @@ def decode_attn(q, codes, W_kv, T, n_kv, G, code_batch_stride=None, opts=None, w
         elif codes.dim() == 3:
             code_batch_stride = codes.shape[1] * codes.shape[2]
         else:
-            code_batch_stride = T * (G // 2)
+            code_batch_stride = T * row_bytes(G, opts.levels or 16)
     nbytes = workspace_size(B, T, n_q, n_kv, d_h, G, opts)
     if nbytes == 0:
         raise FsqError(FSQ_ERR_INVALID_ARG, "fsq_decode_attn_workspace_size")

@@ -8,20 +8,23 @@
 #include "common.cuh"
 
 namespace fsq {
-cudaError_t launch_encode_pack_simt(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C, const uint16_t *E,
-                                    int G, const Thresholds &th, uint8_t *codes, int64_t ldc, uint32_t *status,
-                                    uint32_t stall_ns, cudaStream_t s);
-cudaError_t launch_quantize_pack_f32(const float *u, int64_t n_tok, int G, const Thresholds &th, uint8_t *codes,
-                                     int64_t ldc, cudaStream_t s);
+cudaError_t launch_encode_pack(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C, const uint16_t *E, int G,
+                               int levels, const float *th, uint8_t *codes, int64_t ldc, uint32_t *status,
+                               uint32_t stall_ns, cudaStream_t s);
+cudaError_t launch_quantize_pack_f32(const float *u, int64_t n_tok, int G, int levels, const float *th,
+                                     uint8_t *codes, int64_t ldc, cudaStream_t s);
 cudaError_t launch_absorbed_simt(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
-                                 const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv,
-                                 float scale, int S, int64_t tps, float *qa, float *part, uint32_t *err,
-                                 MergeScratch ms, void *o, int out_fp32, void *const *prof, cudaStream_t st);
+                                 const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, int bits,
+                                 const uint16_t *W_kv, float scale, int S, int64_t tps, float *qa, float *part,
+                                 uint32_t *err, MergeScratch ms, void *o, int out_fp32, void *const *prof,
+                                 cudaStream_t st);
 cudaError_t launch_expand_simt(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
-                               const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv,
-                               float scale, int S, int64_t tps, int rope_knorm, float rope_base,
-                               const uint16_t *gain, float eps, float *part, uint32_t *err, void *o, int out_fp32,
-                               void *const *prof, cudaStream_t st);
+                               const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, int bits,
+                               const uint16_t *W_kv, float scale, int S, int64_t tps, int rope_knorm,
+                               float rope_base, const uint16_t *gain, float eps, float *part, uint32_t *err, void *o,
+                               int out_fp32, void *const *prof, cudaStream_t st);
+size_t absorbed_simt_smem(int n_q, int G);
+size_t expand_simt_smem(int G);
 bool expand_tc_supported(int n_q, int n_kv, int G);
 size_t expand_tc_stage_bytes(int G, int variant_expand);
 cudaError_t launch_expand_tc(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
@@ -32,24 +35,39 @@ cudaError_t launch_expand_tc(const uint16_t *q, const uint8_t *codes, int64_t bs
                              uint32_t stall_ns, void *const *prof, cudaStream_t st);
 int simt_max_nq();
 int simt_max_grp();
-bool absorbed_tc_supported(int n_q, int n_kv, int G);
+int absorbed_tc_width(int n_q, int n_kv, int G, int levels);
 size_t absorbed_tc_qphys_bytes(int n_q, int G);
 cudaError_t launch_absorbed_tc(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
-                               const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv,
-                               float scale, int S, int64_t tps, uint8_t *qphys, float *corr, float *part,
-                               uint32_t *err, MergeScratch ms, void *o, int out_fp32, uint32_t stall_ns,
-                               void *const *prof, cudaStream_t st);
+                               const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, int levels,
+                               const uint16_t *W_kv, float scale, int S, int64_t tps, uint8_t *qphys, float *corr,
+                               float *part, uint32_t *err, MergeScratch ms, void *o, int out_fp32,
+                               uint32_t stall_ns, void *const *prof, cudaStream_t st);
 
 namespace {
 
 constexpr int kMaxSplits = 1024;
 constexpr bool kEnableTc = true;  // tensor-core absorbed kernel (being validated)
 
+constexpr size_t kMaxDynSmem = 227 * 1024;  // dynamic shared memory a CTA may request
+
 bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
 
+// Level count of a levels field (0 selects 16); 0 when unsupported.
+int levels_of(int levels) {
+  if (levels == 0) return FSQ_LEVELS;
+  return bits_of_levels(levels) ? levels : 0;
+}
+
+// Latent widths that pack into whole bytes and whole coordinate pairs.
+bool width_ok(int G, int L) { return G >= 2 && G <= FSQ_MAX_G && G % 2 == 0 && (L != 4 || G % 4 == 0); }
+
+// Every level of eq. (2) must lie in {-L/2 .. L/2-1}.
 fsq_status check_quant(fsq_quant_params qp) {
+  const int L = levels_of(qp.levels);
+  if (!L) return FSQ_ERR_UNSUPPORTED;
+  const float top = 0.5f * (float)L;
   if (!(qp.delta > 0.f) || !(qp.h > qp.delta)) return FSQ_ERR_INVALID_ARG;
-  if (!(qp.h - qp.delta <= 7.5f) || !(qp.h + qp.delta <= 8.5f)) return FSQ_ERR_INVALID_ARG;
+  if (!(qp.h - qp.delta <= top - 0.5f) || !(qp.h + qp.delta <= top + 0.5f)) return FSQ_ERR_INVALID_ARG;
   return FSQ_OK;
 }
 
@@ -60,11 +78,13 @@ float ceil_to_float(double x) {
   return f;
 }
 
-void make_thresholds(fsq_quant_params qp, float out[15]) {
+// The L-1 thresholds of eq. (2) at L = levels_of(qp.levels).
+void make_thresholds(fsq_quant_params qp, float *out) {
+  const int L = levels_of(qp.levels);
   const double h = qp.h, dl = qp.delta;
   const double a = atanh(dl / h);
-  for (int k = 0; k < 15; ++k) {
-    const double m = (double)(k - 8);         // boundary between levels m and m+1
+  for (int k = 0; k < L - 1; ++k) {
+    const double m = (double)(k - L / 2);     // boundary between levels m and m+1
     const double arg = (m + 0.5 + dl) / h;    // tanh(u + a) at u~ = m + 1/2
     if (arg >= 1.0) out[k] = INFINITY;
     else if (arg <= -1.0) out[k] = -INFINITY;
@@ -74,6 +94,7 @@ void make_thresholds(fsq_quant_params qp, float out[15]) {
 
 struct Plan {
   int variant;
+  int levels;     // L of the codes
   bool tc;        // tensor-core kernel (absorbed, expand or hybrid form)
   int S;          // splits per batch row
   int64_t tps;    // tokens per split
@@ -85,13 +106,14 @@ struct Plan {
 fsq_status plan_decode(int64_t B, int64_t T, int n_q, int n_kv, int d_h, int G, const fsq_attn_opts &op, Plan *p) {
   if (B < 0 || T < 1 || n_q < 1 || n_kv < 1 || d_h < 1 || G < 2) return FSQ_ERR_INVALID_ARG;
   if (n_q % n_kv) return FSQ_ERR_INVALID_ARG;
-  if (G % 2) return FSQ_ERR_UNSUPPORTED;
-  if (G > FSQ_MAX_G || d_h != FSQ_HEAD_DIM) return FSQ_ERR_UNSUPPORTED;
+  const int L = levels_of(op.levels);
+  if (!L || !width_ok(G, L) || d_h != FSQ_HEAD_DIM) return FSQ_ERR_UNSUPPORTED;
   if (op.variant < FSQ_VARIANT_AUTO || op.variant > FSQ_VARIANT_HYBRID) return FSQ_ERR_INVALID_ARG;
   if (op.num_splits < 0) return FSQ_ERR_INVALID_ARG;
   if (op.rope_knorm != 0 && op.rope_knorm != 1) return FSQ_ERR_INVALID_ARG;
   int variant = op.variant;
-  const bool xtc_shape = kEnableTc && expand_tc_supported(n_q, n_kv, G);
+  // the tensor-core kernels read 16-level codes
+  const bool xtc_shape = kEnableTc && L == 16 && expand_tc_supported(n_q, n_kv, G);
   if (variant == FSQ_VARIANT_AUTO)
     variant = !op.rope_knorm ? FSQ_VARIANT_ABSORBED : (xtc_shape ? FSQ_VARIANT_HYBRID : FSQ_VARIANT_EXPAND);
   if (variant == FSQ_VARIANT_ABSORBED && op.rope_knorm) return FSQ_ERR_UNSUPPORTED;
@@ -102,7 +124,13 @@ fsq_status plan_decode(int64_t B, int64_t T, int n_q, int n_kv, int d_h, int G, 
 
   const int64_t Bc = B > 0 ? B : 1;
   const bool xtc = (variant == FSQ_VARIANT_EXPAND || variant == FSQ_VARIANT_HYBRID) && xtc_shape;
-  const bool tc = (kEnableTc && variant == FSQ_VARIANT_ABSORBED && absorbed_tc_supported(n_q, n_kv, G)) || xtc;
+  // the absorbed tensor-core kernel reads rows of Gn nibbles: 16-level codes,
+  // or 256-level codes read as two nibbles each (Gn = 2G)
+  const int Gn = (kEnableTc && variant == FSQ_VARIANT_ABSORBED) ? absorbed_tc_width(n_q, n_kv, G, L) : 0;
+  const bool tc = Gn > 0 || xtc;
+  // the CUDA-core kernels hold a tile of latents (and, in the expand form, W_kv^(j)) in shared memory
+  if (!tc && variant == FSQ_VARIANT_ABSORBED && absorbed_simt_smem(n_q, G) > kMaxDynSmem) return FSQ_ERR_UNSUPPORTED;
+  if (!tc && variant == FSQ_VARIANT_EXPAND && expand_simt_smem(G) > kMaxDynSmem) return FSQ_ERR_UNSUPPORTED;
   const int64_t ctas_per_row = (variant == FSQ_VARIANT_EXPAND || variant == FSQ_VARIANT_HYBRID) ? n_kv : 1;
   int64_t S = op.num_splits;
   if (S == 0) {
@@ -124,14 +152,15 @@ fsq_status plan_decode(int64_t B, int64_t T, int n_q, int n_kv, int d_h, int G, 
   if (tc) tps = (tps + 127) / 128 * 128;  // whole 128-token tiles, 16-byte aligned split starts
   S = (T + tps - 1) / tps;  // no empty splits
   p->variant = variant;
+  p->levels = L;
   p->tc = tc;
   p->S = (int)S;
   p->tps = tps;
-  const int acc_len = variant == FSQ_VARIANT_EXPAND ? d_h : G;
+  const int acc_len = variant == FSQ_VARIANT_EXPAND ? d_h : (Gn ? Gn : G);  // floats per partial after (m, l)
   size_t off = kWsHeader;
   p->off_qa = off;
   if (xtc) off = align_up(off + (size_t)Bc * n_kv * 16 * d_h * 2, 256);  // staged queries
-  else if (tc) off = align_up(off + absorbed_tc_qphys_bytes(n_q, G) * (size_t)Bc, 256);
+  else if (tc) off = align_up(off + absorbed_tc_qphys_bytes(n_q, Gn) * (size_t)Bc, 256);
   else if (variant == FSQ_VARIANT_ABSORBED) off = align_up(off + sizeof(float) * (size_t)Bc * n_q * G, 256);
   p->off_corr = off;
   if (tc && !xtc) off = align_up(off + 2 * sizeof(float) * (size_t)Bc * n_q, 256);
@@ -149,7 +178,7 @@ fsq_status plan_decode(int64_t B, int64_t T, int n_q, int n_kv, int d_h, int G, 
   }
   p->off_part = off;
   off = align_up(off + sizeof(float) * (size_t)Bc * S * n_q * (2 + acc_len), 256);
-  if (variant == FSQ_VARIANT_ABSORBED || variant == FSQ_VARIANT_HYBRID) p->mp = merge_plan((int)S, Bc, n_q, n_kv, G);
+  if (variant == FSQ_VARIANT_ABSORBED || variant == FSQ_VARIANT_HYBRID) p->mp = merge_plan((int)S, Bc, n_q, n_kv, acc_len);
   p->off_mslab = off;
   off = align_up(off + p->mp.slab_bytes, 256);
   p->off_mcnt = off;
@@ -181,9 +210,10 @@ void fsq_attn_opts_default(fsq_attn_opts *opts) {
   opts->prof_events[0] = opts->prof_events[1] = nullptr;
   opts->seq_lens = nullptr;
   opts->debug_stall_ns = 0;
+  opts->levels = FSQ_LEVELS;
 }
 
-fsq_status fsq_thresholds(fsq_quant_params qp, float theta_out[15]) {
+fsq_status fsq_thresholds(fsq_quant_params qp, float *theta_out) {
   if (!theta_out) return FSQ_ERR_INVALID_ARG;
   fsq_status st = check_quant(qp);
   if (st != FSQ_OK) return st;
@@ -195,34 +225,36 @@ fsq_status fsq_encode_pack(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_
                            fsq_quant_params qp, uint8_t *codes, int64_t ldc_bytes, const fsq_encode_opts *opts,
                            fsq_stream_t stream) {
   if (n_tok < 0 || C < 1 || G < 2) return FSQ_ERR_INVALID_ARG;
-  if (G % 2 || G > FSQ_MAX_G || C % 64) return FSQ_ERR_UNSUPPORTED;
-  if (ldx < C || ldc_bytes < G / 2) return FSQ_ERR_INVALID_ARG;
   fsq_status st = check_quant(qp);
   if (st != FSQ_OK) return st;
+  const int L = levels_of(qp.levels);
+  if (!width_ok(G, L) || C % 64) return FSQ_ERR_UNSUPPORTED;
+  if (ldx < C || ldc_bytes < (int64_t)G * bits_of_levels(L) / 8) return FSQ_ERR_INVALID_ARG;
   if (n_tok == 0) return FSQ_OK;
   if (!x || !E || !codes) return FSQ_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(E) || ldx % 8) return FSQ_ERR_MISALIGNED;
   uint32_t *status = opts ? opts->status_word : nullptr;
   if ((uintptr_t)status & 3u) return FSQ_ERR_MISALIGNED;
-  Thresholds th;
-  make_thresholds(qp, th.th);
-  return from_cuda(launch_encode_pack_simt(x, n_tok, ldx, C, E, G, th, codes, ldc_bytes, status,
-                                           opts ? opts->debug_stall_ns : 0u, (cudaStream_t)stream));
+  float th[kMaxLevels - 1];
+  make_thresholds(qp, th);
+  return from_cuda(launch_encode_pack(x, n_tok, ldx, C, E, G, L, th, codes, ldc_bytes, status,
+                                      opts ? opts->debug_stall_ns : 0u, (cudaStream_t)stream));
 }
 
 fsq_status fsq_quantize_pack_f32(const float *u, int64_t n_tok, int G, fsq_quant_params qp, uint8_t *codes,
                                  int64_t ldc_bytes, fsq_stream_t stream) {
   if (n_tok < 0 || G < 2) return FSQ_ERR_INVALID_ARG;
-  if (G % 2 || G > FSQ_MAX_G) return FSQ_ERR_UNSUPPORTED;
-  if (ldc_bytes < G / 2) return FSQ_ERR_INVALID_ARG;
   fsq_status st = check_quant(qp);
   if (st != FSQ_OK) return st;
+  const int L = levels_of(qp.levels);
+  if (!width_ok(G, L)) return FSQ_ERR_UNSUPPORTED;
+  if (ldc_bytes < (int64_t)G * bits_of_levels(L) / 8) return FSQ_ERR_INVALID_ARG;
   if (n_tok == 0) return FSQ_OK;
   if (!u || !codes) return FSQ_ERR_INVALID_ARG;
   if (!aligned16(u)) return FSQ_ERR_MISALIGNED;
-  Thresholds th;
-  make_thresholds(qp, th.th);
-  return from_cuda(launch_quantize_pack_f32(u, n_tok, G, th, codes, ldc_bytes, (cudaStream_t)stream));
+  float th[kMaxLevels - 1];
+  make_thresholds(qp, th);
+  return from_cuda(launch_quantize_pack_f32(u, n_tok, G, L, th, codes, ldc_bytes, (cudaStream_t)stream));
 }
 
 size_t fsq_decode_attn_workspace_size(int64_t B, int64_t T, int n_q, int n_kv, int d_h, int G,
@@ -247,7 +279,8 @@ fsq_status fsq_decode_attn(const uint16_t *q, int64_t B, int n_q, int d_h, const
   if (st != FSQ_OK) return st;
   if (B == 0) return FSQ_OK;
   if (!q || !codes || !W_kv || !o) return FSQ_ERR_INVALID_ARG;
-  if (code_batch_stride_bytes < T * (G / 2)) return FSQ_ERR_INVALID_ARG;
+  const int bits = bits_of_levels(p.levels);
+  if (code_batch_stride_bytes < T * ((int64_t)G * bits / 8)) return FSQ_ERR_INVALID_ARG;
   if (!aligned16(codes) || code_batch_stride_bytes % 16) return FSQ_ERR_MISALIGNED;
   if (!aligned16(q) || !aligned16(W_kv) || !aligned16(o)) return FSQ_ERR_MISALIGNED;
   if ((uintptr_t)op.seq_lens & 3u) return FSQ_ERR_MISALIGNED;
@@ -268,15 +301,16 @@ fsq_status fsq_decode_attn(const uint16_t *q, int64_t B, int n_q, int d_h, const
                          (float *)(ws + p.off_ck), (float *)(ws + p.off_cv), (uint8_t *)(ws + p.off_qa), part, err,
                          ms, o, op.out_fp32, op.debug_stall_ns, op.prof_events, s);
   } else if (p.tc) {
-    e = launch_absorbed_tc(q, codes, code_batch_stride_bytes, B, T, op.seq_lens, n_q, n_kv, d_h, G, W_kv, scale,
-                           p.S, p.tps, (uint8_t *)(ws + p.off_qa), (float *)(ws + p.off_corr), part, err, ms, o,
-                           op.out_fp32, op.debug_stall_ns, op.prof_events, s);
+    e = launch_absorbed_tc(q, codes, code_batch_stride_bytes, B, T, op.seq_lens, n_q, n_kv, d_h, G, p.levels, W_kv,
+                           scale, p.S, p.tps, (uint8_t *)(ws + p.off_qa), (float *)(ws + p.off_corr), part, err, ms,
+                           o, op.out_fp32, op.debug_stall_ns, op.prof_events, s);
   } else if (p.variant == FSQ_VARIANT_ABSORBED) {
-    e = launch_absorbed_simt(q, codes, code_batch_stride_bytes, B, T, op.seq_lens, n_q, n_kv, d_h, G, W_kv, scale,
-                             p.S, p.tps, (float *)(ws + p.off_qa), part, err, ms, o, op.out_fp32, op.prof_events, s);
+    e = launch_absorbed_simt(q, codes, code_batch_stride_bytes, B, T, op.seq_lens, n_q, n_kv, d_h, G, bits, W_kv,
+                             scale, p.S, p.tps, (float *)(ws + p.off_qa), part, err, ms, o, op.out_fp32,
+                             op.prof_events, s);
   } else {
-    e = launch_expand_simt(q, codes, code_batch_stride_bytes, B, T, op.seq_lens, n_q, n_kv, d_h, G, W_kv, scale,
-                           p.S, p.tps, op.rope_knorm, op.rope_base, op.knorm_gain, op.knorm_eps, part, err, o,
+    e = launch_expand_simt(q, codes, code_batch_stride_bytes, B, T, op.seq_lens, n_q, n_kv, d_h, G, bits, W_kv,
+                           scale, p.S, p.tps, op.rope_knorm, op.rope_base, op.knorm_gain, op.knorm_eps, part, err, o,
                            op.out_fp32, op.prof_events, s);
   }
   return from_cuda(e);

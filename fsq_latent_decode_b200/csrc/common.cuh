@@ -20,8 +20,15 @@ constexpr int kNumSMs = 148;
 // 1/ln(2): scores are kept in the log2 domain so the softmax uses exp2.
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Supported level counts L and their code widths b = log2 L ([D] backup frame
+// "the grid size is an allocation choice", Table 8: 4, 16 and 256 levels).
+constexpr int kMaxLevels = 256;
+__host__ __device__ constexpr int bits_of_levels(int L) { return L == 4 ? 2 : L == 16 ? 4 : L == 256 ? 8 : 0; }
+
+// The L-1 ascending fp32 decision thresholds of eq. (2) at L levels.
+template <int L>
 struct Thresholds {
-  float th[15];
+  float th[L - 1];
 };
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t v) {
@@ -33,11 +40,22 @@ __device__ __forceinline__ uint16_t f32_to_bf16_rn(float f) {
   return *reinterpret_cast<uint16_t *>(&b);
 }
 
-// Nibble = number of thresholds at or below u (0..15); level = nibble - 8.
-__device__ __forceinline__ uint32_t fsq_nibble(float u, const Thresholds &t) {
+// Code = number of thresholds at or below u (0..L-1); level = code - L/2.
+// Up to 16 levels every threshold is compared; at 256 levels a binary search
+// over the ascending table finds the same count (8 comparisons).  Kernels
+// take the table as a __grid_constant__ parameter, so indexing it reads the
+// parameter space directly.
+template <int L>
+__device__ __forceinline__ uint32_t fsq_code(float u, const Thresholds<L> &t) {
   uint32_t n = 0;
+  if constexpr (L <= 16) {
 #pragma unroll
-  for (int k = 0; k < 15; ++k) n += (u >= t.th[k]) ? 1u : 0u;
+    for (int k = 0; k < L - 1; ++k) n += (u >= t.th[k]) ? 1u : 0u;
+  } else {
+#pragma unroll
+    for (uint32_t step = L / 2; step; step >>= 1)
+      if (u >= t.th[n + step - 1]) n += step;  // index <= L - 1 - step
+  }
   return n;
 }
 

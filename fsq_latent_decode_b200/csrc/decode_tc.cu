@@ -756,10 +756,12 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int g = 128 * h + 32 * q + 8 * (sl >> 1) + 4 * (sl & 1) + jn;
+          if (g < G) {  // G < 256: the second half is partly padding
 #pragma unroll
-          for (int n = 0; n < HQ; ++n)
-            out[(size_t)(h0 + n) * (2 + G) + 2 + g] =
-                fmaf(__uint_as_float(h ? a1[n] : a0[n]), vscale, -8.f * Lt[h0 + n]);
+            for (int n = 0; n < HQ; ++n)
+              out[(size_t)(h0 + n) * (2 + G) + 2 + g] =
+                  fmaf(__uint_as_float(h ? a1[n] : a0[n]), vscale, -8.f * Lt[h0 + n]);
+          }
         }
       } else {
         const int g = 32 * q + 8 * (sl >> 1) + 4 * (sl & 1) + jn;
@@ -789,6 +791,12 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
 // kappa = 8w + 4e + i for coordinate 8w + 2i + e (the dequant's byte order).
 // corr[b] = [sigma_h] then [sigma_h * 8 * sum_g (128 a_g + b_g)]: the score is
 // sigma (128 S_a + S_b) - offset, the offset removing the +8 of the bytes.
+// BYTE: the cache holds 256-level codes, one byte per coordinate i, read here
+// as two nibbles (G = 2 x the latent width): with n = lo + 16 hi, the level
+// n - 128 = (lo - 8) + 16 (hi - 8) + 8, so nibble 2i carries weight q'_i and
+// nibble 2i+1 weight 16 q'_i; the constant 8 q'_i shifts every score of a head
+// alike (the softmax ignores it) and the merge folds the pooled nibble pairs
+// back (merge.cu).  W_k^(j) is then [D][G/2].
 // Threads: KPAD coordinates x NDQ slices of the head dimension.  W_k^(j)
 // is staged in shared memory by 16-byte asynchronous copies (requested before
 // q, so the two latencies overlap); thread (dq, g) sums its slice of the head
@@ -798,11 +806,12 @@ template <int GRP>
 struct AbsorbShape {
   static constexpr int NDQ = GRP <= 4 ? 4 : (GRP == 8 ? 2 : 1);
 };
-template <int G, int NQ, int GRP>
+template <int G, int NQ, int GRP, bool BYTE>
 struct AbsorbSmem {
   static constexpr int GS = Cfg<G, NQ>::KPAD;
   static constexpr int NDQ = AbsorbShape<GRP>::NDQ;
-  static constexpr int W_BYTES = FSQ_HEAD_DIM * G * 2;          // W_k^(j), bf16 [D][G]
+  static constexpr int GW = BYTE ? G / 2 : G;                    // columns of W_k^(j)
+  static constexpr int W_BYTES = FSQ_HEAD_DIM * GW * 2;         // W_k^(j), bf16 [D][GW]
   static constexpr int PART_OFF = (W_BYTES + 15) / 16 * 16;
   static constexpr int BYTES = PART_OFF + NDQ * GRP * GS * 4;  // slice sums, fp32 [NDQ][GRP][GS]
 };
@@ -811,13 +820,14 @@ __device__ __forceinline__ void cp_async16_g2s(void *smem_dst, const void *gsrc)
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
 }
 
-template <int G, int NQ, int GRP>
+template <int G, int NQ, int GRP, bool BYTE>
 __global__ void __launch_bounds__(Cfg<G, NQ>::KPAD * AbsorbShape<GRP>::NDQ)
     absorb_query_tc(const uint16_t *__restrict__ q, const uint16_t *__restrict__ W_kv, float c,
                     uint8_t *__restrict__ qphys, float *__restrict__ corr, uint32_t *err, MergeScratch ms) {
   // one CTA per (kv head j, batch row b): the group's heads share W_k^(j), read once
   using C = Cfg<G, NQ>;
-  using SM = AbsorbSmem<G, NQ, GRP>;
+  using SM = AbsorbSmem<G, NQ, GRP, BYTE>;
+  constexpr int GW = SM::GW;
   constexpr int D = FSQ_HEAD_DIM;
   constexpr int NDQ = SM::NDQ;
   constexpr int GS = SM::GS;        // threads per slice (one per padded coordinate)
@@ -842,7 +852,7 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::KPAD * AbsorbShape<GRP>::NDQ)
   // at the end, before releasing the split kernel, whose first code loads
   // precede its own wait.
   {
-    const uint8_t *src = reinterpret_cast<const uint8_t *>(W_kv + (int64_t)j * D * G);
+    const uint8_t *src = reinterpret_cast<const uint8_t *>(W_kv + (int64_t)j * D * GW);
     for (int k = threadIdx.x; k < SM::W_BYTES / 16; k += NT) cp_async16_g2s(asmem + 16 * k, src + 16 * k);
     asm volatile("cp.async.commit_group;" ::: "memory");
   }
@@ -858,11 +868,11 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::KPAD * AbsorbShape<GRP>::NDQ)
 #pragma unroll
   for (int hh = 0; hh < GRP; ++hh) v[hh] = 0.f;
   if (g < G) {
-    const uint16_t *wk = wks + (dq * DS) * G + g;
+    const uint16_t *wk = wks + (dq * DS) * GW + (BYTE ? g >> 1 : g);
 #pragma unroll 8
     for (int u = 0; u < DS; u += 4) {
-      const float w0 = bf16_to_f32(wk[(u + 0) * G]), w1 = bf16_to_f32(wk[(u + 1) * G]);
-      const float w2 = bf16_to_f32(wk[(u + 2) * G]), w3 = bf16_to_f32(wk[(u + 3) * G]);
+      const float w0 = bf16_to_f32(wk[(u + 0) * GW]), w1 = bf16_to_f32(wk[(u + 1) * GW]);
+      const float w2 = bf16_to_f32(wk[(u + 2) * GW]), w3 = bf16_to_f32(wk[(u + 3) * GW]);
 #pragma unroll
       for (int hh = 0; hh < GRP; ++hh) {
         const float4 qv = *reinterpret_cast<const float4 *>(&qs[hh][dq * DS + u]);
@@ -875,6 +885,7 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::KPAD * AbsorbShape<GRP>::NDQ)
   __syncthreads();
   // slice dq finishes heads dq, dq + NDQ, ...
   constexpr int HPS = (GRP + NDQ - 1) / NDQ;  // heads per slice
+  const float cg = (BYTE && (g & 1)) ? 16.f * c : c;  // the high nibble of a byte code weighs 16
   float vf[HPS];
 #pragma unroll
   for (int k = 0; k < HPS; ++k) {
@@ -884,7 +895,7 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::KPAD * AbsorbShape<GRP>::NDQ)
 #pragma unroll
       for (int i = 0; i < NDQ; ++i) t += part[(i * GRP + hh) * GS + g];
     }
-    vf[k] = t * c;
+    vf[k] = t * cg;
     float am = fabsf(vf[k]);
 #pragma unroll
     for (int o = 16; o; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
@@ -930,26 +941,26 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::KPAD * AbsorbShape<GRP>::NDQ)
   pdl_trigger();  // the split kernel may start its prologue and code loads
 }
 
-template <int G, int NQ, int GRP>
+template <int G, int NQ, int GRP, bool BYTE>
 cudaError_t absorb_query_launch(const dim3 &grid, const uint16_t *q, const uint16_t *W_kv, float c, uint8_t *qphys,
                                 float *corr, uint32_t *err, MergeScratch ms, cudaStream_t st) {
-  using SM = AbsorbSmem<G, NQ, GRP>;
-  cudaError_t e = ensure_smem_limit((const void *)absorb_query_tc<G, NQ, GRP>, (size_t)SM::BYTES);
+  using SM = AbsorbSmem<G, NQ, GRP, BYTE>;
+  cudaError_t e = ensure_smem_limit((const void *)absorb_query_tc<G, NQ, GRP, BYTE>, (size_t)SM::BYTES);
   if (e != cudaSuccess) return e;
-  return launch_pdl(absorb_query_tc<G, NQ, GRP>, grid, dim3(Cfg<G, NQ>::KPAD * AbsorbShape<GRP>::NDQ),
+  return launch_pdl(absorb_query_tc<G, NQ, GRP, BYTE>, grid, dim3(Cfg<G, NQ>::KPAD * AbsorbShape<GRP>::NDQ),
                     (size_t)SM::BYTES, st, q, W_kv, c, qphys, corr, err, ms);
 }
 
-template <int G, int NQ>
+template <int G, int NQ, bool BYTE>
 cudaError_t launch_absorb_query(const uint16_t *q, int64_t B, int n_kv, const uint16_t *W_kv, float c,
                                 uint8_t *qphys, float *corr, uint32_t *err, MergeScratch ms, cudaStream_t st) {
   const dim3 grid(n_kv, (unsigned)B);
   switch (NQ / n_kv) {
-    case 1: return absorb_query_launch<G, NQ, 1>(grid, q, W_kv, c, qphys, corr, err, ms, st);
-    case 2: return absorb_query_launch<G, NQ, 2>(grid, q, W_kv, c, qphys, corr, err, ms, st);
-    case 4: return absorb_query_launch<G, NQ, 4>(grid, q, W_kv, c, qphys, corr, err, ms, st);
-    case 8: return absorb_query_launch<G, NQ, 8>(grid, q, W_kv, c, qphys, corr, err, ms, st);
-    case 16: return absorb_query_launch<G, NQ, 16>(grid, q, W_kv, c, qphys, corr, err, ms, st);
+    case 1: return absorb_query_launch<G, NQ, 1, BYTE>(grid, q, W_kv, c, qphys, corr, err, ms, st);
+    case 2: return absorb_query_launch<G, NQ, 2, BYTE>(grid, q, W_kv, c, qphys, corr, err, ms, st);
+    case 4: return absorb_query_launch<G, NQ, 4, BYTE>(grid, q, W_kv, c, qphys, corr, err, ms, st);
+    case 8: return absorb_query_launch<G, NQ, 8, BYTE>(grid, q, W_kv, c, qphys, corr, err, ms, st);
+    case 16: return absorb_query_launch<G, NQ, 16, BYTE>(grid, q, W_kv, c, qphys, corr, err, ms, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -984,13 +995,13 @@ cudaError_t make_code_tensor_map(CUtensorMap *map, const uint8_t *codes, int64_t
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int G, int NQ>
+template <int G, int NQ, bool BYTE>
 cudaError_t launch(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
                    const int32_t *seq_lens, int n_kv, const uint16_t *W_kv, float scale, int S, int64_t tps,
                    uint8_t *qphys, float *corr, float *part, uint32_t *err, MergeScratch ms, uint32_t stall_ns,
                    void *const *prof, cudaStream_t st) {
   using C = Cfg<G, NQ>;
-  cudaError_t e = launch_absorb_query<G, NQ>(q, B, n_kv, W_kv, scale * kLog2e, qphys, corr, err, ms, st);
+  cudaError_t e = launch_absorb_query<G, NQ, BYTE>(q, B, n_kv, W_kv, scale * kLog2e, qphys, corr, err, ms, st);
   if (e != cudaSuccess) return e;
   // one CTA per SM: ask for more shared memory than two CTAs could share
   const int smem = C::SM_TOTAL > 120 * 1024 ? C::SM_TOTAL : 120 * 1024;
@@ -1013,8 +1024,14 @@ cudaError_t launch(const uint16_t *q, const uint8_t *codes, int64_t bstride, int
 
 }  // namespace tc
 
-bool absorbed_tc_supported(int n_q, int n_kv, int G) {
-  return (n_q == 16 || n_q == 32) && (G == 256 || G == 84) && n_kv > 0 && n_q % n_kv == 0 && n_q / n_kv <= 16;
+// Width of the nibble rows the split kernel reads: G at 16 levels; 2G at 256
+// levels (each 8-bit code read as two nibbles); 0 when the kernel does not
+// cover the shape.
+int absorbed_tc_width(int n_q, int n_kv, int G, int levels) {
+  const int Gn = levels == 16 ? G : (levels == 256 ? 2 * G : 0);
+  const bool ok = (n_q == 16 || n_q == 32) && (Gn == 256 || Gn == 160 || Gn == 84) && n_kv > 0 && n_q % n_kv == 0 &&
+                  n_q / n_kv <= 16;
+  return ok ? Gn : 0;
 }
 
 size_t absorbed_tc_qphys_bytes(int n_q, int G) {
@@ -1023,25 +1040,33 @@ size_t absorbed_tc_qphys_bytes(int n_q, int G) {
 }
 
 cudaError_t merge_absorbed_launch(const float *part, int S, int64_t B, int n_q, int n_kv, int d_h, int G,
-                                  const uint16_t *W_kv, void *o, int out_fp32, MergeScratch ms, cudaStream_t st);
+                                  const uint16_t *W_kv, void *o, int out_fp32, MergeScratch ms, cudaStream_t st,
+                                  int fold_bytes);
 
+// G: the latent width of the cache (levels 16 or 256); the partials carry
+// absorbed_tc_width(...) nibble coordinates, folded back by the merge.
 cudaError_t launch_absorbed_tc(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
-                               const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv,
-                               float scale, int S, int64_t tps, uint8_t *qphys, float *corr, float *part,
-                               uint32_t *err, MergeScratch ms, void *o, int out_fp32, uint32_t stall_ns,
-                               void *const *prof, cudaStream_t st) {
-  cudaError_t e;
-#define FSQ_TC_LAUNCH(GG, NN)                                                                                  \
-  tc::launch<GG, NN>(q, codes, bstride, B, T, seq_lens, n_kv, W_kv, scale, S, tps, qphys, corr, part, err, ms, \
-                     stall_ns, prof, st)
-  if (G == 256 && n_q == 32) e = FSQ_TC_LAUNCH(256, 32);
-  else if (G == 256 && n_q == 16) e = FSQ_TC_LAUNCH(256, 16);
-  else if (G == 84 && n_q == 32) e = FSQ_TC_LAUNCH(84, 32);
-  else if (G == 84 && n_q == 16) e = FSQ_TC_LAUNCH(84, 16);
+                               const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, int levels,
+                               const uint16_t *W_kv, float scale, int S, int64_t tps, uint8_t *qphys, float *corr,
+                               float *part, uint32_t *err, MergeScratch ms, void *o, int out_fp32,
+                               uint32_t stall_ns, void *const *prof, cudaStream_t st) {
+  const int Gn = absorbed_tc_width(n_q, n_kv, G, levels);
+  const bool byte = levels == 256;
+  cudaError_t e = cudaErrorInvalidValue;
+#define FSQ_TC_LAUNCH(GG, NN, BB)                                                                                  \
+  tc::launch<GG, NN, BB>(q, codes, bstride, B, T, seq_lens, n_kv, W_kv, scale, S, tps, qphys, corr, part, err, ms, \
+                         stall_ns, prof, st)
+#define FSQ_TC_CASE(GG)                                                       \
+  if (Gn == GG && n_q == 32) e = byte ? FSQ_TC_LAUNCH(GG, 32, true) : FSQ_TC_LAUNCH(GG, 32, false); \
+  else if (Gn == GG && n_q == 16) e = byte ? FSQ_TC_LAUNCH(GG, 16, true) : FSQ_TC_LAUNCH(GG, 16, false);
+  FSQ_TC_CASE(256)
+  else FSQ_TC_CASE(160)
+  else FSQ_TC_CASE(84)
   else return cudaErrorInvalidValue;
+#undef FSQ_TC_CASE
 #undef FSQ_TC_LAUNCH
   if (e != cudaSuccess) return e;
-  return merge_absorbed_launch(part, S, B, n_q, n_kv, d_h, G, W_kv, o, out_fp32, ms, st);
+  return merge_absorbed_launch(part, S, B, n_q, n_kv, d_h, Gn, W_kv, o, out_fp32, ms, st, byte ? 1 : 0);
 }
 
 }  // namespace fsq

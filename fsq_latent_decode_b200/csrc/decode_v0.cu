@@ -8,6 +8,10 @@
 //  * EXPAND: per tile k_t = W_k^(j) z_t (optionally RoPE_t(N_k(.))) and
 //    v_t = W_v^(j) z_t, then standard GQA online-softmax attention
 //    (summary eq. (5)).
+// The code of a coordinate is b = log2 L bits wide (L = 4, 16 or 256 levels;
+// slide deck backup frame "the grid size is an allocation choice"): a byte of
+// a row holds 8/b consecutive coordinates, the first in its lowest bits, and a
+// level is code - L/2.
 // Long contexts are split over token ranges; each split emits (m, l, acc)
 // in the log2 domain and a merge kernel combines them by log-sum-exp
 // (slide deck frame "The kernel reads codes and never writes reconstructed
@@ -50,8 +54,8 @@ __global__ void absorb_query_kernel(const uint16_t *__restrict__ q, const uint16
 __global__ void __launch_bounds__(256) absorbed_split_simt(const float *__restrict__ qa,
                                                            const uint8_t *__restrict__ codes, int64_t bstride,
                                                            int64_t T, const int32_t *__restrict__ seq_lens,
-                                                           int G, int n_q, int64_t tps, float *__restrict__ part,
-                                                           uint32_t *err) {
+                                                           int G, int bits, int n_q, int64_t tps,
+                                                           float *__restrict__ part, uint32_t *err) {
   extern __shared__ float sm[];
   float *qs = sm;                                   // [n_q][G]
   float *acc = qs + n_q * G;                        // [n_q][G]
@@ -64,7 +68,9 @@ __global__ void __launch_bounds__(256) absorbed_split_simt(const float *__restri
   const int s = blockIdx.x, b = blockIdx.y, S = gridDim.x;
   const int64_t t0 = (int64_t)s * tps;
   const int64_t t1 = min(row_len(seq_lens, b, T, err, s == 0 && tid == 0), t0 + tps);  // empty past the row's end
-  const int half = G / 2;
+  const int per = 8 / bits, rb = G / per;  // coordinates per byte, bytes per row
+  const uint32_t mask = (1u << bits) - 1u;
+  const float off = (float)(1 << (bits - 1));  // L/2
   const uint8_t *cb = codes + (int64_t)b * bstride;
 
   for (int i = tid; i < n_q * G; i += nth) {
@@ -79,16 +85,11 @@ __global__ void __launch_bounds__(256) absorbed_split_simt(const float *__restri
 
   for (int64_t tt = t0; tt < t1; tt += kNT) {
     const int nv = (int)min((int64_t)kNT, t1 - tt);
-    for (int i = tid; i < kNT * half; i += nth) {
-      int t = i / half, by = i % half;
-      float lo = 0.f, hi = 0.f;
-      if (t < nv) {
-        uint32_t v = cb[(tt + t) * half + by];
-        lo = (float)(int)(v & 15u) - 8.f;
-        hi = (float)(int)(v >> 4) - 8.f;
-      }
-      cs[t * (G + 1) + 2 * by] = lo;
-      cs[t * (G + 1) + 2 * by + 1] = hi;
+    for (int i = tid; i < kNT * rb; i += nth) {
+      const int t = i / rb, by = i % rb;
+      const uint32_t v = t < nv ? cb[(tt + t) * rb + by] : 0u;
+      for (int c = 0; c < per; ++c)
+        cs[t * (G + 1) + per * by + c] = t < nv ? (float)((v >> (bits * c)) & mask) - off : 0.f;
     }
     __syncthreads();
     for (int i = tid; i < kNT * n_q; i += nth) {
@@ -182,7 +183,8 @@ __global__ void merge_absorbed_kernel(const float *__restrict__ part, int S, int
 __global__ void __launch_bounds__(128) expand_split_simt(const uint16_t *__restrict__ q,
                                                          const uint8_t *__restrict__ codes, int64_t bstride,
                                                          int64_t T, const int32_t *__restrict__ seq_lens, int G,
-                                                         int n_q, int n_kv, const uint16_t *__restrict__ W_kv,
+                                                         int bits, int n_q, int n_kv,
+                                                         const uint16_t *__restrict__ W_kv,
                                                          float c, int64_t tps, int rope_knorm, float rope_base,
                                                          const uint16_t *__restrict__ gain, float eps,
                                                          float *__restrict__ part, uint32_t *err) {
@@ -200,7 +202,9 @@ __global__ void __launch_bounds__(128) expand_split_simt(const uint16_t *__restr
   const int grp = n_q / n_kv;
   const int64_t t0 = (int64_t)s * tps;
   const int64_t t1 = min(row_len(seq_lens, b, T, err, s == 0 && j == 0 && d == 0), t0 + tps);
-  const int half = G / 2;
+  const int per = 8 / bits, rb = G / per;  // coordinates per byte, bytes per row
+  const uint32_t mask = (1u << bits) - 1u;
+  const float off = (float)(1 << (bits - 1));  // L/2
   const uint8_t *cb = codes + (int64_t)b * bstride;
 
   for (int i = d; i < G * D; i += D) {
@@ -219,16 +223,11 @@ __global__ void __launch_bounds__(128) expand_split_simt(const uint16_t *__restr
 
   for (int64_t tt = t0; tt < t1; tt += kNTx) {
     const int nv = (int)min((int64_t)kNTx, t1 - tt);
-    for (int i = d; i < kNTx * half; i += D) {
-      int t = i / half, by = i % half;
-      float lo = 0.f, hi = 0.f;
-      if (t < nv) {
-        uint32_t v = cb[(tt + t) * half + by];
-        lo = (float)(int)(v & 15u) - 8.f;
-        hi = (float)(int)(v >> 4) - 8.f;
-      }
-      cs[t * G + 2 * by] = lo;
-      cs[t * G + 2 * by + 1] = hi;
+    for (int i = d; i < kNTx * rb; i += D) {
+      const int t = i / rb, by = i % rb;
+      const uint32_t v = t < nv ? cb[(tt + t) * rb + by] : 0u;
+      for (int c = 0; c < per; ++c)
+        cs[t * G + per * by + c] = t < nv ? (float)((v >> (bits * c)) & mask) - off : 0.f;
     }
     __syncthreads();
     float vr[kNTx];
@@ -342,14 +341,17 @@ __global__ void clear_err_kernel(uint32_t *err) { *err = 0u; }
 bool merge_grouped_supported(int n_q, int n_kv);
 cudaError_t merge_grouped_launch(const float *part, int S, int64_t B, int n_q, int n_kv, int G,
                                  const uint16_t *W_kv, void *o, int out_fp32, float *slab, uint32_t *cnt,
-                                 cudaStream_t st);
+                                 cudaStream_t st, int fold_bytes);
 
 // Group sizes 1, 2, 4, 8, 16 share W_v^(j) reads across the group (merge.cu);
-// others take one CTA per query head.
+// others take one CTA per query head.  fold_bytes: the partials carry 8-bit
+// codes read as nibble pairs (G of them = 2 x the latent width; grouped merge only).
 cudaError_t merge_absorbed_launch(const float *part, int S, int64_t B, int n_q, int n_kv, int d_h, int G,
-                                  const uint16_t *W_kv, void *o, int out_fp32, MergeScratch ms, cudaStream_t st) {
+                                  const uint16_t *W_kv, void *o, int out_fp32, MergeScratch ms, cudaStream_t st,
+                                  int fold_bytes) {
   if (merge_grouped_supported(n_q, n_kv))
-    return merge_grouped_launch(part, S, B, n_q, n_kv, G, W_kv, o, out_fp32, ms.slab, ms.cnt, st);
+    return merge_grouped_launch(part, S, B, n_q, n_kv, G, W_kv, o, out_fp32, ms.slab, ms.cnt, st, fold_bytes);
+  if (fold_bytes) return cudaErrorInvalidValue;
   merge_absorbed_kernel<<<dim3(n_q, (unsigned)B), 256, 0, st>>>(part, S, n_q, n_kv, d_h, G, W_kv, o, out_fp32);
   return cudaGetLastError();
 }
@@ -374,7 +376,8 @@ int simt_max_nq() { return kMaxNQ; }
 int simt_max_grp() { return kMaxGrp; }
 
 cudaError_t launch_absorbed_simt(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
-                                 const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv,
+                                 const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, int bits,
+                                 const uint16_t *W_kv,
                                  float scale, int S, int64_t tps, float *qa, float *part, uint32_t *err,
                                  MergeScratch ms, void *o, int out_fp32, void *const *prof, cudaStream_t st) {
   absorb_query_kernel<<<dim3(n_q, (unsigned)B), 256, 0, st>>>(q, W_kv, n_q, n_kv, d_h, G, scale * kLog2e, qa, err,
@@ -385,16 +388,17 @@ cudaError_t launch_absorbed_simt(const uint16_t *q, const uint8_t *codes, int64_
   e = ensure_smem_limit((const void *)absorbed_split_simt, smem);
   if (e != cudaSuccess) return e;
   record_prof_event(prof[0], st);
-  absorbed_split_simt<<<dim3(S, (unsigned)B), 256, smem, st>>>(qa, codes, bstride, T, seq_lens, G, n_q, tps, part,
-                                                                err);
+  absorbed_split_simt<<<dim3(S, (unsigned)B), 256, smem, st>>>(qa, codes, bstride, T, seq_lens, G, bits, n_q, tps,
+                                                                part, err);
   e = cudaGetLastError();
   record_prof_event(prof[1], st);
   if (e != cudaSuccess) return e;
-  return merge_absorbed_launch(part, S, B, n_q, n_kv, d_h, G, W_kv, o, out_fp32, ms, st);
+  return merge_absorbed_launch(part, S, B, n_q, n_kv, d_h, G, W_kv, o, out_fp32, ms, st, 0);
 }
 
 cudaError_t launch_expand_simt(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
-                               const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv,
+                               const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, int bits,
+                               const uint16_t *W_kv,
                                float scale, int S, int64_t tps, int rope_knorm, float rope_base,
                                const uint16_t *gain, float eps, float *part, uint32_t *err, void *o, int out_fp32,
                                void *const *prof, cudaStream_t st) {
@@ -406,8 +410,8 @@ cudaError_t launch_expand_simt(const uint16_t *q, const uint8_t *codes, int64_t 
   if (e != cudaSuccess) return e;
   record_prof_event(prof[0], st);
   expand_split_simt<<<dim3(S, (unsigned)B, n_kv), FSQ_HEAD_DIM, smem, st>>>(
-      q, codes, bstride, T, seq_lens, G, n_q, n_kv, W_kv, scale * kLog2e, tps, rope_knorm, rope_base, gain, eps,
-      part, err);
+      q, codes, bstride, T, seq_lens, G, bits, n_q, n_kv, W_kv, scale * kLog2e, tps, rope_knorm, rope_base, gain,
+      eps, part, err);
   e = cudaGetLastError();
   record_prof_event(prof[1], st);
   if (e != cudaSuccess) return e;

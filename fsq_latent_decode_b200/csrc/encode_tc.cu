@@ -1,7 +1,8 @@
 // Append path on the 5th-generation tensor cores (prefill-sized token counts):
 //   u = x E^T      bf16 operands, fp32 accumulation in TMEM   ([S] eq. 4)
-//   level = #{k : u >= theta_k} - 8, nibbles packed in pairs  ([S] eq. 2;
-//   slide deck frame "A wide product code uses four bits per coordinate").
+//   level = #{k : u >= theta_k} - L/2, b-bit codes packed    ([S] eq. 2;
+//   slide deck frames "A wide product code uses four bits per coordinate" and
+//   "the grid size is an allocation choice": L = 4, 16, 256 at b = 2, 4, 8).
 //
 // One CTA computes a tile of 128 tokens x NC coordinates (NC = 64, 48, 32 or
 // 16, whichever divides G rounded up to 16), so that a prefill chunk spreads
@@ -81,11 +82,11 @@ __device__ __forceinline__ bool wait_ok(uint64_t *b, uint32_t parity, volatile u
   return mbar_wait(b, parity, abort, kWaitNs);
 }
 
-template <int NC>
+template <int NC, int L>
 __global__ void __launch_bounds__(kThreads, 1)
     encode_pack_tc(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap te, int64_t n_tok,
-                   int64_t C, int G, Thresholds th, uint8_t *__restrict__ codes, int64_t ldc, uint32_t *status,
-                   uint32_t stall_ns) {
+                   int64_t C, int G, const __grid_constant__ Thresholds<L> th, uint8_t *__restrict__ codes,
+                   int64_t ldc, uint32_t *status, uint32_t stall_ns) {
   using EC = ECfg<NC>;
   extern __shared__ __align__(1024) uint8_t esm[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(esm) + 1023) & ~uintptr_t(1023));
@@ -180,24 +181,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const int64_t row = m0 + 32 * warp + lane;  // this thread's token: TMEM lane 32 warp + lane
     const uint32_t tl = tm + ((uint32_t)(32 * warp) << 16);
+    constexpr int BITS = bits_of_levels(L);
+    constexpr int WORDS = 16 * BITS / 32;  // 32-bit words of packed codes per 16 coordinates
 #pragma unroll
     for (int j0 = 0; j0 < NC; j0 += 16) {
       uint32_t v[16];
       tmem_ld16(tl + j0, v);
       tmem_ld_wait();
       if (row < n_tok) {
-        uint8_t *dst = codes + row * ldc + (n0 + j0) / 2;
-        uint32_t w[2] = {0u, 0u};
+        uint8_t *dst = codes + row * ldc + (n0 + j0) * BITS / 8;
+        uint32_t w[WORDS];
+#pragma unroll
+        for (int k = 0; k < WORDS; ++k) w[k] = 0u;
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const uint32_t nib = fsq_nibble(__uint_as_float(v[e]), th);
-          w[e / 8] |= nib << (4 * (e % 8));
+          const uint32_t code = fsq_code<L>(__uint_as_float(v[e]), th);
+          w[e * BITS / 32] |= code << ((e * BITS) % 32);
         }
         const int nvalid = min(16, G - (n0 + j0));  // coordinates of this group inside G
-        if (nvalid == 16 && ((reinterpret_cast<uintptr_t>(dst) & 7u) == 0)) {
-          *reinterpret_cast<uint2 *>(dst) = make_uint2(w[0], w[1]);
+        if (nvalid == 16 && ((reinterpret_cast<uintptr_t>(dst) & (4u * WORDS - 1u)) == 0)) {
+          if constexpr (WORDS == 1) *reinterpret_cast<uint32_t *>(dst) = w[0];
+          else if constexpr (WORDS == 2) *reinterpret_cast<uint2 *>(dst) = make_uint2(w[0], w[1]);
+          else *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
         } else {
-          for (int bb = 0; bb < nvalid / 2; ++bb) dst[bb] = (uint8_t)(w[bb / 4] >> (8 * (bb % 4)));
+          // a ragged last group (nvalid a multiple of 8 / BITS) or an unaligned row
+          for (int bb = 0; bb < nvalid * BITS / 8; ++bb) dst[bb] = (uint8_t)(w[bb / 4] >> (8 * (bb % 4)));
         }
       }
     }
@@ -239,9 +247,9 @@ cudaError_t make_bf16_map(CUtensorMap *map, const uint16_t *base, int64_t rows, 
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int NC>
+template <int NC, int L>
 cudaError_t launch_nc(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C, const uint16_t *E, int G,
-                      const Thresholds &th, uint8_t *codes, int64_t ldc, uint32_t *status, uint32_t stall_ns,
+                      const Thresholds<L> &th, uint8_t *codes, int64_t ldc, uint32_t *status, uint32_t stall_ns,
                       cudaStream_t s) {
   using EC = ECfg<NC>;
   CUtensorMap tx, te;
@@ -249,26 +257,37 @@ cudaError_t launch_nc(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C, 
   if (e != cudaSuccess) return e;
   e = make_bf16_map(&te, E, G, C, C, NC);
   if (e != cudaSuccess) return e;
-  e = ensure_smem_limit((const void *)encode_pack_tc<NC>, EC::SMEM);
+  e = ensure_smem_limit((const void *)encode_pack_tc<NC, L>, EC::SMEM);
   if (e != cudaSuccess) return e;
   const int gp = (G + 15) / 16 * 16;
   const dim3 grid((unsigned)(gp / NC), (unsigned)((n_tok + kM - 1) / kM));
-  encode_pack_tc<NC><<<grid, kThreads, EC::SMEM, s>>>(tx, te, n_tok, C, G, th, codes, ldc, status, stall_ns);
+  encode_pack_tc<NC, L><<<grid, kThreads, EC::SMEM, s>>>(tx, te, n_tok, C, G, th, codes, ldc, status, stall_ns);
   return cudaGetLastError();
 }
 
 }  // namespace enc
 
-// Tensor-core append for n_tok tokens; C a multiple of 64, G even <= 256.
+// Tensor-core append for n_tok tokens; C a multiple of 64, G even <= FSQ_MAX_G
+// (a multiple of 4 at L = 4).
+template <int L>
 cudaError_t launch_encode_pack_tc(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C, const uint16_t *E, int G,
-                                  const Thresholds &th, uint8_t *codes, int64_t ldc, uint32_t *status,
+                                  const Thresholds<L> &th, uint8_t *codes, int64_t ldc, uint32_t *status,
                                   uint32_t stall_ns, cudaStream_t s) {
   if (n_tok > (int64_t)65535 * enc::kM || C > 0x7fffffffLL) return cudaErrorInvalidValue;
   const int gp = (G + 15) / 16 * 16;
-  if (gp % 64 == 0) return enc::launch_nc<64>(x, n_tok, ldx, C, E, G, th, codes, ldc, status, stall_ns, s);
-  if (gp % 48 == 0) return enc::launch_nc<48>(x, n_tok, ldx, C, E, G, th, codes, ldc, status, stall_ns, s);
-  if (gp % 32 == 0) return enc::launch_nc<32>(x, n_tok, ldx, C, E, G, th, codes, ldc, status, stall_ns, s);
-  return enc::launch_nc<16>(x, n_tok, ldx, C, E, G, th, codes, ldc, status, stall_ns, s);
+  if (gp % 64 == 0) return enc::launch_nc<64, L>(x, n_tok, ldx, C, E, G, th, codes, ldc, status, stall_ns, s);
+  if (gp % 48 == 0) return enc::launch_nc<48, L>(x, n_tok, ldx, C, E, G, th, codes, ldc, status, stall_ns, s);
+  if (gp % 32 == 0) return enc::launch_nc<32, L>(x, n_tok, ldx, C, E, G, th, codes, ldc, status, stall_ns, s);
+  return enc::launch_nc<16, L>(x, n_tok, ldx, C, E, G, th, codes, ldc, status, stall_ns, s);
 }
+template cudaError_t launch_encode_pack_tc<4>(const uint16_t *, int64_t, int64_t, int64_t, const uint16_t *, int,
+                                              const Thresholds<4> &, uint8_t *, int64_t, uint32_t *, uint32_t,
+                                              cudaStream_t);
+template cudaError_t launch_encode_pack_tc<16>(const uint16_t *, int64_t, int64_t, int64_t, const uint16_t *, int,
+                                               const Thresholds<16> &, uint8_t *, int64_t, uint32_t *, uint32_t,
+                                               cudaStream_t);
+template cudaError_t launch_encode_pack_tc<256>(const uint16_t *, int64_t, int64_t, int64_t, const uint16_t *, int,
+                                                const Thresholds<256> &, uint8_t *, int64_t, uint32_t *, uint32_t,
+                                                cudaStream_t);
 
 }  // namespace fsq

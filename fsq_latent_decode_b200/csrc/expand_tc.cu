@@ -912,7 +912,8 @@ bool expand_tc_supported(int n_q, int n_kv, int G) {
 }
 
 cudaError_t merge_absorbed_launch(const float *part, int S, int64_t B, int n_q, int n_kv, int d_h, int G,
-                                  const uint16_t *W_kv, void *o, int out_fp32, MergeScratch ms, cudaStream_t st);
+                                  const uint16_t *W_kv, void *o, int out_fp32, MergeScratch ms, cudaStream_t st,
+                                  int fold_bytes);
 cudaError_t merge_expand_launch(const float *part, int S, int64_t B, int n_q, int d_h, void *o, int out_fp32,
                                 cudaStream_t st);
 
@@ -933,7 +934,7 @@ cudaError_t launch_expand_tc(const uint16_t *q, const uint8_t *codes, int64_t bs
   else return cudaErrorInvalidValue;
 #undef FSQ_X_LAUNCH
   if (e != cudaSuccess) return e;
-  if (hybrid) return merge_absorbed_launch(part, S, B, n_q, n_kv, d_h, G, W_kv, o, out_fp32, ms, st);
+  if (hybrid) return merge_absorbed_launch(part, S, B, n_q, n_kv, d_h, G, W_kv, o, out_fp32, ms, st, 0);
   return merge_expand_launch(part, S, B, n_q, d_h, o, out_fp32, st);
 }
 

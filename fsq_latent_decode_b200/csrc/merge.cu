@@ -23,6 +23,13 @@
 // 32-coordinate slices of G over all splits, write their slices of abar to a
 // slab in the workspace, and the last to finish (an arrival count, zeroed by
 // the query prologue of the same call) applies W_v.
+//
+// Byte fold: with 256-level codes the split kernel pools each 8-bit code as
+// its two nibbles (coordinates 2i and 2i+1 of G = 2 x the latent width, levels
+// lo - 8 and hi - 8).  The code's level is (lo - 8) + 16 (hi - 8) + 8, and the
+// merged weights sum to one, so abar_i = abar'_2i + 16 abar'_2i+1 + 8: the
+// pair a thread merges is exactly one byte, folded as it is written.  W_v^(j)
+// then has G/2 columns.
 #include <algorithm>
 
 #include "common.cuh"
@@ -220,7 +227,7 @@ __global__ void __launch_bounds__(kMT) merge_absorbed_grouped(const float *__res
                                                               int n_kv, int G, const uint16_t *__restrict__ W_kv,
                                                               void *o, int out_fp32, int ngq,
                                                               float *__restrict__ slab, uint32_t *__restrict__ cnt,
-                                                              MergeSmem L) {
+                                                              MergeSmem L, int fold) {
   constexpr int D = FSQ_HEAD_DIM;
   extern __shared__ __align__(16) unsigned char msm[];
   uint16_t *wv = reinterpret_cast<uint16_t *>(msm);           // [D][WS] bf16
@@ -231,9 +238,10 @@ __global__ void __launch_bounds__(kMT) merge_absorbed_grouped(const float *__res
   const int j = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x;
   const bool direct = ngq == 1;
-  const int GP = g_pad(G);
-  const uint16_t *wsrc = W_kv + (int64_t)(n_kv + j) * D * G;
-  if (direct) stage_wv(wv, wsrc, G);  // W_v is not written by the split kernel
+  const int GW = fold ? G / 2 : G;  // latent width: columns of W_v^(j), entries of abar
+  const int GP = g_pad(GW);
+  const uint16_t *wsrc = W_kv + (int64_t)(n_kv + j) * D * GW;
+  if (direct) stage_wv(wv, wsrc, GW);  // W_v is not written by the split kernel
   // the partials come from the split kernel; no early trigger: whatever
   // follows the call starts once o is complete
   pdl_wait();
@@ -263,12 +271,18 @@ __global__ void __launch_bounds__(kMT) merge_absorbed_grouped(const float *__res
     if (sub == 0 && t < items) {
       const float inv = 1.f / st.l;
       const float2 v = make_float2(st.a.x * inv, st.a.y * inv);
-      if (direct) *reinterpret_cast<float2 *>(abar + h * GP + gi) = v;
-      else *reinterpret_cast<float2 *>(sl + h * GP + gi) = v;
+      if (fold) {
+        const float f = fmaf(16.f, v.y, v.x) + 8.f;  // nibbles lo, hi of byte gi / 2
+        (direct ? abar : sl)[h * GP + gi / 2] = f;
+      } else if (direct) {
+        *reinterpret_cast<float2 *>(abar + h * GP + gi) = v;
+      } else {
+        *reinterpret_cast<float2 *>(sl + h * GP + gi) = v;
+      }
     }
   }
   if (direct) {
-    for (int i = tid; i < GRP * (GP - G); i += kMT) abar[(i / (GP - G)) * GP + G + i % (GP - G)] = 0.f;
+    for (int i = tid; i < GRP * (GP - GW); i += kMT) abar[(i / (GP - GW)) * GP + GW + i % (GP - GW)] = 0.f;
   } else {
     // the last CTA of the (j, b) pair gathers abar and applies W_v
     __threadfence();
@@ -277,23 +291,23 @@ __global__ void __launch_bounds__(kMT) merge_absorbed_grouped(const float *__res
     __syncthreads();
     if (!last) return;
     __threadfence();
-    stage_wv(wv, wsrc, G);
-    for (int i = tid; i < GRP * GP; i += kMT) abar[i] = i % GP < G ? __ldcg(sl + i) : 0.f;
+    stage_wv(wv, wsrc, GW);
+    for (int i = tid; i < GRP * GP; i += kMT) abar[i] = i % GP < GW ? __ldcg(sl + i) : 0.f;
   }
   cp_async_wait_all();
   __syncthreads();
-  apply_wv<GRP>(wv, abar, scr, G, ((int64_t)b * n_q + (int64_t)j * GRP) * D, o, out_fp32);
+  apply_wv<GRP>(wv, abar, scr, GW, ((int64_t)b * n_q + (int64_t)j * GRP) * D, o, out_fp32);
 }
 
 template <int GRP>
 cudaError_t merge_launch(const float *part, int S, int64_t B, int n_q, int n_kv, int G, const uint16_t *W_kv, void *o,
-                         int out_fp32, const MergePlan &mp, float *slab, uint32_t *cnt, cudaStream_t st) {
-  const MergeSmem L = merge_smem(G, GRP);
+                         int out_fp32, const MergePlan &mp, float *slab, uint32_t *cnt, cudaStream_t st, int fold) {
+  const MergeSmem L = merge_smem(fold ? G / 2 : G, GRP);
   auto kern = merge_absorbed_grouped<GRP>;
   cudaError_t e = ensure_smem_limit((const void *)kern, L.bytes);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3((unsigned)mp.ngq, (unsigned)n_kv, (unsigned)B), dim3(kMT), L.bytes, st, part, S, n_q,
-                    n_kv, G, W_kv, o, out_fp32, mp.ngq, slab, cnt, L);
+                    n_kv, G, W_kv, o, out_fp32, mp.ngq, slab, cnt, L, fold);
 }
 
 }  // namespace
@@ -316,18 +330,19 @@ MergePlan merge_plan(int S, int64_t B, int n_q, int n_kv, int G) {
   return mp;
 }
 
+// G: coordinates of the partials (with fold, two nibbles per 8-bit code).
 cudaError_t merge_grouped_launch(const float *part, int S, int64_t B, int n_q, int n_kv, int G,
                                  const uint16_t *W_kv, void *o, int out_fp32, float *slab, uint32_t *cnt,
-                                 cudaStream_t st) {
-  if (B > 65535 || n_kv > 65535 || G > FSQ_MAX_G) return cudaErrorInvalidValue;
+                                 cudaStream_t st, int fold) {
+  if (B > 65535 || n_kv > 65535 || G > 2 * FSQ_MAX_G || (!fold && G > FSQ_MAX_G)) return cudaErrorInvalidValue;
   const MergePlan mp = merge_plan(S, B, n_q, n_kv, G);
   if (mp.ngq > 1 && (!slab || !cnt)) return cudaErrorInvalidValue;
   switch (n_q / n_kv) {
-    case 1: return merge_launch<1>(part, S, B, n_q, n_kv, G, W_kv, o, out_fp32, mp, slab, cnt, st);
-    case 2: return merge_launch<2>(part, S, B, n_q, n_kv, G, W_kv, o, out_fp32, mp, slab, cnt, st);
-    case 4: return merge_launch<4>(part, S, B, n_q, n_kv, G, W_kv, o, out_fp32, mp, slab, cnt, st);
-    case 8: return merge_launch<8>(part, S, B, n_q, n_kv, G, W_kv, o, out_fp32, mp, slab, cnt, st);
-    case 16: return merge_launch<16>(part, S, B, n_q, n_kv, G, W_kv, o, out_fp32, mp, slab, cnt, st);
+    case 1: return merge_launch<1>(part, S, B, n_q, n_kv, G, W_kv, o, out_fp32, mp, slab, cnt, st, fold);
+    case 2: return merge_launch<2>(part, S, B, n_q, n_kv, G, W_kv, o, out_fp32, mp, slab, cnt, st, fold);
+    case 4: return merge_launch<4>(part, S, B, n_q, n_kv, G, W_kv, o, out_fp32, mp, slab, cnt, st, fold);
+    case 8: return merge_launch<8>(part, S, B, n_q, n_kv, G, W_kv, o, out_fp32, mp, slab, cnt, st, fold);
+    case 16: return merge_launch<16>(part, S, B, n_q, n_kv, G, W_kv, o, out_fp32, mp, slab, cnt, st, fold);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -8,7 +8,10 @@ to the CPU oracle.
 Distributions (per token, per layer):
   x     ~ N(0, 1)        residual states [N, C]          (bf16)
   E     ~ N(0, 4/C)      encoder [G, C]                   (bf16)
-  W_kv  ~ N(0, 1/G)      shared decoder [2*n_kv*d_h, G]   (bf16)
+  W_kv  ~ N(0, 1/G)      shared decoder [2*n_kv*d_h, G]   (bf16); at L levels
+                         other than 16 the standard deviation is scaled by
+                         16/L (exact in bf16: a power of two), so that keys
+                         and values keep the magnitude they have at 16 levels
   q     ~ N(0, 1)        queries [B, n_q, d_h]            (bf16)
   u     ~ N(0, 4)        pre-activations [N, G] (fp32): the law of E x under
                          the two lines above, used to make large caches
@@ -34,9 +37,13 @@ class Workload:
     lengths: tuple
     n_new: int = 0          # tokens encoded and appended (prefill / append leg)
     note: str = ""
+    levels: int = 16        # L: 4, 16 or 256 levels per coordinate (2, 4, 8 bits)
 
 
-# The five seeded workloads (Qwen3-shaped single layer, L=16 levels).
+# The five seeded workloads (Qwen3-shaped single layer, L=16 levels), then the
+# level-grid comparison: the same 8B-shaped layer at fixed code budgets of 80
+# and 144 B/token with 4 or 256 levels (2- or 8-bit codes), the budget setting
+# the latent width G = 8 * budget / b.
 WORKLOADS = {
     "tiny_0p6b": Workload("tiny_0p6b", 16, 8, 128, 256, 1024, (1,), (1024,), 1024,
                           "0.6B-shaped, codes from encoding x end to end"),
@@ -48,6 +55,14 @@ WORKLOADS = {
                              "8B-shaped layer, 42 B/token"),
     "long_8b_97x": Workload("long_8b_97x", 32, 8, 128, 84, 4096, (1,), (1 << 20,), 4096,
                             "8B-shaped layer, 1,048,576 cached tokens, chunked prefill of 4096"),
+    "qwen3_8b_l4_80B": Workload("qwen3_8b_l4_80B", 32, 8, 128, 320, 4096, (16,), (32768,), 4096,
+                                "8B-shaped layer, 4 levels (2-bit codes), 80 B/token", 4),
+    "qwen3_8b_l256_80B": Workload("qwen3_8b_l256_80B", 32, 8, 128, 80, 4096, (16,), (32768,), 4096,
+                                  "8B-shaped layer, 256 levels (8-bit codes), 80 B/token", 256),
+    "qwen3_8b_l4_144B": Workload("qwen3_8b_l4_144B", 32, 8, 128, 576, 4096, (16,), (32768,), 4096,
+                                 "8B-shaped layer, 4 levels (2-bit codes), 144 B/token", 4),
+    "qwen3_8b_l256_144B": Workload("qwen3_8b_l256_144B", 32, 8, 128, 144, 4096, (16,), (32768,), 4096,
+                                   "8B-shaped layer, 256 levels (8-bit codes), 144 B/token", 256),
 }
 
 
@@ -72,9 +87,11 @@ def encoder_inputs(n_tok, C, G, gen, device="cpu"):
     return x, E
 
 
-def decoder_inputs(B, n_q, n_kv, d_h, G, gen, device="cpu"):
-    """W_kv [2*n_kv*d_h, G] ~ N(0, 1/G) then q [B, n_q, d_h] ~ N(0,1), bf16."""
+def decoder_inputs(B, n_q, n_kv, d_h, G, gen, device="cpu", levels=16):
+    """W_kv [2*n_kv*d_h, G] ~ N(0, 1/G) (std x 16/L) then q [B, n_q, d_h] ~ N(0,1), bf16."""
     W_kv = normal((2 * n_kv * d_h, G), (1.0 / G) ** 0.5, gen, device=device)
+    if levels != 16:
+        W_kv = W_kv * (16.0 / levels)  # a power of two: exact in bf16
     q = normal((B, n_q, d_h), 1.0, gen, device=device)
     return W_kv, q
 
@@ -85,7 +102,7 @@ def preactivations(n_tok, G, gen, std=2.0, device="cpu"):
 
 
 def random_bytes(shape, gen, device="cpu"):
-    """Uniform bytes (any byte is a valid pair of 4-bit codes)."""
+    """Uniform bytes (any byte is a valid group of 2-, 4- or 8-bit codes)."""
     return torch.randint(0, 256, shape, generator=gen, dtype=torch.uint8, device=device)
 
 

@@ -1,8 +1,9 @@
 /*
  * fsq.h — C ABI of the B200 (sm_100a) library for Transformer-FSQ's decode
- * hot path: appending tokens to a KV cache that holds only nibble-packed
- * 4-bit FSQ latent codes, and single-token grouped-query attention read
- * directly from those codes through the shared decoder W_kv.
+ * hot path: appending tokens to a KV cache that holds only bit-packed FSQ
+ * latent codes (4-bit nibbles at the default 16 levels; 2- and 8-bit codes at
+ * 4 and 256 levels), and single-token grouped-query attention read directly
+ * from those codes through the shared decoder W_kv.
  *
  * Sources (page titles):
  *  [S] "Transformer-FSQ: Discrete Latents for Extreme KV-Cache Compression",
@@ -36,12 +37,18 @@
  *    it must not write q or W_kv.  Ordinary kernels are unaffected.
  *
  * Cache format (FSQ_FORMAT_VERSION 1)
- *  - A token's G levels z_i in {-8..7} are stored as nibbles n_i = z_i + 8.
- *    Byte i of the token's row holds coordinate 2i in its low nibble and
- *    coordinate 2i+1 in its high nibble.  A row is exactly G/2 bytes; no
- *    scale, zero point or norm is stored ([S] Summary; [D] product-code frame).
- *  - A layer's cache is [B, T_max, G/2] bytes; row t of batch b starts at
- *    codes + b*code_batch_stride_bytes + t*G/2.
+ *  - L levels per coordinate (L = 16 by default; 4 and 256 also supported,
+ *    [D] backup frame "the grid size is an allocation choice", Table 8), so
+ *    b = log2(L) bits per coordinate.  A token's G levels z_i in
+ *    {-L/2 .. L/2-1} are stored as codes n_i = z_i + L/2 of b bits.  Byte k
+ *    of the token's row holds coordinates k*(8/b) .. k*(8/b) + 8/b - 1, the
+ *    first in its lowest b bits.  At L = 16: coordinate 2i in the low nibble
+ *    of byte i and coordinate 2i+1 in its high nibble; at L = 256 one byte per
+ *    coordinate; at L = 4 four coordinates per byte.
+ *  - A row is exactly R = G*b/8 bytes; no scale, zero point or norm is stored
+ *    ([S] Summary; [D] product-code frame: ceil(G*b/8) bytes per token).
+ *  - A layer's cache is [B, T_max, R] bytes; row t of batch b starts at
+ *    codes + b*code_batch_stride_bytes + t*R.
  */
 #ifndef FSQ_H_
 #define FSQ_H_
@@ -54,8 +61,8 @@ extern "C" {
 #endif
 
 #define FSQ_FORMAT_VERSION 1
-#define FSQ_LEVELS 16
-#define FSQ_MAX_G 256
+#define FSQ_LEVELS 16   /* default level count (levels field 0) */
+#define FSQ_MAX_G 576   /* widest latent: Table 8's 144 B/token at L = 4 */
 #define FSQ_HEAD_DIM 128
 
 #if defined(__GNUC__)
@@ -77,12 +84,15 @@ typedef enum {
 } fsq_status;
 
 /* eq. (2) of [S]: u~ = h*tanh(u + atanh(delta/h)) - delta, level = round(u~).
- * Requires 0 < delta < h, h - delta <= 7.5 and h + delta <= 8.5 so that every
- * level lies in {-8..7}.  The acceptance default is {7.5, 0.5}; the deck
- * prints h=7.5075 for L=16 ([D] product-code frame). */
+ * levels: L in {4, 16, 256}; 0 selects 16.  Requires 0 < delta < h,
+ * h - delta <= L/2 - 1/2 and h + delta <= L/2 + 1/2 so that every level lies
+ * in {-L/2 .. L/2-1}.  The acceptance default at L = 16 is {7.5, 0.5}; the
+ * deck prints h=7.5075 for L=16 ([D] product-code frame); for the other level
+ * counts h = (L-1)/2, delta = 0.5 is the same choice. */
 typedef struct {
   float h;
   float delta;
+  int levels;
 } fsq_quant_params;
 
 enum {
@@ -93,7 +103,8 @@ enum {
   FSQ_VARIANT_HYBRID = 3    /* rebuild K per tile through W_k (then N_k and RoPE_t
                                when rope_knorm), pool codes with the weights and
                                apply W_v once ([D] kernel frame, steps 1-4);
-                               tensor cores; G in {84, 256}, n_q / n_kv <= 8 */
+                               tensor cores; G in {84, 256}, n_q / n_kv <= 8,
+                               16 levels */
 };
 
 typedef struct {
@@ -123,19 +134,27 @@ typedef struct {
                              output is undefined.  Only that wait uses the
                              limit; the waits that let in-flight copies and
                              tensor-core operations finish keep their own. */
+  int levels;             /* L of the cache's codes: 4, 16 or 256; 0 = 16.  The
+                             tensor-core kernels read 16-level codes; at L = 4
+                             and L = 256 the library runs its CUDA-core forms
+                             (ABSORBED, EXPAND) and AUTO picks among those. */
 } fsq_attn_opts;
 
 /* Fills *opts with {AUTO, 1/sqrt(d_h), auto splits, rope off, 1e6, NULL,
- * 1e-6, bf16 output, no profiling events, no per-row lengths, no stall}. */
+ * 1e-6, bf16 output, no profiling events, no per-row lengths, no stall,
+ * 16 levels}. */
 FSQ_API void fsq_attn_opts_default(fsq_attn_opts *opts);
 
-/* Host-side: the 15 ascending u-space decision thresholds the kernels
- * compare against.  A level is -8 + #{k : u >= theta_k}.  theta_k is the
- * smallest fp32 value not below the exact preimage of the half-integer
- * boundary m + 1/2 (m = -8..6) under eq. (2), so for any fp32 u the count
- * equals the exact rounding of eq. (2) except at an exact tie.  Unreachable
- * boundaries are +/-infinity.  Returns FSQ_ERR_INVALID_ARG for bad params. */
-FSQ_API fsq_status fsq_thresholds(fsq_quant_params qp, float theta_out[15]);
+/* Host-side: the L-1 ascending u-space decision thresholds the kernels
+ * compare against (L = qp.levels; theta_out has room for L-1 floats).  A
+ * level is -L/2 + #{k : u >= theta_k}.  theta_k is the smallest fp32 value not
+ * below the exact preimage of the half-integer boundary m + 1/2
+ * (m = -L/2 .. L/2-2) under eq. (2), so for any fp32 u the count equals the
+ * exact rounding of eq. (2) except at an exact tie.  Unreachable boundaries
+ * are +/-infinity.  Returns FSQ_ERR_INVALID_ARG for bad h or delta and
+ * FSQ_ERR_UNSUPPORTED for a level count other than 4, 16 or 256 (the append
+ * calls return the same for such parameters). */
+FSQ_API fsq_status fsq_thresholds(fsq_quant_params qp, float *theta_out);
 
 /* Options of the append path. */
 typedef struct {
@@ -159,21 +178,23 @@ typedef struct {
  *   u = E x_t (bf16 operands, fp32 accumulation), level = eq. (2), packed.
  *  x      bf16 [n_tok, ldx], row t = x_t (C used entries)      — read
  *  E      bf16 [G, C] encoder                                    — read
- *  codes  uint8 [n_tok, ldc_bytes]; row t gets G/2 bytes          — written
+ *  codes  uint8 [n_tok, ldc_bytes]; row t gets R = G*b/8 bytes    — written
  *  opts   may be NULL (no status word, no stall)
- * To append at position T of a [T_max, G/2] cache pass codes + T*G/2 and
- * ldc_bytes = G/2.  Needs: G even, 2 <= G <= 256; C a positive multiple of
- * 64; ldx >= C and ldx % 8 == 0; x and E 16-byte aligned.  n_tok == 0 is a
- * no-op.  Codes are bit-exact with eq. (2) applied to the fp32 u; the fp32 u
- * itself differs from exact arithmetic by the GEMM's rounding. */
+ * To append at position T of a [T_max, R] cache pass codes + T*R and
+ * ldc_bytes = R.  Needs: G even, 2 <= G <= FSQ_MAX_G, G % 4 == 0 at L = 4;
+ * C a positive multiple of 64; ldx >= C and ldx % 8 == 0; x and E 16-byte
+ * aligned.  n_tok == 0 is a no-op.  Codes are bit-exact with eq. (2) applied
+ * to the fp32 u; the fp32 u itself differs from exact arithmetic by the
+ * GEMM's rounding. */
 FSQ_API fsq_status fsq_encode_pack(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C,
                            const uint16_t *E, int G, fsq_quant_params qp,
                            uint8_t *codes, int64_t ldc_bytes, const fsq_encode_opts *opts,
                            fsq_stream_t stream);
 
 /* Quantiser + packing alone on given fp32 pre-activations u [n_tok, G]
- * (row-major, contiguous).  Same codes as fsq_encode_pack would write for
- * that u.  Used to test eq. (2) in isolation. */
+ * (row-major, contiguous; u 16-byte aligned).  Same codes as fsq_encode_pack
+ * would write for that u, under the same G rules.  Used to test eq. (2) in
+ * isolation. */
 FSQ_API fsq_status fsq_quantize_pack_f32(const float *u, int64_t n_tok, int G, fsq_quant_params qp,
                                  uint8_t *codes, int64_t ldc_bytes, fsq_stream_t stream);
 
@@ -198,9 +219,12 @@ FSQ_API size_t fsq_decode_attn_workspace_size(int64_t B, int64_t T, int n_q, int
  *  o        [B, n_q, d_h], bf16 or fp32 (opts->out_fp32)          — written
  *  workspace  >= fsq_decode_attn_workspace_size(...) bytes, 256-byte aligned,
  *             owned by the caller; contents need no initialisation
- * Needs: d_h == 128, n_q % n_kv == 0, G even, 2 <= G <= 256, T >= 1; codes
- * and code_batch_stride_bytes 16-byte aligned, code_batch_stride_bytes >=
- * T*G/2; q, W_kv, o 16-byte aligned.  B == 0 is a no-op.  opts may be NULL
+ * Needs: d_h == 128, n_q % n_kv == 0, G even, 2 <= G <= FSQ_MAX_G (G % 4 == 0
+ * at L = 4), T >= 1; codes and code_batch_stride_bytes 16-byte aligned,
+ * code_batch_stride_bytes >= T*R (R = G*b/8 bytes per row); q, W_kv, o 16-byte
+ * aligned.  Shapes whose CUDA-core kernels would not fit in shared memory
+ * (large n_q * G, or G above 372 for EXPAND) return FSQ_ERR_UNSUPPORTED.
+ * B == 0 is a no-op.  opts may be NULL
  * (defaults).  The absorbed form on the tensor cores reads each code tile once
  * with an L2 evict-first hint, so the call's code stream does not displace
  * other data from L2 (the weights, the workspace, the caller's tensors). */

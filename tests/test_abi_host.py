@@ -87,9 +87,59 @@ def test_workspace_plan_is_deterministic_and_validates():
     assert F.workspace_size(1, 10, 16, 8, 64, 84, _opts()) == 0          # d_h != 128
     assert F.workspace_size(1, 10, 12, 8, 128, 84, _opts()) == 0         # n_q % n_kv
     assert F.workspace_size(1, 10, 16, 8, 128, 85, _opts()) == 0         # odd G
-    assert F.workspace_size(1, 10, 16, 8, 128, 258, _opts()) == 0        # G > 256
+    assert F.workspace_size(1, 10, 16, 8, 128, 578, _opts()) == 0        # G > FSQ_MAX_G
+    assert F.workspace_size(1, 10, 16, 8, 128, 258, _opts()) > 0         # CUDA-core absorbed form
     assert F.workspace_size(1, 10, 16, 8, 128, 84, _opts(variant="absorbed", rope_knorm=True)) == 0
     assert F.workspace_size(1, 10, 16, 8, 128, 84, _opts(rope_knorm=True)) > 0  # auto -> expand
+
+
+def test_level_count_plans():
+    """4 and 256 levels run the CUDA-core forms; shapes whose shared-memory
+    tiles would not fit are refused before any launch."""
+    def ws(G, L, n_q=32, **kw):
+        return F.workspace_size(2, 4096, n_q, 8, 128, G, _opts(levels=L, **kw))
+    for L, G in ((4, 320), (4, 576), (16, 160), (16, 288), (256, 80), (256, 144)):
+        assert ws(G, L) > 0, (L, G)                    # Table 8 widths at 80 and 144 B/token
+    assert ws(86, 4) == 0                               # 2-bit rows need G % 4 == 0
+    assert ws(84, 8) == 0 and ws(84, 2) == 0            # unsupported level counts
+    assert ws(576, 4, n_q=64) == 0                      # absorbed tile exceeds shared memory
+    assert ws(144, 256, variant="hybrid", rope_knorm=True) == 0  # tensor-core forms read 16 levels
+    assert ws(320, 4, rope_knorm=True) > 0              # AUTO + rope -> CUDA-core expand form
+    assert ws(576, 4, rope_knorm=True) == 0             # W_kv^(j) of G=576 exceeds shared memory
+    # levels 0 selects 16: same plan as 16
+    assert ws(256, 0) == ws(256, 16)
+    # 256-level codes on the tensor-core absorbed kernel read each byte as two
+    # nibbles: the plan of G = 80 at 256 levels is that of G = 160 at 16 levels
+    assert ws(80, 256) == ws(160, 16)
+    assert ws(128, 256) == ws(256, 16)
+    assert ws(144, 256) != ws(288, 16)  # 2 x 144 exceeds the kernel's widths: CUDA-core form
+
+
+@pytest.mark.parametrize("L", [4, 256])
+def test_threshold_table_other_levels_agrees_with_oracle(L):
+    h = (L - 1) / 2
+    th = np.array(F.thresholds(h, 0.5, levels=L), dtype=np.float32)
+    assert len(th) == L - 1 and np.all(np.diff(th) > 0)
+    for k, t in enumerate(th):
+        below = np.nextafter(t, np.float32(-np.inf), dtype=np.float32)
+        lv = O.fsq_quantize(np.array([float(t), float(below)]), h, 0.5, L)
+        assert lv[0] == k + 1 - L // 2 and lv[1] == k - L // 2, (k, t)
+
+
+def test_level_param_checks():
+    for h, d, L in [(1.5, 0.5, 8), (2.1, 0.5, 4), (127.5, 1.5, 256), (1.0, 1.0, 4)]:
+        with pytest.raises(F.FsqError):
+            F.thresholds(h, d, levels=L)
+    qp = F.quant_params(levels=4)
+    assert (qp.h, qp.delta, qp.levels) == (1.5, 0.5, 4)
+    # encode: 2-bit rows need G % 4 == 0; the row must hold G*b/8 bytes
+    assert F.encode_pack_raw(16, 4, 64, 64, 16, 86, qp, 16, 64, None) == F.FSQ_ERR_UNSUPPORTED
+    assert F.encode_pack_raw(16, 4, 64, 64, 16, 88, qp, 16, 21, None) == F.FSQ_ERR_INVALID_ARG
+    assert F.encode_pack_raw(16, 4, 64, 64, 16, 578, F.quant_params(levels=256), 16, 578, None) == \
+        F.FSQ_ERR_UNSUPPORTED
+    assert F.quantize_pack_f32_raw(16, 3, 144, F.quant_params(levels=256), 16, 143, None) == F.FSQ_ERR_INVALID_ARG
+    assert F.encode_pack_raw(16, 4, 64, 64, 16, 88, F.quant_params(1.5, 0.5, 8), 16, 64, None) == \
+        F.FSQ_ERR_UNSUPPORTED
 
 
 def test_invalid_arguments_return_before_launch():
@@ -126,7 +176,7 @@ def test_invalid_arguments_return_before_launch():
     assert call(n_q=12) == F.FSQ_ERR_INVALID_ARG
     assert call(G=85) == F.FSQ_ERR_UNSUPPORTED
     assert call(codes=None) == F.FSQ_ERR_INVALID_ARG
-    assert call(bs=100) == F.FSQ_ERR_INVALID_ARG          # stride < T*G/2
+    assert call(bs=100) == F.FSQ_ERR_INVALID_ARG          # stride < T*G*b/8
     assert call(bs=4104) == F.FSQ_ERR_MISALIGNED          # stride % 16
     assert call(codes=24) == F.FSQ_ERR_MISALIGNED
     assert call(q=18) == F.FSQ_ERR_MISALIGNED

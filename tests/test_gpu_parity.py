@@ -13,7 +13,8 @@ import fsq_latent_decode_b200 as F
 from fsq_latent_decode_b200 import synth
 from oracle import fsq_oracle as O
 
-from cases import TOL, decoder_weights, fp16_key_floor, gemm_error_bound, oracle_cache, padded_len, record, rel_err
+from cases import (TOL, decoder_weights, fp16_key_floor, gemm_error_bound, oracle_cache, padded_len, query_grid_floor,
+                   record, rel_err)
 
 pytestmark = pytest.mark.gpu
 
@@ -51,17 +52,18 @@ def test_quantize_pack_bit_exact(G, h, n_tok):
 
 
 # ---------------------------------------------------------------- encoder + FSQ + pack
-def check_codes(got, x, E, G, label):
+def check_codes(got, x, E, G, label, levels=16):
     """Codes are bit-exact with the oracle's eq. (2) on the exact u, except
     where the exact u lies within the fp32 GEMM's forward-error bound of a
     rounding boundary; those mismatches (always one level apart) are counted
     and recorded, split by whether they also lie within 1e-6 of it."""
     x64, E64 = np.asarray(x, np.float64), np.asarray(E, np.float64)
-    lv_r, u = O.encode(x64, E64)
-    lv_g = O.unpack(got, G)
+    h = O.default_h(levels)  # 7.5 at 16 levels, the library's default
+    lv_r, u = O.encode(x64, E64, h, 0.5, levels)
+    lv_g = O.unpack(got, G, levels)
     bad = lv_g != lv_r
     n_bad = int(bad.sum())
-    d = O.fsq_boundary_distance(u[bad]) if n_bad else np.zeros(0)
+    d = O.fsq_boundary_distance(u[bad], h, 0.5, levels) if n_bad else np.zeros(0)
     if n_bad:
         bound = gemm_error_bound(x64, E64)[bad]
         assert (np.abs(lv_g[bad] - lv_r[bad]) == 1).all()
@@ -228,15 +230,15 @@ def test_workload_append_leg(name):
 
 
 # ---------------------------------------------------------------- softmax edge cases
-def _edge_inputs(case, B, n_q, n_kv, G, T, seed):
+def _edge_inputs(case, B, n_q, n_kv, G, T, seed, levels=16):
     """Inputs that drive the online softmax to its corners (summary eqs. 5-6):
     equal scores, a near one-hot softmax, scores that rise along the cache
     (the running maximum grows on every tile; fast: by more than the lazy
     rescale's 2^8 per pair of tiles, slow: by less, so the weights climb
     toward that ceiling without a rescale) and saturated code rows."""
     d_h = 128
-    codes = oracle_cache(B, T, G, seed=seed)
-    W, q = decoder_weights(n_q, n_kv, G, B, seed=seed + 1)
+    codes = oracle_cache(B, T, G, seed=seed, levels=levels)
+    W, q = decoder_weights(n_q, n_kv, G, B, seed=seed + 1, levels=levels)
     if case == "q_zero":
         q = torch.zeros_like(q)
     elif case == "q_x30":
@@ -252,14 +254,14 @@ def _edge_inputs(case, B, n_q, n_kv, G, T, seed):
             q = (q.float() * 4.0).to(torch.bfloat16)
         wk = W[:d_h].double().numpy()
         for b in range(B):
-            z = O.unpack(codes[b, :T], G).astype(np.float64)
+            z = O.unpack(codes[b, :T], G, levels).astype(np.float64)
             order = np.argsort(z @ (wk.T @ q[b, 0].double().numpy()), kind="stable")
             codes[b, :T] = codes[b, :T][order]
     elif case == "saturated":
         sel = np.random.default_rng(seed).integers(0, 3, size=(B, T))
         rows = codes[:, :T]
-        rows[sel == 1] = 0x00   # every level -8
-        rows[sel == 2] = 0xFF   # every level +7
+        rows[sel == 1] = 0x00   # every level -L/2
+        rows[sel == 2] = 0xFF   # every level L/2 - 1
     elif case == "all_low":
         codes[:, :T] = 0x00
     elif case == "all_high":
@@ -478,4 +480,148 @@ def test_decode_flat_softmax_long_single_split(variant, n_q, G, rope, T):
     ref = O.decode_attn(q.float().numpy(), codes[:, :T], W.float().numpy(), n_kv, G, rope_knorm=rk if rope else None)
     got = _decode(q, codes, W, T, n_kv, G, variant=variant, num_splits=1, out_fp32=True, rope_knorm=rope,
                   rope_base=1.0e6, knorm_gain=_dev(gain) if rope else None, knorm_eps=1e-6).cpu().numpy()
+    assert rel_err(got, ref) <= TOL
+
+
+# ---------------------------------------------------------------- level-count variants (4 and 256 levels)
+# The deck's backup frame on grid size (Table 8) compares 4, 16 and 256 levels
+# at fixed byte budgets; the widths below are the table's at 80 and 144 B/token
+# (G = 8 * budget / b) plus small ragged ones.
+@pytest.mark.parametrize("L,G", [(4, 320), (4, 576), (4, 12), (256, 80), (256, 144), (256, 6)])
+@pytest.mark.parametrize("n_tok", [1, 7, 129, 4099])
+def test_quantize_pack_levels_bit_exact(L, G, n_tok):
+    h = O.default_h(L)
+    gen = synth._gen(synth.workload_seed(111, L, G, n_tok))
+    u = synth.preactivations(n_tok, G, gen)
+    th = np.array(F.thresholds(h, 0.5, levels=L), dtype=np.float32)
+    flat = u.view(-1)
+    planted = np.concatenate([th, np.nextafter(th, np.float32(np.inf)), np.nextafter(th, np.float32(-np.inf))])
+    k = min(flat.numel(), planted.size)
+    flat[:k] = torch.from_numpy(planted[:k])
+    got = F.quantize_pack_f32(_dev(u), h, 0.5, levels=L).cpu().numpy()
+    assert got.shape == (n_tok, G * O.bits_per_coordinate(L) // 8)
+    ref = O.quantize_pack(u.numpy().astype(np.float64), h, 0.5, L)
+    bad = O.unpack(got, G, L) != O.unpack(ref, G, L)
+    if bad.any():
+        d = O.fsq_boundary_distance(u.numpy()[bad].astype(np.float64), h, 0.5, L)
+        assert (d < 1e-6).all(), f"{bad.sum()} mismatches outside the 1e-6 band"
+
+
+@pytest.mark.parametrize("L,G", [(4, 320), (4, 576), (4, 12), (256, 80), (256, 144), (256, 6)])
+@pytest.mark.parametrize("n_tok,C", [(1, 1024), (16, 4096), (17, 2048), (64, 1024), (65, 2048), (4096, 4096)])
+def test_encode_pack_levels_parity(L, G, n_tok, C):
+    gen = synth._gen(synth.workload_seed(121, L, n_tok, C, G))
+    x, E = synth.encoder_inputs(n_tok, C, G, gen)
+    word = torch.zeros(1, dtype=torch.int32, device=DEV)
+    got = F.encode_pack(_dev(x), _dev(E), status_word=word, levels=L).cpu().numpy()
+    assert F.workspace_status(word) == F.FSQ_OK
+    check_codes(got, x.float().numpy(), E.float().numpy(), G, f"L={L} n_tok={n_tok} C={C} G={G}", levels=L)
+
+
+def test_encode_pack_levels_append_into_cache_rows():
+    """Appending at row T of a larger cache writes exactly rows T..T+n-1 (row
+    stride G*b/8), leaving the bytes around them as they were."""
+    for L, G in ((4, 320), (256, 144)):
+        rb = G * O.bits_per_coordinate(L) // 8
+        for n_tok in (3, 40, 300):
+            gen = synth._gen(synth.workload_seed(131, L, n_tok))
+            x, E = synth.encoder_inputs(n_tok, 1024, G, gen)
+            cache = torch.full((n_tok + 9, rb), 0xA5, dtype=torch.uint8, device=DEV)
+            F.encode_pack(_dev(x), _dev(E), out=cache[5:5 + n_tok], levels=L)
+            c = cache.cpu().numpy()
+            assert (c[:5] == 0xA5).all() and (c[5 + n_tok:] == 0xA5).all()
+            check_codes(c[5:5 + n_tok], x.float().numpy(), E.float().numpy(), G, f"append L={L} n={n_tok}", levels=L)
+
+
+LEVEL_SHAPES = [
+    # L, B, n_q, n_kv, G, T
+    (4, 2, 32, 8, 320, 777), (4, 1, 32, 8, 576, 300), (4, 3, 16, 8, 12, 1000), (4, 1, 8, 2, 88, 4099),
+    (256, 2, 32, 8, 80, 777), (256, 1, 32, 8, 144, 1025), (256, 3, 16, 8, 6, 1000), (256, 1, 8, 2, 146, 4099),
+    (256, 2, 16, 8, 128, 4099), (256, 1, 32, 8, 42, 1000), (256, 2, 16, 4, 80, 129),
+    (16, 1, 32, 8, 160, 513), (16, 2, 16, 8, 160, 4099), (16, 1, 32, 8, 288, 300),
+]
+
+
+@pytest.mark.parametrize("variant", ["auto", "absorbed", "expand"])
+@pytest.mark.parametrize("L,B,n_q,n_kv,G,T", LEVEL_SHAPES)
+def test_decode_levels_parity(variant, L, B, n_q, n_kv, G, T):
+    if variant == "expand" and G > 372:
+        pytest.skip("the CUDA-core expand form holds W_kv^(j) in shared memory: G <= 372")
+    codes = oracle_cache(B, T, G, seed=141 + T, levels=L)
+    W, q = decoder_weights(n_q, n_kv, G, B, seed=142 + T, levels=L)
+    ref = O.decode_attn(q.float().numpy(), codes[:, :T], W.float().numpy(), n_kv, G, levels=L)
+    got = _decode(q, codes, W, T, n_kv, G, variant=variant, out_fp32=True, levels=L).cpu().numpy()
+    assert rel_err(got, ref) <= TOL
+
+
+@pytest.mark.parametrize("L,G", [(4, 320), (256, 144), (256, 80)])
+def test_decode_levels_ragged_split_and_rope(L, G):
+    """Per-row lengths, explicit split counts and the key norm + RoPE flag at
+    4 and 256 levels (CUDA-core forms)."""
+    B, n_q, n_kv, T = 4, 32, 8, 3000
+    lengths = [1, 129, 1000, T]
+    codes = oracle_cache(B, T, G, seed=151, levels=L)
+    W, q = decoder_weights(n_q, n_kv, G, B, seed=152, levels=L)
+    lens = torch.tensor(lengths, dtype=torch.int32, device=DEV)
+    ref = O.decode_attn(q.float().numpy(), codes[:, :T], W.float().numpy(), n_kv, G, lengths=lengths, levels=L)
+    for variant in ("absorbed", "expand"):
+        for splits in (0, 1, 23):
+            ws = F.Workspace(DEV)
+            got = F.decode_attn(_dev(q), _dev(codes), _dev(W), T, n_kv, G, workspace=ws,
+                                opts=F.attn_opts(variant=variant, out_fp32=True, seq_lens=lens, num_splits=splits,
+                                                 levels=L))
+            assert F.workspace_status(ws.buf) == F.FSQ_OK
+            assert rel_err(got.cpu().numpy(), ref) <= TOL, (variant, splits)
+    gain, rk = _rope_args(153)
+    ref = O.decode_attn(q.float().numpy(), codes[:, :T], W.float().numpy(), n_kv, G, rope_knorm=rk, levels=L)
+    got = _decode(q, codes, W, T, n_kv, G, rope_knorm=True, rope_base=1.0e6, knorm_gain=_dev(gain), knorm_eps=1e-6,
+                  out_fp32=True, levels=L).cpu().numpy()
+    assert rel_err(got, ref) <= TOL
+
+
+@pytest.mark.parametrize("name", ["qwen3_8b_l4_80B", "qwen3_8b_l256_80B", "qwen3_8b_l256_144B", "qwen3_8b_l4_144B"])
+def test_level_grid_workloads_sampled(name):
+    """The level-grid workloads at their full size (B=16, T=32768) in the
+    benchmark's launch configuration, checked on sampled batch rows and heads."""
+    wl = synth.WORKLOADS[name]
+    B, T, L, G = wl.batches[0], wl.lengths[0], wl.levels, wl.G
+    rows = [0, B - 1]
+    codes = oracle_cache(B, T, G, seed=161, rows=rows, levels=L)
+    W, q = decoder_weights(wl.n_q, wl.n_kv, G, B, seed=162, levels=L)
+    heads = [0, 13, wl.n_q - 1]
+    ref = O.decode_attn(q.float().numpy(), codes[:, :T], W.float().numpy(), wl.n_kv, G, rows=rows, heads=heads,
+                        levels=L)
+    got = _decode(q, codes, W, T, wl.n_kv, G, levels=L).float().cpu().numpy()
+    assert rel_err(got[rows][:, heads], ref[rows][:, heads]) <= TOL
+
+
+@pytest.mark.parametrize("splits", [1, 0])
+@pytest.mark.parametrize("case", EDGE_CASES)
+@pytest.mark.parametrize("L,n_q,G", [(256, 32, 80), (256, 16, 128), (16, 32, 160)])
+def test_decode_levels_softmax_edge_cases(case, L, n_q, G, splits):
+    """The softmax edge cases on the tensor-core path of 256-level codes (each
+    8-bit code read as two nibbles) and of 16 levels at G = 160."""
+    B, n_kv, T = 2, 8, 2048 + 77
+    q, codes, W = _edge_inputs(case, B, n_q, n_kv, G, T, seed=700 + n_q + G, levels=L)
+    ref = O.decode_attn(q.float().numpy(), codes[:, :T], W.float().numpy(), n_kv, G, levels=L)
+    got = _decode(q, codes, W, T, n_kv, G, variant="absorbed", num_splits=splits, out_fp32=True,
+                  levels=L).cpu().numpy()
+    assert np.isfinite(got).all()
+    bound = TOL
+    if case == "q_x30":  # scores span hundreds of log2 units: the query-weight grid sets the floor
+        bound = max(TOL, 1.1 * query_grid_floor(q.float().numpy(), codes[:, :T], W.float().numpy(), n_kv, G, ref, L))
+    assert rel_err(got, ref) <= bound
+
+
+@pytest.mark.parametrize("L,G", [(256, 80), (16, 160)])
+@pytest.mark.parametrize("T", [16384 - 77, 20000 + 77])
+def test_decode_levels_flat_softmax_long_single_split(L, G, T):
+    """A nearly flat softmax over one long split (one accumulation run, or
+    runs folded every 64 tiles) at the new tensor-core widths."""
+    B, n_q, n_kv = 1, 32, 8
+    codes = oracle_cache(B, T, G, seed=801 + G, levels=L)
+    W, q = decoder_weights(n_q, n_kv, G, B, seed=802 + G, levels=L)
+    q = (q.float() * 0.05).to(torch.bfloat16)
+    ref = O.decode_attn(q.float().numpy(), codes[:, :T], W.float().numpy(), n_kv, G, levels=L)
+    got = _decode(q, codes, W, T, n_kv, G, variant="absorbed", num_splits=1, out_fp32=True, levels=L).cpu().numpy()
     assert rel_err(got, ref) <= TOL

@@ -410,3 +410,16 @@ def test_level_variant_attention_matches_sdpa():
             torch.from_numpy(q)[:, :, None, :], torch.from_numpy(K), torch.from_numpy(V),
             enable_gqa=True)[:, :, 0, :].numpy()
         assert np.abs(o - ref).max() <= 1e-12 * max(1.0, np.abs(ref).max())
+
+
+def test_byte_code_equals_its_nibble_pair():
+    """An 8-bit code n (256 levels, level n - 128) read as the nibbles lo = n % 16
+    and hi = n // 16 (each a 16-level code, level nibble - 8) has level
+    (lo - 8) + 16 (hi - 8) + 8: a 256-level row of G coordinates is a 16-level
+    row of 2G nibbles with weights 1 and 16 and a constant offset."""
+    n = np.arange(256)
+    lv = O.unpack(n[:, None].astype(np.uint8), 1, 256)[:, 0]
+    lo = O.unpack(n[:, None].astype(np.uint8), 2, 16)[:, 0]
+    hi = O.unpack(n[:, None].astype(np.uint8), 2, 16)[:, 1]
+    assert np.array_equal(lv, n - 128)
+    assert np.array_equal(lo + 16 * hi + 8, lv)
