@@ -471,6 +471,88 @@ def points(args, torch, F, synth, peaks):
     return rows
 
 
+# Multi-query points: speculative verification of n_new draft tokens per row,
+# and one chunked-prefill chunk attending to a long cache.
+MULTI_POINTS = (("qwen3_8b_32x", 16, 4, 32768), ("qwen3_8b_32x", 16, 8, 32768), ("qwen3_8b_97x", 16, 8, 32768),
+                ("qwen3_8b_32x", 1, 256, 32768))
+
+
+def multi_points(args, torch, F, synth, peaks):
+    """fsq_decode_attn_multi: n_new queries per row, each attending causally to
+    the code cache.  A step appends each row's n_new new tokens (one append
+    call per row: the rows' new tokens are not one strided block) and runs the
+    multi-query attention.  One JSON line per point with the step time, the
+    split kernel's time and its roofline (codes read once; FLOPs of n_new
+    queries per cached token)."""
+    device = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream()
+    sptr = stream.cuda_stream
+    out_rows = []
+    for wl_name, B, n_new, T in MULTI_POINTS:
+        wl = synth.WORKLOADS[wl_name]
+        G, rb = wl.G, F.row_bytes(wl.G, wl.levels)
+        qp = F.quant_params(levels=wl.levels)
+        code_bytes = B * T * rb
+        n_copies = min(8, max(1, math.ceil(2 * L2_BYTES / code_bytes)))
+        st = build_state(torch, F, synth, wl, B, T, 0, device, n_copies)
+        bstride = st["T_max"] * rb
+        gen = torch.Generator(device=device)
+        gen.manual_seed(synth.workload_seed(5, B, n_new, T))
+        q = synth.normal((B, n_new, wl.n_q, wl.d_h), 1.0, gen, device=device)
+        x_new = synth.normal((B * n_new, wl.C), 1.0, gen, device=device)
+        out = torch.empty((B, n_new, wl.n_q, wl.d_h), dtype=torch.bfloat16, device=device)
+        opts = F.attn_opts(levels=wl.levels)
+        wbuf = F.Workspace(device).get(F.multi_workspace_size(B, n_new, T, wl.n_q, wl.n_kv, wl.d_h, G, opts))
+
+        def step(i, prof=None):
+            cache = st["caches"][i % n_copies]
+            for b in range(B):  # row b's n_new new tokens at positions T - n_new .. T - 1
+                rc = F.encode_pack_raw(x_new.data_ptr() + b * n_new * wl.C * 2, n_new, wl.C, wl.C, st["E"].data_ptr(),
+                                       G, qp, cache.data_ptr() + b * bstride + (T - n_new) * rb, rb, sptr)
+                if rc:
+                    raise F.FsqError(rc, "fsq_encode_pack")
+            rc = F.decode_attn_multi_raw(q.data_ptr(), B, n_new, wl.n_q, wl.d_h, cache.data_ptr(), bstride, T, G,
+                                         st["W_kv"].data_ptr(), wl.n_kv,
+                                         F.attn_opts(levels=wl.levels, prof_events=prof), wbuf.data_ptr(),
+                                         wbuf.numel(), out.data_ptr(), sptr)
+            if rc:
+                raise F.FsqError(rc, "fsq_decode_attn_multi")
+
+        for i in range(max(3, args.warmup)):
+            step(i)
+        torch.cuda.synchronize()
+        K = max(5, args.steps)
+        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_.record(stream)
+        for i in range(K):
+            step(i)
+        b_.record(stream)
+        torch.cuda.synchronize()
+        step_ms = a_.elapsed_time(b_) / K
+        evs = RawEvents(K)
+        for i in range(K):
+            step(i, evs.pair(i))
+        torch.cuda.synchronize()
+        kern_ms = sum(evs.elapsed_ms(i) for i in range(K)) / K
+        evs.close()
+        t = kern_ms * 1e-3
+        flops = B * n_new * (T - (n_new - 1) / 2) * 4 * wl.n_q * G  # scores + pooling over each query's prefix
+        t_b = code_bytes / (peaks["hbm_gbs"] * 1e9)
+        t_f = flops / (peaks["bf16_tflops"] * 1e12)
+        row = {"multi_query": wl_name, "what": "speculative verification" if n_new <= 16 else "chunked prefill chunk",
+               "B": B, "n_new": n_new, "T": T, "G": G, "n_q": wl.n_q, "step_us": step_ms * 1e3,
+               "kernel_us": kern_ms * 1e3, "query_context_tok_s": B * n_new * T / (step_ms * 1e-3),
+               "roofline_bound": "tensor" if t_f >= t_b else "hbm", "roofline_frac": max(t_b, t_f) / t,
+               "tflops": flops / t / 1e12, "code_gbs": code_bytes / t / 1e9,
+               "l2": f"{n_copies} rotating caches" if n_copies > 1 else "codes larger than L2",
+               "launches_per_step": B + 3, "peak_source": peaks["source"] + " (burst)"}
+        print(json.dumps(row), flush=True)
+        out_rows.append(row)
+        del st, q, x_new, out, wbuf
+        torch.cuda.empty_cache()
+    return out_rows
+
+
 def _oracle_setup(wl_name, Ts):
     from fsq_latent_decode_b200 import synth
     from oracle import fsq_oracle as O
@@ -615,12 +697,14 @@ def main():
     ap.add_argument("--no-append", action="store_true", help="skip the 4096-token prefill append measurement")
     ap.add_argument("--points", action="store_true",
                     help="time every (workload, batch, length) point of the five configurations, one JSON line each")
+    ap.add_argument("--multi", action="store_true",
+                    help="time the multi-query points (speculative verification, chunked prefill), one line each")
     args = ap.parse_args()
-    if args.points:
+    if args.points or args.multi:
         import torch
         import fsq_latent_decode_b200 as F
         from fsq_latent_decode_b200 import synth
-        points(args, torch, F, synth, load_peaks())
+        (points if args.points else multi_points)(args, torch, F, synth, load_peaks())
         return
     rank, world, local = dist_env()
     wl_name = args.workload

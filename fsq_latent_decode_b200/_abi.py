@@ -30,7 +30,7 @@ VARIANTS = {"auto": VARIANT_AUTO, "absorbed": VARIANT_ABSORBED, "expand": VARIAN
 EXPORTED = ("fsq_attn_opts_default", "fsq_thresholds", "fsq_encode_pack", "fsq_quantize_pack_f32",
             "fsq_decode_attn_workspace_size", "fsq_decode_attn", "fsq_workspace_status",
             "fsq_status_string", "fsq_format_version", "fsq_decode_attn_noalloc",
-            "fsq_decode_attn_noalloc_status")
+            "fsq_decode_attn_noalloc_status", "fsq_decode_attn_multi_workspace_size", "fsq_decode_attn_multi")
 # FSQ_NOALLOC_SCRATCH_BYTES of include/fsq.h (a host test checks the two agree)
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -75,6 +75,11 @@ def _load() -> C.CDLL:
     lib.fsq_decode_attn.argtypes = [vp, i64, i32, i32, vp, i64, i64, i32, vp, i32, C.POINTER(AttnOpts),
                                     vp, C.c_size_t, vp, vp]
     lib.fsq_decode_attn.restype = i32
+    lib.fsq_decode_attn_multi_workspace_size.argtypes = [i64, i32, i64, i32, i32, i32, i32, C.POINTER(AttnOpts)]
+    lib.fsq_decode_attn_multi_workspace_size.restype = C.c_size_t
+    lib.fsq_decode_attn_multi.argtypes = [vp, i64, i32, i32, i32, vp, i64, i64, i32, vp, i32, C.POINTER(AttnOpts),
+                                          vp, C.c_size_t, vp, vp]
+    lib.fsq_decode_attn_multi.restype = i32
     lib.fsq_decode_attn_noalloc.argtypes = [vp, i64, i32, i32, vp, i64, i64, i32, vp, i32, C.POINTER(AttnOpts),
                                             vp, vp]
     lib.fsq_decode_attn_noalloc.restype = i32
@@ -201,6 +206,17 @@ def decode_attn_raw(q_ptr, B, n_q, d_h, codes_ptr, bstride, T, G, wkv_ptr, n_kv,
                                   None if opts is None else C.byref(opts), ws_ptr, ws_bytes, o_ptr, stream_ptr)
 
 
+def multi_workspace_size(B, n_new, T, n_q, n_kv, d_h, G, opts: AttnOpts | None = None) -> int:
+    return int(_lib().fsq_decode_attn_multi_workspace_size(B, n_new, T, n_q, n_kv, d_h, G,
+                                                           None if opts is None else C.byref(opts)))
+
+
+def decode_attn_multi_raw(q_ptr, B, n_new, n_q, d_h, codes_ptr, bstride, T, G, wkv_ptr, n_kv, opts, ws_ptr,
+                          ws_bytes, o_ptr, stream_ptr) -> int:
+    return _lib().fsq_decode_attn_multi(q_ptr, B, n_new, n_q, d_h, codes_ptr, bstride, T, G, wkv_ptr, n_kv,
+                                        None if opts is None else C.byref(opts), ws_ptr, ws_bytes, o_ptr, stream_ptr)
+
+
 def decode_attn_noalloc_raw(q_ptr, B, n_q, d_h, codes_ptr, bstride, T, G, wkv_ptr, n_kv, opts, o_ptr,
                             stream_ptr) -> int:
     return _lib().fsq_decode_attn_noalloc(q_ptr, B, n_q, d_h, codes_ptr, bstride, T, G, wkv_ptr, n_kv,
@@ -286,6 +302,34 @@ def decode_attn(q, codes, W_kv, T, n_kv, G, code_batch_stride=None, opts=None, w
     st = decode_attn_raw(_ptr(q), B, n_q, d_h, _ptr(codes), code_batch_stride, T, G, _ptr(W_kv), n_kv, opts,
                          _ptr(ws), ws.numel(), _ptr(out), _stream_ptr(stream))
     _check(st, "fsq_decode_attn")
+    return out
+
+
+def decode_attn_multi(q, codes, W_kv, T, n_kv, G, code_batch_stride=None, opts=None, workspace=None, out=None,
+                      stream=None):
+    """o[B, n_new, n_q, d_h]: query i of row b (q[b, i]) attends causally to the
+    first L_b - n_new + i + 1 cached tokens of codes[b] (L_b = T or seq_lens[b])."""
+    import torch
+    B, n_new, n_q, d_h = q.shape
+    if opts is None:
+        opts = attn_opts()
+    if code_batch_stride is None:
+        if codes.dim() == 3 and codes.shape[0] > 1:
+            code_batch_stride = codes.stride(0)
+        elif codes.dim() == 3:
+            code_batch_stride = codes.shape[1] * codes.shape[2]
+        else:
+            code_batch_stride = T * row_bytes(G, opts.levels or 16)
+    nbytes = multi_workspace_size(B, n_new, T, n_q, n_kv, d_h, G, opts)
+    if nbytes == 0:
+        raise FsqError(FSQ_ERR_INVALID_ARG, "fsq_decode_attn_multi_workspace_size")
+    ws = (workspace or Workspace(q.device)).get(nbytes)
+    if out is None:
+        out = torch.empty((B, n_new, n_q, d_h), dtype=torch.float32 if opts.out_fp32 else torch.bfloat16,
+                          device=q.device)
+    st = decode_attn_multi_raw(_ptr(q), B, n_new, n_q, d_h, _ptr(codes), code_batch_stride, T, G, _ptr(W_kv), n_kv,
+                               opts, _ptr(ws), ws.numel(), _ptr(out), _stream_ptr(stream))
+    _check(st, "fsq_decode_attn_multi")
     return out
 
 

@@ -13,13 +13,13 @@ cudaError_t launch_encode_pack(const uint16_t *x, int64_t n_tok, int64_t ldx, in
                                uint32_t stall_ns, cudaStream_t s);
 cudaError_t launch_quantize_pack_f32(const float *u, int64_t n_tok, int G, int levels, const float *th,
                                      uint8_t *codes, int64_t ldc, cudaStream_t s);
-cudaError_t launch_absorbed_simt(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
-                                 const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, int bits,
+cudaError_t launch_absorbed_simt(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int n_new,
+                                 int64_t T, const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, int bits,
                                  const uint16_t *W_kv, float scale, int S, int64_t tps, float *qa, float *part,
                                  uint32_t *err, MergeScratch ms, void *o, int out_fp32, void *const *prof,
                                  cudaStream_t st);
-cudaError_t launch_expand_simt(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
-                               const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, int bits,
+cudaError_t launch_expand_simt(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int n_new,
+                               int64_t T, const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, int bits,
                                const uint16_t *W_kv, float scale, int S, int64_t tps, int rope_knorm,
                                float rope_base, const uint16_t *gain, float eps, float *part, uint32_t *err, void *o,
                                int out_fp32, void *const *prof, cudaStream_t st);
@@ -27,8 +27,8 @@ size_t absorbed_simt_smem(int n_q, int G);
 size_t expand_simt_smem(int G);
 bool expand_tc_supported(int n_q, int n_kv, int G);
 size_t expand_tc_stage_bytes(int G, int variant_expand);
-cudaError_t launch_expand_tc(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
-                             const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv,
+cudaError_t launch_expand_tc(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int n_new,
+                             int64_t T, const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv,
                              float scale, int S, int64_t tps, int hybrid, int rope, float rope_base,
                              const uint16_t *gain, float eps, uint8_t *wk, uint8_t *wv, float *ck, float *cv,
                              uint8_t *qs, float *part, uint32_t *err, MergeScratch ms, void *o, int out_fp32,
@@ -37,8 +37,8 @@ int simt_max_nq();
 int simt_max_grp();
 int absorbed_tc_width(int n_q, int n_kv, int G, int levels);
 size_t absorbed_tc_qphys_bytes(int n_q, int G);
-cudaError_t launch_absorbed_tc(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
-                               const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, int levels,
+cudaError_t launch_absorbed_tc(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int n_new,
+                               int64_t T, const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, int levels,
                                const uint16_t *W_kv, float scale, int S, int64_t tps, uint8_t *qphys, float *corr,
                                float *part, uint32_t *err, MergeScratch ms, void *o, int out_fp32,
                                uint32_t stall_ns, void *const *prof, cudaStream_t st);
@@ -46,6 +46,7 @@ cudaError_t launch_absorbed_tc(const uint16_t *q, const uint8_t *codes, int64_t 
 namespace {
 
 constexpr int kMaxSplits = 1024;
+constexpr int64_t kMaxGridRows = 65535;  // grid rows of a call: batch rows x queries per row (grid y)
 constexpr bool kEnableTc = true;  // tensor-core absorbed kernel (being validated)
 
 constexpr size_t kMaxDynSmem = 227 * 1024;  // dynamic shared memory a CTA may request
@@ -259,11 +260,17 @@ fsq_status fsq_quantize_pack_f32(const float *u, int64_t n_tok, int G, fsq_quant
 
 size_t fsq_decode_attn_workspace_size(int64_t B, int64_t T, int n_q, int n_kv, int d_h, int G,
                                       const fsq_attn_opts *opts) {
+  return fsq_decode_attn_multi_workspace_size(B, 1, T, n_q, n_kv, d_h, G, opts);
+}
+
+size_t fsq_decode_attn_multi_workspace_size(int64_t B, int n_new, int64_t T, int n_q, int n_kv, int d_h, int G,
+                                            const fsq_attn_opts *opts) {
   fsq_attn_opts op;
   if (opts) op = *opts;
   else fsq_attn_opts_default(&op);
   Plan p;
-  if (plan_decode(B, T, n_q, n_kv, d_h, G, op, &p) != FSQ_OK) return 0;
+  if (n_new < 1 || B < 0 || B * n_new > kMaxGridRows) return 0;
+  if (plan_decode(B * n_new, T, n_q, n_kv, d_h, G, op, &p) != FSQ_OK) return 0;
   return p.total;
 }
 
@@ -271,11 +278,25 @@ fsq_status fsq_decode_attn(const uint16_t *q, int64_t B, int n_q, int d_h, const
                            int64_t code_batch_stride_bytes, int64_t T, int G, const uint16_t *W_kv, int n_kv,
                            const fsq_attn_opts *opts, void *workspace, size_t workspace_bytes, void *o,
                            fsq_stream_t stream) {
+  return fsq_decode_attn_multi(q, B, 1, n_q, d_h, codes, code_batch_stride_bytes, T, G, W_kv, n_kv, opts, workspace,
+                               workspace_bytes, o, stream);
+}
+
+// The queries of a cache row run as n_new consecutive grid rows of the same
+// kernels (R = B * n_new rows); only the split kernels map a grid row to its
+// cache row and causal length.
+fsq_status fsq_decode_attn_multi(const uint16_t *q, int64_t B, int n_new, int n_q, int d_h, const uint8_t *codes,
+                                 int64_t code_batch_stride_bytes, int64_t T, int G, const uint16_t *W_kv, int n_kv,
+                                 const fsq_attn_opts *opts, void *workspace, size_t workspace_bytes, void *o,
+                                 fsq_stream_t stream) {
   fsq_attn_opts op;
   if (opts) op = *opts;
   else fsq_attn_opts_default(&op);
+  if (n_new < 1 || B < 0) return FSQ_ERR_INVALID_ARG;
+  if (B * n_new > kMaxGridRows) return FSQ_ERR_UNSUPPORTED;
+  const int64_t R = B * n_new;
   Plan p;
-  fsq_status st = plan_decode(B, T, n_q, n_kv, d_h, G, op, &p);
+  fsq_status st = plan_decode(R, T, n_q, n_kv, d_h, G, op, &p);
   if (st != FSQ_OK) return st;
   if (B == 0) return FSQ_OK;
   if (!q || !codes || !W_kv || !o) return FSQ_ERR_INVALID_ARG;
@@ -292,26 +313,26 @@ fsq_status fsq_decode_attn(const uint16_t *q, int64_t B, int n_q, int d_h, const
   float *part = (float *)(ws + p.off_part);
   cudaStream_t s = (cudaStream_t)stream;
   MergeScratch ms{nullptr, nullptr, 0};
-  if (p.mp.cnt_bytes) ms = {(float *)(ws + p.off_mslab), (uint32_t *)(ws + p.off_mcnt), (int)(B * n_kv)};
+  if (p.mp.cnt_bytes) ms = {(float *)(ws + p.off_mslab), (uint32_t *)(ws + p.off_mcnt), (int)(R * n_kv)};
   cudaError_t e;
   if (p.tc && (p.variant == FSQ_VARIANT_EXPAND || p.variant == FSQ_VARIANT_HYBRID)) {
-    e = launch_expand_tc(q, codes, code_batch_stride_bytes, B, T, op.seq_lens, n_q, n_kv, d_h, G, W_kv, scale, p.S,
-                         p.tps, p.variant == FSQ_VARIANT_HYBRID, op.rope_knorm, op.rope_base, op.knorm_gain,
+    e = launch_expand_tc(q, codes, code_batch_stride_bytes, R, n_new, T, op.seq_lens, n_q, n_kv, d_h, G, W_kv, scale,
+                         p.S, p.tps, p.variant == FSQ_VARIANT_HYBRID, op.rope_knorm, op.rope_base, op.knorm_gain,
                          op.knorm_eps, (uint8_t *)(ws + p.off_wk), (uint8_t *)(ws + p.off_wv),
                          (float *)(ws + p.off_ck), (float *)(ws + p.off_cv), (uint8_t *)(ws + p.off_qa), part, err,
                          ms, o, op.out_fp32, op.debug_stall_ns, op.prof_events, s);
   } else if (p.tc) {
-    e = launch_absorbed_tc(q, codes, code_batch_stride_bytes, B, T, op.seq_lens, n_q, n_kv, d_h, G, p.levels, W_kv,
-                           scale, p.S, p.tps, (uint8_t *)(ws + p.off_qa), (float *)(ws + p.off_corr), part, err, ms,
-                           o, op.out_fp32, op.debug_stall_ns, op.prof_events, s);
+    e = launch_absorbed_tc(q, codes, code_batch_stride_bytes, R, n_new, T, op.seq_lens, n_q, n_kv, d_h, G, p.levels,
+                           W_kv, scale, p.S, p.tps, (uint8_t *)(ws + p.off_qa), (float *)(ws + p.off_corr), part, err,
+                           ms, o, op.out_fp32, op.debug_stall_ns, op.prof_events, s);
   } else if (p.variant == FSQ_VARIANT_ABSORBED) {
-    e = launch_absorbed_simt(q, codes, code_batch_stride_bytes, B, T, op.seq_lens, n_q, n_kv, d_h, G, bits, W_kv,
-                             scale, p.S, p.tps, (float *)(ws + p.off_qa), part, err, ms, o, op.out_fp32,
+    e = launch_absorbed_simt(q, codes, code_batch_stride_bytes, R, n_new, T, op.seq_lens, n_q, n_kv, d_h, G, bits,
+                             W_kv, scale, p.S, p.tps, (float *)(ws + p.off_qa), part, err, ms, o, op.out_fp32,
                              op.prof_events, s);
   } else {
-    e = launch_expand_simt(q, codes, code_batch_stride_bytes, B, T, op.seq_lens, n_q, n_kv, d_h, G, bits, W_kv,
-                           scale, p.S, p.tps, op.rope_knorm, op.rope_base, op.knorm_gain, op.knorm_eps, part, err, o,
-                           op.out_fp32, op.prof_events, s);
+    e = launch_expand_simt(q, codes, code_batch_stride_bytes, R, n_new, T, op.seq_lens, n_q, n_kv, d_h, G, bits,
+                           W_kv, scale, p.S, p.tps, op.rope_knorm, op.rope_base, op.knorm_gain, op.knorm_eps, part,
+                           err, o, op.out_fp32, op.prof_events, s);
   }
   return from_cuda(e);
 }

@@ -95,6 +95,22 @@ __device__ __forceinline__ int64_t row_len(const int32_t *seq_lens, int64_t b, i
   return v < 1 ? 1 : T;
 }
 
+// Multi-query calls (chunked prefill, speculative decoding) run the n_new
+// queries of a cache row as consecutive virtual rows r = b * n_new + i of the
+// same kernels.  Query i of cache row b (whose length is L_b, the new tokens
+// included) sits at position L_b - n_new + i and attends causally to the
+// first L_b - n_new + i + 1 cached tokens.  One thread per cache row reports
+// (from its query 0) a row too short for its queries, clamped to length 1.
+__device__ __forceinline__ int64_t query_len(const int32_t *seq_lens, int64_t r, int n_new, int64_t T, uint32_t *err,
+                                             bool report) {
+  const int64_t b = r / n_new;
+  const int i = (int)(r - b * n_new);
+  const int64_t len = row_len(seq_lens, b, T, err, report && i == 0) - (n_new - 1 - i);
+  if (len >= 1) return len;
+  if (report && i == 0) record_error(err, FSQ_ERR_INVALID_ARG);
+  return 1;
+}
+
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Raise a kernel's dynamic shared-memory limit on the current device, once:

@@ -143,6 +143,7 @@ struct Params {
   uint64_t wait_ns;      // limit of every hand-off wait
   const int32_t *seq_lens;  // per-row lengths (ragged batch) or null
   uint32_t stall_ns;     // test-only: > 0 makes the softmax wait on `never` first
+  int n_new;             // queries per cache row: grid row r reads cache row r / n_new (causal)
 };
 
 struct Misc {
@@ -190,9 +191,9 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int split = blockIdx.x, b = blockIdx.y;
   const int64_t t0 = (int64_t)split * p.tps;
-  const int64_t t1 = min(row_len(p.seq_lens, b, p.T, p.err, false), t0 + p.tps);
+  const int64_t t1 = min(query_len(p.seq_lens, b, p.n_new, p.T, p.err, false), t0 + p.tps);
   if (t1 <= t0) {
-    // this split lies wholly past its row's length (ragged batch): an empty
+    // this split lies wholly past its row's length (ragged batch, causal query): an empty
     // partial, which the merge weighs by 2^-inf = 0
     pdl_wait();
     float *out = p.part + (((size_t)b * p.S + split) * NQ) * (2 + G);
@@ -200,7 +201,8 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
     return;
   }
   const int n_tiles = (int)((t1 - t0 + kTile - 1) / kTile);
-  const uint8_t *gcodes = p.codes + (int64_t)b * p.bstride + t0 * C::HALF;
+  const int crow = b / p.n_new;  // cache row
+  const uint8_t *gcodes = p.codes + (int64_t)crow * p.bstride + t0 * C::HALF;
   volatile uint32_t *abort = &ms.abort;
   constexpr uint32_t kPoolIssuers = 2;
 
@@ -253,7 +255,7 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
     // The codes were written before the query prologue kernel started, so the
     // first ring-full of tiles is requested before waiting for that kernel;
     // Q' (its output) right after, before the first wait for a free stage.
-    const uint64_t pol = l2_evict_first();
+    const uint64_t pol = p.n_new > 1 ? l2_evict_normal() : l2_evict_first();
     auto load_q = [&]() {
       if (lane == 0) {
         pdl_wait();
@@ -281,7 +283,7 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
         // rows past T arrive as zeros; rows past this split's end are masked by the softmax
         if (lane == 0) {
           mbar_arrive_expect_tx(&ms.full[st], C::TILE_BYTES);
-          tma_load_3d(dst, &tmap, 0, (int)(t0 + (int64_t)i * kTile), b, &ms.full[st], pol);
+          tma_load_3d(dst, &tmap, 0, (int)(t0 + (int64_t)i * kTile), crow, &ms.full[st], pol);
         }
       } else if (rows == kTile) {
         if (lane == 0) {
@@ -507,7 +509,7 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
       ms.sig[h0 + gtid] = p.corr[(size_t)b * 2 * NQ + h0 + gtid];
       ms.corr[h0 + gtid] = p.corr[(size_t)b * 2 * NQ + NQ + h0 + gtid];
       // a bad per-row length is reported once, after the prologue cleared the error word
-      if (split == 0 && hh == 0 && gtid == 0) row_len(p.seq_lens, b, p.T, p.err, true);
+      if (split == 0 && hh == 0 && gtid == 0) query_len(p.seq_lens, b, p.n_new, p.T, p.err, true);
     }
     named_bar(barid, 128);
     bool ok = true;
@@ -996,7 +998,7 @@ cudaError_t make_code_tensor_map(CUtensorMap *map, const uint8_t *codes, int64_t
 }
 
 template <int G, int NQ, bool BYTE>
-cudaError_t launch(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
+cudaError_t launch(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int n_new, int64_t T,
                    const int32_t *seq_lens, int n_kv, const uint16_t *W_kv, float scale, int S, int64_t tps,
                    uint8_t *qphys, float *corr, float *part, uint32_t *err, MergeScratch ms, uint32_t stall_ns,
                    void *const *prof, cudaStream_t st) {
@@ -1009,11 +1011,11 @@ cudaError_t launch(const uint16_t *q, const uint8_t *codes, int64_t bstride, int
   auto kern = fold ? absorbed_split_tc<G, NQ, true> : absorbed_split_tc<G, NQ, false>;
   e = ensure_smem_limit((const void *)kern, (size_t)smem);
   if (e != cudaSuccess) return e;
-  Params p{codes, bstride, T, tps, S, qphys, corr, part, err, kWaitLimitNs, seq_lens, stall_ns};
+  Params p{codes, bstride, T, tps, S, qphys, corr, part, err, kWaitLimitNs, seq_lens, stall_ns, n_new};
   CUtensorMap tmap;
   memset(&tmap, 0, sizeof(tmap));
   if constexpr (C::TMA) {
-    e = make_code_tensor_map(&tmap, codes, bstride, T, B, C::HALF);
+    e = make_code_tensor_map(&tmap, codes, bstride, T, B / n_new, C::HALF);
     if (e != cudaSuccess) return e;
   }
   record_prof_event(prof[0], st);
@@ -1045,8 +1047,9 @@ cudaError_t merge_absorbed_launch(const float *part, int S, int64_t B, int n_q, 
 
 // G: the latent width of the cache (levels 16 or 256); the partials carry
 // absorbed_tc_width(...) nibble coordinates, folded back by the merge.
-cudaError_t launch_absorbed_tc(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
-                               const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, int levels,
+// B: grid rows (cache rows x n_new queries).
+cudaError_t launch_absorbed_tc(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int n_new,
+                               int64_t T, const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, int levels,
                                const uint16_t *W_kv, float scale, int S, int64_t tps, uint8_t *qphys, float *corr,
                                float *part, uint32_t *err, MergeScratch ms, void *o, int out_fp32,
                                uint32_t stall_ns, void *const *prof, cudaStream_t st) {
@@ -1054,8 +1057,8 @@ cudaError_t launch_absorbed_tc(const uint16_t *q, const uint8_t *codes, int64_t 
   const bool byte = levels == 256;
   cudaError_t e = cudaErrorInvalidValue;
 #define FSQ_TC_LAUNCH(GG, NN, BB)                                                                                  \
-  tc::launch<GG, NN, BB>(q, codes, bstride, B, T, seq_lens, n_kv, W_kv, scale, S, tps, qphys, corr, part, err, ms, \
-                         stall_ns, prof, st)
+  tc::launch<GG, NN, BB>(q, codes, bstride, B, n_new, T, seq_lens, n_kv, W_kv, scale, S, tps, qphys, corr, part, \
+                         err, ms, stall_ns, prof, st)
 #define FSQ_TC_CASE(GG)                                                       \
   if (Gn == GG && n_q == 32) e = byte ? FSQ_TC_LAUNCH(GG, 32, true) : FSQ_TC_LAUNCH(GG, 32, false); \
   else if (Gn == GG && n_q == 16) e = byte ? FSQ_TC_LAUNCH(GG, 16, true) : FSQ_TC_LAUNCH(GG, 16, false);

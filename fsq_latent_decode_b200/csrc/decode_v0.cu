@@ -54,7 +54,7 @@ __global__ void absorb_query_kernel(const uint16_t *__restrict__ q, const uint16
 __global__ void __launch_bounds__(256) absorbed_split_simt(const float *__restrict__ qa,
                                                            const uint8_t *__restrict__ codes, int64_t bstride,
                                                            int64_t T, const int32_t *__restrict__ seq_lens,
-                                                           int G, int bits, int n_q, int64_t tps,
+                                                           int n_new, int G, int bits, int n_q, int64_t tps,
                                                            float *__restrict__ part, uint32_t *err) {
   extern __shared__ float sm[];
   float *qs = sm;                                   // [n_q][G]
@@ -67,11 +67,12 @@ __global__ void __launch_bounds__(256) absorbed_split_simt(const float *__restri
   const int tid = threadIdx.x, nth = blockDim.x;
   const int s = blockIdx.x, b = blockIdx.y, S = gridDim.x;
   const int64_t t0 = (int64_t)s * tps;
-  const int64_t t1 = min(row_len(seq_lens, b, T, err, s == 0 && tid == 0), t0 + tps);  // empty past the row's end
+  // empty past the row's end (ragged batch, causal query); grid row b reads cache row b / n_new
+  const int64_t t1 = min(query_len(seq_lens, b, n_new, T, err, s == 0 && tid == 0), t0 + tps);
   const int per = 8 / bits, rb = G / per;  // coordinates per byte, bytes per row
   const uint32_t mask = (1u << bits) - 1u;
   const float off = (float)(1 << (bits - 1));  // L/2
-  const uint8_t *cb = codes + (int64_t)b * bstride;
+  const uint8_t *cb = codes + (int64_t)(b / n_new) * bstride;
 
   for (int i = tid; i < n_q * G; i += nth) {
     qs[i] = qa[(int64_t)b * n_q * G + i];
@@ -182,8 +183,8 @@ __global__ void merge_absorbed_kernel(const float *__restrict__ part, int S, int
 // part layout: [B][S][n_q][2 + d_h].
 __global__ void __launch_bounds__(128) expand_split_simt(const uint16_t *__restrict__ q,
                                                          const uint8_t *__restrict__ codes, int64_t bstride,
-                                                         int64_t T, const int32_t *__restrict__ seq_lens, int G,
-                                                         int bits, int n_q, int n_kv,
+                                                         int64_t T, const int32_t *__restrict__ seq_lens,
+                                                         int n_new, int G, int bits, int n_q, int n_kv,
                                                          const uint16_t *__restrict__ W_kv,
                                                          float c, int64_t tps, int rope_knorm, float rope_base,
                                                          const uint16_t *__restrict__ gain, float eps,
@@ -201,11 +202,11 @@ __global__ void __launch_bounds__(128) expand_split_simt(const uint16_t *__restr
   const int s = blockIdx.x, b = blockIdx.y, j = blockIdx.z, S = gridDim.x;
   const int grp = n_q / n_kv;
   const int64_t t0 = (int64_t)s * tps;
-  const int64_t t1 = min(row_len(seq_lens, b, T, err, s == 0 && j == 0 && d == 0), t0 + tps);
+  const int64_t t1 = min(query_len(seq_lens, b, n_new, T, err, s == 0 && j == 0 && d == 0), t0 + tps);
   const int per = 8 / bits, rb = G / per;  // coordinates per byte, bytes per row
   const uint32_t mask = (1u << bits) - 1u;
   const float off = (float)(1 << (bits - 1));  // L/2
-  const uint8_t *cb = codes + (int64_t)b * bstride;
+  const uint8_t *cb = codes + (int64_t)(b / n_new) * bstride;
 
   for (int i = d; i < G * D; i += D) {
     int dd = i / G, g = i % G;
@@ -375,8 +376,8 @@ size_t expand_simt_smem(int G) {
 int simt_max_nq() { return kMaxNQ; }
 int simt_max_grp() { return kMaxGrp; }
 
-cudaError_t launch_absorbed_simt(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
-                                 const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, int bits,
+cudaError_t launch_absorbed_simt(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int n_new,
+                                 int64_t T, const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, int bits,
                                  const uint16_t *W_kv,
                                  float scale, int S, int64_t tps, float *qa, float *part, uint32_t *err,
                                  MergeScratch ms, void *o, int out_fp32, void *const *prof, cudaStream_t st) {
@@ -388,16 +389,16 @@ cudaError_t launch_absorbed_simt(const uint16_t *q, const uint8_t *codes, int64_
   e = ensure_smem_limit((const void *)absorbed_split_simt, smem);
   if (e != cudaSuccess) return e;
   record_prof_event(prof[0], st);
-  absorbed_split_simt<<<dim3(S, (unsigned)B), 256, smem, st>>>(qa, codes, bstride, T, seq_lens, G, bits, n_q, tps,
-                                                                part, err);
+  absorbed_split_simt<<<dim3(S, (unsigned)B), 256, smem, st>>>(qa, codes, bstride, T, seq_lens, n_new, G, bits,
+                                                                n_q, tps, part, err);
   e = cudaGetLastError();
   record_prof_event(prof[1], st);
   if (e != cudaSuccess) return e;
   return merge_absorbed_launch(part, S, B, n_q, n_kv, d_h, G, W_kv, o, out_fp32, ms, st, 0);
 }
 
-cudaError_t launch_expand_simt(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
-                               const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, int bits,
+cudaError_t launch_expand_simt(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int n_new,
+                               int64_t T, const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, int bits,
                                const uint16_t *W_kv,
                                float scale, int S, int64_t tps, int rope_knorm, float rope_base,
                                const uint16_t *gain, float eps, float *part, uint32_t *err, void *o, int out_fp32,
@@ -410,8 +411,8 @@ cudaError_t launch_expand_simt(const uint16_t *q, const uint8_t *codes, int64_t 
   if (e != cudaSuccess) return e;
   record_prof_event(prof[0], st);
   expand_split_simt<<<dim3(S, (unsigned)B, n_kv), FSQ_HEAD_DIM, smem, st>>>(
-      q, codes, bstride, T, seq_lens, G, bits, n_q, n_kv, W_kv, scale * kLog2e, tps, rope_knorm, rope_base, gain,
-      eps, part, err);
+      q, codes, bstride, T, seq_lens, n_new, G, bits, n_q, n_kv, W_kv, scale * kLog2e, tps, rope_knorm, rope_base,
+      gain, eps, part, err);
   e = cudaGetLastError();
   record_prof_event(prof[1], st);
   if (e != cudaSuccess) return e;

@@ -145,6 +145,7 @@ struct XParams {
   uint32_t *err;
   const int32_t *seq_lens;
   uint32_t stall_ns;
+  int n_new;                 // queries per cache row: grid row r reads cache row r / n_new (causal)
 };
 
 struct XMisc {
@@ -179,16 +180,17 @@ __global__ void __launch_bounds__(XC<G, VEXP>::THREADS, 1)
   const int GRP = p.grp;
   constexpr int REC = 2 + (VEXP ? 128 : G);  // floats per partial record
   const int64_t t0 = (int64_t)split * p.tps;
-  const int64_t t1 = min(row_len(p.seq_lens, b, p.T, p.err, false), t0 + p.tps);
+  const int64_t t1 = min(query_len(p.seq_lens, b, p.n_new, p.T, p.err, false), t0 + p.tps);
   float *prec = p.part + (((size_t)b * p.S + split) * p.n_q + (size_t)j * GRP) * REC;
   if (t1 <= t0) {
-    // a split wholly past its row's length (ragged batch): empty partials
+    // a split wholly past its row's length (ragged batch, causal query): empty partials
     pdl_wait();
     for (int i = tid; i < GRP * REC; i += C::THREADS) prec[i] = (i % REC) == 0 ? -INFINITY : 0.f;
     return;
   }
   const int n_tiles = (int)((t1 - t0 + kT - 1) / kT);
-  const uint8_t *gcodes = p.codes + (int64_t)b * p.bstride + t0 * C::HALF;
+  const int crow = b / p.n_new;  // cache row
+  const uint8_t *gcodes = p.codes + (int64_t)crow * p.bstride + t0 * C::HALF;
   volatile uint32_t *abort = &ms.abort;
 
   if (tid == 0) {
@@ -251,7 +253,7 @@ __global__ void __launch_bounds__(XC<G, VEXP>::THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     uint8_t *ring = smem + C::SM_CODES;
-    const uint64_t pol = l2_evict_first();
+    const uint64_t pol = p.n_new > 1 ? l2_evict_normal() : l2_evict_first();
     int issued = 0;
     bool ok = true, w_loaded = false;
     auto load_w = [&]() {
@@ -282,7 +284,7 @@ __global__ void __launch_bounds__(XC<G, VEXP>::THREADS, 1)
       if constexpr (C::TMA) {
         if (lane == 0) {
           mbar_arrive_expect_tx(&ms.full[st], C::TILE_BYTES);
-          tma_load_3d(dst, &tmap, 0, (int)(t0 + (int64_t)i * kT), b, &ms.full[st], pol);
+          tma_load_3d(dst, &tmap, 0, (int)(t0 + (int64_t)i * kT), crow, &ms.full[st], pol);
         }
       } else if (rows == kT) {
         if (lane == 0) {
@@ -463,7 +465,7 @@ __global__ void __launch_bounds__(XC<G, VEXP>::THREADS, 1)
     const int gt = tid - 256;                  // 0..255 over the eight token warps
     pdl_wait();                                // the offset terms come from the prologue kernel
     // a bad per-row length is reported once, after the prologue cleared the error word
-    if (split == 0 && j == 0 && gt == 0) row_len(p.seq_lens, b, p.T, p.err, true);
+    if (split == 0 && j == 0 && gt == 0) query_len(p.seq_lens, b, p.n_new, p.T, p.err, true);
     for (int d = gt; d < 128; d += 256) {
       const int dk = (d >> 1) + 64 * (d & 1);  // pair order: column 2i + e is dimension i + 64 e
       ms.ck[d] = p.ck[(size_t)j * 128 + d];
@@ -870,8 +872,8 @@ __global__ void __launch_bounds__(256) expand_prep(const uint16_t *__restrict__ 
 }  // namespace x
 
 template <int G, bool VEXP>
-cudaError_t launch_expand_tc_t(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
-                               const int32_t *seq_lens, int n_q, int n_kv, const uint16_t *W_kv, float scale, int S,
+cudaError_t launch_expand_tc_t(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int n_new,
+                               int64_t T, const int32_t *seq_lens, int n_q, int n_kv, const uint16_t *W_kv, float scale, int S,
                                int64_t tps, int rope, float rope_base, const uint16_t *gain, float eps, uint8_t *wk,
                                uint8_t *wv, float *ck, float *cv, uint8_t *qs, float *part, uint32_t *err,
                                MergeScratch msc, uint32_t stall_ns, void *const *prof, cudaStream_t st) {
@@ -885,11 +887,11 @@ cudaError_t launch_expand_tc_t(const uint16_t *q, const uint8_t *codes, int64_t 
   e = ensure_smem_limit((const void *)x::expand_split_tc<G, VEXP>, (size_t)C::SM_TOTAL);
   if (e != cudaSuccess) return e;
   x::XParams p{codes, bstride, T, tps, S, n_q, n_kv, grp, wk, wv, ck, cv, qs, gain, c / pow2, eps, rope_base, rope,
-               part, err, seq_lens, stall_ns};
+               part, err, seq_lens, stall_ns, n_new};
   CUtensorMap tmap;
   memset(&tmap, 0, sizeof(tmap));
   if constexpr (C::TMA) {
-    e = make_code_tensor_map(&tmap, codes, bstride, T, B, C::HALF);
+    e = make_code_tensor_map(&tmap, codes, bstride, T, B / n_new, C::HALF);
     if (e != cudaSuccess) return e;
   }
   record_prof_event(prof[0], st);
@@ -919,7 +921,8 @@ cudaError_t merge_expand_launch(const float *part, int S, int64_t B, int n_q, in
 
 // Keys rebuilt per tile on the tensor cores; values pooled in latent space
 // (hybrid, W_v applied by the merge) or rebuilt per tile as well (expand).
-cudaError_t launch_expand_tc(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int64_t T,
+// B: grid rows (cache rows x n_new queries).
+cudaError_t launch_expand_tc(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int n_new, int64_t T,
                              const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, const uint16_t *W_kv,
                              float scale, int S, int64_t tps, int hybrid, int rope, float rope_base,
                              const uint16_t *gain, float eps, uint8_t *wk, uint8_t *wv, float *ck, float *cv,
@@ -927,8 +930,8 @@ cudaError_t launch_expand_tc(const uint16_t *q, const uint8_t *codes, int64_t bs
                              uint32_t stall_ns, void *const *prof, cudaStream_t st) {
   cudaError_t e;
 #define FSQ_X_LAUNCH(GG, VV)                                                                                         \
-  tc::launch_expand_tc_t<GG, VV>(q, codes, bstride, B, T, seq_lens, n_q, n_kv, W_kv, scale, S, tps, rope, rope_base, \
-                                 gain, eps, wk, wv, ck, cv, qs, part, err, ms, stall_ns, prof, st)
+  tc::launch_expand_tc_t<GG, VV>(q, codes, bstride, B, n_new, T, seq_lens, n_q, n_kv, W_kv, scale, S, tps, rope,    \
+                                 rope_base, gain, eps, wk, wv, ck, cv, qs, part, err, ms, stall_ns, prof, st)
   if (G == 256) e = hybrid ? FSQ_X_LAUNCH(256, false) : FSQ_X_LAUNCH(256, true);
   else if (G == 84) e = hybrid ? FSQ_X_LAUNCH(84, false) : FSQ_X_LAUNCH(84, true);
   else return cudaErrorInvalidValue;

@@ -74,6 +74,14 @@ __device__ __forceinline__ uint64_t l2_evict_first() {
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
   return pol;
 }
+// With several queries per cache row (virtual rows of one call) the CTAs of
+// the row's queries read the same tiles at about the same time: keep them in
+// L2 at normal priority so that each tile crosses HBM about once.
+__device__ __forceinline__ uint64_t l2_evict_normal() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
 __device__ __forceinline__ void tma_load_3d(void *dst, const CUtensorMap *map, int c0, int c1, int c2, uint64_t *bar,
                                             uint64_t pol) {
   asm volatile(

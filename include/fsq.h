@@ -222,7 +222,7 @@ FSQ_API size_t fsq_decode_attn_workspace_size(int64_t B, int64_t T, int n_q, int
  * Needs: d_h == 128, n_q % n_kv == 0, G even, 2 <= G <= FSQ_MAX_G (G % 4 == 0
  * at L = 4), T >= 1; codes and code_batch_stride_bytes 16-byte aligned,
  * code_batch_stride_bytes >= T*R (R = G*b/8 bytes per row); q, W_kv, o 16-byte
- * aligned.  Shapes whose CUDA-core kernels would not fit in shared memory
+ * aligned; B <= 65535.  Shapes whose CUDA-core kernels would not fit in shared memory
  * (large n_q * G, or G above 372 for EXPAND) return FSQ_ERR_UNSUPPORTED.
  * B == 0 is a no-op.  opts may be NULL
  * (defaults).  The absorbed form on the tensor cores reads each code tile once
@@ -232,6 +232,31 @@ FSQ_API fsq_status fsq_decode_attn(const uint16_t *q, int64_t B, int n_q, int d_
                            const uint8_t *codes, int64_t code_batch_stride_bytes, int64_t T, int G,
                            const uint16_t *W_kv, int n_kv, const fsq_attn_opts *opts,
                            void *workspace, size_t workspace_bytes, void *o, fsq_stream_t stream);
+
+/* Multi-query attention over the code cache: n_new query positions per batch
+ * row, each attending causally to the cache (chunked prefill, where a chunk's
+ * tokens attend to the cache they were just appended to, or speculative
+ * decoding, where draft tokens are verified together).  [S] Methodology
+ * eq. (4)-(5) applied to several queries; the deck's backup frame "capacity and
+ * accuracy are counted by different protocols" counts prefill peak memory,
+ * which a code-only cache keeps small.
+ *   q   bf16 [B, n_new, n_q, d_h]: query i of row b, projected/normed/rotated
+ *   o   [B, n_new, n_q, d_h], bf16 or fp32 (opts->out_fp32)      — written
+ * Row b holds L_b cached tokens (T, or opts->seq_lens[b]) whose last n_new are
+ * the new tokens, already appended; query i sits at position L_b - n_new + i
+ * and attends to tokens 0 .. L_b - n_new + i.  A row shorter than n_new is
+ * clamped (its early queries see one token) and records FSQ_ERR_INVALID_ARG in
+ * the workspace's error word.  Same forms, options, alignment rules and errors
+ * as fsq_decode_attn, which is the case n_new == 1.  Needs n_new >= 1 and
+ * B * n_new <= 65535.  The queries of a row run as consecutive rows of the same
+ * kernels and share each code tile through L2 (read at normal L2 priority).
+ * Workspace: fsq_decode_attn_multi_workspace_size(...). */
+FSQ_API size_t fsq_decode_attn_multi_workspace_size(int64_t B, int n_new, int64_t T, int n_q, int n_kv, int d_h,
+                                                    int G, const fsq_attn_opts *opts);
+FSQ_API fsq_status fsq_decode_attn_multi(const uint16_t *q, int64_t B, int n_new, int n_q, int d_h,
+                                         const uint8_t *codes, int64_t code_batch_stride_bytes, int64_t T, int G,
+                                         const uint16_t *W_kv, int n_kv, const fsq_attn_opts *opts,
+                                         void *workspace, size_t workspace_bytes, void *o, fsq_stream_t stream);
 
 /* Allocation-free decode attention.  There is no counterpart in the paper:
  * this entry point exists for callers that cannot allocate device memory at

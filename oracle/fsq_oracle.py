@@ -274,6 +274,34 @@ def decode_attn(q, codes, W_kv, n_kv, G, scale=None, rope_knorm=None, rows=None,
     return o
 
 
+def decode_attn_multi(q, codes, W_kv, n_kv, G, scale=None, rope_knorm=None, lengths=None, levels=LEVELS,
+                      rows=None, heads=None):
+    """Several new queries per batch row attending to the code cache, causally
+    (chunked prefill or speculative decoding: [S] Methodology eqs. 4-5 for more
+    than one query).
+
+    q: [B, n_new, n_q, d_h].  Row b holds L_b cached tokens (lengths[b], else
+    all T rows of codes), the last n_new of them the new tokens; query i sits
+    at position L_b - n_new + i and attends to tokens 0 .. L_b - n_new + i.
+    Each query is therefore a single-token decode over its own prefix of the
+    cache.  rows / heads optionally restrict the computation (others left NaN).
+    Returns o [B, n_new, n_q, d_h] fp64.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    B, n_new, n_q, d_h = q.shape
+    T = codes.shape[1]
+    o = np.full(q.shape, np.nan)
+    for b in (range(B) if rows is None else rows):
+        L = T if lengths is None else int(lengths[b])
+        if L < n_new:
+            raise ValueError("a row must hold at least its n_new new tokens")
+        for i in range(n_new):
+            n = L - n_new + i + 1
+            o[b, i] = decode_attn(q[b, i][None], codes[b:b + 1, :n], W_kv, n_kv, G, scale=scale,
+                                  rope_knorm=rope_knorm, levels=levels, heads=heads)[0]
+    return o
+
+
 def decode_attn_pooled(q, codes, W_kv, n_kv, G, scale=None):
     """eq. (6) form, for cross-checks only: pool codes with the attention
     weights, then apply W_v once; keys scored as (W_k^T q) . z_t.

@@ -142,6 +142,21 @@ def test_level_param_checks():
         F.FSQ_ERR_UNSUPPORTED
 
 
+def test_multi_query_plans_and_checks():
+    o = _opts()
+    # n_new queries per row plan as B * n_new grid rows
+    assert F.multi_workspace_size(4, 8, 4096, 32, 8, 128, 256, o) == F.workspace_size(32, 4096, 32, 8, 128, 256, o)
+    assert F.multi_workspace_size(4, 1, 4096, 32, 8, 128, 84, o) == F.workspace_size(4, 4096, 32, 8, 128, 84, o)
+    assert F.multi_workspace_size(4, 0, 4096, 32, 8, 128, 84, o) == 0
+    assert F.multi_workspace_size(8192, 8, 4096, 32, 8, 128, 84, o) == 0  # 65536 grid rows
+    args = (16, 4, 0, 32, 128, 16, 4096 * 128, 4096, 256, 16, 8, o, 256, 1 << 30, 16, None)
+    assert F.decode_attn_multi_raw(*args) == F.FSQ_ERR_INVALID_ARG                     # n_new = 0
+    assert F.decode_attn_multi_raw(16, 9000, 8, 32, 128, 16, 4096 * 128, 4096, 256, 16, 8, o, 256, 1 << 30, 16,
+                                   None) == F.FSQ_ERR_UNSUPPORTED                         # B * n_new > 65535
+    assert F.decode_attn_multi_raw(None, 0, 4, 32, 128, None, 4096 * 128, 4096, 256, None, 8, o, None, 0, None,
+                                   None) == F.FSQ_OK                                      # empty batch
+
+
 def test_invalid_arguments_return_before_launch():
     qp = F.quant_params()
     null = None

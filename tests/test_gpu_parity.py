@@ -625,3 +625,95 @@ def test_decode_levels_flat_softmax_long_single_split(L, G, T):
     ref = O.decode_attn(q.float().numpy(), codes[:, :T], W.float().numpy(), n_kv, G, levels=L)
     got = _decode(q, codes, W, T, n_kv, G, variant="absorbed", num_splits=1, out_fp32=True, levels=L).cpu().numpy()
     assert rel_err(got, ref) <= TOL
+
+
+# ---------------------------------------------------------------- multi-query attention (causal)
+def _multi(q, codes, W, T, n_kv, G, ws=None, **kw):
+    return F.decode_attn_multi(_dev(q), _dev(codes), _dev(W), T, n_kv, G, opts=F.attn_opts(**kw), workspace=ws)
+
+
+MULTI_SHAPES = [
+    # variant, L, B, n_new, n_q, n_kv, G, T
+    ("absorbed", 16, 2, 4, 32, 8, 256, 1000), ("absorbed", 16, 1, 8, 16, 8, 84, 2049),
+    ("absorbed", 16, 3, 2, 32, 8, 160, 777), ("absorbed", 256, 2, 3, 32, 8, 80, 513),
+    ("absorbed", 16, 2, 5, 8, 2, 12, 300), ("absorbed", 4, 1, 4, 32, 8, 320, 400),
+    ("hybrid", 16, 2, 4, 32, 8, 256, 1000), ("hybrid", 16, 1, 8, 16, 8, 84, 2049),
+    ("expand", 16, 2, 4, 32, 8, 256, 1000), ("expand", 16, 2, 3, 8, 2, 12, 300),
+    ("absorbed", 16, 1, 64, 32, 8, 256, 700), ("absorbed", 16, 1, 1, 32, 8, 84, 129),
+]
+
+
+@pytest.mark.parametrize("variant,L,B,n_new,n_q,n_kv,G,T", MULTI_SHAPES)
+def test_decode_multi_query_parity(variant, L, B, n_new, n_q, n_kv, G, T):
+    codes = oracle_cache(B, T, G, seed=901 + T, levels=L)
+    W, _ = decoder_weights(n_q, n_kv, G, B, seed=902 + T, levels=L)
+    gen = synth._gen(903 + T)
+    q = synth.normal((B, n_new, n_q, 128), 1.0, gen)
+    ref = O.decode_attn_multi(q.float().numpy(), codes[:, :T], W.float().numpy(), n_kv, G, levels=L)
+    ws = F.Workspace(DEV)
+    got = _multi(q, codes, W, T, n_kv, G, ws, variant=variant, out_fp32=True, levels=L).cpu().numpy()
+    assert F.workspace_status(ws.buf) == F.FSQ_OK
+    assert rel_err(got, ref) <= TOL
+
+
+def test_decode_multi_query_one_query_equals_decode():
+    B, n_q, n_kv, G, T = 2, 32, 8, 256, 1500
+    codes = oracle_cache(B, T, G, seed=911)
+    W, q = decoder_weights(n_q, n_kv, G, B, seed=912)
+    for variant in ("absorbed", "hybrid", "expand"):
+        a = _decode(q, codes, W, T, n_kv, G, variant=variant, out_fp32=True)
+        b = _multi(q[:, None], codes, W, T, n_kv, G, variant=variant, out_fp32=True)[:, 0]
+        assert torch.equal(a, b), variant
+
+
+@pytest.mark.parametrize("variant", ["absorbed", "hybrid", "expand"])
+@pytest.mark.parametrize("splits", [0, 1, 17])
+def test_decode_multi_query_ragged_rope_and_splits(variant, splits):
+    """Per-row lengths with several queries per row (row b's queries sit at its
+    last n_new positions), the key norm + RoPE flag (hybrid, expand) and
+    explicit split counts."""
+    B, n_new, n_q, n_kv, G, T = 3, 4, 32, 8, 84, 2500
+    lengths = [4, 1000, T]
+    rope = variant != "absorbed"
+    codes = oracle_cache(B, T, G, seed=921)
+    W, _ = decoder_weights(n_q, n_kv, G, B, seed=922)
+    q = synth.normal((B, n_new, n_q, 128), 1.0, synth._gen(923))
+    gain, rk = _rope_args(924)
+    lens = torch.tensor(lengths, dtype=torch.int32, device=DEV)
+    ref = O.decode_attn_multi(q.float().numpy(), codes[:, :T], W.float().numpy(), n_kv, G, lengths=lengths,
+                              rope_knorm=rk if rope else None)
+    ws = F.Workspace(DEV)
+    got = _multi(q, codes, W, T, n_kv, G, ws, variant=variant, out_fp32=True, seq_lens=lens, num_splits=splits,
+                 rope_knorm=rope, rope_base=1.0e6, knorm_gain=_dev(gain) if rope else None,
+                 knorm_eps=1e-6).cpu().numpy()
+    assert F.workspace_status(ws.buf) == F.FSQ_OK
+    assert rel_err(got, ref) <= TOL
+
+
+def test_decode_multi_query_short_row_is_clamped_and_reported():
+    B, n_new, n_q, n_kv, G, T = 2, 4, 16, 8, 256, 300
+    codes = oracle_cache(B, T, G, seed=931)
+    W, _ = decoder_weights(n_q, n_kv, G, B, seed=932)
+    q = synth.normal((B, n_new, n_q, 128), 1.0, synth._gen(933))
+    lens = torch.tensor([2, T], dtype=torch.int32, device=DEV)  # row 0 is shorter than its queries
+    ws = F.Workspace(DEV)
+    got = _multi(q, codes, W, T, n_kv, G, ws, out_fp32=True, seq_lens=lens).cpu().numpy()
+    assert F.workspace_status(ws.buf) == F.FSQ_ERR_INVALID_ARG
+    ref = O.decode_attn_multi(q[1:].float().numpy(), codes[1:, :T], W.float().numpy(), n_kv, G)
+    assert rel_err(got[1:], ref) <= TOL  # the well-formed row is unaffected
+    assert np.isfinite(got).all()
+
+
+def test_decode_multi_query_full_size_sampled():
+    """Speculative verification of 4 draft tokens on the 8B-shaped layer at 32x
+    (B=16, T=32768), in the benchmark's launch configuration, on sampled rows
+    and heads."""
+    wl = synth.WORKLOADS["qwen3_8b_32x"]
+    B, n_new, T, G = 16, 4, 32768, wl.G
+    rows, heads = [0, B - 1], [0, 17, wl.n_q - 1]
+    codes = oracle_cache(B, T, G, seed=941, rows=rows)
+    W, _ = decoder_weights(wl.n_q, wl.n_kv, G, B, seed=942)
+    q = synth.normal((B, n_new, wl.n_q, 128), 1.0, synth._gen(943))
+    ref = O.decode_attn_multi(q.float().numpy(), codes[:, :T], W.float().numpy(), wl.n_kv, G, rows=rows, heads=heads)
+    got = _multi(q, codes, W, T, wl.n_kv, G).float().cpu().numpy()
+    assert rel_err(got[rows][:, :, heads], ref[rows][:, :, heads]) <= TOL

@@ -423,3 +423,51 @@ def test_byte_code_equals_its_nibble_pair():
     hi = O.unpack(n[:, None].astype(np.uint8), 2, 16)[:, 1]
     assert np.array_equal(lv, n - 128)
     assert np.array_equal(lo + 16 * hi + 8, lv)
+
+
+# ---------------------------------------------------------------- multi-query (causal) attention
+def _multi_inputs(B=2, n_new=5, n_q=4, n_kv=2, d_h=8, G=6, T=23, seed=0):
+    rng = np.random.default_rng(seed)
+    codes = rng.integers(0, 256, size=(B, T, G // 2), dtype=np.uint8)
+    W = rng.normal(size=(2 * n_kv * d_h, G)) / math.sqrt(G)
+    q = rng.normal(size=(B, n_new, n_q, d_h))
+    return q, codes, W, n_kv, G
+
+
+def test_multi_query_single_query_is_decode():
+    q, codes, W, n_kv, G = _multi_inputs(n_new=1)
+    o = O.decode_attn_multi(q, codes, W, n_kv, G)
+    assert np.array_equal(o[:, 0], O.decode_attn(q[:, 0], codes, W, n_kv, G))
+
+
+def test_multi_query_matches_masked_sdpa():
+    """Against torch SDPA in fp64 on the expanded K, V with an explicit causal
+    mask: query i of a row of T tokens sees tokens t <= T - n_new + i."""
+    q, codes, W, n_kv, G = _multi_inputs()
+    B, n_new, n_q, d_h = q.shape
+    T = codes.shape[1]
+    o = O.decode_attn_multi(q, codes, W, n_kv, G)
+    K = np.stack([O.reconstruct_kv(O.unpack(codes[b], G), W, n_kv, d_h)[0] for b in range(B)])
+    V = np.stack([O.reconstruct_kv(O.unpack(codes[b], G), W, n_kv, d_h)[1] for b in range(B)])
+    mask = torch.tensor([[t <= T - n_new + i for t in range(T)] for i in range(n_new)])
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q).permute(0, 2, 1, 3), torch.from_numpy(K), torch.from_numpy(V), attn_mask=mask,
+        enable_gqa=True).permute(0, 2, 1, 3).numpy()
+    assert np.abs(o - ref).max() <= 1e-12 * np.abs(ref).max()
+
+
+def test_multi_query_is_causal_and_honours_lengths():
+    q, codes, W, n_kv, G = _multi_inputs(B=1, n_new=4, T=30)
+    lengths = [26]
+    o = O.decode_attn_multi(q, codes, W, n_kv, G, lengths=lengths)
+    # query i sits at position 26 - 4 + i: tokens after it (and past the row's length) do not matter
+    c2 = codes.copy()
+    c2[0, 23:] ^= 0x5A  # changes tokens 23.. : seen by queries 1..3 only (positions 23, 24, 25)
+    o2 = O.decode_attn_multi(q, c2, W, n_kv, G, lengths=lengths)
+    assert np.array_equal(o[0, 0], o2[0, 0])
+    assert not np.allclose(o[0, 1:], o2[0, 1:])
+    c3 = codes.copy()
+    c3[0, 26:] ^= 0x5A  # past the row's length: nothing changes
+    assert np.array_equal(O.decode_attn_multi(q, c3, W, n_kv, G, lengths=lengths), o)
+    with pytest.raises(ValueError):
+        O.decode_attn_multi(q, codes, W, n_kv, G, lengths=[3])
