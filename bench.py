@@ -44,12 +44,14 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-# Source files that make up each timed kernel (its digest voids a stored
-# traffic figure once any of them changes).
+# Source files that make up each split kernel (its digest voids a stored
+# traffic figure once any of them changes).  Names as fsq_decode_attn_kernel
+# reports them.
 KERNEL_SOURCES = {
-    "absorbed_split": ("decode_tc.cu", "tc_decode.cuh", "tc_ptx.cuh", "common.cuh"),
-    "hybrid_split": ("expand_tc.cu", "tc_decode.cuh", "tc_ptx.cuh", "common.cuh"),
-    "expand_split": ("expand_tc.cu", "tc_decode.cuh", "tc_ptx.cuh", "common.cuh"),
+    "absorbed_split_tc": ("decode_tc.cu", "tc_decode.cuh", "tc_ptx.cuh", "common.cuh"),
+    "absorbed_split_gen": ("absorbed_gen.cu", "tc_decode.cuh", "tc_ptx.cuh", "common.cuh"),
+    "hybrid_split_tc": ("expand_tc.cu", "tc_decode.cuh", "tc_ptx.cuh", "common.cuh"),
+    "expand_split_tc": ("expand_tc.cu", "tc_decode.cuh", "tc_ptx.cuh", "common.cuh"),
     "absorbed_split_simt": ("decode_v0.cu", "common.cuh"),
     "expand_split_simt": ("decode_v0.cu", "common.cuh"),
 }
@@ -61,19 +63,6 @@ def src_digest(kernel):
     for f in KERNEL_SOURCES[kernel]:
         h.update(open(os.path.join(csrc, f), "rb").read())
     return h.hexdigest()[:16]
-
-
-def split_kernel_name(variant, wl):
-    """Which split kernel the library runs for this workload: its tensor-core
-    kernels read 16-level rows of 84, 160 or 256 nibbles (a 256-level code is
-    read as two nibbles; the key-expanding forms take 16 levels at G = 84 or
-    256 only); every other shape runs a CUDA-core form."""
-    nib = wl.G if wl.levels == 16 else (2 * wl.G if wl.levels == 256 else 0)
-    if variant == "absorbed":
-        return "absorbed_split" if nib in (84, 160, 256) and wl.n_q in (16, 32) else "absorbed_split_simt"
-    if wl.levels == 16 and wl.G in (84, 256):
-        return {"expand": "expand_split", "hybrid": "hybrid_split"}[variant]
-    return "expand_split_simt"
 
 
 def traffic_record(kernel, workload_key):
@@ -482,7 +471,8 @@ def points(args, torch, F, synth, peaks):
                 step_ms = sorted(a.elapsed_time(b) for a, b in ab)[K // 2]
                 kern_ms = sorted(evs.elapsed_ms(i) for i in range(K))[K // 2]
                 evs.close()
-                rf = roofline(dict(wl=wl, B=B, T=T, kern_ms=kern_ms), peaks, split_kernel_name("absorbed", wl))
+                rf = roofline(dict(wl=wl, B=B, T=T, kern_ms=kern_ms), peaks,
+                              F.split_kernel(B, T, wl.n_q, wl.n_kv, wl.d_h, G, F.attn_opts(variant="absorbed")))
                 row = {"point": wl_name, "G": G, "n_q": wl.n_q, "C": wl.C, "B": B, "T": T,
                        "step_us": step_ms * 1e3, "kernel_us": kern_ms * 1e3,
                        "ctx_tok_s": B * T / (step_ms * 1e-3), "code_gbs": rf["code_gbs"],
@@ -769,7 +759,8 @@ def main():
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     peaks = load_peaks()
-    kernel_name = split_kernel_name(args.variant, wl)
+    kernel_name = F.split_kernel(B, T, wl.n_q, wl.n_kv, wl.d_h, wl.G,
+                                 F.attn_opts(variant=args.variant, rope_knorm=args.rope, levels=wl.levels))
     res = run_gpu(args, wl_name, B, T, torch, F, synth, dist, rank, world, device)
     also = None
     if not args.no_second and wl_name == DEFAULT_WORKLOAD[0] and args.B is None and args.T is None:
@@ -812,15 +803,17 @@ def main():
                 "value": value, "unit": "context tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": res["ms"], "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None,
-                "dtype": ({"absorbed_split": "u4 codes; s8 x u8 score MMA (s32), f16 pooling MMA (f32), f32 "
-                                             "softmax/merge, bf16 in/out",
-                           "hybrid_split": "u4 codes; f16 key, score and pooling MMAs (f32), f32 key norm/RoPE/"
-                                           "softmax/merge, bf16 in/out",
-                           "expand_split": "u4 codes; f16 key, value, score and output MMAs (f32), f32 softmax/merge, "
-                                           "bf16 in/out"}.get(kernel_name,
-                                                              f"u{rbytes * 8 // wl.G} codes; f32 CUDA-core scores, "
-                                                              "pooling, softmax and merge, bf16 in/out")
-                          if wl.levels == 16 or kernel_name != "absorbed_split" else
+                "dtype": ({"absorbed_split_tc": "u4 codes; s8 x u8 score MMA (s32), f16 pooling MMA (f32), f32 "
+                                                "softmax/merge, bf16 in/out",
+                           "absorbed_split_gen": f"u{rbytes * 8 // wl.G} codes as f16 levels; f16 score MMA (two-term "
+                                                 "query, f32), f16 pooling MMA (f32), f32 softmax/merge, bf16 in/out",
+                           "hybrid_split_tc": "u4 codes; f16 key, score and pooling MMAs (f32), f32 key norm/RoPE/"
+                                              "softmax/merge, bf16 in/out",
+                           "expand_split_tc": "u4 codes; f16 key, value, score and output MMAs (f32), f32 softmax/"
+                                              "merge, bf16 in/out"}.get(kernel_name,
+                                                                        f"u{rbytes * 8 // wl.G} codes; f32 CUDA-core "
+                                                                        "scores, pooling, softmax and merge, bf16 in/out")
+                          if wl.levels == 16 or kernel_name != "absorbed_split_tc" else
                           "u8 codes read as u4 nibble pairs; s8 x u8 score MMA (s32), f16 pooling MMA (f32), f32 "
                           "softmax/merge, bf16 in/out"),
                 "data": "synthetic (seeded; cache = FSQ codes of u ~ N(0,4), the law of E x; new token x ~ N(0,1) appended each step)",

@@ -11,7 +11,7 @@ from ._abi import (  # noqa: F401
     EXPORTED, FSQ_OK, FSQ_ERR_CUDA, FSQ_ERR_INVALID_ARG, FSQ_ERR_MISALIGNED, FSQ_ERR_TIMEOUT,
     FSQ_ERR_UNSUPPORTED, FSQ_ERR_WORKSPACE, AttnOpts, EncodeOpts, FsqError, QuantParams, Workspace, attn_opts,
     decode_attn, decode_attn_multi, decode_attn_multi_raw, decode_attn_noalloc_status, decode_attn_raw,
-    multi_workspace_size, encode_opts, encode_pack, encode_pack_raw, quant_params,
+    multi_workspace_size, split_kernel, encode_opts, encode_pack, encode_pack_raw, quant_params,
     quantize_pack_f32, quantize_pack_f32_raw, row_bytes, bits_of_levels, status_string, thresholds, workspace_size,
     workspace_status,
 )

@@ -30,7 +30,8 @@ VARIANTS = {"auto": VARIANT_AUTO, "absorbed": VARIANT_ABSORBED, "expand": VARIAN
 EXPORTED = ("fsq_attn_opts_default", "fsq_thresholds", "fsq_encode_pack", "fsq_quantize_pack_f32",
             "fsq_decode_attn_workspace_size", "fsq_decode_attn", "fsq_workspace_status",
             "fsq_status_string", "fsq_format_version", "fsq_decode_attn_noalloc",
-            "fsq_decode_attn_noalloc_status", "fsq_decode_attn_multi_workspace_size", "fsq_decode_attn_multi")
+            "fsq_decode_attn_noalloc_status", "fsq_decode_attn_multi_workspace_size", "fsq_decode_attn_multi",
+            "fsq_decode_attn_kernel")
 # FSQ_NOALLOC_SCRATCH_BYTES of include/fsq.h (a host test checks the two agree)
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
@@ -80,6 +81,8 @@ def _load() -> C.CDLL:
     lib.fsq_decode_attn_multi.argtypes = [vp, i64, i32, i32, i32, vp, i64, i64, i32, vp, i32, C.POINTER(AttnOpts),
                                           vp, C.c_size_t, vp, vp]
     lib.fsq_decode_attn_multi.restype = i32
+    lib.fsq_decode_attn_kernel.argtypes = [i64, i32, i64, i32, i32, i32, i32, C.POINTER(AttnOpts)]
+    lib.fsq_decode_attn_kernel.restype = C.c_char_p
     lib.fsq_decode_attn_noalloc.argtypes = [vp, i64, i32, i32, vp, i64, i64, i32, vp, i32, C.POINTER(AttnOpts),
                                             vp, vp]
     lib.fsq_decode_attn_noalloc.restype = i32
@@ -209,6 +212,12 @@ def decode_attn_raw(q_ptr, B, n_q, d_h, codes_ptr, bstride, T, G, wkv_ptr, n_kv,
 def multi_workspace_size(B, n_new, T, n_q, n_kv, d_h, G, opts: AttnOpts | None = None) -> int:
     return int(_lib().fsq_decode_attn_multi_workspace_size(B, n_new, T, n_q, n_kv, d_h, G,
                                                            None if opts is None else C.byref(opts)))
+
+
+def split_kernel(B, T, n_q, n_kv, d_h, G, opts: AttnOpts | None = None, n_new=1):
+    """Name of the attention (split) kernel a call with these arguments launches, or None."""
+    r = _lib().fsq_decode_attn_kernel(B, n_new, T, n_q, n_kv, d_h, G, None if opts is None else C.byref(opts))
+    return None if r is None else r.decode()
 
 
 def decode_attn_multi_raw(q_ptr, B, n_new, n_q, d_h, codes_ptr, bstride, T, G, wkv_ptr, n_kv, opts, ws_ptr,

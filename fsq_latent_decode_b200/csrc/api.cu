@@ -36,6 +36,14 @@ cudaError_t launch_expand_tc(const uint16_t *q, const uint8_t *codes, int64_t bs
 int simt_max_nq();
 int simt_max_grp();
 int absorbed_tc_width(int n_q, int n_kv, int G, int levels);
+bool absorbed_gen_supported(int n_q, int n_kv, int G, int levels);
+size_t absorbed_gen_qbuf_bytes(int n_q, int G);
+int absorbed_gen_ctas_per_sm(int n_q, int G, int levels);
+cudaError_t launch_absorbed_gen(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t R, int n_new,
+                                int64_t T, const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, int levels,
+                                const uint16_t *W_kv, float scale, int S, int64_t tps, uint8_t *qbuf, float *part,
+                                uint32_t *err, MergeScratch ms, void *o, int out_fp32, uint32_t stall_ns,
+                                void *const *prof, cudaStream_t st);
 size_t absorbed_tc_qphys_bytes(int n_q, int G);
 cudaError_t launch_absorbed_tc(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int n_new,
                                int64_t T, const int32_t *seq_lens, int n_q, int n_kv, int d_h, int G, int levels,
@@ -96,6 +104,7 @@ void make_thresholds(fsq_quant_params qp, float *out) {
 struct Plan {
   int variant;
   int levels;     // L of the codes
+  bool gen;       // generic tensor-core absorbed kernel
   bool tc;        // tensor-core kernel (absorbed, expand or hybrid form)
   int S;          // splits per batch row
   int64_t tps;    // tokens per split
@@ -128,7 +137,9 @@ fsq_status plan_decode(int64_t B, int64_t T, int n_q, int n_kv, int d_h, int G, 
   // the absorbed tensor-core kernel reads rows of Gn nibbles: 16-level codes,
   // or 256-level codes read as two nibbles each (Gn = 2G)
   const int Gn = (kEnableTc && variant == FSQ_VARIANT_ABSORBED) ? absorbed_tc_width(n_q, n_kv, G, L) : 0;
-  const bool tc = Gn > 0 || xtc;
+  // other absorbed shapes: the generic tensor-core kernel (codes unpacked to fp16 in shared memory)
+  const bool gen = !Gn && kEnableTc && variant == FSQ_VARIANT_ABSORBED && absorbed_gen_supported(n_q, n_kv, G, L);
+  const bool tc = Gn > 0 || xtc || gen;
   // the CUDA-core kernels hold a tile of latents (and, in the expand form, W_kv^(j)) in shared memory
   if (!tc && variant == FSQ_VARIANT_ABSORBED && absorbed_simt_smem(n_q, G) > kMaxDynSmem) return FSQ_ERR_UNSUPPORTED;
   if (!tc && variant == FSQ_VARIANT_EXPAND && expand_simt_smem(G) > kMaxDynSmem) return FSQ_ERR_UNSUPPORTED;
@@ -136,8 +147,10 @@ fsq_status plan_decode(int64_t B, int64_t T, int n_q, int n_kv, int d_h, int G, 
   int64_t S = op.num_splits;
   if (S == 0) {
     if (tc) {
-      // one CTA per SM (each holds all of TMEM): fill the 148 SMs in a single wave
-      S = kNumSMs / (Bc * ctas_per_row);
+      // one wave of CTAs: one per SM (each holds all of TMEM), or as many as
+      // an SM holds of the generic kernel
+      const int per_sm = gen ? absorbed_gen_ctas_per_sm(n_q, G, L) : 1;
+      S = (int64_t)kNumSMs * per_sm / (Bc * ctas_per_row);
       if (S < 1) S = 1;
     } else {
       const int64_t target = 2 * kNumSMs;
@@ -155,16 +168,18 @@ fsq_status plan_decode(int64_t B, int64_t T, int n_q, int n_kv, int d_h, int G, 
   p->variant = variant;
   p->levels = L;
   p->tc = tc;
+  p->gen = gen;
   p->S = (int)S;
   p->tps = tps;
   const int acc_len = variant == FSQ_VARIANT_EXPAND ? d_h : (Gn ? Gn : G);  // floats per partial after (m, l)
   size_t off = kWsHeader;
   p->off_qa = off;
   if (xtc) off = align_up(off + (size_t)Bc * n_kv * 16 * d_h * 2, 256);  // staged queries
+  else if (gen) off = align_up(off + absorbed_gen_qbuf_bytes(n_q, G) * (size_t)Bc, 256);
   else if (tc) off = align_up(off + absorbed_tc_qphys_bytes(n_q, Gn) * (size_t)Bc, 256);
   else if (variant == FSQ_VARIANT_ABSORBED) off = align_up(off + sizeof(float) * (size_t)Bc * n_q * G, 256);
   p->off_corr = off;
-  if (tc && !xtc) off = align_up(off + 2 * sizeof(float) * (size_t)Bc * n_q, 256);
+  if (tc && !xtc && !gen) off = align_up(off + 2 * sizeof(float) * (size_t)Bc * n_q, 256);  // per-head scales / offsets
   p->off_wk = p->off_wv = p->off_ck = p->off_cv = off;
   if (xtc) {
     const size_t slice = expand_tc_stage_bytes(G, 0);
@@ -274,6 +289,20 @@ size_t fsq_decode_attn_multi_workspace_size(int64_t B, int n_new, int64_t T, int
   return p.total;
 }
 
+const char *fsq_decode_attn_kernel(int64_t B, int n_new, int64_t T, int n_q, int n_kv, int d_h, int G,
+                                   const fsq_attn_opts *opts) {
+  fsq_attn_opts op;
+  if (opts) op = *opts;
+  else fsq_attn_opts_default(&op);
+  Plan p;
+  if (n_new < 1 || B < 0 || B * n_new > kMaxGridRows) return nullptr;
+  if (plan_decode(B * n_new, T, n_q, n_kv, d_h, G, op, &p) != FSQ_OK) return nullptr;
+  if (p.variant == FSQ_VARIANT_HYBRID) return "hybrid_split_tc";
+  if (p.variant == FSQ_VARIANT_EXPAND) return p.tc ? "expand_split_tc" : "expand_split_simt";
+  if (p.gen) return "absorbed_split_gen";
+  return p.tc ? "absorbed_split_tc" : "absorbed_split_simt";
+}
+
 fsq_status fsq_decode_attn(const uint16_t *q, int64_t B, int n_q, int d_h, const uint8_t *codes,
                            int64_t code_batch_stride_bytes, int64_t T, int G, const uint16_t *W_kv, int n_kv,
                            const fsq_attn_opts *opts, void *workspace, size_t workspace_bytes, void *o,
@@ -321,6 +350,10 @@ fsq_status fsq_decode_attn_multi(const uint16_t *q, int64_t B, int n_new, int n_
                          op.knorm_eps, (uint8_t *)(ws + p.off_wk), (uint8_t *)(ws + p.off_wv),
                          (float *)(ws + p.off_ck), (float *)(ws + p.off_cv), (uint8_t *)(ws + p.off_qa), part, err,
                          ms, o, op.out_fp32, op.debug_stall_ns, op.prof_events, s);
+  } else if (p.gen) {
+    e = launch_absorbed_gen(q, codes, code_batch_stride_bytes, R, n_new, T, op.seq_lens, n_q, n_kv, d_h, G, p.levels,
+                            W_kv, scale, p.S, p.tps, (uint8_t *)(ws + p.off_qa), part, err, ms, o, op.out_fp32,
+                            op.debug_stall_ns, op.prof_events, s);
   } else if (p.tc) {
     e = launch_absorbed_tc(q, codes, code_batch_stride_bytes, R, n_new, T, op.seq_lens, n_q, n_kv, d_h, G, p.levels,
                            W_kv, scale, p.S, p.tps, (uint8_t *)(ws + p.off_qa), (float *)(ws + p.off_corr), part, err,

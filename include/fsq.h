@@ -258,6 +258,17 @@ FSQ_API fsq_status fsq_decode_attn_multi(const uint16_t *q, int64_t B, int n_new
                                          const uint16_t *W_kv, int n_kv, const fsq_attn_opts *opts,
                                          void *workspace, size_t workspace_bytes, void *o, fsq_stream_t stream);
 
+/* Host-side: the name of the attention (split) kernel that
+ * fsq_decode_attn_multi would launch for these arguments — one of
+ * "absorbed_split_tc" (tensor cores, 16-level rows of 84, 160 or 256 nibbles;
+ * 256-level codes read as nibble pairs), "absorbed_split_gen" (tensor cores,
+ * codes unpacked to fp16 levels in shared memory), "hybrid_split_tc",
+ * "expand_split_tc", "absorbed_split_simt", "expand_split_simt" — or NULL when
+ * the arguments are invalid or unsupported.  For logs and benchmarks; the
+ * returned string is static. */
+FSQ_API const char *fsq_decode_attn_kernel(int64_t B, int n_new, int64_t T, int n_q, int n_kv, int d_h, int G,
+                                           const fsq_attn_opts *opts);
+
 /* Allocation-free decode attention.  There is no counterpart in the paper:
  * this entry point exists for callers that cannot allocate device memory at
  * the point where they decode — for example a plugin whose host framework

@@ -717,3 +717,73 @@ def test_decode_multi_query_full_size_sampled():
     ref = O.decode_attn_multi(q.float().numpy(), codes[:, :T], W.float().numpy(), wl.n_kv, G, rows=rows, heads=heads)
     got = _multi(q, codes, W, T, wl.n_kv, G).float().cpu().numpy()
     assert rel_err(got[rows][:, :, heads], ref[rows][:, :, heads]) <= TOL
+
+
+# ---------------------------------------------------------------- generic tensor-core absorbed kernel
+# Widths, level counts and head counts outside the nibble kernel's (codes
+# unpacked to fp16 levels in shared memory; two-term fp16 query weights).
+GEN_SHAPES = [
+    # L, B, n_q, n_kv, G, T
+    (16, 2, 32, 8, 200, 777), (16, 1, 64, 8, 128, 1500), (16, 2, 16, 8, 96, 4099), (16, 1, 64, 16, 288, 300),
+    (256, 2, 32, 8, 144, 1025), (256, 1, 16, 4, 200, 2049), (256, 3, 64, 8, 6, 129),
+    (4, 2, 32, 8, 320, 777), (4, 1, 16, 8, 64, 3000), (4, 1, 64, 8, 160, 513),
+    # Z in two chunks (one does not fit in shared memory next to the rest)
+    (4, 1, 32, 8, 576, 1500), (16, 2, 32, 8, 448, 777), (4, 2, 16, 4, 576, 300),
+]
+
+
+@pytest.mark.parametrize("L,B,n_q,n_kv,G,T", GEN_SHAPES)
+def test_decode_generic_tc_parity(L, B, n_q, n_kv, G, T):
+    codes = oracle_cache(B, T, G, seed=1001 + T, levels=L)
+    W, q = decoder_weights(n_q, n_kv, G, B, seed=1002 + T, levels=L)
+    ref = O.decode_attn(q.float().numpy(), codes[:, :T], W.float().numpy(), n_kv, G, levels=L)
+    for splits in (0, 1, 7):
+        ws = F.Workspace(DEV)
+        got = F.decode_attn(_dev(q), _dev(codes), _dev(W), T, n_kv, G, workspace=ws,
+                            opts=F.attn_opts(variant="absorbed", out_fp32=True, levels=L, num_splits=splits))
+        assert F.workspace_status(ws.buf) == F.FSQ_OK
+        assert rel_err(got.cpu().numpy(), ref) <= TOL, splits
+
+
+@pytest.mark.parametrize("case", EDGE_CASES)
+@pytest.mark.parametrize("L,n_q,G", [(16, 32, 200), (256, 32, 144), (4, 64, 160), (4, 32, 576)])
+def test_decode_generic_tc_softmax_edge_cases(case, L, n_q, G):
+    B, n_kv, T = 2, 8, 2048 + 77
+    q, codes, W = _edge_inputs(case, B, n_q, n_kv, G, T, seed=1100 + n_q + G, levels=L)
+    ref = O.decode_attn(q.float().numpy(), codes[:, :T], W.float().numpy(), n_kv, G, levels=L)
+    got = _decode(q, codes, W, T, n_kv, G, variant="absorbed", num_splits=0, out_fp32=True, levels=L).cpu().numpy()
+    assert np.isfinite(got).all()
+    assert rel_err(got, ref) <= TOL
+
+
+@pytest.mark.parametrize("L,G", [(256, 144), (4, 320), (16, 200), (4, 576)])
+def test_decode_generic_tc_flat_softmax_long_single_split(L, G):
+    """One split of ~20k tokens with a nearly flat softmax: the pooled sums of
+    every token stay within tolerance (signed fp16 levels, so the fp32 sums do
+    not drift one way)."""
+    B, n_q, n_kv, T = 1, 32, 8, 20000 + 77
+    codes = oracle_cache(B, T, G, seed=1201 + G, levels=L)
+    W, q = decoder_weights(n_q, n_kv, G, B, seed=1202 + G, levels=L)
+    q = (q.float() * 0.05).to(torch.bfloat16)
+    ref = O.decode_attn(q.float().numpy(), codes[:, :T], W.float().numpy(), n_kv, G, levels=L)
+    got = _decode(q, codes, W, T, n_kv, G, variant="absorbed", num_splits=1, out_fp32=True, levels=L).cpu().numpy()
+    assert rel_err(got, ref) <= TOL
+
+
+def test_decode_generic_tc_ragged_multi_and_bounded_wait():
+    B, n_new, n_q, n_kv, G, T, L = 3, 3, 32, 8, 320, 2600, 4
+    lengths = [5, 1000, T]
+    codes = oracle_cache(B, T, G, seed=1301, levels=L)
+    W, _ = decoder_weights(n_q, n_kv, G, B, seed=1302, levels=L)
+    q = synth.normal((B, n_new, n_q, 128), 1.0, synth._gen(1303))
+    lens = torch.tensor(lengths, dtype=torch.int32, device=DEV)
+    ref = O.decode_attn_multi(q.float().numpy(), codes[:, :T], W.float().numpy(), n_kv, G, lengths=lengths, levels=L)
+    ws = F.Workspace(DEV)
+    qd, cd, Wd = _dev(q), _dev(codes), _dev(W)
+    F.decode_attn_multi(qd, cd, Wd, T, n_kv, G, workspace=ws,
+                        opts=F.attn_opts(levels=L, seq_lens=lens, debug_stall_ns=2_000_000))
+    assert F.workspace_status(ws.buf) == F.FSQ_ERR_TIMEOUT
+    got = F.decode_attn_multi(qd, cd, Wd, T, n_kv, G, workspace=ws,
+                              opts=F.attn_opts(levels=L, seq_lens=lens, out_fp32=True))
+    assert F.workspace_status(ws.buf) == F.FSQ_OK
+    assert rel_err(got.cpu().numpy(), ref) <= TOL
