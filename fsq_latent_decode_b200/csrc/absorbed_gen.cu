@@ -15,6 +15,9 @@
 //      coordinates that block is a K-major core matrix of the score MMA's A;
 //      read along the tokens it is an MN-major core matrix of the pooling
 //      MMA's A (Z^T), so one copy serves both products with no transpose.
+//      The unpack also writes each token's row of Z to TMEM (lane = token),
+//      the A operand of the score MMA, so that product reads only Q' from
+//      shared memory.
 //   -> S [128 x 2 NQ] = Z . Q'^T on tcgen05 (kind::f16, fp32 in TMEM), Q' the
 //      absorbed query weights as two fp16 terms (hi, lo) per head, stacked
 //      along N: the score is 2^24 (S_hi + S_lo), with about 22 significant bits
@@ -63,16 +66,16 @@ constexpr uint64_t kDrainNs = 1000000000ull;      // 1 s for in-flight copies an
 constexpr size_t kSmemMax = 227 * 1024;
 constexpr int kMiscBytes = 4096;
 
-// Shared-memory plan of one CTA (host and device agree on it).  Z holds the
-// unpacked tile in one piece (nch = 1) or, when that does not fit, in two
-// chunks of whole 128-coordinate blocks (nch = 2): the first nmb0 blocks, then
-// the rest.  The scores accumulate over the chunks; the pooling runs on the
-// resident second chunk, then on the first chunk unpacked again.
+// Shared-memory plan of one CTA (host and device agree on it).  The pooling's
+// copy of Z holds the unpacked tile in one piece (nch = 1) or, when that does
+// not fit, in two chunks of whole 128-coordinate blocks (nch = 2): the first
+// nmb0 blocks, then the rest.  The pooling runs on the resident second chunk,
+// then on the first chunk unpacked again (the scores read Z from TMEM).
 struct Plan {
   int G, Gp, NMB, RB;            // latent width, width padded to 16, 128-coordinate blocks, code bytes per row
   int nq, nch, nmb0;
   size_t off_z, off_q, off_p, off_c, off_misc, total;
-  int tmem_cols;
+  int tmem_cols, off_za;          // TMEM: S [0, 2 nq), ACC [2 nq, 2 nq + NMB nq), Z (score A) from off_za
 };
 __host__ __device__ inline Plan plan_with(int G, int nq, int bits, int nch) {
   Plan p;
@@ -100,7 +103,8 @@ __host__ __device__ inline Plan plan_with(int G, int nq, int bits, int nch) {
   // discarded), which must lie inside the allocation.
   const size_t zread = (size_t)p.nmb0 * 128 * kTile * 2;
   p.total = off > zread ? off : zread;
-  const int cols = 2 * nq + p.NMB * nq;
+  p.off_za = 2 * nq + p.NMB * nq;
+  const int cols = p.off_za + p.Gp / 2;  // Z as fp16 pairs: Gp / 2 columns
   int c = 32;
   while (c < cols) c *= 2;
   p.tmem_cols = c;
@@ -263,7 +267,7 @@ __global__ void __launch_bounds__(NT, Shape<NQ, NT>::MINB) absorbed_split_gen(Pa
 #pragma unroll
   for (int k = 0; k < NH; ++k) lsum[k] = 0.f;
   const uint32_t lane_base = (uint32_t)(32 * q4) << 16;
-  constexpr uint32_t id_s = idesc_f16(128, 2 * NQ, 0, 0);
+  constexpr uint32_t id_s = idesc_f16(128, 2 * NQ, 0, 0);  // A (TMEM) and B K-major
   constexpr uint32_t id_p = idesc_f16(128, NQ, 1, 1);
   const uint32_t z_a = smem_u32(zs), q_a = smem_u32(qs), p_a = smem_u32(ps);
 
@@ -274,7 +278,8 @@ __global__ void __launch_bounds__(NT, Shape<NQ, NT>::MINB) absorbed_split_gen(Pa
   // unpack chunk c of the tile's codes into Z: thread -> token (tid % 128) and
   // every NP-th 8-coordinate block; a warp covers 32 consecutive tokens of one
   // block (512 contiguous bytes of Z)
-  auto unpack = [&](const uint8_t *ct, int c) {
+  auto unpack = [&](const uint8_t *ct, int c, bool to_tmem) {
+    const uint32_t za = tm + ((uint32_t)(32 * (warp & 3)) << 16) + pl.off_za;  // this warp's lanes of Z in TMEM
     constexpr int NP = kThreads / kTile;
     constexpr int U = 4;                       // blocks whose code loads are issued together
     const int t = tid & (kTile - 1);
@@ -308,8 +313,10 @@ __global__ void __launch_bounds__(NT, Shape<NQ, NT>::MINB) absorbed_split_gen(Pa
           uint32_t o[4];
           unpack_word<BITS>(w[u][0], o);
           if constexpr (BITS == 8) unpack_word<8>(w[u][1], o + 2);
-          *reinterpret_cast<uint4 *>(zt + (size_t)(cb - cbA) * (kTile / 8) * 128) =
-              make_uint4(to_level<BITS>(o[0]), to_level<BITS>(o[1]), to_level<BITS>(o[2]), to_level<BITS>(o[3]));
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o[e] = to_level<BITS>(o[e]);
+          *reinterpret_cast<uint4 *>(zt + (size_t)(cb - cbA) * (kTile / 8) * 128) = make_uint4(o[0], o[1], o[2], o[3]);
+          if (to_tmem) tmem_st4(za + 4 * cb, o[0], o[1], o[2], o[3]);  // warp-uniform: cb is the warp's
         }
       }
     }
@@ -321,21 +328,21 @@ __global__ void __launch_bounds__(NT, Shape<NQ, NT>::MINB) absorbed_split_gen(Pa
         const int g = 8 * cb + e;
         v[e] = g < G ? (row[g * BITS / 8] >> ((g * BITS) % 8)) & ((1u << BITS) - 1u) : 0u;
       }
-      *reinterpret_cast<uint4 *>(zt + (size_t)(cb - cbA) * (kTile / 8) * 128) =
-          make_uint4(to_level<BITS>(v[0] | (v[1] << 16)), to_level<BITS>(v[2] | (v[3] << 16)),
-                     to_level<BITS>(v[4] | (v[5] << 16)), to_level<BITS>(v[6] | (v[7] << 16)));
+      const uint32_t o0 = to_level<BITS>(v[0] | (v[1] << 16)), o1 = to_level<BITS>(v[2] | (v[3] << 16));
+      const uint32_t o2 = to_level<BITS>(v[4] | (v[5] << 16)), o3 = to_level<BITS>(v[6] | (v[7] << 16));
+      *reinterpret_cast<uint4 *>(zt + (size_t)(cb - cbA) * (kTile / 8) * 128) = make_uint4(o0, o1, o2, o3);
+      if (to_tmem) tmem_st4(za + 4 * cb, o0, o1, o2, o3);
     }
     fence_proxy_async_smem();
+    if (to_tmem) tmem_st_wait();
   };
-  // S (+)= Z[chunk c] . Q'[chunk c]^T: the K steps of 16 coordinates inside the chunk (thread 0)
-  auto score_mmas = [&](int c) {
+  // S = Z . Q'^T over all Gp coordinates: A from TMEM (8 columns per 16 coordinates), B from shared memory (thread 0)
+  auto score_mmas = [&]() {
     tc_fence_after();
-    const int k0 = 8 * mb_lo(c), k1 = min(8 * mb_hi(c), pl.Gp / 16);
 #pragma unroll 1
-    for (int k = k0; k < k1; ++k) {
-      const uint64_t da = smem_desc(z_a + (uint32_t)((k - k0) * 2 * (kTile / 8) * 128), (kTile / 8) * 128, 128);
+    for (int k = 0; k < pl.Gp / 16; ++k) {
       const uint64_t db = smem_desc(q_a + (uint32_t)(k * 2 * (2 * NQ / 8) * 128), (2 * NQ / 8) * 128, 128);
-      mma_ss(tm, da, db, id_s, k > 0 ? 1u : 0u);
+      mma_ts(tm, tm + pl.off_za + 8 * k, db, id_s, k > 0 ? 1u : 0u);
     }
   };
   // ACC[mb] += Z^T[mb] . P over the tile's 128 tokens for the 128-blocks of chunk c (thread 0)
@@ -373,25 +380,15 @@ __global__ void __launch_bounds__(NT, Shape<NQ, NT>::MINB) absorbed_split_gen(Pa
       for (int k = tid; k < kTile * pl.RB; k += kThreads) dst[k] = k < nb ? src[k] : (uint8_t)0;
       __syncthreads();
     }
-    // ---- scores over the chunks
-    unpack(ct, 0);
+    // ---- unpack (Z to TMEM for the scores and to shared memory for the pooling), then the scores
+    unpack(ct, 0, true);
+    if (nch == 2) unpack(ct, 1, true);  // shared memory keeps the second chunk
+    else issue_copy(i + 2);             // this tile's code buffer has been read
+    tc_fence_before();
     __syncthreads();
     if (tid == 0) {
-      score_mmas(0);
-      tc_commit(nch == 2 ? &ms.s_mid : &ms.s_full);
-    }
-    if (nch == 2) {
-      // the first chunk's score MMAs must be done before Z is overwritten
-      if (!wait_bar(&ms.s_mid, (uint32_t)i & 1u, abort, kWaitNs)) ok = false;
-      if (__syncthreads_or(!ok)) break;
-      unpack(ct, 1);
-      __syncthreads();
-      if (tid == 0) {
-        score_mmas(1);
-        tc_commit(&ms.s_full);
-      }
-    } else {
-      issue_copy(i + 2);  // this tile's code buffer has been read
+      score_mmas();
+      tc_commit(&ms.s_full);
     }
     if (!wait_bar(&ms.s_full, (uint32_t)i & 1u, abort, kWaitNs)) ok = false;
     tc_fence_after();
@@ -498,7 +495,7 @@ __global__ void __launch_bounds__(NT, Shape<NQ, NT>::MINB) absorbed_split_gen(Pa
       }
       if (!wait_bar(&ms.p_mid, (uint32_t)i & 1u, abort, kWaitNs)) ok = false;
       if (__syncthreads_or(!ok)) break;
-      unpack(ct, 0);
+      unpack(ct, 0, false);
       __syncthreads();
       issue_copy(i + 2);  // this tile's code buffer has been read
       if (tid == 0) {
