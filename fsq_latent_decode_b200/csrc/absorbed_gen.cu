@@ -278,7 +278,7 @@ __global__ void __launch_bounds__(NT, Shape<NQ, NT>::MINB) absorbed_split_gen(Pa
   // unpack chunk c of the tile's codes into Z: thread -> token (tid % 128) and
   // every NP-th 8-coordinate block; a warp covers 32 consecutive tokens of one
   // block (512 contiguous bytes of Z)
-  auto unpack = [&](const uint8_t *ct, int c, bool to_tmem) {
+  auto unpack = [&](const uint8_t *ct, int c, bool to_tmem, bool to_smem) {
     const uint32_t za = tm + ((uint32_t)(32 * (warp & 3)) << 16) + pl.off_za;  // this warp's lanes of Z in TMEM
     constexpr int NP = kThreads / kTile;
     constexpr int U = 4;                       // blocks whose code loads are issued together
@@ -315,7 +315,8 @@ __global__ void __launch_bounds__(NT, Shape<NQ, NT>::MINB) absorbed_split_gen(Pa
           if constexpr (BITS == 8) unpack_word<8>(w[u][1], o + 2);
 #pragma unroll
           for (int e = 0; e < 4; ++e) o[e] = to_level<BITS>(o[e]);
-          *reinterpret_cast<uint4 *>(zt + (size_t)(cb - cbA) * (kTile / 8) * 128) = make_uint4(o[0], o[1], o[2], o[3]);
+          if (to_smem)
+            *reinterpret_cast<uint4 *>(zt + (size_t)(cb - cbA) * (kTile / 8) * 128) = make_uint4(o[0], o[1], o[2], o[3]);
           if (to_tmem) tmem_st4(za + 4 * cb, o[0], o[1], o[2], o[3]);  // warp-uniform: cb is the warp's
         }
       }
@@ -330,10 +331,10 @@ __global__ void __launch_bounds__(NT, Shape<NQ, NT>::MINB) absorbed_split_gen(Pa
       }
       const uint32_t o0 = to_level<BITS>(v[0] | (v[1] << 16)), o1 = to_level<BITS>(v[2] | (v[3] << 16));
       const uint32_t o2 = to_level<BITS>(v[4] | (v[5] << 16)), o3 = to_level<BITS>(v[6] | (v[7] << 16));
-      *reinterpret_cast<uint4 *>(zt + (size_t)(cb - cbA) * (kTile / 8) * 128) = make_uint4(o0, o1, o2, o3);
+      if (to_smem) *reinterpret_cast<uint4 *>(zt + (size_t)(cb - cbA) * (kTile / 8) * 128) = make_uint4(o0, o1, o2, o3);
       if (to_tmem) tmem_st4(za + 4 * cb, o0, o1, o2, o3);
     }
-    fence_proxy_async_smem();
+    if (to_smem) fence_proxy_async_smem();
     if (to_tmem) tmem_st_wait();
   };
   // S = Z . Q'^T over all Gp coordinates: A from TMEM (8 columns per 16 coordinates), B from shared memory (thread 0)
@@ -360,30 +361,135 @@ __global__ void __launch_bounds__(NT, Shape<NQ, NT>::MINB) absorbed_split_gen(Pa
     }
   };
 
-  int i = 0;
-  for (; i < n_tiles; ++i) {
-    if (__syncthreads_or(!ok)) break;
+  // softmax of tile i (every thread: one token row, NH heads) and its P in
+  // shared memory.  The previous tile's pooling must be complete (P is one
+  // buffer; a rescale scales ACC).  Returns false when a failed wait ends the
+  // tile loop (every thread the same).
+  auto softmax_tile = [&](int i, int rows) -> bool {
+      // ---- softmax (every thread: one token row, NH heads)
+      float x[NH];
+      {
+        uint32_t sv[2 * NH];
+        if constexpr (NH == 32) {
+          tmem_ld32(tm + lane_base + hh * 2 * NH, sv);
+          tmem_ld32(tm + lane_base + hh * 2 * NH + 32, sv + 32);
+        } else if constexpr (NH == 16) {
+          tmem_ld32(tm + lane_base + hh * 2 * NH, sv);
+        } else {
+          tmem_ld16(tm + lane_base + hh * 2 * NH, sv);
+        }
+        tmem_ld_wait();
+        const bool valid = r < rows;
+  #pragma unroll
+        for (int k = 0; k < NH; ++k) {
+          const float s = __uint_as_float(sv[k]) + __uint_as_float(sv[NH + k]);
+          x[k] = valid ? fmaf(s, 16777216.f, ms.cneg[hh * NH + k]) : -INFINITY;
+        }
+      }
+      float xm = -INFINITY;
+  #pragma unroll
+      for (int k = 0; k < NH; ++k) xm = fmaxf(xm, x[k]);
+      // the rescale decision is the CTA's (every token of a head shares one max);
+      // a failed wait ends the loop for every thread (two barriers, in this order)
+      const int vote = __syncthreads_count((i == 0 || xm > kTau) ? 1 : 0);
+      if (__syncthreads_or(!ok)) return false;
+      if (vote > 0) {
+        // raise the running max of each head: m <- m + max(0, tile max of x) (the first tile: its max)
+  #pragma unroll
+        for (int k = 0; k < NH; ++k) {
+          float v = x[k];
+  #pragma unroll
+          for (int off = 16; off; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+          if (lane == 0) ms.red[warp][hh * NH + k] = v;
+        }
+        __syncthreads();
+        float f[NH];
+  #pragma unroll
+        for (int k = 0; k < NH; ++k) {
+          const int h = hh * NH + k;
+          const int w0 = 4 * hh;  // the four warps holding head h's tokens
+          const float d = fmaxf(fmaxf(ms.red[w0][h], ms.red[w0 + 1][h]), fmaxf(ms.red[w0 + 2][h], ms.red[w0 + 3][h]));
+          const float sh = (i == 0) ? (d == -INFINITY ? 0.f : d) : fmaxf(d, 0.f);
+          f[k] = (i == 0) ? 0.f : exp2f(-sh);
+          x[k] -= sh;
+          lsum[k] *= f[k];
+          if (q4 == 0 && lane == 0) ms.cneg[h] -= sh;
+        }
+        if (i > 0) {
+          // ACC holds every earlier tile (its pooling is done): scale this warp's lanes of its heads
+  #pragma unroll 1
+          for (int mb = 0; mb < pl.NMB; ++mb) {
+            uint32_t a[NH];
+            const uint32_t ta = tm + lane_base + 2 * NQ + mb * NQ + hh * NH;
+            if constexpr (NH == 32) tmem_ld32(ta, a);
+            else if constexpr (NH == 16) tmem_ld16(ta, a);
+            else tmem_ld8(ta, a);
+            tmem_ld_wait();
+  #pragma unroll
+            for (int k = 0; k < NH; ++k) a[k] = __float_as_uint(__uint_as_float(a[k]) * f[k]);
+            if constexpr (NH == 32) tmem_st32(ta, a);
+            else if constexpr (NH == 16) tmem_st16(ta, a);
+            else tmem_st8(ta, a);
+          }
+          tmem_st_wait();
+        }
+      }
+      // P row of this token (fp16, MN-major blocks: 8 tokens x 8 heads); the sum
+      // takes the rounded weights the pooling MMA sees
+  #pragma unroll
+      for (int k8 = 0; k8 < NH / 8; ++k8) {
+        uint32_t hv[4];
+  #pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int k = 8 * k8 + 2 * e;
+          const __half2 h2 = __floats2half2_rn(ex2_approx(x[k]), ex2_approx(x[k + 1]));
+          const float2 back = __half22float2(h2);
+          lsum[k] += back.x;
+          lsum[k + 1] += back.y;
+          hv[e] = *reinterpret_cast<const uint32_t *>(&h2);
+        }
+        const int hb = (hh * NH) / 8 + k8;
+        *reinterpret_cast<uint4 *>(ps + ((size_t)hb * (kTile / 8) + (r >> 3)) * 128 + (r & 7) * 16) =
+            make_uint4(hv[0], hv[1], hv[2], hv[3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncthreads();
+    return true;
+  };
+  // the tile's codes (full tiles: the bulk copy; the ragged last tile: plain loads, zero past its rows)
+  auto take_codes = [&](int i) -> bool {
     const int rows = tile_rows(i);
-    const uint8_t *ct = cs + (i & 1) * cbb;
-    // ---- this tile's codes; Z is free once the previous tile's pooling is done
-    if (rows == kTile) {
-      if (!wait_bar(&ms.full[i & 1], (uint32_t)(i >> 1) & 1u, abort, kWaitNs)) ok = false;
-    }
-    if (i > 0 && !wait_bar(&ms.p_done, (uint32_t)(i - 1) & 1u, abort, kWaitNs)) ok = false;
-    if (__syncthreads_or(!ok)) break;
+    if (rows == kTile && !wait_bar(&ms.full[i & 1], (uint32_t)(i >> 1) & 1u, abort, kWaitNs)) ok = false;
+    if (__syncthreads_or(!ok)) return false;
     if (pend[i & 1] == i) pend[i & 1] = -1;  // every thread saw the copy complete
     if (rows < kTile) {
-      // ragged last tile: its buffer is free (no copy was issued into it); zero past the rows
+      // ragged last tile: its buffer is free (no copy was issued into it)
       uint8_t *dst = cs + (i & 1) * cbb;
       const uint8_t *src = gcodes + (int64_t)i * kTile * pl.RB;
       const int nb = rows * pl.RB;
       for (int k = tid; k < kTile * pl.RB; k += kThreads) dst[k] = k < nb ? src[k] : (uint8_t)0;
       __syncthreads();
     }
-    // ---- unpack (Z to TMEM for the scores and to shared memory for the pooling), then the scores
-    unpack(ct, 0, true);
-    if (nch == 2) unpack(ct, 1, true);  // shared memory keeps the second chunk
-    else issue_copy(i + 2);             // this tile's code buffer has been read
+    return true;
+  };
+
+  int i = 0;
+  for (; i < n_tiles; ++i) {
+    if (__syncthreads_or(!ok)) break;
+    const uint8_t *ct = cs + (i & 1) * cbb;
+    // Z is free once the previous tile's pooling is done
+    if (i > 0 && !wait_bar(&ms.p_done, (uint32_t)(i - 1) & 1u, abort, kWaitNs)) ok = false;
+    if (!take_codes(i)) break;
+    // Z to TMEM for the scores and to shared memory for the pooling (with two
+    // chunks, shared memory keeps the second)
+    if (nch == 1) {
+      unpack(ct, 0, true, true);
+      issue_copy(i + 2);  // this tile's code buffer has been read
+    } else {
+      unpack(ct, 0, true, false);
+      unpack(ct, 1, true, true);
+    }
     tc_fence_before();
     __syncthreads();
     if (tid == 0) {
@@ -392,96 +498,7 @@ __global__ void __launch_bounds__(NT, Shape<NQ, NT>::MINB) absorbed_split_gen(Pa
     }
     if (!wait_bar(&ms.s_full, (uint32_t)i & 1u, abort, kWaitNs)) ok = false;
     tc_fence_after();
-    // ---- softmax (every thread: one token row, NH heads)
-    float x[NH];
-    {
-      uint32_t sv[2 * NH];
-      if constexpr (NH == 32) {
-        tmem_ld32(tm + lane_base + hh * 2 * NH, sv);
-        tmem_ld32(tm + lane_base + hh * 2 * NH + 32, sv + 32);
-      } else if constexpr (NH == 16) {
-        tmem_ld32(tm + lane_base + hh * 2 * NH, sv);
-      } else {
-        tmem_ld16(tm + lane_base + hh * 2 * NH, sv);
-      }
-      tmem_ld_wait();
-      const bool valid = r < rows;
-#pragma unroll
-      for (int k = 0; k < NH; ++k) {
-        const float s = __uint_as_float(sv[k]) + __uint_as_float(sv[NH + k]);
-        x[k] = valid ? fmaf(s, 16777216.f, ms.cneg[hh * NH + k]) : -INFINITY;
-      }
-    }
-    float xm = -INFINITY;
-#pragma unroll
-    for (int k = 0; k < NH; ++k) xm = fmaxf(xm, x[k]);
-    // the rescale decision is the CTA's (every token of a head shares one max);
-    // a failed wait ends the loop for every thread (two barriers, in this order)
-    const int vote = __syncthreads_count((i == 0 || xm > kTau) ? 1 : 0);
-    if (__syncthreads_or(!ok)) break;
-    if (vote > 0) {
-      // raise the running max of each head: m <- m + max(0, tile max of x) (the first tile: its max)
-#pragma unroll
-      for (int k = 0; k < NH; ++k) {
-        float v = x[k];
-#pragma unroll
-        for (int off = 16; off; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-        if (lane == 0) ms.red[warp][hh * NH + k] = v;
-      }
-      __syncthreads();
-      float f[NH];
-#pragma unroll
-      for (int k = 0; k < NH; ++k) {
-        const int h = hh * NH + k;
-        const int w0 = 4 * hh;  // the four warps holding head h's tokens
-        const float d = fmaxf(fmaxf(ms.red[w0][h], ms.red[w0 + 1][h]), fmaxf(ms.red[w0 + 2][h], ms.red[w0 + 3][h]));
-        const float sh = (i == 0) ? (d == -INFINITY ? 0.f : d) : fmaxf(d, 0.f);
-        f[k] = (i == 0) ? 0.f : exp2f(-sh);
-        x[k] -= sh;
-        lsum[k] *= f[k];
-        if (q4 == 0 && lane == 0) ms.cneg[h] -= sh;
-      }
-      if (i > 0) {
-        // ACC holds every earlier tile (its pooling is done): scale this warp's lanes of its heads
-#pragma unroll 1
-        for (int mb = 0; mb < pl.NMB; ++mb) {
-          uint32_t a[NH];
-          const uint32_t ta = tm + lane_base + 2 * NQ + mb * NQ + hh * NH;
-          if constexpr (NH == 32) tmem_ld32(ta, a);
-          else if constexpr (NH == 16) tmem_ld16(ta, a);
-          else tmem_ld8(ta, a);
-          tmem_ld_wait();
-#pragma unroll
-          for (int k = 0; k < NH; ++k) a[k] = __float_as_uint(__uint_as_float(a[k]) * f[k]);
-          if constexpr (NH == 32) tmem_st32(ta, a);
-          else if constexpr (NH == 16) tmem_st16(ta, a);
-          else tmem_st8(ta, a);
-        }
-        tmem_st_wait();
-      }
-    }
-    // P row of this token (fp16, MN-major blocks: 8 tokens x 8 heads); the sum
-    // takes the rounded weights the pooling MMA sees
-#pragma unroll
-    for (int k8 = 0; k8 < NH / 8; ++k8) {
-      uint32_t hv[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int k = 8 * k8 + 2 * e;
-        const __half2 h2 = __floats2half2_rn(ex2_approx(x[k]), ex2_approx(x[k + 1]));
-        const float2 back = __half22float2(h2);
-        lsum[k] += back.x;
-        lsum[k + 1] += back.y;
-        hv[e] = *reinterpret_cast<const uint32_t *>(&h2);
-      }
-      const int hb = (hh * NH) / 8 + k8;
-      *reinterpret_cast<uint4 *>(ps + ((size_t)hb * (kTile / 8) + (r >> 3)) * 128 + (r & 7) * 16) =
-          make_uint4(hv[0], hv[1], hv[2], hv[3]);
-    }
-    fence_proxy_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    // ---- pooling
+    if (!softmax_tile(i, tile_rows(i))) break;
     if (nch == 1) {
       if (tid == 0) {
         pool_mmas(0, i);
@@ -495,7 +512,7 @@ __global__ void __launch_bounds__(NT, Shape<NQ, NT>::MINB) absorbed_split_gen(Pa
       }
       if (!wait_bar(&ms.p_mid, (uint32_t)i & 1u, abort, kWaitNs)) ok = false;
       if (__syncthreads_or(!ok)) break;
-      unpack(ct, 0, false);
+      unpack(ct, 0, false, true);
       __syncthreads();
       issue_copy(i + 2);  // this tile's code buffer has been read
       if (tid == 0) {
