@@ -166,6 +166,13 @@ __device__ __forceinline__ void unpack_word(uint32_t w, uint32_t *o) {
   }
 }
 
+// 32 lanes x 32 bit, 4 consecutive columns: thread i <-> lane (base + i)
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(r0), "r"(r1), "r"(r2),
+               "r"(r3)
+               : "memory");
+}
+
 // (n 2^-24, m 2^-24) -> ((n - L/2) 2^-24, (m - L/2) 2^-24): an fp16 subtraction
 // of subnormals whose result is a subnormal, so exact
 template <int BITS>
