@@ -397,13 +397,20 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
         if constexpr (C::TMA) {
           const int rr = 32 * q + lane;
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const uint4 u = *reinterpret_cast<const uint4 *>(tile + swz(rr, c0 / 4 + v));
-            r[8 * v + 0] = nib_even(u.x); r[8 * v + 1] = nib_odd(u.x);
-            r[8 * v + 2] = nib_even(u.y); r[8 * v + 3] = nib_odd(u.y);
-            r[8 * v + 4] = nib_even(u.z); r[8 * v + 5] = nib_odd(u.z);
-            r[8 * v + 6] = nib_even(u.w); r[8 * v + 7] = nib_odd(u.w);
+          for (int hv = 0; hv < 2; ++hv) {
+            uint32_t r16[16];
+#pragma unroll
+            for (int v2 = 0; v2 < 2; ++v2) {
+              const int v = 2 * hv + v2;
+              const uint4 u = *reinterpret_cast<const uint4 *>(tile + swz(rr, c0 / 4 + v));
+              r16[8 * v2 + 0] = nib_even(u.x); r16[8 * v2 + 1] = nib_odd(u.x);
+              r16[8 * v2 + 2] = nib_even(u.y); r16[8 * v2 + 3] = nib_odd(u.y);
+              r16[8 * v2 + 4] = nib_even(u.z); r16[8 * v2 + 5] = nib_odd(u.z);
+              r16[8 * v2 + 6] = nib_even(u.w); r16[8 * v2 + 7] = nib_odd(u.w);
+            }
+            tmem_st16(cbase + 2 * c0 + 16 * hv, r16);
           }
+          continue;
         } else {
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
@@ -452,7 +459,7 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
       for (int h = 0; h < C::NH; ++h) {
         const int byte0 = 64 * h + 16 * q;  // first byte of this warp's 32 coordinates
         if (byte0 >= C::HALF) continue;
-        uint32_t lo[16], hi[16];
+        uint32_t lo[16];
         // y[2j + e]: the 8x8 block of 16-bit groups (four nibbles of one token)
         // of tokens 8 tb .. 8 tb + 7, tb = 8c + 2j + e, transposed, so this
         // thread holds one group (four coordinates) of two tokens
@@ -474,15 +481,27 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
             y[m] = movmatrix_trans(lds_u32_a2(tile + rr * C::HALF + byte0 + 4 * (lane & 3)));
           }
         }
+        // nibbles 0, 1 of each group (n 2^-24, n 2^-20) to lanes +0..15, then
+        // nibbles 2, 3 to lanes +16..31: 16 live results at a time
+        const uint32_t cbase = tm + lane_base + C::OFF_CP + cb * C::CP_CHUNK + h * 32;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
 #pragma unroll
-          for (int e = 0; e < 2; ++e)
-            nib_sub4(y[2 * j + e], lo[4 * j + e], lo[4 * j + 2 + e], hi[4 * j + e], hi[4 * j + 2 + e]);
+          for (int e = 0; e < 2; ++e) {
+            lo[4 * j + e] = y[2 * j + e] & 0x000F000Fu;
+            lo[4 * j + 2 + e] = y[2 * j + e] & 0x00F000F0u;
+          }
         }
-        const uint32_t cbase = tm + lane_base + C::OFF_CP + cb * C::CP_CHUNK + h * 32;
         tmem_st_16x256b_x4(cbase, lo);
-        tmem_st_16x256b_x4(cbase + (16u << 16), hi);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            lo[4 * j + e] = (y[2 * j + e] >> 8) & 0x000F000Fu;
+            lo[4 * j + 2 + e] = (y[2 * j + e] >> 8) & 0x00F000F0u;
+          }
+        }
+        tmem_st_16x256b_x4(cbase + (16u << 16), lo);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&ms.empty[st]);
@@ -541,14 +560,17 @@ __global__ void __launch_bounds__(Cfg<G, NQ>::THREADS, 1) absorbed_split_tc(cons
     static_assert(HQ == 8, "softmax warps own eight heads");
     // x <- score - m of one tile from its raw S (a, b terms); rows past the
     // split's end (ragged last tile only) take no weight; returns the row max
+    float sgr[HQ];  // the group's per-head scales, held for the whole split
+#pragma unroll
+    for (int n = 0; n < HQ; ++n) sgr[n] = ms.sig[h0 + n];
     auto scores = [&](int i, const uint32_t (&ra)[HQ], const uint32_t (&rb)[HQ], float (&x)[HQ]) -> float {
-      const float4 *sg4 = reinterpret_cast<const float4 *>(ms.sig + h0);
       const float4 *cm4 = reinterpret_cast<const float4 *>(cm);
       float lm = -INFINITY;
 #pragma unroll
       for (int n4 = 0; n4 < HQ / 4; ++n4) {
-        const float4 sg = sg4[n4], cc = cm4[n4];
-        const float sv[4] = {sg.x, sg.y, sg.z, sg.w}, cv[4] = {cc.x, cc.y, cc.z, cc.w};
+        const float4 cc = cm4[n4];
+        const float sv[4] = {sgr[4 * n4], sgr[4 * n4 + 1], sgr[4 * n4 + 2], sgr[4 * n4 + 3]};
+        const float cv[4] = {cc.x, cc.y, cc.z, cc.w};
 #pragma unroll
         for (int e = 0; e < 4; e += 2) {
           const int n = 4 * n4 + e;
