@@ -4,17 +4,21 @@
 //   slide deck frames "A wide product code uses four bits per coordinate" and
 //   "the grid size is an allocation choice": L = 4, 16, 256 at b = 2, 4, 8).
 //
-// One CTA computes a tile of 128 tokens x NC coordinates (NC = 64, 48, 32 or
-// 16, whichever divides G rounded up to 16), so that a prefill chunk spreads
-// over many SMs.  Warp 0 streams 64-wide slices of C of x and E into a ring of
-// shared-memory stages by TMA (128-byte swizzle, rows past the tensor read as
-// zero); one lane of warp 1 issues tcgen05.mma kind::f16 (bf16 x bf16 -> fp32)
-// with both operands K-major in that swizzled layout; after the last slice
-// all four warps read their 32 token rows of the accumulator from TMEM, count
-// thresholds and store the packed bytes.  Every wait is bounded; a wait that
-// gives up records FSQ_ERR_TIMEOUT in the caller's status word (if any), and
-// the CTA lets its copies and MMAs finish (waits with their own fixed limit)
-// and exits.
+// Two kernels share the operand pipeline: warp 0 streams 64-wide slices of C
+// of x and E into a ring of shared-memory stages by TMA (128-byte swizzle,
+// rows past the tensor read as zero); one lane of warp 1 issues tcgen05.mma
+// kind::f16 (bf16 x bf16 -> fp32) with both operands K-major in that swizzled
+// layout.
+//  - encode_pack_ks (G <= 256): a CTA owns 128 tokens x all coordinates of a
+//    coordinate tile, over a slice of C; the CTAs of a thread-block cluster
+//    add their partial sums through distributed shared memory (below).
+//  - encode_pack_tc (wider G): a CTA owns 128 tokens x NC coordinates (NC =
+//    64, 48, 32 or 16, whichever divides G rounded up to 16) over all of C;
+//    after the last slice its four warps read their token rows of the
+//    accumulator from TMEM, count thresholds and store the packed bytes.
+// Every wait is bounded; a wait that gives up records FSQ_ERR_TIMEOUT in the
+// caller's status word (if any), and the CTA lets its copies and MMAs finish
+// (waits with their own fixed limit) and exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
