@@ -75,11 +75,14 @@ def check_codes(got, x, E, G, label, levels=16):
 # Past 64 tokens at G <= 256 the append splits C over a cluster of ks = 1..8
 # CTAs (ks = 8 up to 18 token tiles, 4 up to 37, then 2 and 1; never more
 # than the 64-wide slices of C): the last four cases take ks = 1 (one slice),
-# ks = 2, an uneven split (three slices over two CTAs) and ks = 1 by token count.
+# ks = 2, an uneven split (three slices over two CTAs) and ks = 1 by token count;
+# then widths whose coordinate tiles are ragged: G = 2 (one 16-wide tile), and
+# G = 144 and 240, split into two tiles of 80 and 128 whose second tile holds
+# only 64 and 112 coordinates of G.
 @pytest.mark.parametrize("n_tok,C,G", [(1024, 1024, 256), (4096, 2048, 256), (4096, 4096, 256), (4096, 4096, 84),
                                        (1, 1024, 84), (16, 4096, 256), (17, 2048, 84), (37, 2048, 256),
                                        (129, 4096, 84), (300, 64, 256), (200, 128, 84), (1000, 192, 256),
-                                       (16384, 1024, 84)])
+                                       (16384, 1024, 84), (130, 1024, 2), (777, 1024, 144), (500, 2048, 240)])
 def test_encode_pack_parity(n_tok, C, G):
     gen = synth._gen(synth.workload_seed(21, n_tok, C, G))
     x, E = synth.encoder_inputs(n_tok, C, G, gen)
