@@ -1,5 +1,5 @@
 // Inline-PTX building blocks for sm_100a: mbarriers with bounded waits, 1-D
-// bulk copies (no multicast), tcgen05 TMEM allocation / MMA / ld / st, and
+// bulk copies into this CTA's shared memory, tcgen05 TMEM allocation / MMA / ld / st, and
 // shared-memory matrix descriptors.  Written from the PTX ISA's descriptions
 // of these instructions.
 #pragma once
