@@ -493,8 +493,8 @@ MULTI_POINTS = (("qwen3_8b_32x", 16, 4, 32768), ("qwen3_8b_32x", 16, 8, 32768), 
 def multi_points(args, torch, F, synth, peaks):
     """fsq_decode_attn_multi: n_new queries per row, each attending causally to
     the code cache.  A step appends each row's n_new new tokens (one append
-    call per row: the rows' new tokens are not one strided block) and runs the
-    multi-query attention.  One JSON line per point with the step time, the
+    call for all rows: groups of n_new tokens, one group per cache row) and
+    runs the multi-query attention.  One JSON line per point with the step time, the
     split kernel's time and its roofline (codes read once; FLOPs of n_new
     queries per cached token)."""
     device = torch.device("cuda", 0)
@@ -517,13 +517,15 @@ def multi_points(args, torch, F, synth, peaks):
         opts = F.attn_opts(levels=wl.levels)
         wbuf = F.Workspace(device).get(F.multi_workspace_size(B, n_new, T, wl.n_q, wl.n_kv, wl.d_h, G, opts))
 
+        grouped = F.encode_opts(tokens_per_row=n_new, row_stride_bytes=bstride)
+
         def step(i, prof=None):
             cache = st["caches"][i % n_copies]
-            for b in range(B):  # row b's n_new new tokens at positions T - n_new .. T - 1
-                rc = F.encode_pack_raw(x_new.data_ptr() + b * n_new * wl.C * 2, n_new, wl.C, wl.C, st["E"].data_ptr(),
-                                       G, qp, cache.data_ptr() + b * bstride + (T - n_new) * rb, rb, sptr)
-                if rc:
-                    raise F.FsqError(rc, "fsq_encode_pack")
+            # row b's n_new new tokens (x_new rows b*n_new ..) at positions T - n_new .. T - 1
+            rc = F.encode_pack_raw(x_new.data_ptr(), B * n_new, wl.C, wl.C, st["E"].data_ptr(), G, qp,
+                                   cache.data_ptr() + (T - n_new) * rb, rb, sptr, grouped)
+            if rc:
+                raise F.FsqError(rc, "fsq_encode_pack")
             rc = F.decode_attn_multi_raw(q.data_ptr(), B, n_new, wl.n_q, wl.d_h, cache.data_ptr(), bstride, T, G,
                                          st["W_kv"].data_ptr(), wl.n_kv,
                                          F.attn_opts(levels=wl.levels, prof_events=prof), wbuf.data_ptr(),
@@ -558,7 +560,7 @@ def multi_points(args, torch, F, synth, peaks):
                "roofline_bound": "tensor" if t_f >= t_b else "hbm", "roofline_frac": max(t_b, t_f) / t,
                "tflops": flops / t / 1e12, "code_gbs": code_bytes / t / 1e9,
                "l2": f"{n_copies} rotating caches" if n_copies > 1 else "codes larger than L2",
-               "launches_per_step": B + 3, "peak_source": peaks["source"] + " (burst)"}
+               "launches_per_step": 4, "peak_source": peaks["source"] + " (burst)"}
         print(json.dumps(row), flush=True)
         out_rows.append(row)
         del st, q, x_new, out, wbuf

@@ -8,7 +8,7 @@ ctypes binding plus seeded synthetic inputs.  PyTorch only provides device
 memory and streams.  The library is loaded on first use.
 """
 from ._abi import (  # noqa: F401
-    EXPORTED, FSQ_OK, FSQ_ERR_CUDA, FSQ_ERR_INVALID_ARG, FSQ_ERR_MISALIGNED, FSQ_ERR_TIMEOUT,
+    EXPORTED, FSQ_OK, append_rows, FSQ_ERR_CUDA, FSQ_ERR_INVALID_ARG, FSQ_ERR_MISALIGNED, FSQ_ERR_TIMEOUT,
     FSQ_ERR_UNSUPPORTED, FSQ_ERR_WORKSPACE, AttnOpts, EncodeOpts, FsqError, QuantParams, Workspace, attn_opts,
     decode_attn, decode_attn_multi, decode_attn_multi_raw, decode_attn_noalloc_status, decode_attn_raw,
     multi_workspace_size, split_kernel, encode_opts, encode_pack, encode_pack_raw, quant_params,

@@ -48,7 +48,8 @@ class AttnOpts(C.Structure):
 
 
 class EncodeOpts(C.Structure):
-    _fields_ = [("status_word", C.c_void_p), ("debug_stall_ns", C.c_uint32)]
+    _fields_ = [("status_word", C.c_void_p), ("debug_stall_ns", C.c_uint32), ("tokens_per_row", C.c_int64),
+                ("row_stride_bytes", C.c_int64)]
 
 
 class FsqError(RuntimeError):
@@ -171,9 +172,12 @@ def attn_opts(variant="auto", scale=0.0, num_splits=0, rope_knorm=False, rope_ba
     return o
 
 
-def encode_opts(status_word=None, debug_stall_ns=0) -> EncodeOpts:
-    """status_word: a device tensor whose first 4 bytes are the caller's status word."""
-    o = EncodeOpts(None if status_word is None else int(status_word.data_ptr()), int(debug_stall_ns))
+def encode_opts(status_word=None, debug_stall_ns=0, tokens_per_row=0, row_stride_bytes=0) -> EncodeOpts:
+    """status_word: a device tensor whose first 4 bytes are the caller's status
+    word; tokens_per_row / row_stride_bytes: groups of consecutive tokens, each
+    group written at its own cache row (0: one stride between tokens)."""
+    o = EncodeOpts(None if status_word is None else int(status_word.data_ptr()), int(debug_stall_ns),
+                   int(tokens_per_row), int(row_stride_bytes))
     o._tensors = (status_word,)  # keeps the word's memory alive with the struct
     return o
 
@@ -259,6 +263,25 @@ def encode_pack(x, E, h=None, delta=0.5, out=None, stream=None, status_word=None
                          ldc, _stream_ptr(stream), encode_opts(status_word))
     _check(st, "fsq_encode_pack")
     return out
+
+
+def append_rows(x, E, cache, t0, h=None, delta=0.5, stream=None, status_word=None, levels=16):
+    """One call appends n new tokens to each of the B rows of a [B, T_max, R]
+    uint8 code cache: x is [B * n, C] (row b's tokens are x[b*n:(b+1)*n]) and
+    they go to cache[b, t0:t0+n] (fsq_encode_opts.tokens_per_row = n)."""
+    B, T_max, rb = cache.shape
+    n_tok, C_ = x.shape
+    G = E.shape[0]
+    if B < 1 or n_tok % B or rb != row_bytes(G, levels) or cache.stride(2) != 1 or cache.stride(1) != rb:
+        raise ValueError("append_rows: x must hold B * n rows and cache must be [B, T_max, G*b/8], rows contiguous")
+    n = n_tok // B
+    if not 0 <= t0 <= T_max - n:
+        raise ValueError("append_rows: positions t0 .. t0+n-1 must lie inside the cache")
+    st = encode_pack_raw(_ptr(x), n_tok, x.stride(0), C_, _ptr(E), G, quant_params(h, delta, levels),
+                         int(cache.data_ptr()) + t0 * rb, rb, _stream_ptr(stream),
+                         encode_opts(status_word, tokens_per_row=n, row_stride_bytes=cache.stride(0)))
+    _check(st, "fsq_encode_pack")
+    return cache
 
 
 def quantize_pack_f32(u, h=None, delta=0.5, out=None, stream=None, levels=16):

@@ -9,8 +9,8 @@
 
 namespace fsq {
 cudaError_t launch_encode_pack(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C, const uint16_t *E, int G,
-                               int levels, const float *th, uint8_t *codes, int64_t ldc, uint32_t *status,
-                               uint32_t stall_ns, cudaStream_t s);
+                               int levels, const float *th, uint8_t *codes, int64_t ldc, int64_t per_row,
+                               int64_t row_stride, uint32_t *status, uint32_t stall_ns, cudaStream_t s);
 cudaError_t launch_quantize_pack_f32(const float *u, int64_t n_tok, int G, int levels, const float *th,
                                      uint8_t *codes, int64_t ldc, cudaStream_t s);
 cudaError_t launch_absorbed_simt(const uint16_t *q, const uint8_t *codes, int64_t bstride, int64_t B, int n_new,
@@ -251,9 +251,12 @@ fsq_status fsq_encode_pack(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_
   if (!aligned16(x) || !aligned16(E) || ldx % 8) return FSQ_ERR_MISALIGNED;
   uint32_t *status = opts ? opts->status_word : nullptr;
   if ((uintptr_t)status & 3u) return FSQ_ERR_MISALIGNED;
+  const int64_t per_row = opts ? opts->tokens_per_row : 0;
+  const int64_t row_stride = opts ? opts->row_stride_bytes : 0;
+  if (per_row < 0 || (per_row > 0 && row_stride < 0)) return FSQ_ERR_INVALID_ARG;
   float th[kMaxLevels - 1];
   make_thresholds(qp, th);
-  return from_cuda(launch_encode_pack(x, n_tok, ldx, C, E, G, L, th, codes, ldc_bytes, status,
+  return from_cuda(launch_encode_pack(x, n_tok, ldx, C, E, G, L, th, codes, ldc_bytes, per_row, row_stride, status,
                                       opts ? opts->debug_stall_ns : 0u, (cudaStream_t)stream));
 }
 

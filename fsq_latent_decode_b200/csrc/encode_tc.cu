@@ -25,6 +25,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "encode.cuh"
 #include "tc_ptx.cuh"
 
 namespace fsq {
@@ -131,8 +132,8 @@ __device__ __forceinline__ void pack_store16(const uint32_t (&v)[16], const Thre
 template <int NC, int L>
 __global__ void __launch_bounds__(kThreads, 1)
     encode_pack_tc(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap te, int64_t n_tok,
-                   int64_t C, int G, const __grid_constant__ Thresholds<L> th, uint8_t *__restrict__ codes,
-                   int64_t ldc, uint32_t *status, uint32_t stall_ns) {
+                   int64_t C, int G, const __grid_constant__ Thresholds<L> th, const CodeRows dst,
+                   uint32_t *status, uint32_t stall_ns) {
   using EC = ECfg<NC>;
   extern __shared__ __align__(1024) uint8_t esm[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(esm) + 1023) & ~uintptr_t(1023));
@@ -233,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t v[16];
       tmem_ld16(tl + j0, v);
       tmem_ld_wait();
-      if (row < n_tok) pack_store16<L>(v, th, codes + row * ldc + (n0 + j0) * BITS / 8, min(16, G - (n0 + j0)));
+      if (row < n_tok) pack_store16<L>(v, th, dst.row(row) + (n0 + j0) * BITS / 8, min(16, G - (n0 + j0)));
     }
   }
   tc_fence_before();
@@ -275,7 +276,7 @@ cudaError_t make_bf16_map(CUtensorMap *map, const uint16_t *base, int64_t rows, 
 
 template <int NC, int L>
 cudaError_t launch_nc(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C, const uint16_t *E, int G,
-                      const Thresholds<L> &th, uint8_t *codes, int64_t ldc, uint32_t *status, uint32_t stall_ns,
+                      const Thresholds<L> &th, const CodeRows &dst, uint32_t *status, uint32_t stall_ns,
                       cudaStream_t s) {
   using EC = ECfg<NC>;
   CUtensorMap tx, te;
@@ -287,7 +288,7 @@ cudaError_t launch_nc(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C, 
   if (e != cudaSuccess) return e;
   const int gp = (G + 15) / 16 * 16;
   const dim3 grid((unsigned)(gp / NC), (unsigned)((n_tok + kM - 1) / kM));
-  encode_pack_tc<NC, L><<<grid, kThreads, EC::SMEM, s>>>(tx, te, n_tok, C, G, th, codes, ldc, status, stall_ns);
+  encode_pack_tc<NC, L><<<grid, kThreads, EC::SMEM, s>>>(tx, te, n_tok, C, G, th, dst, status, stall_ns);
   return cudaGetLastError();
 }
 
@@ -383,8 +384,8 @@ __device__ __forceinline__ void cluster_sync_all() {
 template <int TN, int L>
 __global__ void __launch_bounds__(kKsThreads, 1)
     encode_pack_ks(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap te, int64_t n_tok,
-                   int64_t C, int G, const __grid_constant__ Thresholds<L> th, uint8_t *__restrict__ codes,
-                   int64_t ldc, uint32_t *status, uint32_t stall_ns) {
+                   int64_t C, int G, const __grid_constant__ Thresholds<L> th, const CodeRows dst,
+                   uint32_t *status, uint32_t stall_ns) {
   using KC = KsCfg<TN>;
   extern __shared__ __align__(1024) uint8_t esm[];
   uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(esm) + 1023) & ~uintptr_t(1023));
@@ -497,7 +498,7 @@ __global__ void __launch_bounds__(kKsThreads, 1)
         tmem_ld16(tl + 16 * g, v);
         tmem_ld_wait();
         if (row < n_tok)
-          pack_store16<L>(v, th, codes + row * ldc + (n0 + 16 * g) * BITS / 8, min(16, Gt - 16 * g), ms.th);
+          pack_store16<L>(v, th, dst.row(row) + (n0 + 16 * g) * BITS / 8, min(16, Gt - 16 * g), ms.th);
       }
     }
   } else {
@@ -584,7 +585,7 @@ __global__ void __launch_bounds__(kKsThreads, 1)
           uint32_t v[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(acc[e]);
-          pack_store16<L>(v, th, codes + row * ldc + (n0 + 16 * g) * BITS / 8, min(16, Gt - 16 * g), ms.th);
+          pack_store16<L>(v, th, dst.row(row) + (n0 + 16 * g) * BITS / 8, min(16, Gt - 16 * g), ms.th);
         }
       }
     }
@@ -617,7 +618,7 @@ inline int tn_of(int gp, int64_t n_tiles) { return gp >= 128 && 2 * n_tiles <= 1
 
 template <int TN, int L>
 cudaError_t launch_ks(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C, const uint16_t *E, int G,
-                      const Thresholds<L> &th, uint8_t *codes, int64_t ldc, uint32_t *status, uint32_t stall_ns,
+                      const Thresholds<L> &th, const CodeRows &dst, uint32_t *status, uint32_t stall_ns,
                       cudaStream_t s) {
   using KC = KsCfg<TN>;
   CUtensorMap tx, te;
@@ -642,19 +643,19 @@ cudaError_t launch_ks(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C, 
   at[0].val.clusterDim.z = 1;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, encode_pack_ks<TN, L>, tx, te, n_tok, C, G, th, codes, ldc, status, stall_ns);
+  e = cudaLaunchKernelEx(&cfg, encode_pack_ks<TN, L>, tx, te, n_tok, C, G, th, dst, status, stall_ns);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
 template <int L>
 cudaError_t launch_ks_g(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C, const uint16_t *E, int G,
-                        const Thresholds<L> &th, uint8_t *codes, int64_t ldc, uint32_t *status, uint32_t stall_ns,
+                        const Thresholds<L> &th, const CodeRows &dst, uint32_t *status, uint32_t stall_ns,
                         cudaStream_t s) {
   switch (tn_of((G + 15) / 16 * 16, (n_tok + kM - 1) / kM) / 16) {
 #define FSQ_KS_CASE(n) \
   case n:              \
-    return launch_ks<16 * n, L>(x, n_tok, ldx, C, E, G, th, codes, ldc, status, stall_ns, s);
+    return launch_ks<16 * n, L>(x, n_tok, ldx, C, E, G, th, dst, status, stall_ns, s);
     FSQ_KS_CASE(1) FSQ_KS_CASE(2) FSQ_KS_CASE(3) FSQ_KS_CASE(4) FSQ_KS_CASE(5) FSQ_KS_CASE(6) FSQ_KS_CASE(7)
     FSQ_KS_CASE(8) FSQ_KS_CASE(9) FSQ_KS_CASE(10) FSQ_KS_CASE(11) FSQ_KS_CASE(12) FSQ_KS_CASE(13)
     FSQ_KS_CASE(14) FSQ_KS_CASE(15) FSQ_KS_CASE(16)
@@ -670,24 +671,24 @@ cudaError_t launch_ks_g(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C
 // (a multiple of 4 at L = 4).
 template <int L>
 cudaError_t launch_encode_pack_tc(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C, const uint16_t *E, int G,
-                                  const Thresholds<L> &th, uint8_t *codes, int64_t ldc, uint32_t *status,
+                                  const Thresholds<L> &th, const CodeRows &dst, uint32_t *status,
                                   uint32_t stall_ns, cudaStream_t s) {
   if (n_tok > (int64_t)65535 * enc::kM || C > 0x7fffffffLL) return cudaErrorInvalidValue;
   const int gp = (G + 15) / 16 * 16;
-  if (gp <= 256) return enc::launch_ks_g<L>(x, n_tok, ldx, C, E, G, th, codes, ldc, status, stall_ns, s);
-  if (gp % 64 == 0) return enc::launch_nc<64, L>(x, n_tok, ldx, C, E, G, th, codes, ldc, status, stall_ns, s);
-  if (gp % 48 == 0) return enc::launch_nc<48, L>(x, n_tok, ldx, C, E, G, th, codes, ldc, status, stall_ns, s);
-  if (gp % 32 == 0) return enc::launch_nc<32, L>(x, n_tok, ldx, C, E, G, th, codes, ldc, status, stall_ns, s);
-  return enc::launch_nc<16, L>(x, n_tok, ldx, C, E, G, th, codes, ldc, status, stall_ns, s);
+  if (gp <= 256) return enc::launch_ks_g<L>(x, n_tok, ldx, C, E, G, th, dst, status, stall_ns, s);
+  if (gp % 64 == 0) return enc::launch_nc<64, L>(x, n_tok, ldx, C, E, G, th, dst, status, stall_ns, s);
+  if (gp % 48 == 0) return enc::launch_nc<48, L>(x, n_tok, ldx, C, E, G, th, dst, status, stall_ns, s);
+  if (gp % 32 == 0) return enc::launch_nc<32, L>(x, n_tok, ldx, C, E, G, th, dst, status, stall_ns, s);
+  return enc::launch_nc<16, L>(x, n_tok, ldx, C, E, G, th, dst, status, stall_ns, s);
 }
 template cudaError_t launch_encode_pack_tc<4>(const uint16_t *, int64_t, int64_t, int64_t, const uint16_t *, int,
-                                              const Thresholds<4> &, uint8_t *, int64_t, uint32_t *, uint32_t,
+                                              const Thresholds<4> &, const CodeRows &, uint32_t *, uint32_t,
                                               cudaStream_t);
 template cudaError_t launch_encode_pack_tc<16>(const uint16_t *, int64_t, int64_t, int64_t, const uint16_t *, int,
-                                               const Thresholds<16> &, uint8_t *, int64_t, uint32_t *, uint32_t,
+                                               const Thresholds<16> &, const CodeRows &, uint32_t *, uint32_t,
                                                cudaStream_t);
 template cudaError_t launch_encode_pack_tc<256>(const uint16_t *, int64_t, int64_t, int64_t, const uint16_t *, int,
-                                                const Thresholds<256> &, uint8_t *, int64_t, uint32_t *, uint32_t,
+                                                const Thresholds<256> &, const CodeRows &, uint32_t *, uint32_t,
                                                 cudaStream_t);
 
 }  // namespace fsq

@@ -4,6 +4,7 @@
 // bits per coordinate" (ceil(G*b/8) bytes per token) and backup frame "the
 // grid size is an allocation choice" (L = 4, 16, 256 at b = 2, 4, 8 bits).
 #include "common.cuh"
+#include "encode.cuh"
 
 namespace fsq {
 
@@ -26,7 +27,7 @@ template <int L>
 __global__ void __launch_bounds__(256) encode_pack_rows(const uint16_t *__restrict__ x, int64_t n_tok, int64_t ldx,
                                                         int64_t C, const uint16_t *__restrict__ E, int G,
                                                         const __grid_constant__ Thresholds<L> th,
-                                                        uint8_t *__restrict__ codes, int64_t ldc) {
+                                                        const CodeRows dst) {
   constexpr int P = Pk<L>::PER, BITS = Pk<L>::BITS;
   const int rb = G / P;  // bytes per token row
   const int64_t wid = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
@@ -64,7 +65,7 @@ __global__ void __launch_bounds__(256) encode_pack_rows(const uint16_t *__restri
     uint32_t v = 0;
 #pragma unroll
     for (int c = 0; c < P; ++c) v |= fsq_code<L>(a[c], th) << (BITS * c);
-    codes[t * ldc + by] = (uint8_t)v;
+    dst.row(t)[by] = (uint8_t)v;
   }
 }
 
@@ -81,7 +82,7 @@ template <int L>
 __global__ void __launch_bounds__(kFewWarps * 32, 1)
     encode_pack_few(const uint16_t *__restrict__ x, int n_tok, int64_t ldx, int64_t C,
                     const uint16_t *__restrict__ E, int G, const __grid_constant__ Thresholds<L> th,
-                    uint8_t *__restrict__ codes, int64_t ldc) {
+                    const CodeRows dst) {
   constexpr int P = Pk<L>::PER, BITS = Pk<L>::BITS, CP = Pk<L>::CP, NPAIR = CP / 2;
   __shared__ float red[NPAIR][kFewWarps][2 * kFewTok];
   const int c0 = blockIdx.x * CP;  // first coordinate of this chunk
@@ -148,7 +149,7 @@ __global__ void __launch_bounds__(kFewWarps * 32, 1)
       uint32_t v = 0;
 #pragma unroll
       for (int c = 0; c < P; ++c) v |= cw[by * P + c] << (BITS * c);
-      codes[(int64_t)t * ldc + c0 / P + by] = (uint8_t)v;
+      dst.row(t)[c0 / P + by] = (uint8_t)v;
     }
   }
 }
@@ -182,7 +183,7 @@ Thresholds<L> table_of(const float *th) {
 
 template <int L>
 cudaError_t launch_encode_pack_tc(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C, const uint16_t *E, int G,
-                                  const Thresholds<L> &th, uint8_t *codes, int64_t ldc, uint32_t *status,
+                                  const Thresholds<L> &th, const CodeRows &dst, uint32_t *status,
                                   uint32_t stall_ns, cudaStream_t s);
 
 namespace {
@@ -190,19 +191,19 @@ namespace {
 // the tensor cores (encode_tc.cu).
 template <int L>
 cudaError_t encode_levels(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C, const uint16_t *E, int G,
-                          const float *th_host, uint8_t *codes, int64_t ldc, uint32_t *status, uint32_t stall_ns,
+                          const float *th_host, const CodeRows &dst, uint32_t *status, uint32_t stall_ns,
                           cudaStream_t s) {
   const Thresholds<L> th = table_of<L>(th_host);
   if (n_tok <= kFewTok) {
     return launch_pdl(encode_pack_few<L>, dim3((unsigned)(G / Pk<L>::CP)), dim3(kFewWarps * 32), 0, s, x, (int)n_tok,
-                      ldx, C, E, G, th, codes, ldc);
+                      ldx, C, E, G, th, dst);
   }
   if (n_tok <= 64) {
     const int64_t warps = n_tok * (G / Pk<L>::PER);
-    encode_pack_rows<L><<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(x, n_tok, ldx, C, E, G, th, codes, ldc);
+    encode_pack_rows<L><<<(unsigned)((warps + 7) / 8), 256, 0, s>>>(x, n_tok, ldx, C, E, G, th, dst);
     return cudaGetLastError();
   }
-  return launch_encode_pack_tc<L>(x, n_tok, ldx, C, E, G, th, codes, ldc, status, stall_ns, s);
+  return launch_encode_pack_tc<L>(x, n_tok, ldx, C, E, G, th, dst, status, stall_ns, s);
 }
 
 template <int L>
@@ -215,14 +216,16 @@ cudaError_t quantize_levels(const float *u, int64_t n_tok, int G, const float *t
 }
 }  // namespace
 
-// th: the levels-1 thresholds of fsq_thresholds.
+// th: the levels-1 thresholds of fsq_thresholds; per_row / row_stride: the
+// grouping of the destination rows (CodeRows; per_row = 0: one stride ldc).
 cudaError_t launch_encode_pack(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C, const uint16_t *E, int G,
-                               int levels, const float *th, uint8_t *codes, int64_t ldc, uint32_t *status,
-                               uint32_t stall_ns, cudaStream_t s) {
+                               int levels, const float *th, uint8_t *codes, int64_t ldc, int64_t per_row,
+                               int64_t row_stride, uint32_t *status, uint32_t stall_ns, cudaStream_t s) {
+  const CodeRows dst{codes, ldc, per_row, row_stride};
   switch (levels) {
-    case 4: return encode_levels<4>(x, n_tok, ldx, C, E, G, th, codes, ldc, status, stall_ns, s);
-    case 16: return encode_levels<16>(x, n_tok, ldx, C, E, G, th, codes, ldc, status, stall_ns, s);
-    case 256: return encode_levels<256>(x, n_tok, ldx, C, E, G, th, codes, ldc, status, stall_ns, s);
+    case 4: return encode_levels<4>(x, n_tok, ldx, C, E, G, th, dst, status, stall_ns, s);
+    case 16: return encode_levels<16>(x, n_tok, ldx, C, E, G, th, dst, status, stall_ns, s);
+    case 256: return encode_levels<256>(x, n_tok, ldx, C, E, G, th, dst, status, stall_ns, s);
   }
   return cudaErrorInvalidValue;
 }

@@ -172,6 +172,16 @@ typedef struct {
                              with this limit in nanoseconds, for a barrier that
                              nothing completes, so that its bounded-wait failure
                              path runs (FSQ_ERR_TIMEOUT in status_word). */
+  int64_t tokens_per_row;  /* 0: token t's codes go to codes + t*ldc_bytes.  When
+                             > 0, the n_tok tokens are groups of tokens_per_row
+                             consecutive tokens (the last group may be shorter),
+                             one group per cache row: token t goes to codes +
+                             (t / tokens_per_row)*row_stride_bytes + (t %
+                             tokens_per_row)*ldc_bytes, so one call appends the
+                             new tokens of several rows of a [B, T_max, R] cache
+                             (codes = &cache[0][T0], row_stride_bytes = T_max*R,
+                             ldc_bytes = R).  Destinations must not overlap. */
+  int64_t row_stride_bytes; /* bytes between groups (>= 0) when tokens_per_row > 0 */
 } fsq_encode_opts;
 
 /* Append path ([S] eq. 4 then packing; [D] product-code frame):
@@ -179,7 +189,7 @@ typedef struct {
  *  x      bf16 [n_tok, ldx], row t = x_t (C used entries)      — read
  *  E      bf16 [G, C] encoder                                    — read
  *  codes  uint8 [n_tok, ldc_bytes]; row t gets R = G*b/8 bytes    — written
- *  opts   may be NULL (no status word, no stall)
+ *  opts   may be NULL (no status word, no stall, one stride ldc_bytes)
  * To append at position T of a [T_max, R] cache pass codes + T*R and
  * ldc_bytes = R.  Needs: G even, 2 <= G <= FSQ_MAX_G, G % 4 == 0 at L = 4;
  * C a positive multiple of 64; ldx >= C and ldx % 8 == 0; x and E 16-byte

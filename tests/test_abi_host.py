@@ -173,6 +173,11 @@ def test_invalid_arguments_return_before_launch():
     bad_word = F.encode_opts()
     bad_word.status_word = 18  # a status word must be 4-byte aligned
     assert F.encode_pack_raw(16, 4, 64, 64, 16, 256, qp, 16, 128, null, bad_word) == F.FSQ_ERR_MISALIGNED
+    # grouped destination rows: a negative group size or row stride
+    assert F.encode_pack_raw(16, 4, 64, 64, 16, 256, qp, 16, 128, null,
+                             F.encode_opts(tokens_per_row=-1)) == F.FSQ_ERR_INVALID_ARG
+    assert F.encode_pack_raw(16, 4, 64, 64, 16, 256, qp, 16, 128, null,
+                             F.encode_opts(tokens_per_row=2, row_stride_bytes=-128)) == F.FSQ_ERR_INVALID_ARG
     assert F.quantize_pack_f32_raw(null, 3, 256, qp, null, 128, null) == F.FSQ_ERR_INVALID_ARG
     assert F.quantize_pack_f32_raw(8, 3, 256, qp, 16, 128, null) == F.FSQ_ERR_MISALIGNED
     # decode

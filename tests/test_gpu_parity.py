@@ -526,6 +526,29 @@ def test_encode_pack_levels_parity(L, G, n_tok, C):
     check_codes(got, x.float().numpy(), E.float().numpy(), G, f"L={L} n_tok={n_tok} C={C} G={G}", levels=L)
 
 
+@pytest.mark.parametrize("L,G", [(16, 256), (16, 84), (4, 320), (256, 144)])
+@pytest.mark.parametrize("n", [3, 13, 30])
+def test_append_rows_grouped(L, G, n):
+    """One call appends n tokens to each of B rows of a [B, T_max, R] cache
+    (tokens_per_row = n): every code matches the oracle, and no byte outside
+    cache[b, t0:t0+n] changes.  B*n = 15, 65, 150 tokens take the three
+    append kernels (CUDA cores up to 16 and 64 tokens, then tensor cores)."""
+    B, T_max, t0, C_ = 5, 41, 7, 1024
+    rb = G * O.bits_per_coordinate(L) // 8
+    gen = synth._gen(synth.workload_seed(141, L, G, n))
+    x, E = synth.encoder_inputs(B * n, C_, G, gen)
+    cache = torch.full((B, T_max, rb), 0xA5, dtype=torch.uint8, device=DEV)
+    word = torch.zeros(1, dtype=torch.int32, device=DEV)
+    F.append_rows(_dev(x), _dev(E), cache, t0, status_word=word, levels=L)
+    assert F.workspace_status(word) == F.FSQ_OK
+    c = cache.cpu().numpy()
+    keep = np.ones(c.shape, dtype=bool)
+    keep[:, t0:t0 + n] = False
+    assert (c[keep] == 0xA5).all()
+    check_codes(c[:, t0:t0 + n].reshape(B * n, rb), x.float().numpy(), E.float().numpy(), G,
+                f"grouped rows L={L} G={G} B={B} n={n}", levels=L)
+
+
 def test_encode_pack_levels_append_into_cache_rows():
     """Appending at row T of a larger cache writes exactly rows T..T+n-1 (row
     stride G*b/8), leaving the bytes around them as they were."""
