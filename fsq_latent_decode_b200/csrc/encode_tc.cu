@@ -293,12 +293,14 @@ cudaError_t launch_nc(const uint16_t *x, int64_t n_tok, int64_t ldx, int64_t C, 
 }
 
 // ---------------------------------------------------------------------------
-// K-split form for G <= 256: one CTA computes ALL coordinates of its 128
-// tokens (MMA N = G rounded up to 16) over a slice of C, and the ks CTAs of a
-// thread-block cluster (one per slice of C) add their fp32 partial sums
+// K-split form for G <= 256: one CTA computes every coordinate of a
+// coordinate tile for its 128 tokens (MMA N = TN: G rounded up to 16, or half
+// of that past 128 coordinates, see tn_of) over a slice of C, and the ks CTAs
+// of a thread-block cluster (one per slice of C) add their fp32 partial sums
 // through distributed shared memory.  The operand bytes a CTA streams per
 // output fall from (1/64 + 1/128) to (1/TN + 1/128) of a C-long row pair,
-// while the K split keeps as many SMs busy as the N split did.
+// while the split of C keeps as many SMs busy as a split into 64-wide
+// coordinate tiles would.
 //
 // CTA rank r owns the 16-column groups g = r, r + ks, ... of the tile.  Once
 // every CTA of the cluster has finished its MMAs (cluster barrier A: the
