@@ -211,3 +211,20 @@ def test_invalid_arguments_return_before_launch():
     assert F.lib.fsq_workspace_status(None, 256, None) == F.FSQ_ERR_INVALID_ARG
     assert F.lib.fsq_workspace_status(16, 2, None) == F.FSQ_ERR_INVALID_ARG
     assert F.lib.fsq_workspace_status(18, 4, None) == F.FSQ_ERR_MISALIGNED
+
+
+def test_append_rows_rejects_bad_shapes_before_any_call():
+    """append_rows checks the cache shape, the token count and the positions
+    on the host, before it reaches the library."""
+    import torch
+    x = torch.zeros((10, 64), dtype=torch.bfloat16)
+    E = torch.zeros((256, 64), dtype=torch.bfloat16)
+    cache = torch.zeros((5, 40, 128), dtype=torch.uint8)
+    with pytest.raises(ValueError):
+        F.append_rows(x[:9], E, cache, 0)                   # 9 tokens over 5 rows
+    with pytest.raises(ValueError):
+        F.append_rows(x, E, cache[:, :, :64], 0)            # rows of 64 bytes for G=256 at 4 bits
+    with pytest.raises(ValueError):
+        F.append_rows(x, E, cache, 39)                      # positions 39, 40 past T_max = 40
+    with pytest.raises(ValueError):
+        F.append_rows(x, E, cache[:, ::2], 0)               # every other position: token rows 256 bytes apart
